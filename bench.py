@@ -1,0 +1,454 @@
+"""Benchmark of the Nemotron-H non-gated MoE block forward on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME]
+                    [--impl ours|reference] [--no-cpu-baseline]
+
+One step = one whole block call (router, permute, routed up/down experts,
+shared expert on a second stream, finalize) over one batch of T seeded
+synthetic tokens, replayed as a CUDA graph with weights and inputs resident
+in HBM.  The timed region holds exactly K steps between two barriers +
+device synchronisations and is measured with CUDA events; with N GPUs
+(torchrun) every rank runs its own batch (token data parallelism: no
+collective on the data path) and the max over ranks is reported.
+
+Rank 0 prints one JSON line with the throughput (tokens/s), the TFLOP/s and
+roofline fractions, the dominant kernel's roofline (CUDA-event timed), the
+end-to-end throughput through the public host API, the oracle's CPU
+throughput on a bounded sample, and the SM clocks sampled during the timed
+region.  ``--impl reference`` times the fp64 CPU oracle on the same workload
+(rank 0 only) and prints the same line with ``"impl": "reference"``.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "MoE-block tokens/s and TFLOP/s (frac of bf16 peak / HBM roofline), 1×B200"
+DEFAULT_WORKLOAD = "decode_bf16_t8"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+KERNEL_SOURCES = ["non_gated_relu_b200/csrc/gemm_tc.cuh", "non_gated_relu_b200/csrc/common.cuh",
+                  "non_gated_relu_b200/csrc/nh_moe.cu"]
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=0, help="timed steps (0: about 2 s of work)")
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=synth.CONFIG_ORDER)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--batches", type=int, default=4, help="distinct input batches cycled")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+def skew_b(cfg):
+    if not cfg.skew_hot_groups:
+        return None
+    with open(os.path.join(ROOT, "tests", "golden", "skew_prefill_t2048.json")) as f:
+        return json.load(f)["b"]
+
+
+def batch_x(cfg, i):
+    """Input batch i: batch 0 is the workload's own x; others use seed offsets."""
+    c = cfg if i == 0 else cfg.replace(seed=cfg.seed + 1000 * i)
+    x, _, _, _, _ = synth.make_router_and_x(c, skew_b(cfg))
+    return x
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.idx = gpu_index
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.idx}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.t = threading.Thread(target=self._read, daemon=True)
+            self.t.start()
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.t.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [v.strip() for v in ln.split(",")]
+            if len(f) < 9:
+                continue
+            try:
+                sm.append(float(f[1]))
+                smax.append(float(f[2]))
+            except ValueError:
+                continue
+            for n, v in zip(names, f[5:9]):
+                if v.lower().startswith("active"):
+                    reasons.add(n)
+        return {"sm_mhz": float(np.median(sm)) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_rate(inp, budget_s=12.0, sample_tokens=None):
+    """Oracle tokens/s on a bounded sample (single-threaded fp64 C)."""
+    import oracle
+    cfg = inp.cfg
+    n = sample_tokens or min(cfg.T, 8)
+    tok = np.arange(n, dtype=np.int64)
+    done, t0 = 0, time.perf_counter()
+    while True:
+        oracle.forward(inp, tokens=tok)
+        done += n
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return done / el, done, el
+
+
+# ----------------------------------------------------------------------------- ours
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import non_gated_relu_b200 as nh
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = synth.CONFIGS[args.workload]
+    inp = synth.make_inputs(cfg, skew_b=skew_b(cfg))
+    blk = nh.NemotronHMoE(cfg, inp.w_router, inp.w_up, inp.w_down, inp.w_shared_up,
+                          inp.w_shared_down, device=dev)
+    T = cfg.T
+    nb = max(1, args.batches)
+    xs = []
+    for i in range(nb):
+        xi = inp.x if (i == 0 and rank == 0) else batch_x(cfg, i + nb * rank)
+        t = torch.from_numpy(xi)
+        t = t.view(torch.bfloat16) if xi.dtype == np.uint16 else t
+        xs.append(t.to(dev))
+    # one graph per input batch (buffers shared: the replays are stream-ordered)
+    graphs = []
+    b = blk.buffers(T)
+    for i in range(nb):
+        s = torch.cuda.Stream(dev)
+        s.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(s):
+            blk.forward(xs[i], b)
+        torch.cuda.current_stream(dev).wait_stream(s)
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            blk.forward(xs[i], b)
+        graphs.append(g)
+    rc = blk.check(T)
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} after warm-up")
+
+    main = torch.cuda.current_stream(dev)
+    for i in range(max(3, args.warmup)):
+        graphs[i % nb].replay()
+    torch.cuda.synchronize(dev)
+
+    # step-time estimate -> default number of steps (about 2 s timed)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(main)
+    for i in range(20):
+        graphs[i % nb].replay()
+    e1.record(main)
+    e1.synchronize()
+    est = e0.elapsed_time(e1) / 20.0
+    steps = args.steps if args.steps > 0 else int(max(20, min(20000, 2000.0 / max(est, 1e-3))))
+
+    dist = None
+    if world > 1:
+        import torch.distributed as dist
+    clocks = ClockSampler(local_rank)
+    if rank == 0:
+        clocks.start()
+        time.sleep(0.3)
+    if dist:
+        dist.barrier()
+    torch.cuda.synchronize(dev)
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t_start.record(main)
+    for i in range(steps):
+        graphs[i % nb].replay()
+    t_end.record(main)
+    torch.cuda.synchronize(dev)
+    if dist:
+        dist.barrier()
+    elapsed_ms = t_start.elapsed_time(t_end)
+    clk = clocks.stop() if rank == 0 else None
+    if dist:
+        tt = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        elapsed_ms = float(tt.item())
+    rc = blk.check(T)
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} after the timed region")
+
+    # per-kernel durations (eager calls, events on the launching streams)
+    kern = kernel_times(blk, xs, b, nb, steps=min(steps, 200))
+
+    # end to end through the public host API (pinned H2D, graph, D2H)
+    xh = [x.cpu().pin_memory() for x in xs]
+    for i in range(3):
+        blk(xh[i % nb])
+    e2e_steps = min(steps, 2000)
+    torch.cuda.synchronize(dev)
+    h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h0.record(main)
+    for i in range(e2e_steps):
+        blk(xh[i % nb])
+    h1.record(main)
+    torch.cuda.synchronize(dev)
+    e2e_ms = h0.elapsed_time(h1) / e2e_steps
+
+    result = None
+    if rank == 0:
+        result = report(args, cfg, inp, world, steps, elapsed_ms, clk, kern, e2e_ms, blk)
+    if dist:
+        dist.barrier()
+    del graphs
+    return result
+
+
+def kernel_times(blk, xs, b, nb, steps):
+    """Average CUDA-event duration of each phase of the block, eager, on its stream."""
+    import torch
+    import non_gated_relu_b200 as nh
+    main = torch.cuda.current_stream(blk.device)
+    T = xs[0].shape[0]
+    names = ["route", "permute", "experts_up", "experts_down", "shared", "finalize"]
+    acc = {n: 0.0 for n in names}
+    ev = {n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for n in names}
+    for i in range(steps):
+        x = xs[i % nb]
+        def timed(n, fn, stream=main):
+            ev[n][0].record(stream)
+            fn()
+            ev[n][1].record(stream)
+        if blk.has_shared:
+            timed("shared", lambda: nh.shared(blk.c, x, blk.w_shared_up, blk.w_shared_down,
+                                               b.y_shared, b.ws_shared, stream=main))
+        timed("route", lambda: nh.route(blk.c, x, blk.w_router, blk.bias, b.topk_idx, b.topk_w,
+                                         b.ws, stream=main))
+        timed("permute", lambda: nh.permute(blk.c, x, b.topk_idx, b.topk_w, b.ws, stream=main))
+        nh.zero(b.y_acc, stream=main)
+        timed("experts_up", lambda: nh.experts_up(blk.c, T, blk.w_up, b.ws, stream=main))
+        timed("experts_down", lambda: nh.experts_down(blk.c, T, blk.w_down, b.y_acc, b.ws,
+                                                       stream=main))
+        timed("finalize", lambda: nh.finalize(blk.c, T, b.y_acc, b.y_shared, b.y, stream=main))
+        torch.cuda.synchronize(blk.device)
+        for n in names:
+            if n == "shared" and not blk.has_shared:
+                continue
+            acc[n] += ev[n][0].elapsed_time(ev[n][1])
+    return {n: acc[n] / steps for n in names}
+
+
+def distinct_experts(cfg, idx):
+    return int(len(np.unique(idx)))
+
+
+def report(args, cfg, inp, world, steps, elapsed_ms, clk, kern, e2e_ms, blk):
+    import torch
+    pk, pk_kind = peaks()
+    T = cfg.T
+    ms = elapsed_ms / steps
+    tokens = T * world * steps
+    value = tokens / (elapsed_ms / 1e3)
+    flops_tok = cfg.flops_per_token()
+    tflops = flops_tok * T * world / (ms / 1e3) / 1e12
+    elem = 2 if cfg.dtype == "bf16" else 4
+    b = blk.buffers(T)
+    idx = b.topk_idx.cpu().numpy()
+    D = distinct_experts(cfg, idx)
+    expert_bytes = cfg.I * cfg.H * elem            # one projection of one expert
+    shared_bytes = 2 * cfg.S * cfg.H * elem if cfg.n_shared_experts else 0
+    rows = T * cfg.k
+    # algorithmic bytes of one step: touched weights + router + x in + y out
+    step_bytes = (D * 2 * expert_bytes + shared_bytes + cfg.E * cfg.H * 4
+                  + 2 * T * cfg.H * elem)
+    hbm_step = step_bytes / (ms / 1e3) / 1e9
+    # dominant kernel roofline
+    decode = T <= 64
+    if decode:
+        dom = "experts_up" if kern["experts_up"] >= kern["experts_down"] else "experts_down"
+        kb = D * expert_bytes + rows * (cfg.H + cfg.I) * elem
+        ach = kb / (kern[dom] / 1e3) / 1e9
+        peak = pk["hbm_gbs"]
+        roof = {"bound": "hbm", "kernel": dom, "achieved": round(ach, 1), "peak": peak,
+                "unit": "GB/s", "frac": round(ach / peak, 4), "peak_kind": pk_kind,
+                "algorithmic_bytes_per_launch": kb, "ms_per_launch": round(kern[dom], 5)}
+    else:
+        dom = "experts_up" if kern["experts_up"] >= kern["experts_down"] else "experts_down"
+        kf = 2.0 * rows * cfg.H * cfg.I
+        ach = kf / (kern[dom] / 1e3) / 1e12
+        peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"]) if pk_kind == "measured" else pk["bf16_tflops"]
+        roof = {"bound": "tensor", "kernel": dom, "achieved": round(ach, 1), "peak": peak,
+                "unit": "TFLOP/s", "frac": round(ach / peak, 4),
+                "peak_kind": pk_kind + (" sustained" if pk_kind == "measured" else ""),
+                "algorithmic_flops_per_launch": kf, "ms_per_launch": round(kern[dom], 5)}
+    roof["traffic"] = ncu_traffic(args.workload, roof["kernel"])
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
+        "steps": steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16" if cfg.dtype == "bf16" else "f32", "data": "synthetic",
+        "config": {"workload": cfg.name, "tokens_per_step_per_gpu": T, "hidden_size": cfg.H,
+                   "n_routed_experts": cfg.E, "n_group": cfg.G, "topk_group": cfg.tg,
+                   "num_experts_per_tok": cfg.k, "moe_intermediate_size": cfg.I,
+                   "moe_shared_expert_intermediate_size": cfg.S,
+                   "parallelism": f"dp{world} (token batches, replicated weights)",
+                   "input_batches_cycled": args.batches,
+                   "l2": (f"inputs larger than L2: {step_bytes / 1e6:.0f} MB of weights and "
+                          f"activations touched per step, {D} distinct experts")},
+        "tflops": round(tflops, 3),
+        "tflops_frac": round(tflops / (pk.get("bf16_tflops_sustained") or pk["bf16_tflops"]), 4),
+        "hbm_gbs_step": round(hbm_step, 1), "hbm_frac_step": round(hbm_step / pk["hbm_gbs"], 4),
+        "roofline": roof,
+        "kernel_ms": {k: round(v, 5) for k, v in kern.items()},
+        "e2e": {"value": round(T / (e2e_ms / 1e3), 2), "unit": "tokens/s",
+                "ms_per_step": round(e2e_ms, 5),
+                "h2d_bytes_per_step": T * cfg.H * elem, "d2h_bytes_per_step": T * cfg.H * elem},
+        "gpu_launches": 11 * steps if cfg.n_shared_experts else 9 * steps,
+        "clocks": clk,
+        "peaks": {"kind": pk_kind, "hbm_gbs": pk["hbm_gbs"], "bf16_tflops": pk["bf16_tflops"],
+                  "bf16_tflops_sustained": pk.get("bf16_tflops_sustained")},
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        rate, n, el = oracle_rate(inp)
+        out["cpu_baseline"] = {"value": round(rate, 4), "unit": "tokens/s", "cores": 1,
+                               "kind": "oracle",
+                               "sample": f"{n} tokens (first {min(cfg.T, 8)} of the batch, "
+                                         f"repeated) in {el:.1f} s, single-threaded fp64 C"}
+    return out
+
+
+def kernel_hash():
+    h = hashlib.sha256()
+    for p in KERNEL_SOURCES:
+        with open(os.path.join(ROOT, p), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def ncu_traffic(workload, kernel):
+    """DRAM bytes per launch from the committed ncu summary, or None when the
+    kernel sources changed since the counters were taken."""
+    p = os.path.join(ROOT, "profiles", "traffic.json")
+    if not os.path.exists(p):
+        return None
+    with open(p) as f:
+        d = json.load(f)
+    rec = d.get(workload, {}).get(kernel)
+    if not rec or rec.get("kernel_hash") != kernel_hash():
+        return None
+    return rec.get("dram_bytes_per_launch")
+
+
+# ----------------------------------------------------------------------------- reference
+def run_reference(args, rank, world):
+    if rank != 0:
+        return None
+    cfg = synth.CONFIGS[args.workload]
+    import oracle
+    inp = synth.make_inputs(cfg, skew_b=skew_b(cfg))
+    n = min(cfg.T, 8)
+    tok = np.arange(n, dtype=np.int64)
+    for _ in range(max(0, min(args.warmup, 1))):
+        oracle.forward(inp, tokens=tok)
+    steps = args.steps if args.steps > 0 else 10
+    t0 = time.perf_counter()
+    for _ in range(steps):
+        oracle.forward(inp, tokens=tok)
+    el = time.perf_counter() - t0
+    value = n * steps / el
+    return {"metric": METRIC, "impl": "reference", "value": round(value, 4), "unit": "tokens/s",
+            "n_gpus": world, "steps": steps, "warmup": args.warmup,
+            "ms_per_step": round(el / steps * 1e3, 3), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": cfg.name, "tokens_per_step_per_gpu": cfg.T,
+                       "sample_tokens_per_step": n},
+            "cpu_baseline": {"value": round(value, 4), "unit": "tokens/s", "cores": 1,
+                             "kind": "oracle",
+                             "sample": f"{n} tokens per step (first {n} of the batch), "
+                                       f"single-threaded fp64 C oracle"},
+            "e2e": {"value": round(value, 4), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        out = run_reference(args, rank, world)
+        if out is not None:
+            print(json.dumps(out), flush=True)
+        return 0
+    if world > 1:
+        import datetime
+        import torch
+        import torch.distributed as dist
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        out = run_ours(args, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+    if rank == 0 and out is not None:
+        print(json.dumps(out), flush=True)
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

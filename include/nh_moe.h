@@ -1,0 +1,220 @@
+/*
+ * nh_moe.h -- C ABI of the B200 (sm_100a) Nemotron-H non-gated MoE block.
+ *
+ * The MoE block of Nemotron-H (`NemotronHMoE(config)`, `__call__(x) -> y`,
+ * exo commit "Add support for Nemotron sharding", nemotron_h.pyi) is
+ *
+ *   y = sum_{j<k} w_j * down_e_j( relu( up_e_j(x) )^2 )  +  shared_down( relu( shared_up(x) )^2 )
+ *
+ * with (e_j, w_j) chosen per token by a grouped top-k sigmoid router and
+ * experts that have no gate_proj ("Non-gated MoE", vllm.cpp PR #518; baseRT
+ * issue #46, "Architecture (config.json)"; expert shapes in the auto-round PR
+ * #1712 log).  One block call is, in stream order:
+ *
+ *   stream A:  nh_moe_route -> nh_moe_permute -> nh_moe_forward ---+
+ *   stream B:  nh_moe_shared ---------------------------------------+-> nh_moe_finalize
+ *
+ * Conventions (every entry point):
+ *   - All pointers named x, w_*, topk_*, y*, ws* are DEVICE pointers of the
+ *     current CUDA device; `cfg` and `out`-structs are HOST pointers.
+ *   - Arrays are dense row-major; weights use the PyTorch Linear layout
+ *     [out_features, in_features].  Device pointers must be 16-byte aligned.
+ *   - The caller owns every buffer and stream.  The library allocates no
+ *     device memory and keeps no state across calls except a thread-local
+ *     error string and per-device caches of kernel attributes.
+ *   - `stream` is a cudaStream_t (NULL = the legacy default stream).  Every
+ *     call only enqueues work; nothing synchronises the host.
+ *   - Errors: a non-NH_OK status is returned and nh_last_error() describes
+ *     it; nothing is enqueued when an argument check fails.  Faults found on
+ *     the device (bounded waits that ran out, index checks) are recorded in
+ *     the workspace status word and read back by nh_moe_check_device.
+ *   - dtype NH_BF16: x, expert weights and y are bf16 (uint16 bit patterns);
+ *     the tensor-core path needs hidden_size, moe_intermediate_size and
+ *     moe_shared_expert_intermediate_size to be multiples of 64, else the
+ *     call returns NH_ERR_UNSUPPORTED.  dtype NH_F32: everything float32,
+ *     any size.  The router weight and all accumulation are float32.
+ */
+#ifndef NH_MOE_H
+#define NH_MOE_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    NH_OK = 0,
+    NH_ERR_INVALID_ARG = 1,   /* config or argument fails validation            */
+    NH_ERR_UNSUPPORTED = 2,   /* valid, but outside what the kernels implement  */
+    NH_ERR_CUDA = 3,          /* a CUDA runtime/driver call failed              */
+    NH_ERR_TIMEOUT = 4,       /* a bounded device-side wait ran out             */
+    NH_ERR_DEVICE_CHECK = 5   /* a device-side index/shape check failed         */
+} nh_status;
+
+typedef enum { NH_F32 = 0, NH_BF16 = 1 } nh_dtype;
+
+/* Group score of the router's group stage. */
+typedef enum {
+    NH_GROUP_SCORE_MAX = 0,   /* max selection score of the group's experts */
+    NH_GROUP_SCORE_TOP2 = 1   /* sum of the two largest (needs >= 2 experts per group) */
+} nh_group_score;
+
+/*
+ * Block configuration.  Field names are the model's config.json / MLX
+ * ModelArgs names (exo commit "Add support for Nemotron sharding",
+ * nemotron_h.pyi, ModelArgs.moe_intermediate_size .. routed_scaling_factor).
+ * `n_group` is the router's group count, which the baseRT issue #46 summary
+ * writes as "n_groups=8" (in ModelArgs, n_groups is the Mamba-2 field).
+ */
+typedef struct {
+    int32_t hidden_size;                          /* H                            */
+    int32_t n_routed_experts;                     /* E, at most 512               */
+    int32_t n_group;                              /* G, E % G == 0                */
+    int32_t topk_group;                           /* tg, 1 <= tg <= G             */
+    int32_t num_experts_per_tok;                  /* k, 1 <= k <= tg * E / G, <= 32 */
+    int32_t moe_intermediate_size;                /* I                            */
+    int32_t moe_shared_expert_intermediate_size;  /* S (ignored if no shared)     */
+    int32_t n_shared_experts;                     /* 0 or 1                       */
+    int32_t norm_topk_prob;                       /* bool                         */
+    float routed_scaling_factor;                  /* alpha, finite                */
+    int32_t dtype;                                /* nh_dtype                     */
+    int32_t group_score;                          /* nh_group_score               */
+} nh_moe_config;
+
+/* Byte offsets of the regions inside the routed-path workspace `ws`. */
+typedef struct {
+    size_t total_bytes;
+    size_t status;        /* int32[4]: status word, first bad index, spare      */
+    size_t logits;        /* float [T, E] router logits                         */
+    size_t counts;        /* int32 [E] assignments per expert                   */
+    size_t offsets;       /* int32 [E + 1] exclusive scan of counts             */
+    size_t chunk_counts;  /* int32 [n_chunks, E] per-chunk histograms           */
+    size_t perm_token;    /* int32 [T * k] token of each permuted row           */
+    size_t perm_w;        /* float [T * k] routing weight of each permuted row  */
+    size_t inv_row;       /* int32 [T, k] permuted row of assignment (t, j)     */
+    size_t tiles;         /* int32 [max_tiles, 4] (expert, first row, rows, 0)  */
+    size_t num_tiles;     /* int32 [1] number of valid tile entries             */
+    size_t x_perm;        /* dtype [rows_alloc, H] x gathered in permuted order */
+    size_t h;             /* dtype [rows_alloc, I] relu^2(up) in permuted order */
+    int64_t rows_alloc;   /* T * k rounded up to the tile height                */
+    int32_t tile_rows;    /* rows per tile entry of this (cfg, T)               */
+    int32_t max_tiles;
+    int32_t n_chunks;     /* token chunks of the permute histogram              */
+    int32_t swap_ab;      /* 1: weights on the MMA M side (small T)             */
+} nh_moe_ws_layout;
+
+/* Validate a configuration (no device work). */
+nh_status nh_moe_validate(const nh_moe_config *cfg);
+
+/* Size of the routed-path workspace for T tokens (T >= 0). */
+nh_status nh_moe_workspace_size(const nh_moe_config *cfg, int64_t T, size_t *bytes);
+
+/* Region offsets of the routed-path workspace (for inspection and tests). */
+nh_status nh_moe_workspace_layout(const nh_moe_config *cfg, int64_t T, nh_moe_ws_layout *out);
+
+/* Size of the shared-expert workspace (relu^2 hidden [T, S] in dtype). */
+nh_status nh_moe_shared_workspace_size(const nh_moe_config *cfg, int64_t T, size_t *bytes);
+
+/*
+ * Router: logits l = x Wr^T (float32 accumulate), scores s = sigmoid(l),
+ * selection score s + e_score_correction_bias (bias may be NULL = 0; with
+ * no bias and the max group score the selection runs on the logits, which
+ * the sigmoid orders identically), group score, topk_group groups kept,
+ * top-k experts among them, ties to the lower group / expert id, output in
+ * (score desc, id asc) order; weights alpha * s_j / sum s (norm_topk_prob)
+ * or alpha * s_j, from the unbiased s.  (baseRT issue #46 MoE summary;
+ * ModelArgs.n_group .. routed_scaling_factor; the router correction bias is
+ * a float32 tensor of the checkpoint, auto-round PR #1712.)
+ *   x [T, H] dtype; w_router [E, H] float32; bias [E] float32 or NULL;
+ *   topk_idx [T, k] int32 (out); topk_w [T, k] float32 (out);
+ *   ws / ws_bytes: routed-path workspace (holds the status word and logits).
+ * The status word is cleared here: nh_moe_route starts a block call.
+ */
+nh_status nh_moe_route(const nh_moe_config *cfg, int64_t T, const void *x, const float *w_router,
+                       const float *e_score_correction_bias, int32_t *topk_idx, float *topk_w,
+                       void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * Token permute: per-expert histogram, exclusive scan, stable scatter of the
+ * (t, j) assignments in (t, j) order, the tile table of the expert GEMMs and
+ * the gather x_perm[row] = x[perm_token[row]].  The routed experts are
+ * applied per expert id (MLX SwitchMLP fc1/fc2 indexed by the router's
+ * expert ids, exo commit "Add support for Nemotron sharding").
+ *   topk_idx / topk_w as produced by nh_moe_route (any valid ids in [0, E)
+ *   are accepted; an id out of range sets NH_ERR_DEVICE_CHECK on the device).
+ */
+nh_status nh_moe_permute(const nh_moe_config *cfg, int64_t T, const void *x,
+                         const int32_t *topk_idx, const float *topk_w, void *ws, size_t ws_bytes,
+                         void *stream);
+
+/*
+ * Routed experts: h = relu(x_perm W_up[e]^T)^2 (float32 accumulate, h stored
+ * in dtype), then y_acc[perm_token[r]] += perm_w[r] * (h[r] W_down[e]^T).
+ * y_acc is zero-filled first by this call.
+ *   w_up [E, I, H] dtype; w_down [E, H, I] dtype; y_acc [T, H] float32 (out).
+ * Needs nh_moe_permute's workspace contents.
+ */
+nh_status nh_moe_forward(const nh_moe_config *cfg, int64_t T, const void *w_up, const void *w_down,
+                         float *y_acc, void *ws, size_t ws_bytes, void *stream);
+
+/*
+ * The two phases of nh_moe_forward, for callers that schedule or time them
+ * separately (same arguments and requirements):
+ *   nh_moe_experts_up:   h = relu(x_perm W_up[e]^T)^2 into the workspace;
+ *   nh_moe_experts_down: y_acc[perm_token[r]] += perm_w[r] * (h[r] W_down[e]^T)
+ *                        (accumulates: y_acc must hold the running sum, e.g. zeros).
+ */
+nh_status nh_moe_experts_up(const nh_moe_config *cfg, int64_t T, const void *w_up, void *ws,
+                            size_t ws_bytes, void *stream);
+nh_status nh_moe_experts_down(const nh_moe_config *cfg, int64_t T, const void *w_down,
+                              float *y_acc, void *ws, size_t ws_bytes, void *stream);
+
+/* Zero-fill n floats of device memory (n >= 0) on `stream`. */
+nh_status nh_moe_zero(float *buf, int64_t n, void *stream);
+
+/*
+ * Shared expert (NemotronHMLP up_proj / down_proj, always on, unscaled):
+ * y_shared = relu(x W_su^T)^2 W_sd^T, written (not accumulated).
+ *   w_shared_up [S, H]; w_shared_down [H, S] (dtype); y_shared [T, H] float32;
+ *   ws_shared: nh_moe_shared_workspace_size bytes.
+ * Independent of the routed path: may run on a second stream.
+ */
+nh_status nh_moe_shared(const nh_moe_config *cfg, int64_t T, const void *x, const void *w_shared_up,
+                        const void *w_shared_down, float *y_shared, void *ws_shared,
+                        size_t ws_shared_bytes, void *stream);
+
+/*
+ * y = dtype(y_acc + y_shared) (y_shared may be NULL when there is no shared
+ * expert).  y [T, H] dtype.
+ */
+nh_status nh_moe_finalize(const nh_moe_config *cfg, int64_t T, const float *y_acc,
+                          const float *y_shared, void *y, void *stream);
+
+/*
+ * Synchronises `stream`, reads the workspace status word and returns it
+ * (NH_OK, NH_ERR_TIMEOUT or NH_ERR_DEVICE_CHECK); a pending CUDA error is
+ * returned as NH_ERR_CUDA.  `ws` is a routed-path workspace.
+ */
+nh_status nh_moe_check_device(void *ws, void *stream);
+
+/*
+ * Failure-detection self test: launches one kernel whose bounded wait on an
+ * mbarrier that nothing arrives on runs out after `timeout_ns`; the kernel
+ * records NH_ERR_TIMEOUT in the status word of `ws` and returns, leaving the
+ * context usable.  Read the result with nh_moe_check_device.
+ */
+nh_status nh_moe_selftest_timeout(void *ws, uint64_t timeout_ns, void *stream);
+
+/* Message of the last non-OK status returned on this host thread. */
+const char *nh_last_error(void);
+
+/* Library version string. */
+const char *nh_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* NH_MOE_H */

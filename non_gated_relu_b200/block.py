@@ -1,0 +1,185 @@
+"""Block-level API: ``NemotronHMoE(cfg, weights...)(x) -> y``.
+
+The Nemotron-H MoE block (``NemotronHMoE.__call__(x) -> y`` with a
+``switch_mlp`` of routed experts and a ``shared_experts`` NemotronHMLP, exo
+commit "Add support for Nemotron sharding", nemotron_h.pyi) on one GPU.  One
+call runs, on the caller's stream and a side stream:
+
+    main: route -> permute -> forward (routed experts) --+
+    side: shared expert ----------------------------------+-> finalize
+
+All arithmetic happens in libnhmoe's kernels; this class only owns buffers,
+streams, events and (optionally) a CUDA graph of the call sequence.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+from typing import Dict, Optional
+
+import numpy as np
+import torch
+
+from . import (check_device, config_from, finalize, forward, permute, route, shared,
+               shared_workspace_size, validate, workspace_size, NH_BF16)
+
+
+def _to_device(a, dtype: torch.dtype, device) -> torch.Tensor:
+    if a is None:
+        return None
+    if isinstance(a, np.ndarray):
+        t = torch.from_numpy(np.ascontiguousarray(a))
+        if a.dtype == np.uint16:
+            t = t.view(torch.bfloat16)
+    else:
+        t = a
+    if t.dtype != dtype:
+        raise TypeError(f"expected {dtype}, got {t.dtype}")
+    return t.to(device).contiguous()
+
+
+@dataclass
+class Buffers:
+    T: int
+    ws: torch.Tensor
+    ws_shared: Optional[torch.Tensor]
+    topk_idx: torch.Tensor
+    topk_w: torch.Tensor
+    y_acc: torch.Tensor
+    y_shared: Optional[torch.Tensor]
+    y: torch.Tensor
+
+
+class NemotronHMoE:
+    """One MoE block with resident weights.
+
+    Weights use the PyTorch Linear layout: ``w_router [E, H]`` float32,
+    ``w_up [E, I, H]``, ``w_down [E, H, I]``, ``w_shared_up [S, H]``,
+    ``w_shared_down [H, S]`` in the block dtype (bf16 or float32), and an
+    optional router correction bias ``[E]`` float32.  numpy uint16 arrays are
+    taken as bf16 bit patterns.
+    """
+
+    def __init__(self, cfg, w_router, w_up, w_down, w_shared_up=None, w_shared_down=None,
+                 bias=None, device=None):
+        self.cfg = cfg
+        self.c = config_from(cfg)
+        validate(self.c)
+        self.device = torch.device(device if device is not None else "cuda")
+        if self.device.type != "cuda":
+            raise ValueError("NemotronHMoE runs on a CUDA device only")
+        self.dtype = torch.bfloat16 if self.c.dtype == NH_BF16 else torch.float32
+        self.H = self.c.hidden_size
+        self.k = self.c.num_experts_per_tok
+        self.has_shared = bool(self.c.n_shared_experts)
+        self.w_router = _to_device(w_router, torch.float32, self.device)
+        self.bias = _to_device(bias, torch.float32, self.device)
+        self.w_up = _to_device(w_up, self.dtype, self.device)
+        self.w_down = _to_device(w_down, self.dtype, self.device)
+        self.w_shared_up = _to_device(w_shared_up, self.dtype, self.device)
+        self.w_shared_down = _to_device(w_shared_down, self.dtype, self.device)
+        if self.has_shared and (self.w_shared_up is None or self.w_shared_down is None):
+            raise ValueError("config has a shared expert but no shared weights were given")
+        with torch.cuda.device(self.device):
+            self.side = torch.cuda.Stream()
+        self._bufs: Dict[int, Buffers] = {}
+        self._graphs: Dict[int, tuple] = {}
+        self._host: Dict[int, tuple] = {}
+
+    # ------------------------------------------------------------------ buffers
+    def buffers(self, T: int) -> Buffers:
+        b = self._bufs.get(T)
+        if b is None:
+            dev = self.device
+            ws = torch.empty(workspace_size(self.c, T), dtype=torch.uint8, device=dev)
+            wss = ys = None
+            if self.has_shared:
+                wss = torch.empty(shared_workspace_size(self.c, T), dtype=torch.uint8, device=dev)
+                ys = torch.empty((T, self.H), dtype=torch.float32, device=dev)
+            b = Buffers(T, ws, wss,
+                        torch.empty((T, self.k), dtype=torch.int32, device=dev),
+                        torch.empty((T, self.k), dtype=torch.float32, device=dev),
+                        torch.empty((T, self.H), dtype=torch.float32, device=dev), ys,
+                        torch.empty((T, self.H), dtype=self.dtype, device=dev))
+            self._bufs[T] = b
+        return b
+
+    # ------------------------------------------------------------------ compute
+    def forward(self, x: torch.Tensor, bufs: Optional[Buffers] = None) -> torch.Tensor:
+        """y for a device tensor x [T, H]; returns the buffer-owned y [T, H]."""
+        T = x.shape[0]
+        b = bufs or self.buffers(T)
+        main = torch.cuda.current_stream(self.device)
+        if self.has_shared:
+            fork = torch.cuda.Event()
+            fork.record(main)
+            self.side.wait_event(fork)
+            shared(self.c, x, self.w_shared_up, self.w_shared_down, b.y_shared, b.ws_shared,
+                   stream=self.side)
+            join = torch.cuda.Event()
+            join.record(self.side)
+        route(self.c, x, self.w_router, self.bias, b.topk_idx, b.topk_w, b.ws, stream=main)
+        permute(self.c, x, b.topk_idx, b.topk_w, b.ws, stream=main)
+        forward(self.c, T, self.w_up, self.w_down, b.y_acc, b.ws, stream=main)
+        if self.has_shared:
+            main.wait_event(join)
+        finalize(self.c, T, b.y_acc, b.y_shared, b.y, stream=main)
+        return b.y
+
+    def capture(self, T: int):
+        """Capture the call sequence for T tokens in a CUDA graph.
+
+        Returns (graph, x_static, y): write the input into ``x_static`` and
+        ``graph.replay()`` writes ``y``."""
+        g = self._graphs.get(T)
+        if g is None:
+            x_static = torch.zeros((T, self.H), dtype=self.dtype, device=self.device)
+            b = self.buffers(T)
+            s = torch.cuda.Stream(self.device)
+            s.wait_stream(torch.cuda.current_stream(self.device))
+            with torch.cuda.stream(s):           # warm up outside the graph
+                self.forward(x_static, b)
+            torch.cuda.current_stream(self.device).wait_stream(s)
+            torch.cuda.synchronize(self.device)
+            graph = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(graph):
+                y = self.forward(x_static, b)
+            g = (graph, x_static, y)
+            self._graphs[T] = g
+        return g
+
+    def check(self, T: int) -> int:
+        """Status word of the last call for T tokens (synchronises)."""
+        b = self.buffers(T)
+        rc = check_device(b.ws)
+        if rc == 0 and b.ws_shared is not None:
+            rc = check_device(b.ws_shared)
+        return rc
+
+    def __call__(self, x, use_graph: bool = True):
+        """y = block(x).  A device tensor is computed in place on the current
+        stream; a host tensor (or numpy array) goes through pinned staging
+        buffers: host->device copy, the block (as a CUDA graph when
+        ``use_graph``), device->host copy; returns a host tensor."""
+        if isinstance(x, torch.Tensor) and x.is_cuda:
+            return self.forward(x)
+        xh = _to_device(x, self.dtype, "cpu") if isinstance(x, np.ndarray) else x
+        T = xh.shape[0]
+        st = self._host.get(T)
+        if st is None:
+            st = (torch.empty((T, self.H), dtype=self.dtype).pin_memory(),
+                  torch.empty((T, self.H), dtype=self.dtype).pin_memory())
+            self._host[T] = st
+        xin, yout = st
+        if not xh.is_pinned():
+            xin.copy_(xh)
+            xh = xin
+        if use_graph:
+            graph, x_static, y = self.capture(T)
+            x_static.copy_(xh, non_blocking=True)
+            graph.replay()
+        else:
+            xd = xh.to(self.device, non_blocking=True)
+            y = self.forward(xd)
+        yout.copy_(y, non_blocking=True)
+        torch.cuda.current_stream(self.device).synchronize()
+        return yout

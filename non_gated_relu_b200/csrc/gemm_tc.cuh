@@ -1,0 +1,311 @@
+// gemm_tc.cuh -- persistent grouped expert GEMM on the sm_100a tensor cores.
+//
+// For every tile entry (expert e, first row r0, rows) of the permute's tile
+// table and every block of output features, D = A[r0 : r0+rows, :] . W[e]^T
+// is accumulated in tensor memory by tcgen05.mma (bf16 in, f32 accumulate)
+// from operand tiles that TMA stages in shared memory with 128-byte swizzle,
+// and a fused epilogue turns it into
+//   up_proj:   h = relu(D)^2 stored in bf16              (non-gated expert,
+//              "up_proj -> relu^2 -> down_proj", vllm.cpp PR #518)
+//   down_proj: y_acc[token] += routing weight * D          (weighted combine)
+//   shared:    y_shared = D                                 (always-on expert)
+//
+// Two orientations:
+//   prefill (SWAP = false): MMA M = 128 activation rows, N = NT weight rows;
+//   decode  (SWAP = true):  MMA M = 128 weight rows, N = NT activation rows,
+//     so that a handful of tokens per expert still fill the 128-row side and
+//     the kernel streams each expert's weights once.
+//
+// Warp roles (192 threads): warp 0 lane 0 issues TMA loads into a STAGES-deep
+// ring; warp 1 owns tensor memory and lane 0 issues the MMAs; warps 2..5 read
+// the accumulator (each its 32-lane quarter) and run the epilogue.  Two
+// accumulators in tensor memory let the epilogue of one tile overlap the
+// main loop of the next.  Every mbarrier wait is bounded: when one runs out
+// the CTA records NH_ERR_TIMEOUT, drains its copies and MMAs in flight, frees
+// its tensor memory and returns.
+#pragma once
+
+#include "common.cuh"
+#include "gemm_simt.cuh"  // Epilogue codes
+
+namespace nh {
+namespace tc {
+
+constexpr int BK = 64;       // K per stage: 64 bf16 = one 128-byte swizzle row
+constexpr int UMMA_K = 16;   // K of one kind::f16 MMA
+constexpr int M = 128;       // MMA M (one CTA)
+constexpr int THREADS = 192;
+
+struct TcArgs {
+  const int4* tiles;          // (expert, first row, rows, 0) or null: dense rows
+  const int32_t* num_tiles;
+  int dense_rows;
+  int tile_rows;
+  int N;                      // output features (weight rows)
+  int K;                      // multiple of 64
+  int epi;                    // Epilogue
+  void* out;
+  int64_t ldo;                // row stride of out, elements
+  const int32_t* perm_token;
+  const float* perm_w;
+  int* status;
+  uint64_t timeout_ns;
+};
+
+template <bool SWAP, int NT, int STAGES>
+struct Shape {
+  static constexpr int A_BYTES = M * BK * 2;     // M-side tile
+  static constexpr int B_BYTES = NT * BK * 2;    // N-side tile
+  static constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+  static_assert(STAGE_BYTES % 1024 == 0, "stages must keep 1024-byte alignment");
+  static_assert(NT % 16 == 0 && NT >= 16 && NT <= 256, "MMA N");
+  static constexpr int ACC_COLS = NT;
+  static constexpr int TMEM_COLS = (2 * NT < 32) ? 32 : 2 * NT;
+  static_assert((TMEM_COLS & (TMEM_COLS - 1)) == 0 && TMEM_COLS <= 512, "TMEM alloc");
+  static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8 + 16;
+  static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + BAR_BYTES;
+};
+
+__device__ __forceinline__ int4 tile_entry_of(const TcArgs& g, int m) {
+  if (g.tiles) return g.tiles[m];
+  const int r0 = m * g.tile_rows;
+  return make_int4(0, r0, min(g.tile_rows, g.dense_rows - r0), 0);
+}
+
+// Wait that ignores the abort flag: used only to drain work already issued.
+__device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, uint64_t timeout_ns,
+                                           int* status) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > timeout_ns) {
+      record_status(status, NH_ERR_TIMEOUT, SITE_TC_DRAIN, 0);
+      return;
+    }
+  }
+}
+
+// epilogue of 32 consecutive output features of one row (prefill orientation)
+__device__ __forceinline__ void epi_row32(const TcArgs& g, int r, int n, const float* v) {
+  if (g.epi == EPI_UP_RELU2) {
+    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) + (size_t)r * g.ldo + n);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      uint4 p;
+      p.x = pack_bf16x2(relu2(v[8 * i + 0]), relu2(v[8 * i + 1]));
+      p.y = pack_bf16x2(relu2(v[8 * i + 2]), relu2(v[8 * i + 3]));
+      p.z = pack_bf16x2(relu2(v[8 * i + 4]), relu2(v[8 * i + 5]));
+      p.w = pack_bf16x2(relu2(v[8 * i + 6]), relu2(v[8 * i + 7]));
+      dst[i] = p;
+    }
+  } else if (g.epi == EPI_DOWN_SCATTER) {
+    const float w = g.perm_w[r];
+    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.out) +
+                                            (size_t)g.perm_token[r] * g.ldo + n);
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      atomicAdd(dst + i, make_float4(w * v[4 * i], w * v[4 * i + 1], w * v[4 * i + 2],
+                                     w * v[4 * i + 3]));
+  } else {
+    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.out) + (size_t)r * g.ldo + n);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+  }
+}
+
+// epilogue of one element (decode orientation: feature f of row r)
+__device__ __forceinline__ void epi_elem(const TcArgs& g, int r, int f, float v) {
+  if (g.epi == EPI_UP_RELU2) {
+    static_cast<__nv_bfloat16*>(g.out)[(size_t)r * g.ldo + f] = __float2bfloat16_rn(relu2(v));
+  } else if (g.epi == EPI_DOWN_SCATTER) {
+    atomicAdd(static_cast<float*>(g.out) + (size_t)g.perm_token[r] * g.ldo + f, g.perm_w[r] * v);
+  } else {
+    static_cast<float*>(g.out)[(size_t)r * g.ldo + f] = v;
+  }
+}
+
+template <bool SWAP, int NT, int STAGES>
+__global__ void __launch_bounds__(THREADS, 1)
+    tc_grouped_gemm(const __grid_constant__ CUtensorMap map_act,
+                    const __grid_constant__ CUtensorMap map_w, const TcArgs g) {
+  using S = Shape<SWAP, NT, STAGES>;
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t base = (raw + 1023u) & ~1023u;
+  uint8_t* const base_ptr = smem_raw + (base - raw);
+  const uint32_t bar0 = base + STAGES * S::STAGE_BYTES;
+  auto full_bar = [&](int s) { return bar0 + 8u * s; };
+  auto empty_bar = [&](int s) { return bar0 + 8u * (STAGES + s); };
+  auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
+  auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
+  const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
+  uint32_t* const tmem_slot =
+      reinterpret_cast<uint32_t*>(base_ptr + STAGES * S::STAGE_BYTES + (2 * STAGES + 5) * 8);
+  volatile int* const abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < STAGES; ++s) {
+      mbar_init(full_bar(s), 1);
+      mbar_init(empty_bar(s), 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(tfull_bar(a), 1);
+      mbar_init(tempty_bar(a), 128);
+    }
+    mbar_init(drain_bar, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_map(&map_act);
+    tma_prefetch_map(&map_w);
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_slot), S::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  const WaitCtl wc{abort_flag, g.status, g.timeout_ns};
+
+  const int num_m = g.tiles ? *g.num_tiles : (g.dense_rows + g.tile_rows - 1) / g.tile_rows;
+  const int n_blocks = SWAP ? (g.N + M - 1) / M : (g.N + NT - 1) / NT;
+  const int total = num_m * n_blocks;
+  const int nk = g.K / BK;
+
+  if (warp == 0 && lane == 0) {
+    // ---------------- TMA producer ----------------
+    int stage = 0;
+    uint32_t phase = 0;
+    long issued = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      const int m = tile / n_blocks, nb = tile - m * n_blocks;
+      const int4 ent = tile_entry_of(g, m);
+      for (int kb = 0; kb < nk; ++kb) {
+        if (!mbar_wait(empty_bar(stage), phase ^ 1u, wc, SITE_TC_PRODUCER)) {
+          ok = false;
+          break;
+        }
+        const uint32_t sa = base + stage * S::STAGE_BYTES, sb = sa + S::A_BYTES;
+        mbar_arrive_expect_tx(full_bar(stage), S::STAGE_BYTES);
+        if (!SWAP) {
+          tma_load_2d(sa, &map_act, full_bar(stage), kb * BK, ent.y);
+          tma_load_3d(sb, &map_w, full_bar(stage), kb * BK, nb * NT, ent.x);
+        } else {
+          tma_load_3d(sa, &map_w, full_bar(stage), kb * BK, nb * M, ent.x);
+          tma_load_2d(sb, &map_act, full_bar(stage), kb * BK, ent.y);
+        }
+        ++issued;
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+    }
+    if (!ok) {
+      // let the copies already issued land before the CTA exits
+      const long first = issued > STAGES ? issued - STAGES : 0;
+      for (long i = first; i < issued; ++i)
+        mbar_drain(full_bar((int)(i % STAGES)), (uint32_t)((i / STAGES) & 1), g.timeout_ns,
+                   g.status);
+    }
+  } else if (warp == 1 && lane == 0) {
+    // ---------------- MMA issuer ----------------
+    int stage = 0;
+    uint32_t phase = 0;
+    int it = 0;
+    bool ok = true, any = false;
+    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+      const int m = tile / n_blocks, nb = tile - m * n_blocks;
+      const int acc = it & 1;
+      const uint32_t aph = (uint32_t)((it >> 1) & 1);
+      if (!mbar_wait(tempty_bar(acc), aph ^ 1u, wc, SITE_TC_MMA)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const int n_mma = SWAP ? NT : min(NT, g.N - nb * NT);
+      const uint32_t idesc = make_idesc_bf16(M, n_mma);
+      const uint32_t d_tmem = tmem_base + (uint32_t)(acc * S::ACC_COLS);
+      (void)m;
+      for (int kb = 0; kb < nk; ++kb) {
+        if (!mbar_wait(full_bar(stage), phase, wc, SITE_TC_MMA)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t sa = base + stage * S::STAGE_BYTES, sb = sa + S::A_BYTES;
+#pragma unroll
+        for (int kk = 0; kk < BK / UMMA_K; ++kk) {
+          umma_bf16(d_tmem, make_sdesc_sw128(sa + kk * UMMA_K * 2),
+                    make_sdesc_sw128(sb + kk * UMMA_K * 2), idesc, (kb | kk) != 0);
+        }
+        any = true;
+        umma_commit(empty_bar(stage));
+        if (++stage == STAGES) {
+          stage = 0;
+          phase ^= 1u;
+        }
+      }
+      if (!ok) break;
+      umma_commit(tfull_bar(acc));
+      ++it;
+    }
+    if (!ok && any) {
+      // all MMAs issued so far must finish before tensor memory is released
+      umma_commit(drain_bar);
+      mbar_drain(drain_bar, 0, g.timeout_ns, g.status);
+    }
+  } else if (warp >= 2) {
+    // ---------------- epilogue: 4 warps, one TMEM lane quarter each ----------------
+    const int q = warp & 3;
+    int it = 0;
+    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+      const int m = tile / n_blocks, nb = tile - m * n_blocks;
+      const int acc = it & 1;
+      const uint32_t aph = (uint32_t)((it >> 1) & 1);
+      int ok = 1;
+      if (lane == 0) ok = mbar_wait(tfull_bar(acc), aph, wc, SITE_TC_EPILOGUE) ? 1 : 0;
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      const int4 ent = tile_entry_of(g, m);
+      const uint32_t tq = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * S::ACC_COLS);
+      if (!SWAP) {
+        const int row = q * 32 + lane;
+        const bool valid = row < ent.z;
+        const int n0 = nb * NT;
+        const int n_eff = min(NT, g.N - n0);
+        for (int c = 0; c < n_eff; c += 32) {
+          float v[32];
+          tmem_ld_x32(tq + (uint32_t)c, v);
+          if (valid) epi_row32(g, ent.y + row, n0 + c, v);
+        }
+      } else {
+        const int f = nb * M + q * 32 + lane;
+        const bool valid = f < g.N;
+#pragma unroll
+        for (int c = 0; c < NT; c += 16) {
+          float v[16];
+          tmem_ld_x16(tq + (uint32_t)c, v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (valid && c + j < ent.z) epi_elem(g, ent.y + c + j, f, v[j]);
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(tempty_bar(acc));
+      ++it;
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, S::TMEM_COLS);
+  }
+}
+
+}  // namespace tc
+}  // namespace nh

@@ -1,0 +1,766 @@
+// nh_moe.cu -- C ABI of libnhmoe: argument checks, workspace plan, tensor
+// maps and kernel launches of the Nemotron-H non-gated MoE block forward.
+// Declarations and the contract of every entry point: include/nh_moe.h.
+#include <cudaTypedefs.h>
+
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+
+#include "common.cuh"
+#include "gemm_simt.cuh"
+#include "gemm_tc.cuh"
+#include "permute.cuh"
+#include "route.cuh"
+
+namespace nh {
+
+// ----------------------------------------------------------------------------
+// errors
+// ----------------------------------------------------------------------------
+static thread_local std::string g_last_error;
+
+static nh_status fail(nh_status s, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof buf, fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return s;
+}
+
+#define NH_CUDA(call)                                                                      \
+  do {                                                                                     \
+    cudaError_t e_ = (call);                                                               \
+    if (e_ != cudaSuccess)                                                                 \
+      return fail(NH_ERR_CUDA, "%s failed: %s (%s:%d)", #call, cudaGetErrorString(e_),    \
+                  __FILE__, __LINE__);                                                     \
+  } while (0)
+
+#define NH_TRY(expr)                     \
+  do {                                   \
+    nh_status s_ = (expr);               \
+    if (s_ != NH_OK) return s_;          \
+  } while (0)
+
+static nh_status launch_check(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess)
+    return fail(NH_ERR_CUDA, "launch of %s failed: %s", what, cudaGetErrorString(e));
+  return NH_OK;
+}
+
+// ----------------------------------------------------------------------------
+// configuration and workspace plan
+// ----------------------------------------------------------------------------
+constexpr int MAX_E = 512;
+constexpr int MAX_G = 64;
+constexpr int MAX_K = 32;
+constexpr size_t ALIGN = 256;
+
+static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+static nh_status validate(const nh_moe_config* c) {
+  if (!c) return fail(NH_ERR_INVALID_ARG, "cfg is NULL");
+  if (c->hidden_size < 1) return fail(NH_ERR_INVALID_ARG, "hidden_size must be >= 1");
+  if (c->n_routed_experts < 1) return fail(NH_ERR_INVALID_ARG, "n_routed_experts must be >= 1");
+  if (c->n_group < 1 || c->n_routed_experts % c->n_group != 0)
+    return fail(NH_ERR_INVALID_ARG, "n_routed_experts (%d) must be a multiple of n_group (%d)",
+                c->n_routed_experts, c->n_group);
+  if (c->topk_group < 1 || c->topk_group > c->n_group)
+    return fail(NH_ERR_INVALID_ARG, "topk_group must be in [1, n_group]");
+  const int g = c->n_routed_experts / c->n_group;
+  if (c->num_experts_per_tok < 1 || c->num_experts_per_tok > c->topk_group * g)
+    return fail(NH_ERR_INVALID_ARG, "num_experts_per_tok must be in [1, topk_group * E / n_group]");
+  if (c->moe_intermediate_size < 1) return fail(NH_ERR_INVALID_ARG, "moe_intermediate_size must be >= 1");
+  if (c->n_shared_experts != 0 && c->n_shared_experts != 1)
+    return fail(NH_ERR_INVALID_ARG, "n_shared_experts must be 0 or 1");
+  if (c->n_shared_experts == 1 && c->moe_shared_expert_intermediate_size < 1)
+    return fail(NH_ERR_INVALID_ARG, "moe_shared_expert_intermediate_size must be >= 1");
+  if (c->norm_topk_prob != 0 && c->norm_topk_prob != 1)
+    return fail(NH_ERR_INVALID_ARG, "norm_topk_prob must be 0 or 1");
+  if (!std::isfinite(c->routed_scaling_factor))
+    return fail(NH_ERR_INVALID_ARG, "routed_scaling_factor must be finite");
+  if (c->dtype != NH_F32 && c->dtype != NH_BF16) return fail(NH_ERR_INVALID_ARG, "unknown dtype");
+  if (c->group_score != NH_GROUP_SCORE_MAX && c->group_score != NH_GROUP_SCORE_TOP2)
+    return fail(NH_ERR_INVALID_ARG, "unknown group_score");
+  if (c->group_score == NH_GROUP_SCORE_TOP2 && g < 2)
+    return fail(NH_ERR_INVALID_ARG, "the top-2 group score needs >= 2 experts per group");
+  // valid; now what the kernels implement
+  if (c->n_routed_experts > MAX_E)
+    return fail(NH_ERR_UNSUPPORTED, "n_routed_experts > %d", MAX_E);
+  if (c->n_group > MAX_G) return fail(NH_ERR_UNSUPPORTED, "n_group > %d", MAX_G);
+  if (c->num_experts_per_tok > MAX_K) return fail(NH_ERR_UNSUPPORTED, "num_experts_per_tok > %d", MAX_K);
+  if (c->dtype == NH_BF16) {
+    if (c->hidden_size % 64 || c->moe_intermediate_size % 64 ||
+        (c->n_shared_experts && c->moe_shared_expert_intermediate_size % 64))
+      return fail(NH_ERR_UNSUPPORTED,
+                  "bf16 tensor-core path needs hidden, intermediate and shared sizes that are "
+                  "multiples of 64");
+  }
+  return NH_OK;
+}
+
+struct Plan {
+  int H, E, G, tg, k, I, S;
+  int64_t T, rows;
+  bool bf16;
+  size_t elem;
+  nh_moe_ws_layout lay;
+};
+
+// rows of one tile entry for T tokens: decode-sized T puts the weights on the
+// MMA M side (swap), with all of an expert's rows in one entry
+static void tile_plan(const nh_moe_config* c, int64_t T, int* tile_rows, int* swap) {
+  if (c->dtype == NH_F32) {
+    *tile_rows = SG_BM;
+    *swap = 0;
+  } else if (T <= 16) {
+    *tile_rows = 16;
+    *swap = 1;
+  } else if (T <= 32) {
+    *tile_rows = 32;
+    *swap = 1;
+  } else if (T <= 64) {
+    *tile_rows = 64;
+    *swap = 1;
+  } else {
+    *tile_rows = tc::M;
+    *swap = 0;
+  }
+}
+
+static nh_status make_plan(const nh_moe_config* c, int64_t T, Plan* p) {
+  NH_TRY(validate(c));
+  if (T < 0) return fail(NH_ERR_INVALID_ARG, "T must be >= 0");
+  const int64_t rows = T * c->num_experts_per_tok;
+  if (rows >= (int64_t(1) << 31) - 4096) return fail(NH_ERR_UNSUPPORTED, "T * k must be < 2^31");
+  p->H = c->hidden_size;
+  p->E = c->n_routed_experts;
+  p->G = c->n_group;
+  p->tg = c->topk_group;
+  p->k = c->num_experts_per_tok;
+  p->I = c->moe_intermediate_size;
+  p->S = c->moe_shared_expert_intermediate_size;
+  p->T = T;
+  p->rows = rows;
+  p->bf16 = c->dtype == NH_BF16;
+  p->elem = p->bf16 ? 2 : 4;
+  nh_moe_ws_layout& L = p->lay;
+  memset(&L, 0, sizeof L);
+  int tr, sw;
+  tile_plan(c, T, &tr, &sw);
+  L.tile_rows = tr;
+  L.swap_ab = sw;
+  L.max_tiles = (int)((rows + tr - 1) / tr + p->E);
+  L.n_chunks = (int)((T + PERM_CHUNK - 1) / PERM_CHUNK);
+  L.rows_alloc = rows;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o = align_up(o + (bytes ? bytes : 1), ALIGN);
+    return at;
+  };
+  L.status = take(16);
+  L.logits = take((size_t)T * p->E * 4);
+  L.counts = take((size_t)p->E * 4);
+  L.offsets = take((size_t)(p->E + 1) * 4);
+  L.chunk_counts = take((size_t)L.n_chunks * p->E * 4);
+  L.perm_token = take((size_t)rows * 4);
+  L.perm_w = take((size_t)rows * 4);
+  L.inv_row = take((size_t)rows * 4);
+  L.tiles = take((size_t)L.max_tiles * 16);
+  L.num_tiles = take(4);
+  L.x_perm = take((size_t)rows * p->H * p->elem);
+  L.h = take((size_t)rows * p->I * p->elem);
+  L.total_bytes = o;
+  return NH_OK;
+}
+
+static nh_status check_ptr(const void* p, const char* name) {
+  if (!p) return fail(NH_ERR_INVALID_ARG, "%s is NULL", name);
+  if (reinterpret_cast<uintptr_t>(p) % 16)
+    return fail(NH_ERR_INVALID_ARG, "%s must be 16-byte aligned", name);
+  return NH_OK;
+}
+
+static nh_status check_ws(const Plan& p, void* ws, size_t ws_bytes) {
+  NH_TRY(check_ptr(ws, "ws"));
+  if (reinterpret_cast<uintptr_t>(ws) % ALIGN)
+    return fail(NH_ERR_INVALID_ARG, "ws must be %zu-byte aligned", ALIGN);
+  if (ws_bytes < p.lay.total_bytes)
+    return fail(NH_ERR_INVALID_ARG, "ws holds %zu bytes, %zu needed", ws_bytes, p.lay.total_bytes);
+  return NH_OK;
+}
+
+template <typename T>
+static T* at(void* ws, size_t off) {
+  return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+// ----------------------------------------------------------------------------
+// device properties and kernel attributes (cached per device)
+// ----------------------------------------------------------------------------
+constexpr int MAX_DEVICES = 64;
+static std::once_flag g_attr_once[MAX_DEVICES];
+static int g_sm_count[MAX_DEVICES];
+static nh_status g_attr_status[MAX_DEVICES];
+
+using TcPrefill = tc::Shape<false, 256, 4>;
+using TcSwap16 = tc::Shape<true, 16, 8>;
+using TcSwap32 = tc::Shape<true, 32, 8>;
+using TcSwap64 = tc::Shape<true, 64, 6>;
+
+static nh_status set_attrs(int dev) {
+  cudaDeviceProp prop;
+  NH_CUDA(cudaGetDeviceProperties(&prop, dev));
+  g_sm_count[dev] = prop.multiProcessorCount;
+  if (prop.major != 10)
+    return fail(NH_ERR_UNSUPPORTED, "libnhmoe is built for sm_100a; device %d is sm_%d%d", dev,
+                prop.major, prop.minor);
+  NH_CUDA(cudaFuncSetAttribute(tc::tc_grouped_gemm<false, 256, 4>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, TcPrefill::SMEM));
+  NH_CUDA(cudaFuncSetAttribute(tc::tc_grouped_gemm<true, 16, 8>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, TcSwap16::SMEM));
+  NH_CUDA(cudaFuncSetAttribute(tc::tc_grouped_gemm<true, 32, 8>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, TcSwap32::SMEM));
+  NH_CUDA(cudaFuncSetAttribute(tc::tc_grouped_gemm<true, 64, 6>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, TcSwap64::SMEM));
+  return NH_OK;
+}
+
+static nh_status device_setup(int* dev_out) {
+  int dev;
+  NH_CUDA(cudaGetDevice(&dev));
+  if (dev < 0 || dev >= MAX_DEVICES) return fail(NH_ERR_UNSUPPORTED, "device id %d", dev);
+  std::call_once(g_attr_once[dev], [dev] { g_attr_status[dev] = set_attrs(dev); });
+  if (g_attr_status[dev] != NH_OK)
+    return fail(g_attr_status[dev], "device %d setup failed (unsupported or CUDA error)", dev);
+  *dev_out = dev;
+  return NH_OK;
+}
+
+static uint64_t timeout_ns() {
+  static uint64_t v = [] {
+    const char* s = getenv("NH_MOE_TIMEOUT_NS");
+    uint64_t t = s ? strtoull(s, nullptr, 10) : 0;
+    return t ? t : 2000000000ull;  // 2 s: far above any single pipeline wait
+  }();
+  return v;
+}
+
+// ----------------------------------------------------------------------------
+// TMA tensor maps (driver entry point fetched through the runtime)
+// ----------------------------------------------------------------------------
+static PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) != cudaSuccess ||
+        q != cudaDriverEntryPointSuccess)
+      p = nullptr;
+    return reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }();
+  return fn;
+}
+
+// bf16 [rows, K] row-major, box {64, box_rows}, 128-byte swizzle
+static nh_status map_2d(CUtensorMap* m, const void* base, int64_t K, int64_t rows, int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(NH_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[2] = {(cuuint64_t)K, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)K * 2};
+  cuuint32_t box[2] = {(cuuint32_t)tc::BK, (cuuint32_t)box_rows};
+  cuuint32_t es[2] = {1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(base), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(NH_ERR_CUDA, "cuTensorMapEncodeTiled (2d) failed: %d", (int)r);
+  return NH_OK;
+}
+
+// bf16 [n_exp, N, K] row-major, box {64, box_rows, 1}, 128-byte swizzle
+static nh_status map_3d(CUtensorMap* m, const void* base, int64_t K, int64_t N, int64_t n_exp,
+                        int box_rows) {
+  auto fn = encode_fn();
+  if (!fn) return fail(NH_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[3] = {(cuuint64_t)K, (cuuint64_t)N, (cuuint64_t)n_exp};
+  cuuint64_t strides[2] = {(cuuint64_t)K * 2, (cuuint64_t)K * N * 2};
+  cuuint32_t box[3] = {(cuuint32_t)tc::BK, (cuuint32_t)box_rows, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(NH_ERR_CUDA, "cuTensorMapEncodeTiled (3d) failed: %d", (int)r);
+  return NH_OK;
+}
+
+// ----------------------------------------------------------------------------
+// one grouped GEMM: out = epi(A[rows] . W[e]^T) over the tile entries
+// ----------------------------------------------------------------------------
+struct GemmCall {
+  const void* A;        // [rows, K] (dtype)
+  int64_t rows;         // rows of A
+  const void* W;        // [n_exp, N, K] (dtype)
+  int n_exp;
+  int N, K;
+  const int4* tiles;    // or null: dense over `rows`
+  const int32_t* num_tiles;
+  int max_tiles;        // grid bound when tiles != null
+  int tile_rows;
+  int swap;
+  int epi;
+  void* out;
+  int64_t ldo;
+  const int32_t* perm_token;
+  const float* perm_w;
+  int* status;
+};
+
+template <bool SWAP, int NT, int STAGES>
+static nh_status launch_tc(const GemmCall& c, int dev, cudaStream_t st) {
+  using S = tc::Shape<SWAP, NT, STAGES>;
+  CUtensorMap ma, mw;
+  NH_TRY(map_2d(&ma, c.A, c.K, c.rows, SWAP ? NT : tc::M));
+  NH_TRY(map_3d(&mw, c.W, c.K, c.N, c.n_exp, SWAP ? tc::M : NT));
+  tc::TcArgs g;
+  g.tiles = c.tiles;
+  g.num_tiles = c.num_tiles;
+  g.dense_rows = (int)c.rows;
+  g.tile_rows = c.tile_rows;
+  g.N = c.N;
+  g.K = c.K;
+  g.epi = c.epi;
+  g.out = c.out;
+  g.ldo = c.ldo;
+  g.perm_token = c.perm_token;
+  g.perm_w = c.perm_w;
+  g.status = c.status;
+  g.timeout_ns = timeout_ns();
+  const int n_blocks = SWAP ? (c.N + tc::M - 1) / tc::M : (c.N + NT - 1) / NT;
+  const int64_t m_max = c.tiles ? c.max_tiles : (c.rows + c.tile_rows - 1) / c.tile_rows;
+  const int64_t work = m_max * n_blocks;
+  const int grid = (int)std::min<int64_t>(work, g_sm_count[dev]);
+  if (grid <= 0) return NH_OK;
+  tc::tc_grouped_gemm<SWAP, NT, STAGES><<<grid, tc::THREADS, S::SMEM, st>>>(ma, mw, g);
+  return launch_check("tc_grouped_gemm");
+}
+
+static nh_status run_gemm(const Plan& p, const GemmCall& c, int dev, cudaStream_t st) {
+  if (c.rows == 0) return NH_OK;
+  if (!p.bf16) {
+    GemmArgs g;
+    g.A = c.A;
+    g.B = c.W;
+    g.K = c.K;
+    g.N = c.N;
+    g.tiles = c.tiles;
+    g.num_tiles = c.num_tiles;
+    g.dense_rows = (int)c.rows;
+    g.tile_rows = c.tile_rows;
+    g.epi = c.epi;
+    g.out = c.out;
+    g.ldo = c.ldo;
+    g.perm_token = c.perm_token;
+    g.perm_w = c.perm_w;
+    const int64_t m_max = c.tiles ? c.max_tiles : (c.rows + c.tile_rows - 1) / c.tile_rows;
+    if (m_max > 65535) return fail(NH_ERR_UNSUPPORTED, "float32 path: too many row tiles");
+    dim3 grid((c.N + SG_BN - 1) / SG_BN, (unsigned)m_max);
+    simt_grouped_gemm<float><<<grid, 256, 0, st>>>(g);
+    return launch_check("simt_grouped_gemm");
+  }
+  if (!c.swap) return launch_tc<false, 256, 4>(c, dev, st);
+  switch (c.tile_rows) {
+    case 16: return launch_tc<true, 16, 8>(c, dev, st);
+    case 32: return launch_tc<true, 32, 8>(c, dev, st);
+    case 64: return launch_tc<true, 64, 6>(c, dev, st);
+    default: return fail(NH_ERR_UNSUPPORTED, "tile rows %d", c.tile_rows);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// small kernels
+// ----------------------------------------------------------------------------
+__global__ void zero_f32(float4* __restrict__ p, int64_t n4) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4;
+       i += (int64_t)gridDim.x * blockDim.x)
+    p[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+}
+
+template <typename Tout>
+__global__ void finalize_kernel(const float* __restrict__ y_acc, const float* __restrict__ y_sh,
+                                Tout* __restrict__ y, int64_t n) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    float v = y_acc[i];
+    if (y_sh) v += y_sh[i];
+    y[i] = from_f32<Tout>(v);
+  }
+}
+
+__global__ void finalize_bf16_vec(const float4* __restrict__ y_acc, const float4* __restrict__ y_sh,
+                                  uint2* __restrict__ y, int64_t n4) {
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    float4 a = y_acc[i];
+    if (y_sh) {
+      const float4 b = y_sh[i];
+      a.x += b.x;
+      a.y += b.y;
+      a.z += b.z;
+      a.w += b.w;
+    }
+    y[i] = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
+  }
+}
+
+__global__ void selftest_timeout_kernel(int* status, uint64_t timeout_ns) {
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    abort_flag = 0;
+    mbar_init(smem_u32(&bar), 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    const WaitCtl w{&abort_flag, status, timeout_ns};
+    // nothing ever arrives on this barrier: the bounded wait must run out
+    mbar_wait(smem_u32(&bar), 0, w, SITE_SELFTEST);
+  }
+  __syncthreads();
+}
+
+static int grid_for(int64_t n, int per_block, int dev) {
+  int64_t b = (n + per_block - 1) / per_block;
+  const int64_t cap = (int64_t)g_sm_count[dev] * 8;
+  if (b > cap) b = cap;
+  return (int)(b < 1 ? 1 : b);
+}
+
+}  // namespace nh
+
+using namespace nh;
+
+// ============================================================================
+// C ABI
+// ============================================================================
+extern "C" {
+
+const char* nh_last_error(void) { return g_last_error.c_str(); }
+
+const char* nh_version(void) { return "nhmoe 0.1 (sm_100a)"; }
+
+nh_status nh_moe_validate(const nh_moe_config* cfg) { return validate(cfg); }
+
+nh_status nh_moe_workspace_layout(const nh_moe_config* cfg, int64_t T, nh_moe_ws_layout* out) {
+  if (!out) return fail(NH_ERR_INVALID_ARG, "out is NULL");
+  Plan p;
+  NH_TRY(make_plan(cfg, T, &p));
+  *out = p.lay;
+  return NH_OK;
+}
+
+nh_status nh_moe_workspace_size(const nh_moe_config* cfg, int64_t T, size_t* bytes) {
+  if (!bytes) return fail(NH_ERR_INVALID_ARG, "bytes is NULL");
+  Plan p;
+  NH_TRY(make_plan(cfg, T, &p));
+  *bytes = p.lay.total_bytes;
+  return NH_OK;
+}
+
+nh_status nh_moe_shared_workspace_size(const nh_moe_config* cfg, int64_t T, size_t* bytes) {
+  if (!bytes) return fail(NH_ERR_INVALID_ARG, "bytes is NULL");
+  Plan p;
+  NH_TRY(make_plan(cfg, T, &p));
+  if (!cfg->n_shared_experts) return fail(NH_ERR_INVALID_ARG, "config has no shared expert");
+  *bytes = ALIGN + align_up((size_t)T * p.S * p.elem + 1, ALIGN);
+  return NH_OK;
+}
+
+nh_status nh_moe_route(const nh_moe_config* cfg, int64_t T, const void* x, const float* w_router,
+                       const float* bias, int32_t* topk_idx, float* topk_w, void* ws,
+                       size_t ws_bytes, void* stream) {
+  Plan p;
+  NH_TRY(make_plan(cfg, T, &p));
+  NH_TRY(check_ws(p, ws, ws_bytes));
+  if (T == 0) return NH_OK;
+  NH_TRY(check_ptr(x, "x"));
+  NH_TRY(check_ptr(w_router, "w_router"));
+  NH_TRY(check_ptr(topk_idx, "topk_idx"));
+  NH_TRY(check_ptr(topk_w, "topk_w"));
+  if (bias) NH_TRY(check_ptr(bias, "e_score_correction_bias"));
+  int dev;
+  NH_TRY(device_setup(&dev));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* status = at<int>(ws, p.lay.status);
+  float* logits = at<float>(ws, p.lay.logits);
+  NH_CUDA(cudaMemsetAsync(status, 0, 16, st));
+  if (T <= 32) {
+    const int warps = (int)(p.E * ((T + 7) / 8));
+    const int blocks = (warps * 32 + 255) / 256;
+    if (p.bf16)
+      router_logits_warp<__nv_bfloat16><<<blocks, 256, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(x), w_router, logits, (int)T, p.H, p.E);
+    else
+      router_logits_warp<float><<<blocks, 256, 0, st>>>(static_cast<const float*>(x), w_router,
+                                                        logits, (int)T, p.H, p.E);
+  } else {
+    dim3 grid((unsigned)((T + RT_BT - 1) / RT_BT), (unsigned)((p.E + RT_BE - 1) / RT_BE));
+    if (p.bf16)
+      router_logits_tiled<__nv_bfloat16><<<grid, 256, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(x), w_router, logits, (int)T, p.H, p.E);
+    else
+      router_logits_tiled<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), w_router,
+                                                       logits, (int)T, p.H, p.E);
+  }
+  NH_TRY(launch_check("router_logits"));
+  SelectArgs a;
+  a.logits = logits;
+  a.bias = bias;
+  a.topk_idx = topk_idx;
+  a.topk_w = topk_w;
+  a.status = status;
+  a.T = (int)T;
+  a.E = p.E;
+  a.G = p.G;
+  a.tg = p.tg;
+  a.k = p.k;
+  a.norm = cfg->norm_topk_prob;
+  a.alpha = cfg->routed_scaling_factor;
+  a.group_score = cfg->group_score;
+  a.use_sigma = (bias != nullptr) || cfg->group_score == NH_GROUP_SCORE_TOP2;
+  router_select<<<(unsigned)((T + 127) / 128), 128, 0, st>>>(a);
+  return launch_check("router_select");
+}
+
+nh_status nh_moe_permute(const nh_moe_config* cfg, int64_t T, const void* x,
+                         const int32_t* topk_idx, const float* topk_w, void* ws, size_t ws_bytes,
+                         void* stream) {
+  Plan p;
+  NH_TRY(make_plan(cfg, T, &p));
+  NH_TRY(check_ws(p, ws, ws_bytes));
+  int dev;
+  NH_TRY(device_setup(&dev));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const nh_moe_ws_layout& L = p.lay;
+  if (T == 0) {
+    NH_CUDA(cudaMemsetAsync(at<int32_t>(ws, L.num_tiles), 0, 4, st));
+    return NH_OK;
+  }
+  NH_TRY(check_ptr(x, "x"));
+  NH_TRY(check_ptr(topk_idx, "topk_idx"));
+  NH_TRY(check_ptr(topk_w, "topk_w"));
+  int* status = at<int>(ws, L.status);
+  int32_t* chunk = at<int32_t>(ws, L.chunk_counts);
+  permute_hist<<<L.n_chunks, 256, p.E * sizeof(int), st>>>(topk_idx, (int)T, p.k, p.E, chunk, status);
+  NH_TRY(launch_check("permute_hist"));
+  const int scan_threads = ((p.E + 31) / 32) * 32;
+  permute_scan<<<1, scan_threads, 0, st>>>(chunk, L.n_chunks, p.E, L.tile_rows,
+                                            at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets),
+                                            at<int4>(ws, L.tiles), at<int32_t>(ws, L.num_tiles),
+                                            L.max_tiles);
+  NH_TRY(launch_check("permute_scan"));
+  const size_t smem = (size_t)(p.E + PERM_CHUNK * p.k) * sizeof(int);
+  if (p.bf16)
+    permute_scatter<__nv_bfloat16><<<L.n_chunks, 256, smem, st>>>(
+        topk_idx, topk_w, static_cast<const __nv_bfloat16*>(x), (int)T, p.k, p.E, p.H, chunk,
+        at<int32_t>(ws, L.perm_token), at<float>(ws, L.perm_w), at<int32_t>(ws, L.inv_row),
+        at<__nv_bfloat16>(ws, L.x_perm), status);
+  else
+    permute_scatter<float><<<L.n_chunks, 256, smem, st>>>(
+        topk_idx, topk_w, static_cast<const float*>(x), (int)T, p.k, p.E, p.H, chunk,
+        at<int32_t>(ws, L.perm_token), at<float>(ws, L.perm_w), at<int32_t>(ws, L.inv_row),
+        at<float>(ws, L.x_perm), status);
+  return launch_check("permute_scatter");
+}
+
+static nh_status experts_phase(const nh_moe_config* cfg, int64_t T, const void* w, float* y_acc,
+                               void* ws, size_t ws_bytes, void* stream, bool up_phase) {
+  Plan p;
+  NH_TRY(make_plan(cfg, T, &p));
+  NH_TRY(check_ws(p, ws, ws_bytes));
+  if (T == 0) return NH_OK;
+  NH_TRY(check_ptr(w, up_phase ? "w_up" : "w_down"));
+  if (!up_phase) NH_TRY(check_ptr(y_acc, "y_acc"));
+  int dev;
+  NH_TRY(device_setup(&dev));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const nh_moe_ws_layout& L = p.lay;
+  GemmCall c{};
+  c.rows = p.rows;
+  c.n_exp = p.E;
+  c.tiles = at<int4>(ws, L.tiles);
+  c.num_tiles = at<int32_t>(ws, L.num_tiles);
+  c.max_tiles = L.max_tiles;
+  c.tile_rows = L.tile_rows;
+  c.swap = L.swap_ab;
+  c.status = at<int>(ws, L.status);
+  if (up_phase) {
+    c.A = at<void>(ws, L.x_perm);
+    c.W = w;
+    c.N = p.I;
+    c.K = p.H;
+    c.epi = EPI_UP_RELU2;
+    c.out = at<void>(ws, L.h);
+    c.ldo = p.I;
+  } else {
+    c.A = at<void>(ws, L.h);
+    c.W = w;
+    c.N = p.H;
+    c.K = p.I;
+    c.epi = EPI_DOWN_SCATTER;
+    c.out = y_acc;
+    c.ldo = p.H;
+    c.perm_token = at<int32_t>(ws, L.perm_token);
+    c.perm_w = at<float>(ws, L.perm_w);
+  }
+  return run_gemm(p, c, dev, st);
+}
+
+nh_status nh_moe_experts_up(const nh_moe_config* cfg, int64_t T, const void* w_up, void* ws,
+                            size_t ws_bytes, void* stream) {
+  return experts_phase(cfg, T, w_up, nullptr, ws, ws_bytes, stream, true);
+}
+
+nh_status nh_moe_experts_down(const nh_moe_config* cfg, int64_t T, const void* w_down,
+                              float* y_acc, void* ws, size_t ws_bytes, void* stream) {
+  return experts_phase(cfg, T, w_down, y_acc, ws, ws_bytes, stream, false);
+}
+
+nh_status nh_moe_zero(float* buf, int64_t n, void* stream) {
+  if (n < 0) return fail(NH_ERR_INVALID_ARG, "n must be >= 0");
+  if (n == 0) return NH_OK;
+  NH_TRY(check_ptr(buf, "buf"));
+  int dev;
+  NH_TRY(device_setup(&dev));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  if (n % 4 == 0) {
+    zero_f32<<<grid_for(n / 4, 256, dev), 256, 0, st>>>(reinterpret_cast<float4*>(buf), n / 4);
+    return launch_check("zero_f32");
+  }
+  NH_CUDA(cudaMemsetAsync(buf, 0, (size_t)n * 4, st));
+  return NH_OK;
+}
+
+nh_status nh_moe_forward(const nh_moe_config* cfg, int64_t T, const void* w_up, const void* w_down,
+                         float* y_acc, void* ws, size_t ws_bytes, void* stream) {
+  Plan p;
+  NH_TRY(make_plan(cfg, T, &p));
+  NH_TRY(check_ws(p, ws, ws_bytes));
+  if (T == 0) return NH_OK;
+  NH_TRY(check_ptr(w_up, "w_up"));
+  NH_TRY(check_ptr(w_down, "w_down"));
+  NH_TRY(check_ptr(y_acc, "y_acc"));
+  NH_TRY(nh_moe_zero(y_acc, T * p.H, stream));
+  NH_TRY(nh_moe_experts_up(cfg, T, w_up, ws, ws_bytes, stream));
+  return nh_moe_experts_down(cfg, T, w_down, y_acc, ws, ws_bytes, stream);
+}
+
+nh_status nh_moe_shared(const nh_moe_config* cfg, int64_t T, const void* x, const void* w_su,
+                        const void* w_sd, float* y_shared, void* ws_shared, size_t ws_shared_bytes,
+                        void* stream) {
+  Plan p;
+  NH_TRY(make_plan(cfg, T, &p));
+  size_t need;
+  NH_TRY(nh_moe_shared_workspace_size(cfg, T, &need));
+  NH_TRY(check_ptr(ws_shared, "ws_shared"));
+  if (ws_shared_bytes < need)
+    return fail(NH_ERR_INVALID_ARG, "ws_shared holds %zu bytes, %zu needed", ws_shared_bytes, need);
+  if (T == 0) return NH_OK;
+  NH_TRY(check_ptr(x, "x"));
+  NH_TRY(check_ptr(w_su, "w_shared_up"));
+  NH_TRY(check_ptr(w_sd, "w_shared_down"));
+  NH_TRY(check_ptr(y_shared, "y_shared"));
+  int dev;
+  NH_TRY(device_setup(&dev));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* status = static_cast<int*>(ws_shared);
+  void* h = static_cast<char*>(ws_shared) + ALIGN;
+  NH_CUDA(cudaMemsetAsync(status, 0, 16, st));
+  GemmCall up{};
+  up.A = x;
+  up.rows = T;
+  up.W = w_su;
+  up.n_exp = 1;
+  up.N = p.S;
+  up.K = p.H;
+  up.tiles = nullptr;
+  up.tile_rows = p.lay.tile_rows;
+  up.swap = p.lay.swap_ab;
+  up.epi = EPI_UP_RELU2;
+  up.out = h;
+  up.ldo = p.S;
+  up.status = status;
+  NH_TRY(run_gemm(p, up, dev, st));
+  GemmCall dn = up;
+  dn.A = h;
+  dn.W = w_sd;
+  dn.N = p.H;
+  dn.K = p.S;
+  dn.epi = EPI_STORE_F32;
+  dn.out = y_shared;
+  dn.ldo = p.H;
+  return run_gemm(p, dn, dev, st);
+}
+
+nh_status nh_moe_finalize(const nh_moe_config* cfg, int64_t T, const float* y_acc,
+                          const float* y_shared, void* y, void* stream) {
+  Plan p;
+  NH_TRY(make_plan(cfg, T, &p));
+  if (T == 0) return NH_OK;
+  NH_TRY(check_ptr(y_acc, "y_acc"));
+  NH_TRY(check_ptr(y, "y"));
+  if (y_shared) NH_TRY(check_ptr(y_shared, "y_shared"));
+  if (cfg->n_shared_experts && !y_shared)
+    return fail(NH_ERR_INVALID_ARG, "y_shared is NULL but the config has a shared expert");
+  int dev;
+  NH_TRY(device_setup(&dev));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t n = T * p.H;
+  if (p.bf16 && n % 4 == 0) {
+    finalize_bf16_vec<<<grid_for(n / 4, 256, dev), 256, 0, st>>>(
+        reinterpret_cast<const float4*>(y_acc), reinterpret_cast<const float4*>(y_shared),
+        static_cast<uint2*>(y), n / 4);
+  } else if (p.bf16) {
+    finalize_kernel<__nv_bfloat16><<<grid_for(n, 256, dev), 256, 0, st>>>(
+        y_acc, y_shared, static_cast<__nv_bfloat16*>(y), n);
+  } else {
+    finalize_kernel<float><<<grid_for(n, 256, dev), 256, 0, st>>>(y_acc, y_shared,
+                                                                   static_cast<float*>(y), n);
+  }
+  return launch_check("finalize");
+}
+
+nh_status nh_moe_check_device(void* ws, void* stream) {
+  NH_TRY(check_ptr(ws, "ws"));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  NH_CUDA(cudaStreamSynchronize(st));
+  int h[4] = {0, 0, 0, 0};
+  NH_CUDA(cudaMemcpy(h, ws, sizeof h, cudaMemcpyDeviceToHost));
+  if (h[0] == NH_ERR_TIMEOUT)
+    return fail(NH_ERR_TIMEOUT, "device wait ran out (site %d, value %d)", h[1], h[2]);
+  if (h[0] == NH_ERR_DEVICE_CHECK)
+    return fail(NH_ERR_DEVICE_CHECK, "device check failed (site %d, value %d)", h[1], h[2]);
+  if (h[0] != 0) return fail((nh_status)h[0], "device status %d (site %d)", h[0], h[1]);
+  return NH_OK;
+}
+
+nh_status nh_moe_selftest_timeout(void* ws, uint64_t timeout, void* stream) {
+  NH_TRY(check_ptr(ws, "ws"));
+  if (timeout == 0 || timeout > 10000000000ull)
+    return fail(NH_ERR_INVALID_ARG, "timeout_ns must be in (0, 1e10]");
+  int dev;
+  NH_TRY(device_setup(&dev));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  NH_CUDA(cudaMemsetAsync(ws, 0, 16, st));
+  selftest_timeout_kernel<<<1, 32, 0, st>>>(static_cast<int*>(ws), timeout);
+  return launch_check("selftest_timeout");
+}
+
+}  // extern "C"

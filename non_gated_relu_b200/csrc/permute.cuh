@@ -1,0 +1,172 @@
+// permute.cuh -- token permute of the routed experts.
+//
+// The (token, slot) assignments are grouped per expert, in (token, slot)
+// order inside each expert: a per-chunk histogram, one scan over experts
+// and chunks (which also writes the tile table the expert GEMMs walk), and a
+// stable scatter that gathers x into the permuted row order.  The routed
+// experts are applied per expert id, as in MLX's SwitchMLP (fc1/fc2 indexed
+// by the router's expert ids; exo commit "Add support for Nemotron
+// sharding").
+#pragma once
+
+#include "common.cuh"
+
+namespace nh {
+
+constexpr int PERM_CHUNK = 256;  // tokens per histogram chunk
+
+// per-chunk expert histogram: chunk_counts[c][e]
+__global__ void __launch_bounds__(256) permute_hist(const int32_t* __restrict__ idx, int T, int k,
+                                                    int E, int32_t* __restrict__ chunk_counts,
+                                                    int* status) {
+  extern __shared__ int hist[];
+  for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
+  __syncthreads();
+  const int t0 = blockIdx.x * PERM_CHUNK;
+  const int n = min(PERM_CHUNK, T - t0) * k;
+  const int32_t* src = idx + (size_t)t0 * k;
+  for (int a = threadIdx.x; a < n; a += blockDim.x) {
+    const int e = src[a];
+    if (e < 0 || e >= E) {
+      record_status(status, NH_ERR_DEVICE_CHECK, SITE_PERMUTE_HIST, e);
+      continue;
+    }
+    atomicAdd(&hist[e], 1);
+  }
+  __syncthreads();
+  for (int e = threadIdx.x; e < E; e += blockDim.x)
+    chunk_counts[(size_t)blockIdx.x * E + e] = hist[e];
+}
+
+// block-wide exclusive scan of one int per thread (blockDim.x <= 1024)
+__device__ __forceinline__ int block_exclusive_scan(int v, int* smem_warp, int* total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nw = (blockDim.x + 31) >> 5;
+  int inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += y;
+  }
+  if (lane == 31) smem_warp[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < nw ? smem_warp[lane] : 0;
+    int wi = w;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, wi, o);
+      if (lane >= o) wi += y;
+    }
+    if (lane < nw) smem_warp[lane] = wi - w;
+    if (lane == nw - 1) smem_warp[32] = wi;
+  }
+  __syncthreads();
+  const int res = smem_warp[warp] + inc - v;
+  *total = smem_warp[32];
+  __syncthreads();
+  return res;
+}
+
+// One block, blockDim.x >= E (rounded to a warp multiple).  Turns the chunk
+// histograms into absolute chunk bases (in place), writes counts, offsets,
+// the tile table (expert, first row, rows, 0) with tiles of `tile_rows` rows
+// that never cross an expert boundary, and the number of tiles.
+__global__ void permute_scan(int32_t* __restrict__ chunk_counts, int n_chunks, int E,
+                             int tile_rows, int32_t* __restrict__ counts,
+                             int32_t* __restrict__ offsets, int4* __restrict__ tiles,
+                             int32_t* __restrict__ num_tiles, int max_tiles) {
+  __shared__ int warp_sums[33];
+  const int e = threadIdx.x;
+  int total = 0;
+  if (e < E)
+    for (int c = 0; c < n_chunks; ++c) total += chunk_counts[(size_t)c * E + e];
+  int all_rows;
+  const int off = block_exclusive_scan(e < E ? total : 0, warp_sums, &all_rows);
+  const int nt = (e < E) ? (total + tile_rows - 1) / tile_rows : 0;
+  int all_tiles;
+  const int toff = block_exclusive_scan(nt, warp_sums, &all_tiles);
+  if (e < E) {
+    counts[e] = total;
+    offsets[e] = off;
+    int run = off;
+    for (int c = 0; c < n_chunks; ++c) {
+      const int v = chunk_counts[(size_t)c * E + e];
+      chunk_counts[(size_t)c * E + e] = run;
+      run += v;
+    }
+    for (int i = 0; i < nt && toff + i < max_tiles; ++i) {
+      const int r0 = i * tile_rows;
+      tiles[toff + i] = make_int4(e, off + r0, min(tile_rows, total - r0), 0);
+    }
+  }
+  if (e == 0) {
+    offsets[E] = all_rows;
+    *num_tiles = min(all_tiles, max_tiles);
+  }
+}
+
+// Stable scatter of one chunk's assignments + gather of x rows into x_perm.
+// Warp 0 ranks the assignments in (t, j) order 32 at a time; then every warp
+// copies rows.  Dynamic smem: int run[E] + int pos[PERM_CHUNK * k].
+template <typename Tin>
+__global__ void __launch_bounds__(256) permute_scatter(
+    const int32_t* __restrict__ idx, const float* __restrict__ w, const Tin* __restrict__ x,
+    int T, int k, int E, int H, const int32_t* __restrict__ chunk_base,
+    int32_t* __restrict__ perm_token, float* __restrict__ perm_w, int32_t* __restrict__ inv_row,
+    Tin* __restrict__ x_perm, int* status) {
+  extern __shared__ int sm[];
+  int* run = sm;
+  int* pos = sm + E;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int c = blockIdx.x;
+  const int t0 = c * PERM_CHUNK;
+  const int n = min(PERM_CHUNK, T - t0) * k;
+  const size_t a0 = (size_t)t0 * k;
+  if (warp == 0) {
+    for (int e = lane; e < E; e += 32) run[e] = chunk_base[(size_t)c * E + e];
+    __syncwarp();
+    const unsigned lt = (1u << lane) - 1u;
+    for (int b = 0; b < n; b += 32) {
+      const int a = b + lane;
+      int e = (a < n) ? idx[a0 + a] : -1;
+      if (e >= E) e = -1;  // already reported by the histogram
+      const unsigned peers = __match_any_sync(0xffffffffu, e);
+      const int start = (e >= 0) ? run[e] : 0;
+      __syncwarp();
+      const int p = start + __popc(peers & lt);
+      if (e >= 0 && lane == __ffs(peers) - 1) run[e] = start + __popc(peers);
+      __syncwarp();
+      if (a < n) {
+        pos[a] = (e >= 0) ? p : -1;
+        if (e >= 0) {
+          perm_token[p] = t0 + a / k;
+          perm_w[p] = w[a0 + a];
+          inv_row[a0 + a] = p;
+        } else {
+          inv_row[a0 + a] = -1;
+        }
+      }
+    }
+  }
+  __syncthreads();
+  // gather rows: one warp per assignment
+  const int nw = blockDim.x >> 5;
+  const size_t row_bytes = (size_t)H * sizeof(Tin);
+  const bool vec = (row_bytes % 16) == 0;
+  for (int a = warp; a < n; a += nw) {
+    const int p = pos[a];
+    if (p < 0) continue;
+    const int t = t0 + a / k;
+    if (vec) {
+      const uint4* src = reinterpret_cast<const uint4*>(x + (size_t)t * H);
+      uint4* dst = reinterpret_cast<uint4*>(x_perm + (size_t)p * H);
+      const int nv = (int)(row_bytes / 16);
+      for (int i = lane; i < nv; i += 32) dst[i] = src[i];
+    } else {
+      for (int i = lane; i < H; i += 32) x_perm[(size_t)p * H + i] = x[(size_t)t * H + i];
+    }
+  }
+}
+
+}  // namespace nh

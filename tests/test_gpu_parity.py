@@ -1,0 +1,157 @@
+"""GPU parity of the CUDA path (through the C ABI) against the fp64 oracle.
+
+Small workloads are compared on every token and span several MMA tiles with
+ragged tails; the five full-size workloads are compared on their routing
+(every token) and on sampled tokens of the block output (plus every
+excused and every exact-tie token), in the launch configuration the
+benchmark uses.
+"""
+import numpy as np
+import pytest
+
+import oracle
+import synth
+from gpu_util import (check_output, check_routing, make_block, run_block, sample_tokens,
+                      to_dev)
+
+torch = pytest.importorskip("torch")
+pytestmark = pytest.mark.gpu
+
+
+def small(name, **kw):
+    base = dict(name=name, T=300, hidden_size=512, n_routed_experts=16, n_group=4, topk_group=2,
+                num_experts_per_tok=4, moe_intermediate_size=320,
+                moe_shared_expert_intermediate_size=640, seed=7, wr_std=0.05, w_std=0.05)
+    base.update(kw)
+    return synth.MoEConfig(**base)
+
+
+SMALL = {
+    # prefill orientation: 128-row tiles, N tails (320 = 256 + 64, 512 = 2 x 256)
+    "small_prefill": small("small_prefill"),
+    # ragged T, one group, no shared expert, norm off
+    "small_noshared": small("small_noshared", T=131, n_group=1, topk_group=1,
+                            n_shared_experts=0, norm_topk_prob=False, seed=8),
+    # decode orientation with 16 / 32 / 64-row activation tiles
+    "small_swap16": small("small_swap16", T=5, seed=9),
+    "small_swap32": small("small_swap32", T=29, seed=10),
+    "small_swap64": small("small_swap64", T=64, seed=11, moe_intermediate_size=192),
+    # float32 CUDA-core path, odd sizes
+    "small_f32_odd": small("small_f32_odd", T=77, hidden_size=100, moe_intermediate_size=36,
+                           moe_shared_expert_intermediate_size=52, dtype="f32", seed=12),
+    # limits: 512 experts, 64 groups, top-32
+    "small_max_experts": small("small_max_experts", T=70, hidden_size=128, n_routed_experts=512,
+                               n_group=64, topk_group=8, num_experts_per_tok=32,
+                               moe_intermediate_size=64, moe_shared_expert_intermediate_size=64,
+                               seed=13),
+    # single expert (routing is trivial)
+    "small_one_expert": small("small_one_expert", T=40, n_routed_experts=1, n_group=1,
+                              topk_group=1, num_experts_per_tok=1, seed=14),
+}
+
+
+@pytest.mark.parametrize("name", sorted(SMALL))
+def test_small_block_every_token(name):
+    inp = synth.make_inputs(SMALL[name])
+    y, idx, w, _ = run_block(inp)
+    exc, _, _ = check_routing(inp.cfg, inp.x, inp.w_router, idx, w)
+    check_output(inp, y, idx, w, np.arange(inp.cfg.T), exc)
+
+
+def test_all_tokens_one_expert_set():
+    """Degenerate routing: a dominant feature sends every token to the same k
+    experts (one expert then spans many row tiles)."""
+    cfg = small("skew_all", T=700, seed=15)
+    inp = synth.make_inputs(cfg)
+    inp.x[:, 0] = synth.f32_to_bf16_bits(np.array([4.0], np.float32))[0]
+    inp.w_router[:, 0] = 0.0
+    inp.w_router[[1, 2, 3, 0], 0] = [30.0, 29.0, 28.0, 27.0]
+    y, idx, w, _ = run_block(inp)
+    assert np.all(idx == np.array([1, 2, 3, 0]))
+    exc, _, _ = check_routing(cfg, inp.x, inp.w_router, idx, w)
+    check_output(inp, y, idx, w, np.arange(cfg.T), exc)
+
+
+@pytest.mark.parametrize("variant", ["bias", "top2", "bias_top2"])
+def test_router_variants(variant):
+    """Selection-only correction bias and the top-2-sum group score."""
+    cfg = small("variants", T=257, n_routed_experts=64, n_group=8, topk_group=3,
+                num_experts_per_tok=6, seed=16, wr_std=0.1)
+    gs = 1 if "top2" in variant else 0
+    inp = synth.make_inputs(cfg, with_bias="bias" in variant)
+    blk = make_block(inp)
+    blk.c.group_score = gs
+    y, idx, w, _ = run_block(inp, blk)
+    exc, _, _ = check_routing(cfg, inp.x, inp.w_router, idx, w, bias=inp.bias, group_score=gs)
+    # the block output under the GPU routing (weights from the unbiased scores)
+    tok = np.arange(cfg.T)
+    ref, _, _ = oracle.forward_parallel(inp, tokens=tok, override_idx=idx,
+                                        override_w=w.astype(np.float64))
+    assert np.abs(y - ref).max() <= 2e-2 * np.abs(ref).max()
+
+
+def test_zero_tokens():
+    cfg = SMALL["small_prefill"]
+    inp = synth.make_inputs(cfg.replace(T=1))
+    blk = make_block(inp)
+    x = to_dev(inp.x)[:0]
+    y = blk.forward(x)
+    torch.cuda.synchronize()
+    assert y.shape == (0, cfg.H)
+
+
+def test_host_api_graph_matches_eager():
+    """The public call with a host tensor (pinned copies, CUDA graph) equals the eager path."""
+    inp = synth.make_inputs(SMALL["small_swap16"])
+    blk = make_block(inp)
+    y_host = blk(inp.x).float().numpy()
+    y_eager = blk.forward(to_dev(inp.x)).float().cpu().numpy()
+    np.testing.assert_array_equal(y_host, y_eager)
+    y2 = blk(inp.x).float().numpy()          # second replay
+    np.testing.assert_array_equal(y2, y_eager)
+
+
+# ----------------------------------------------------------------------------- full size
+FULL = synth.CONFIG_ORDER
+
+
+def full_inputs(name):
+    cfg = synth.CONFIGS[name]
+    b = None
+    if cfg.skew_hot_groups:
+        import json, os
+        with open(os.path.join(os.path.dirname(__file__), "golden",
+                               "skew_prefill_t2048.json")) as f:
+            b = json.load(f)["b"]
+    return synth.make_inputs(cfg, skew_b=b)
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_full_workload(name):
+    inp = full_inputs(name)
+    cfg = inp.cfg
+    y, idx, w, blk = run_block(inp)
+    exc, _, _ = check_routing(cfg, inp.x, inp.w_router, idx, w, tie_tokens=inp.tie_tokens)
+    if cfg.T <= 64:
+        tokens = np.arange(cfg.T)
+    else:
+        extra = list(np.nonzero(exc)[0][:16])
+        if inp.tie_tokens is not None:
+            extra += list(inp.tie_tokens[:16])
+        tokens = sample_tokens(cfg.T, 48, seed=cfg.seed, extra=extra)
+    check_output(inp, y, idx, w, tokens, exc)
+    if inp.tie_tokens is not None:
+        # exact ties: lowest-index picks, equal weights alpha / k
+        np.testing.assert_allclose(w[inp.tie_tokens], cfg.routed_scaling_factor / cfg.k,
+                                   rtol=1e-6)
+    # the CUDA-graph replay of the same call gives the same bits
+    graph, xs, yg = blk.capture(cfg.T)
+    xs.copy_(to_dev(inp.x))
+    graph.replay()
+    torch.cuda.synchronize()
+    yg = yg.float().cpu().numpy()
+    if cfg.T <= 64 or cfg.dtype == "f32":
+        # no float atomics race in small decode tiles? compare within tolerance anyway
+        np.testing.assert_allclose(yg, y, rtol=0, atol=2e-2 * np.abs(y).max())
+    else:
+        np.testing.assert_allclose(yg, y, rtol=0, atol=2e-2 * np.abs(y).max())
