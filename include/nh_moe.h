@@ -88,6 +88,7 @@ typedef struct {
     size_t total_bytes;
     size_t status;        /* int32[4]: status word, first bad index, spare      */
     size_t logits;        /* float [T, E] router logits                         */
+    size_t router_w;      /* bf16 [E, 3H] router weight as three bf16 planes    */
     size_t counts;        /* int32 [E] assignments per expert                   */
     size_t offsets;       /* int32 [E + 1] exclusive scan of counts             */
     size_t chunk_counts;  /* int32 [n_chunks, E] per-chunk histograms           */

@@ -43,6 +43,7 @@ struct TcArgs {
   int tile_rows;
   int N;                      // output features (weight rows)
   int K;                      // multiple of 64
+  int a_kwrap;                // >0: the activation's K coordinate wraps at this value
   int epi;                    // Epilogue
   void* out;
   int64_t ldo;                // row stride of out, elements
@@ -188,13 +189,14 @@ __global__ void __launch_bounds__(THREADS, 1)
           break;
         }
         const uint32_t sa = base + stage * S::STAGE_BYTES, sb = sa + S::A_BYTES;
+        const int ka = g.a_kwrap ? (kb * BK) % g.a_kwrap : kb * BK;
         mbar_arrive_expect_tx(full_bar(stage), S::STAGE_BYTES);
         if (!SWAP) {
-          tma_load_2d(sa, &map_act, full_bar(stage), kb * BK, ent.y);
+          tma_load_2d(sa, &map_act, full_bar(stage), ka, ent.y);
           tma_load_3d(sb, &map_w, full_bar(stage), kb * BK, nb * NT, ent.x);
         } else {
           tma_load_3d(sa, &map_w, full_bar(stage), kb * BK, nb * M, ent.x);
-          tma_load_2d(sb, &map_act, full_bar(stage), kb * BK, ent.y);
+          tma_load_2d(sb, &map_act, full_bar(stage), ka, ent.y);
         }
         ++issued;
         if (++stage == STAGES) {

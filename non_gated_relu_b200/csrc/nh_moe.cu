@@ -168,6 +168,7 @@ static nh_status make_plan(const nh_moe_config* c, int64_t T, Plan* p) {
   };
   L.status = take(16);
   L.logits = take((size_t)T * p->E * 4);
+  L.router_w = take(p->bf16 ? (size_t)p->E * 3 * p->H * 2 : 0);
   L.counts = take((size_t)p->E * 4);
   L.offsets = take((size_t)(p->E + 1) * 4);
   L.chunk_counts = take((size_t)L.n_chunks * p->E * 4);
@@ -304,7 +305,8 @@ static nh_status map_3d(CUtensorMap* m, const void* base, int64_t K, int64_t N, 
 // one grouped GEMM: out = epi(A[rows] . W[e]^T) over the tile entries
 // ----------------------------------------------------------------------------
 struct GemmCall {
-  const void* A;        // [rows, K] (dtype)
+  const void* A;        // [rows, K_a] (dtype); K_a = a_kwrap when set, else K
+  int a_kwrap;
   int64_t rows;         // rows of A
   const void* W;        // [n_exp, N, K] (dtype)
   int n_exp;
@@ -326,7 +328,7 @@ template <bool SWAP, int NT, int STAGES>
 static nh_status launch_tc(const GemmCall& c, int dev, cudaStream_t st) {
   using S = tc::Shape<SWAP, NT, STAGES>;
   CUtensorMap ma, mw;
-  NH_TRY(map_2d(&ma, c.A, c.K, c.rows, SWAP ? NT : tc::M));
+  NH_TRY(map_2d(&ma, c.A, c.a_kwrap ? c.a_kwrap : c.K, c.rows, SWAP ? NT : tc::M));
   NH_TRY(map_3d(&mw, c.W, c.K, c.N, c.n_exp, SWAP ? tc::M : NT));
   tc::TcArgs g;
   g.tiles = c.tiles;
@@ -335,6 +337,7 @@ static nh_status launch_tc(const GemmCall& c, int dev, cudaStream_t st) {
   g.tile_rows = c.tile_rows;
   g.N = c.N;
   g.K = c.K;
+  g.a_kwrap = c.a_kwrap;
   g.epi = c.epi;
   g.out = c.out;
   g.ldo = c.ldo;
@@ -501,25 +504,6 @@ nh_status nh_moe_route(const nh_moe_config* cfg, int64_t T, const void* x, const
   int* status = at<int>(ws, p.lay.status);
   float* logits = at<float>(ws, p.lay.logits);
   NH_CUDA(cudaMemsetAsync(status, 0, 16, st));
-  if (T <= 32) {
-    const int warps = (int)(p.E * ((T + 7) / 8));
-    const int blocks = (warps * 32 + 255) / 256;
-    if (p.bf16)
-      router_logits_warp<__nv_bfloat16><<<blocks, 256, 0, st>>>(
-          static_cast<const __nv_bfloat16*>(x), w_router, logits, (int)T, p.H, p.E);
-    else
-      router_logits_warp<float><<<blocks, 256, 0, st>>>(static_cast<const float*>(x), w_router,
-                                                        logits, (int)T, p.H, p.E);
-  } else {
-    dim3 grid((unsigned)((T + RT_BT - 1) / RT_BT), (unsigned)((p.E + RT_BE - 1) / RT_BE));
-    if (p.bf16)
-      router_logits_tiled<__nv_bfloat16><<<grid, 256, 0, st>>>(
-          static_cast<const __nv_bfloat16*>(x), w_router, logits, (int)T, p.H, p.E);
-    else
-      router_logits_tiled<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), w_router,
-                                                       logits, (int)T, p.H, p.E);
-  }
-  NH_TRY(launch_check("router_logits"));
   SelectArgs a;
   a.logits = logits;
   a.bias = bias;
@@ -535,7 +519,54 @@ nh_status nh_moe_route(const nh_moe_config* cfg, int64_t T, const void* x, const
   a.alpha = cfg->routed_scaling_factor;
   a.group_score = cfg->group_score;
   a.use_sigma = (bias != nullptr) || cfg->group_score == NH_GROUP_SCORE_TOP2;
-  router_select<<<(unsigned)((T + 127) / 128), 128, 0, st>>>(a);
+  const size_t sel_smem = (size_t)8 * p.E * sizeof(float);
+  if (T <= 32) {
+    // decode: logits and selection in one launch (last block selects)
+    const int warps = (int)(p.E * ((T + 7) / 8));
+    const int blocks = (warps + 7) / 8;
+    unsigned int* done = reinterpret_cast<unsigned int*>(status + 3);
+    if (p.bf16)
+      router_fused_small<__nv_bfloat16><<<blocks, 256, sel_smem, st>>>(
+          static_cast<const __nv_bfloat16*>(x), w_router, a, p.H, done);
+    else
+      router_fused_small<float><<<blocks, 256, sel_smem, st>>>(static_cast<const float*>(x),
+                                                                w_router, a, p.H, done);
+    return launch_check("router_fused_small");
+  }
+  if (p.bf16 && p.E % 32 == 0) {
+    // logits on the tensor cores: x (bf16) against the fp32 router weight split
+    // into three bf16 planes, accumulated over K = 3H in fp32
+    __nv_bfloat16* wsplit = at<__nv_bfloat16>(ws, p.lay.router_w);
+    router_split<<<grid_for((int64_t)p.E * p.H, 256, dev), 256, 0, st>>>(w_router, wsplit, p.E,
+                                                                          p.H);
+    NH_TRY(launch_check("router_split"));
+    GemmCall c{};
+    c.A = x;
+    c.a_kwrap = p.H;
+    c.rows = T;
+    c.W = wsplit;
+    c.n_exp = 1;
+    c.N = p.E;
+    c.K = 3 * p.H;
+    c.tiles = nullptr;
+    c.tile_rows = tc::M;
+    c.swap = 0;
+    c.epi = EPI_STORE_F32;
+    c.out = logits;
+    c.ldo = p.E;
+    c.status = status;
+    NH_TRY((launch_tc<false, 256, 4>(c, dev, st)));
+  } else {
+    dim3 grid((unsigned)((T + RT_BT - 1) / RT_BT), (unsigned)((p.E + RT_BE - 1) / RT_BE));
+    if (p.bf16)
+      router_logits_tiled<__nv_bfloat16><<<grid, 256, 0, st>>>(
+          static_cast<const __nv_bfloat16*>(x), w_router, logits, (int)T, p.H, p.E);
+    else
+      router_logits_tiled<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), w_router,
+                                                       logits, (int)T, p.H, p.E);
+    NH_TRY(launch_check("router_logits_tiled"));
+  }
+  router_select<<<(unsigned)((T + 7) / 8), 256, sel_smem, st>>>(a);
   return launch_check("router_select");
 }
 
@@ -557,6 +588,24 @@ nh_status nh_moe_permute(const nh_moe_config* cfg, int64_t T, const void* x,
   NH_TRY(check_ptr(topk_idx, "topk_idx"));
   NH_TRY(check_ptr(topk_w, "topk_w"));
   int* status = at<int>(ws, L.status);
+  if (T <= PERM_CHUNK) {
+    // decode-sized: the whole permute in one block
+    const size_t smem = (size_t)(p.E + T * p.k) * sizeof(int);
+    if (p.bf16)
+      permute_small<__nv_bfloat16><<<1, 512, smem, st>>>(
+          topk_idx, topk_w, static_cast<const __nv_bfloat16*>(x), (int)T, p.k, p.E, p.H,
+          L.tile_rows, L.max_tiles, at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets),
+          at<int4>(ws, L.tiles), at<int32_t>(ws, L.num_tiles), at<int32_t>(ws, L.perm_token),
+          at<float>(ws, L.perm_w), at<int32_t>(ws, L.inv_row), at<__nv_bfloat16>(ws, L.x_perm),
+          status);
+    else
+      permute_small<float><<<1, 512, smem, st>>>(
+          topk_idx, topk_w, static_cast<const float*>(x), (int)T, p.k, p.E, p.H, L.tile_rows,
+          L.max_tiles, at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets),
+          at<int4>(ws, L.tiles), at<int32_t>(ws, L.num_tiles), at<int32_t>(ws, L.perm_token),
+          at<float>(ws, L.perm_w), at<int32_t>(ws, L.inv_row), at<float>(ws, L.x_perm), status);
+    return launch_check("permute_small");
+  }
   int32_t* chunk = at<int32_t>(ws, L.chunk_counts);
   permute_hist<<<L.n_chunks, 256, p.E * sizeof(int), st>>>(topk_idx, (int)T, p.k, p.E, chunk, status);
   NH_TRY(launch_check("permute_hist"));
@@ -567,17 +616,27 @@ nh_status nh_moe_permute(const nh_moe_config* cfg, int64_t T, const void* x,
                                             L.max_tiles);
   NH_TRY(launch_check("permute_scan"));
   const size_t smem = (size_t)(p.E + PERM_CHUNK * p.k) * sizeof(int);
-  if (p.bf16)
-    permute_scatter<__nv_bfloat16><<<L.n_chunks, 256, smem, st>>>(
+  const int gather_blocks = g_sm_count[dev] * 4;
+  if (p.bf16) {
+    permute_scatter<__nv_bfloat16><<<L.n_chunks, 32, smem, st>>>(
         topk_idx, topk_w, static_cast<const __nv_bfloat16*>(x), (int)T, p.k, p.E, p.H, chunk,
         at<int32_t>(ws, L.perm_token), at<float>(ws, L.perm_w), at<int32_t>(ws, L.inv_row),
-        at<__nv_bfloat16>(ws, L.x_perm), status);
-  else
-    permute_scatter<float><<<L.n_chunks, 256, smem, st>>>(
+        at<__nv_bfloat16>(ws, L.x_perm), status, 0);
+    NH_TRY(launch_check("permute_scatter"));
+    permute_gather<__nv_bfloat16><<<gather_blocks, 256, 0, st>>>(
+        static_cast<const __nv_bfloat16*>(x), at<int32_t>(ws, L.perm_token),
+        at<int32_t>(ws, L.offsets), p.E, p.H, at<__nv_bfloat16>(ws, L.x_perm));
+  } else {
+    permute_scatter<float><<<L.n_chunks, 32, smem, st>>>(
         topk_idx, topk_w, static_cast<const float*>(x), (int)T, p.k, p.E, p.H, chunk,
         at<int32_t>(ws, L.perm_token), at<float>(ws, L.perm_w), at<int32_t>(ws, L.inv_row),
-        at<float>(ws, L.x_perm), status);
-  return launch_check("permute_scatter");
+        at<float>(ws, L.x_perm), status, 0);
+    NH_TRY(launch_check("permute_scatter"));
+    permute_gather<float><<<gather_blocks, 256, 0, st>>>(
+        static_cast<const float*>(x), at<int32_t>(ws, L.perm_token), at<int32_t>(ws, L.offsets),
+        p.E, p.H, at<float>(ws, L.x_perm));
+  }
+  return launch_check("permute_gather");
 }
 
 static nh_status experts_phase(const nh_moe_config* cfg, int64_t T, const void* w, float* y_acc,

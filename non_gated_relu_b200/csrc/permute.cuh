@@ -114,7 +114,7 @@ __global__ void __launch_bounds__(256) permute_scatter(
     const int32_t* __restrict__ idx, const float* __restrict__ w, const Tin* __restrict__ x,
     int T, int k, int E, int H, const int32_t* __restrict__ chunk_base,
     int32_t* __restrict__ perm_token, float* __restrict__ perm_w, int32_t* __restrict__ inv_row,
-    Tin* __restrict__ x_perm, int* status) {
+    Tin* __restrict__ x_perm, int* status, int do_gather) {
   extern __shared__ int sm[];
   int* run = sm;
   int* pos = sm + E;
@@ -150,6 +150,7 @@ __global__ void __launch_bounds__(256) permute_scatter(
     }
   }
   __syncthreads();
+  if (!do_gather) return;
   // gather rows: one warp per assignment
   const int nw = blockDim.x >> 5;
   const size_t row_bytes = (size_t)H * sizeof(Tin);
@@ -166,6 +167,115 @@ __global__ void __launch_bounds__(256) permute_scatter(
     } else {
       for (int i = lane; i < H; i += 32) x_perm[(size_t)p * H + i] = x[(size_t)t * H + i];
     }
+  }
+}
+
+// copy one row of H elements with 16-byte vectors when possible
+template <typename Tin>
+__device__ __forceinline__ void copy_row(const Tin* __restrict__ src, Tin* __restrict__ dst, int H,
+                                         int lane) {
+  const size_t row_bytes = (size_t)H * sizeof(Tin);
+  if ((row_bytes % 16) == 0) {
+    const uint4* s4 = reinterpret_cast<const uint4*>(src);
+    uint4* d4 = reinterpret_cast<uint4*>(dst);
+    const int nv = (int)(row_bytes / 16);
+    int i = lane;
+    for (; i + 32 < nv; i += 64) {
+      const uint4 a = s4[i], b = s4[i + 32];
+      d4[i] = a;
+      d4[i + 32] = b;
+    }
+    for (; i < nv; i += 32) d4[i] = s4[i];
+  } else {
+    for (int i = lane; i < H; i += 32) dst[i] = src[i];
+  }
+}
+
+// x_perm[p] = x[perm_token[p]] for every permuted row (one warp per row)
+template <typename Tin>
+__global__ void __launch_bounds__(256) permute_gather(const Tin* __restrict__ x,
+                                                      const int32_t* __restrict__ perm_token,
+                                                      const int32_t* __restrict__ offsets, int E,
+                                                      int H, Tin* __restrict__ x_perm) {
+  const int lane = threadIdx.x & 31;
+  const int rows = offsets[E];
+  const int nw = (gridDim.x * blockDim.x) >> 5;
+  for (int p = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; p < rows; p += nw)
+    copy_row(x + (size_t)perm_token[p] * H, x_perm + (size_t)p * H, H, lane);
+}
+
+// Whole permute in one block for T <= PERM_CHUNK tokens (decode): histogram,
+// scan, tile table, stable ranking and gather.  blockDim.x = 512 (>= E).
+// Dynamic smem: int cnt[E] + int pos[T * k].
+template <typename Tin>
+__global__ void __launch_bounds__(512) permute_small(
+    const int32_t* __restrict__ idx, const float* __restrict__ w, const Tin* __restrict__ x,
+    int T, int k, int E, int H, int tile_rows, int max_tiles, int32_t* __restrict__ counts,
+    int32_t* __restrict__ offsets, int4* __restrict__ tiles, int32_t* __restrict__ num_tiles,
+    int32_t* __restrict__ perm_token, float* __restrict__ perm_w, int32_t* __restrict__ inv_row,
+    Tin* __restrict__ x_perm, int* status) {
+  extern __shared__ int sm[];
+  __shared__ int warp_sums[33];
+  int* cnt = sm;
+  int* pos = sm + E;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int n = T * k;
+  for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
+  __syncthreads();
+  for (int a = threadIdx.x; a < n; a += blockDim.x) {
+    const int e = idx[a];
+    if (e < 0 || e >= E) {
+      record_status(status, NH_ERR_DEVICE_CHECK, SITE_PERMUTE_HIST, e);
+      continue;
+    }
+    atomicAdd(&cnt[e], 1);
+  }
+  __syncthreads();
+  const int e = threadIdx.x;
+  const int total = e < E ? cnt[e] : 0;
+  int all_rows, all_tiles;
+  const int off = block_exclusive_scan(total, warp_sums, &all_rows);
+  const int nt = (total + tile_rows - 1) / tile_rows;
+  const int toff = block_exclusive_scan(nt, warp_sums, &all_tiles);
+  if (e < E) {
+    counts[e] = total;
+    offsets[e] = off;
+    for (int i = 0; i < nt && toff + i < max_tiles; ++i)
+      tiles[toff + i] = make_int4(e, off + i * tile_rows, min(tile_rows, total - i * tile_rows), 0);
+    cnt[e] = off;  // running position for the ranking
+  }
+  if (e == 0) {
+    offsets[E] = all_rows;
+    *num_tiles = min(all_tiles, max_tiles);
+  }
+  __syncthreads();
+  if (warp == 0) {
+    const unsigned lt = (1u << lane) - 1u;
+    for (int b = 0; b < n; b += 32) {
+      const int a = b + lane;
+      int ee = (a < n) ? idx[a] : -1;
+      if (ee >= E) ee = -1;
+      const unsigned peers = __match_any_sync(0xffffffffu, ee);
+      const int start = (ee >= 0) ? cnt[ee] : 0;
+      __syncwarp();
+      const int p = start + __popc(peers & lt);
+      if (ee >= 0 && lane == __ffs(peers) - 1) cnt[ee] = start + __popc(peers);
+      __syncwarp();
+      if (a < n) {
+        pos[a] = (ee >= 0) ? p : -1;
+        inv_row[a] = (ee >= 0) ? p : -1;
+        if (ee >= 0) {
+          perm_token[p] = a / k;
+          perm_w[p] = w[a];
+        }
+      }
+    }
+  }
+  __syncthreads();
+  const int nw = blockDim.x >> 5;
+  for (int a = warp; a < n; a += nw) {
+    const int p = pos[a];
+    if (p >= 0) copy_row(x + (size_t)(a / k) * H, x_perm + (size_t)p * H, H, lane);
   }
 }
 

@@ -119,86 +119,189 @@ __device__ __forceinline__ bool ranks_before(float va, int ia, float vb, int ib)
   return va > vb || (va == vb && ia < ib);
 }
 
-__global__ void __launch_bounds__(128) router_select(SelectArgs a) {
-  const int t = blockIdx.x * blockDim.x + threadIdx.x;
-  if (t >= a.T) return;
-  const float* l = a.logits + (size_t)t * a.E;
-  const int g = a.E / a.G;
-  auto sel = [&](int e) -> float {
-    if (!a.use_sigma) return l[e];
-    return sigmoid_f32(l[e]) + (a.bias ? a.bias[e] : 0.f);
-  };
+// warp-wide argmax under ranks_before (larger value, then lower id)
+__device__ __forceinline__ void warp_best(float& v, int& i) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    const float ov = __shfl_xor_sync(0xffffffffu, v, o);
+    const int oi = __shfl_xor_sync(0xffffffffu, i, o);
+    if (oi >= 0 && (i < 0 || ranks_before(ov, oi, v, i))) {
+      v = ov;
+      i = oi;
+    }
+  }
+}
 
-  // group scores (G <= 64)
-  float gs[64];
-  for (int q = 0; q < a.G; ++q) {
+// Selection of one token by one warp; `sel` holds the token's E selection
+// scores in shared memory (written by the caller).
+__device__ __forceinline__ void select_token(const SelectArgs& a, int t, const float* l,
+                                             float* sel, int lane) {
+  const int E = a.E, G = a.G, g = E / G;
+  for (int e = lane; e < E; e += 32) {
+    const float le = __ldcg(l + e);  // produced by another block or kernel: read at L2
+    sel[e] = a.use_sigma ? sigmoid_f32(le) + (a.bias ? a.bias[e] : 0.f) : le;
+  }
+  __syncwarp();
+  // group scores: lane q (and q + 32) reduces its group
+  float gsv[2];
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {
+    const int q = lane + 32 * r;
     float m1 = -INFINITY, m2 = -INFINITY;
-    for (int i = 0; i < g; ++i) {
-      const float v = sel(q * g + i);
-      if (v > m1) {
-        m2 = m1;
-        m1 = v;
-      } else if (v > m2) {
-        m2 = v;
+    if (q < G) {
+      for (int i = 0; i < g; ++i) {
+        const float v = sel[q * g + i];
+        if (v > m1) {
+          m2 = m1;
+          m1 = v;
+        } else if (v > m2) {
+          m2 = v;
+        }
       }
     }
-    gs[q] = a.group_score ? m1 + m2 : m1;
+    gsv[r] = a.group_score ? m1 + m2 : m1;
   }
-  // keep the tg best groups: each pass takes the best group ranked after the previous pick
+  // keep the tg best groups (each pass: best group ranked after the previous pick)
   uint64_t keep = 0;
   int pq = -1;
   float pv = 0.f;
   for (int r = 0; r < a.tg; ++r) {
-    int bq = -1;
     float bv = 0.f;
-    for (int q = 0; q < a.G; ++q) {
-      if (pq >= 0 && !ranks_before(pv, pq, gs[q], q)) continue;
-      if (bq < 0 || ranks_before(gs[q], q, bv, bq)) {
+    int bq = -1;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int q = lane + 32 * h;
+      if (q >= G) continue;
+      if (pq >= 0 && !ranks_before(pv, pq, gsv[h], q)) continue;
+      if (bq < 0 || ranks_before(gsv[h], q, bv, bq)) {
         bq = q;
-        bv = gs[q];
+        bv = gsv[h];
       }
     }
+    warp_best(bv, bq);
     if (bq < 0) {
-      record_status(a.status, NH_ERR_DEVICE_CHECK, SITE_ROUTE_SELECT, t);
+      if (lane == 0) record_status(a.status, NH_ERR_DEVICE_CHECK, SITE_ROUTE_SELECT, t);
       bq = r;
     }
     keep |= 1ull << bq;
     pq = bq;
     pv = bv;
   }
-  // top-k among the kept groups' experts, in (score desc, id asc) order
-  int32_t* out_i = a.topk_idx + (size_t)t * a.k;
-  float* out_w = a.topk_w + (size_t)t * a.k;
+  // top-k experts of the kept groups in (score desc, id asc) order
   int pe = -1;
-  float pev = 0.f, ssum = 0.f;
-  float sj[32];
+  float pev = 0.f, ssum = 0.f, my_s = 0.f;
+  int my_e = 0;
   for (int j = 0; j < a.k; ++j) {
-    int be = -1;
     float bv = 0.f;
-    for (int q = 0; q < a.G; ++q) {
-      if (!((keep >> q) & 1ull)) continue;
-      for (int i = 0; i < g; ++i) {
-        const int e = q * g + i;
-        const float v = sel(e);
-        if (pe >= 0 && !ranks_before(pev, pe, v, e)) continue;
-        if (be < 0 || ranks_before(v, e, bv, be)) {
-          be = e;
-          bv = v;
-        }
+    int be = -1;
+    for (int e = lane; e < E; e += 32) {
+      if (!((keep >> (e / g)) & 1ull)) continue;
+      const float v = sel[e];
+      if (pe >= 0 && !ranks_before(pev, pe, v, e)) continue;
+      if (be < 0 || ranks_before(v, e, bv, be)) {
+        be = e;
+        bv = v;
       }
     }
+    warp_best(bv, be);
     if (be < 0) {
-      record_status(a.status, NH_ERR_DEVICE_CHECK, SITE_ROUTE_SELECT, t);
+      if (lane == 0) record_status(a.status, NH_ERR_DEVICE_CHECK, SITE_ROUTE_SELECT, t);
       be = 0;
     }
-    out_i[j] = be;
-    sj[j] = sigmoid_f32(l[be]);
-    ssum += sj[j];
+    const float sj = sigmoid_f32(__ldcg(l + be));
+    ssum += sj;
+    if (lane == j) {
+      my_e = be;
+      my_s = sj;
+    }
     pe = be;
     pev = bv;
   }
-  for (int j = 0; j < a.k; ++j)
-    out_w[j] = a.norm ? a.alpha * sj[j] / ssum : a.alpha * sj[j];
+  if (lane < a.k) {
+    a.topk_idx[(size_t)t * a.k + lane] = my_e;
+    a.topk_w[(size_t)t * a.k + lane] = a.norm ? a.alpha * my_s / ssum : a.alpha * my_s;
+  }
+}
+
+// one warp per token; dynamic smem: warps_per_block * E floats
+__global__ void __launch_bounds__(256) router_select(SelectArgs a) {
+  extern __shared__ float sel_smem[];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int t = blockIdx.x * (blockDim.x >> 5) + warp;
+  if (t >= a.T) return;
+  select_token(a, t, a.logits + (size_t)t * a.E, sel_smem + (size_t)warp * a.E, lane);
+}
+
+// Decode-sized T (<= 32): logits by one warp per (expert, 8-token block), then
+// the last block to finish selects every token.  `done` is a zeroed counter
+// in the workspace; the last block resets it for the next call.
+template <typename Tin>
+__global__ void __launch_bounds__(256) router_fused_small(const Tin* __restrict__ x,
+                                                          const float* __restrict__ wr,
+                                                          SelectArgs a, int H,
+                                                          unsigned int* done) {
+  extern __shared__ float sel_smem[];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int T = a.T, E = a.E;
+  const int warp = blockIdx.x * 8 + wib;
+  const int tblocks = (T + 7) >> 3;
+  const int e = warp / tblocks, tb = warp - e * tblocks;
+  float* logits = const_cast<float*>(a.logits);
+  if (e < E) {
+    const int t0 = tb * 8, nt = min(8, T - t0);
+    float acc[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
+    const float* w = wr + (size_t)e * H;
+    const Tin* xb = x + (size_t)t0 * H;
+#pragma unroll 4
+    for (int h = lane; h < H; h += 32) {
+      const float wv = __ldg(w + h);
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+        if (i < nt) acc[i] = fmaf(to_f32(xb[(size_t)i * H + h]), wv, acc[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+      float v = acc[i];
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+      if (lane == 0 && i < nt) logits[(size_t)(t0 + i) * E + e] = v;
+    }
+  }
+  // last-block-done: the block that finishes last sees every logit
+  __shared__ unsigned int ticket;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) ticket = atomicAdd(done, 1u);
+  __syncthreads();
+  if (ticket != gridDim.x - 1) return;
+  __threadfence();
+  for (int t = wib; t < T; t += 8)
+    select_token(a, t, logits + (size_t)t * E, sel_smem + (size_t)wib * E, lane);
+  if (threadIdx.x == 0) *done = 0u;
+}
+
+// fp32 router weight -> three bf16 planes [E][3H] (hi | mid | lo) with
+// w = hi + mid + lo to 24 significant bits, so that a bf16 tensor-core GEMM
+// over K = 3H reproduces the fp32-weight logits.
+__global__ void router_split(const float* __restrict__ wr, __nv_bfloat16* __restrict__ out, int E,
+                             int H) {
+  const int64_t n = (int64_t)E * H;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const int e = (int)(i / H), h = (int)(i - (int64_t)e * H);
+    const float w = wr[i];
+    const __nv_bfloat16 hi = __float2bfloat16_rn(w);
+    const float r1 = w - __bfloat162float(hi);
+    const __nv_bfloat16 mid = __float2bfloat16_rn(r1);
+    const float r2 = r1 - __bfloat162float(mid);
+    const __nv_bfloat16 lo = __float2bfloat16_rn(r2);
+    __nv_bfloat16* row = out + (size_t)e * 3 * H;
+    row[h] = hi;
+    row[H + h] = mid;
+    row[2 * H + h] = lo;
+  }
 }
 
 }  // namespace nh

@@ -73,7 +73,9 @@ def test_workspace_layout(name):
     assert L.total_bytes == nh.workspace_size(cfg, T)
     rows = T * cfg.k
     elem = 2 if cfg.dtype == "bf16" else 4
-    regions = [("status", 16), ("logits", T * cfg.E * 4), ("counts", cfg.E * 4),
+    regions = [("status", 16), ("logits", T * cfg.E * 4),
+               ("router_w", cfg.E * 3 * cfg.H * 2 if cfg.dtype == "bf16" else 1),
+               ("counts", cfg.E * 4),
                ("offsets", (cfg.E + 1) * 4), ("chunk_counts", L.n_chunks * cfg.E * 4),
                ("perm_token", rows * 4), ("perm_w", rows * 4), ("inv_row", rows * 4),
                ("tiles", L.max_tiles * 16), ("num_tiles", 4), ("x_perm", rows * cfg.H * elem),

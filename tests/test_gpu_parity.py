@@ -64,8 +64,10 @@ def test_all_tokens_one_expert_set():
     cfg = small("skew_all", T=700, seed=15)
     inp = synth.make_inputs(cfg)
     inp.x[:, 0] = synth.f32_to_bf16_bits(np.array([4.0], np.float32))[0]
+    inp.w_router[:, 1:] *= np.float32(0.1)       # other features: logits within +-0.6
     inp.w_router[:, 0] = 0.0
-    inp.w_router[[1, 2, 3, 0], 0] = [30.0, 29.0, 28.0, 27.0]
+    # logits 6, 5, 4, 3: well apart, far from sigmoid saturation
+    inp.w_router[[1, 2, 3, 0], 0] = [1.5, 1.25, 1.0, 0.75]
     y, idx, w, _ = run_block(inp)
     assert np.all(idx == np.array([1, 2, 3, 0]))
     exc, _, _ = check_routing(cfg, inp.x, inp.w_router, idx, w)
@@ -150,8 +152,5 @@ def test_full_workload(name):
     graph.replay()
     torch.cuda.synchronize()
     yg = yg.float().cpu().numpy()
-    if cfg.T <= 64 or cfg.dtype == "f32":
-        # no float atomics race in small decode tiles? compare within tolerance anyway
-        np.testing.assert_allclose(yg, y, rtol=0, atol=2e-2 * np.abs(y).max())
-    else:
-        np.testing.assert_allclose(yg, y, rtol=0, atol=2e-2 * np.abs(y).max())
+    # float atomics of the combine may add in another order: compare within tolerance
+    np.testing.assert_allclose(yg, y, rtol=0, atol=1e-2 * np.abs(y).max())
