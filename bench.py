@@ -52,7 +52,24 @@ def parse():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--batches", type=int, default=4, help="distinct input batches cycled")
+    ap.add_argument("--eager", action="store_true",
+                    help="timed loop calls the block eagerly (NVTX range per call) instead of "
+                         "replaying CUDA graphs")
+    ap.add_argument("--only-timed", action="store_true",
+                    help="run the timed loop only (inside an NVTX range 'timed'), for profilers")
+    ap.add_argument("--set", action="append", default=[], metavar="KEY=VALUE",
+                    help="override a workload field (smaller profiling cases of the same kernels)")
     return ap.parse_args()
+
+
+def workload(args):
+    cfg = synth.CONFIGS[args.workload]
+    kw = {}
+    for item in args.set:
+        k, v = item.split("=", 1)
+        cur = getattr(cfg, k)
+        kw[k] = type(cur)(v) if not isinstance(cur, bool) else v.lower() in ("1", "true")
+    return cfg.replace(**kw) if kw else cfg
 
 
 def peaks():
@@ -156,7 +173,7 @@ def run_ours(args, rank, world, local_rank):
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    cfg = synth.CONFIGS[args.workload]
+    cfg = workload(args)
     inp = synth.make_inputs(cfg, skew_b=skew_b(cfg))
     blk = nh.NemotronHMoE(cfg, inp.w_router, inp.w_up, inp.w_down, inp.w_shared_up,
                           inp.w_shared_down, device=dev)
@@ -212,11 +229,17 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     torch.cuda.synchronize(dev)
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.nvtx.range_push("timed")
     t_start.record(main)
-    for i in range(steps):
-        graphs[i % nb].replay()
+    if args.eager:
+        for i in range(steps):
+            blk.forward(xs[i % nb], b, nvtx=True)
+    else:
+        for i in range(steps):
+            graphs[i % nb].replay()
     t_end.record(main)
     torch.cuda.synchronize(dev)
+    torch.cuda.nvtx.range_pop()
     if dist:
         dist.barrier()
     elapsed_ms = t_start.elapsed_time(t_end)
@@ -228,6 +251,11 @@ def run_ours(args, rank, world, local_rank):
     rc = blk.check(T)
     if rc != 0:
         raise RuntimeError(f"device status {rc} after the timed region")
+    if args.only_timed:
+        if rank == 0:
+            return {"workload": cfg.name, "T": T, "E": cfg.E, "steps": steps,
+                    "ms_per_step": round(elapsed_ms / steps, 5), "only_timed": True}
+        return None
 
     # per-kernel durations (eager calls, events on the launching streams)
     kern = kernel_times(blk, xs, b, nb, steps=min(steps, 200))
@@ -395,7 +423,7 @@ def ncu_traffic(workload, kernel):
 def run_reference(args, rank, world):
     if rank != 0:
         return None
-    cfg = synth.CONFIGS[args.workload]
+    cfg = workload(args)
     import oracle
     inp = synth.make_inputs(cfg, skew_b=skew_b(cfg))
     n = min(cfg.T, 8)

@@ -104,25 +104,39 @@ class NemotronHMoE:
         return b
 
     # ------------------------------------------------------------------ compute
-    def forward(self, x: torch.Tensor, bufs: Optional[Buffers] = None) -> torch.Tensor:
-        """y for a device tensor x [T, H]; returns the buffer-owned y [T, H]."""
+    def forward(self, x: torch.Tensor, bufs: Optional[Buffers] = None,
+                nvtx: bool = False) -> torch.Tensor:
+        """y for a device tensor x [T, H]; returns the buffer-owned y [T, H].
+        ``nvtx`` wraps each call in an NVTX range of its name (for profilers)."""
         T = x.shape[0]
         b = bufs or self.buffers(T)
         main = torch.cuda.current_stream(self.device)
+        push = torch.cuda.nvtx.range_push if nvtx else (lambda name: None)
+        pop = torch.cuda.nvtx.range_pop if nvtx else (lambda: None)
         if self.has_shared:
             fork = torch.cuda.Event()
             fork.record(main)
             self.side.wait_event(fork)
+            push("shared")
             shared(self.c, x, self.w_shared_up, self.w_shared_down, b.y_shared, b.ws_shared,
                    stream=self.side)
+            pop()
             join = torch.cuda.Event()
             join.record(self.side)
+        push("route")
         route(self.c, x, self.w_router, self.bias, b.topk_idx, b.topk_w, b.ws, stream=main)
+        pop()
+        push("permute")
         permute(self.c, x, b.topk_idx, b.topk_w, b.ws, stream=main)
+        pop()
+        push("forward")
         forward(self.c, T, self.w_up, self.w_down, b.y_acc, b.ws, stream=main)
+        pop()
         if self.has_shared:
             main.wait_event(join)
+        push("finalize")
         finalize(self.c, T, b.y_acc, b.y_shared, b.y, stream=main)
+        pop()
         return b.y
 
     def capture(self, T: int):
