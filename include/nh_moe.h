@@ -138,6 +138,31 @@ nh_status nh_moe_route(const nh_moe_config *cfg, int64_t T, const void *x, const
                        void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * nh_moe_route_noalloc: the router of nh_moe_route for decode-sized batches,
+ * for callers that cannot allocate device memory or pass a workspace (for
+ * example code running under a CUDA graph capture where allocation is not
+ * allowed, serving stacks whose memory pool has already claimed the device,
+ * or plugin hosts that give an op no scratch buffer).  It has no counterpart
+ * on the pages: it is a packaging choice of this library.
+ *   Same arguments and results as nh_moe_route, without ws / ws_bytes.
+ *   Limits: T <= 32 and T * n_routed_experts <= 16384; larger sizes return
+ *   NH_ERR_INVALID_ARG with a message naming the limit (use nh_moe_route).
+ *   Scratch: a fixed 64 KiB + 256 B array compiled into the library, held by
+ *   every device that loads it until the process exits.  Nothing is
+ *   allocated: no cudaMalloc / cudaFree, no allocating library call.
+ *   The first call on a device looks up that array's device address (a
+ *   one-time set-up per device); make that first call before any stream
+ *   capture.  The array is shared by all calls on a device and keeps the last
+ *   call's contents; each call clears its status word and counter first.
+ *   Calls that overlap on the GPU (different streams, no ordering) race on
+ *   that array: order them on one stream.  Device-side status of these calls
+ *   is not reported through nh_moe_check_device.
+ */
+nh_status nh_moe_route_noalloc(const nh_moe_config *cfg, int64_t T, const void *x,
+                               const float *w_router, const float *e_score_correction_bias,
+                               int32_t *topk_idx, float *topk_w, void *stream);
+
+/*
  * Token permute: per-expert histogram, exclusive scan, stable scatter of the
  * (t, j) assignments in (t, j) order, the tile table of the expert GEMMs and
  * the gather x_perm[row] = x[perm_token[row]].  The routed experts are

@@ -22,7 +22,7 @@ import threading
 from . import build as _build
 
 __all__ = ["NHMoEError", "Config", "Layout", "config_from", "load", "validate", "workspace_size",
-           "workspace_layout", "shared_workspace_size", "route", "permute", "forward", "experts_up", "experts_down",
+           "workspace_layout", "shared_workspace_size", "route", "route_noalloc", "permute", "forward", "experts_up", "experts_down",
            "zero", "shared",
            "finalize", "check_device", "selftest_timeout", "library_path", "NemotronHMoE"]
 
@@ -76,8 +76,8 @@ _lock = threading.Lock()
 _lib = None
 
 _EXPORTS = ["nh_moe_validate", "nh_moe_workspace_size", "nh_moe_workspace_layout",
-            "nh_moe_shared_workspace_size", "nh_moe_route", "nh_moe_permute", "nh_moe_forward",
-            "nh_moe_experts_up", "nh_moe_experts_down", "nh_moe_zero",
+            "nh_moe_shared_workspace_size", "nh_moe_route", "nh_moe_route_noalloc",
+            "nh_moe_permute", "nh_moe_forward", "nh_moe_experts_up", "nh_moe_experts_down", "nh_moe_zero",
             "nh_moe_shared", "nh_moe_finalize", "nh_moe_check_device", "nh_moe_selftest_timeout",
             "nh_last_error", "nh_version"]
 
@@ -102,6 +102,7 @@ def load():
             "nh_moe_workspace_layout": [C, I64, ctypes.POINTER(Layout)],
             "nh_moe_shared_workspace_size": [C, I64, ctypes.POINTER(S)],
             "nh_moe_route": [C, I64, P, P, P, P, P, P, S, P],
+            "nh_moe_route_noalloc": [C, I64, P, P, P, P, P, P],
             "nh_moe_permute": [C, I64, P, P, P, P, S, P],
             "nh_moe_forward": [C, I64, P, P, P, P, S, P],
             "nh_moe_experts_up": [C, I64, P, P, S, P],
@@ -178,6 +179,14 @@ def route(cfg, x, w_router, bias, topk_idx, topk_w, ws, stream=None):
     c = config_from(cfg)
     _check(load().nh_moe_route(ctypes.byref(c), x.shape[0], _p(x), _p(w_router), _p(bias),
                                _p(topk_idx), _p(topk_w), _p(ws), _nbytes(ws), _stream(stream)))
+
+
+def route_noalloc(cfg, x, w_router, bias, topk_idx, topk_w, stream=None):
+    """Router of decode-sized batches (T <= 32) without a workspace argument: its
+    scratch is a fixed array inside the library (see nh_moe_route_noalloc)."""
+    c = config_from(cfg)
+    _check(load().nh_moe_route_noalloc(ctypes.byref(c), x.shape[0], _p(x), _p(w_router),
+                                       _p(bias), _p(topk_idx), _p(topk_w), _stream(stream)))
 
 
 def permute(cfg, x, topk_idx, topk_w, ws, stream=None):

@@ -439,6 +439,40 @@ __global__ void selftest_timeout_kernel(int* status, uint64_t timeout_ns) {
   __syncthreads();
 }
 
+// ----------------------------------------------------------------------------
+// Router without caller-provided scratch (nh_moe_route_noalloc).
+//
+// Some callers cannot hand the library a workspace: code that runs while a
+// CUDA graph is being captured with allocations forbidden, serving stacks
+// whose memory pool reserves all of device memory up front, or plugin hosts
+// that give an op no scratch buffer.  For decode-sized batches the router's
+// only scratch is the logits block, a status word and a completion counter,
+// which fit in a fixed array compiled into the library.  Every device that
+// loads the library holds this array until the process exits.
+// ----------------------------------------------------------------------------
+constexpr int64_t NOALLOC_MAX_T = 32;
+constexpr int64_t NOALLOC_MAX_LOGITS = 16384;  // T * E floats (64 KiB)
+constexpr size_t NOALLOC_HEADER = 256;          // status word + completion counter
+static __device__ __align__(256) unsigned char
+    g_noalloc_scratch[NOALLOC_HEADER + NOALLOC_MAX_LOGITS * sizeof(float)];
+static std::once_flag g_noalloc_once[MAX_DEVICES];
+static void* g_noalloc_ptr[MAX_DEVICES];
+static cudaError_t g_noalloc_err[MAX_DEVICES];
+
+// Device address of the static scratch on `dev` (the current device).  The
+// symbol's name in host code is only a host-side stand-in, so the address is
+// looked up once per device with that device current.
+static nh_status noalloc_scratch(int dev, void** out) {
+  std::call_once(g_noalloc_once[dev], [dev] {
+    g_noalloc_err[dev] = cudaGetSymbolAddress(&g_noalloc_ptr[dev], g_noalloc_scratch);
+  });
+  if (g_noalloc_err[dev] != cudaSuccess)
+    return fail(NH_ERR_CUDA, "cudaGetSymbolAddress of the router scratch failed on device %d: %s",
+                dev, cudaGetErrorString(g_noalloc_err[dev]));
+  *out = g_noalloc_ptr[dev];
+  return NH_OK;
+}
+
 static int grid_for(int64_t n, int per_block, int dev) {
   int64_t b = (n + per_block - 1) / per_block;
   const int64_t cap = (int64_t)g_sm_count[dev] * 8;
@@ -568,6 +602,63 @@ nh_status nh_moe_route(const nh_moe_config* cfg, int64_t T, const void* x, const
   }
   router_select<<<(unsigned)((T + 7) / 8), 256, sel_smem, st>>>(a);
   return launch_check("router_select");
+}
+
+nh_status nh_moe_route_noalloc(const nh_moe_config* cfg, int64_t T, const void* x,
+                               const float* w_router, const float* bias, int32_t* topk_idx,
+                               float* topk_w, void* stream) {
+  NH_TRY(validate(cfg));
+  if (T < 0) return fail(NH_ERR_INVALID_ARG, "T must be >= 0");
+  if (T > NOALLOC_MAX_T)
+    return fail(NH_ERR_INVALID_ARG,
+                "nh_moe_route_noalloc takes at most %lld tokens (got %lld); use nh_moe_route",
+                (long long)NOALLOC_MAX_T, (long long)T);
+  if (T * cfg->n_routed_experts > NOALLOC_MAX_LOGITS)
+    return fail(NH_ERR_INVALID_ARG,
+                "nh_moe_route_noalloc: T * n_routed_experts = %lld exceeds its fixed scratch of "
+                "%lld logits; use nh_moe_route",
+                (long long)(T * cfg->n_routed_experts), (long long)NOALLOC_MAX_LOGITS);
+  if (T == 0) return NH_OK;
+  NH_TRY(check_ptr(x, "x"));
+  NH_TRY(check_ptr(w_router, "w_router"));
+  NH_TRY(check_ptr(topk_idx, "topk_idx"));
+  NH_TRY(check_ptr(topk_w, "topk_w"));
+  if (bias) NH_TRY(check_ptr(bias, "e_score_correction_bias"));
+  int dev;
+  NH_TRY(device_setup(&dev));
+  void* scratch;
+  NH_TRY(noalloc_scratch(dev, &scratch));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* status = static_cast<int*>(scratch);
+  float* logits = reinterpret_cast<float*>(static_cast<char*>(scratch) + NOALLOC_HEADER);
+  // the status word and the completion counter must start at zero each call
+  NH_CUDA(cudaMemsetAsync(status, 0, 16, st));
+  SelectArgs a;
+  a.logits = logits;
+  a.bias = bias;
+  a.topk_idx = topk_idx;
+  a.topk_w = topk_w;
+  a.status = status;
+  a.T = (int)T;
+  a.E = cfg->n_routed_experts;
+  a.G = cfg->n_group;
+  a.tg = cfg->topk_group;
+  a.k = cfg->num_experts_per_tok;
+  a.norm = cfg->norm_topk_prob;
+  a.alpha = cfg->routed_scaling_factor;
+  a.group_score = cfg->group_score;
+  a.use_sigma = (bias != nullptr) || cfg->group_score == NH_GROUP_SCORE_TOP2;
+  const size_t sel_smem = (size_t)8 * a.E * sizeof(float);
+  const int warps = (int)(a.E * ((T + 7) / 8));
+  const int blocks = (warps + 7) / 8;
+  unsigned int* done = reinterpret_cast<unsigned int*>(status + 3);
+  if (cfg->dtype == NH_BF16)
+    router_fused_small<__nv_bfloat16><<<blocks, 256, sel_smem, st>>>(
+        static_cast<const __nv_bfloat16*>(x), w_router, a, cfg->hidden_size, done);
+  else
+    router_fused_small<float><<<blocks, 256, sel_smem, st>>>(static_cast<const float*>(x),
+                                                              w_router, a, cfg->hidden_size, done);
+  return launch_check("router_fused_small (no-alloc)");
 }
 
 nh_status nh_moe_permute(const nh_moe_config* cfg, int64_t T, const void* x,
