@@ -305,17 +305,31 @@ def kernel_times(blk, xs, b, nb, steps):
         timed("route", lambda: nh.route(blk.c, x, blk.w_router, blk.bias, b.topk_idx, b.topk_w,
                                          b.ws, stream=main))
         timed("permute", lambda: nh.permute(blk.c, x, b.topk_idx, b.topk_w, b.ws, stream=main))
-        nh.zero(b.y_acc, stream=main)
         timed("experts_up", lambda: nh.experts_up(blk.c, T, blk.w_up, b.ws, stream=main))
-        timed("experts_down", lambda: nh.experts_down(blk.c, T, blk.w_down, b.y_acc, b.ws,
-                                                       stream=main))
-        timed("finalize", lambda: nh.finalize(blk.c, T, b.y_acc, b.y_shared, b.y, stream=main))
+        timed("experts_down", lambda: nh.experts_down(blk.c, T, blk.w_down, b.ws, stream=main))
+        timed("finalize", lambda: nh.finalize(blk.c, T, b.ws, b.y_shared, b.y, stream=main))
         torch.cuda.synchronize(blk.device)
         for n in names:
             if n == "shared" and not blk.has_shared:
                 continue
             acc[n] += ev[n][0].elapsed_time(ev[n][1])
     return {n: acc[n] / steps for n in names}
+
+
+def launches_per_step(cfg):
+    """Kernels of one block call (memsets excluded), as nh_moe.cu launches them."""
+    T = cfg.T
+    if T <= 32:
+        n = 1                                   # fused router
+    elif cfg.dtype == "bf16" and cfg.E % 32 == 0:
+        n = 3                                   # weight split, tensor-core logits, select
+    else:
+        n = 2                                   # logits, select
+    n += 1 if T <= 256 else 4                   # permute (fused, or hist/scan/scatter/gather)
+    n += 2                                      # routed up, routed down
+    n += 2 if cfg.n_shared_experts else 0       # shared up, shared down
+    n += 1                                      # finalize
+    return n
 
 
 def distinct_experts(cfg, idx):
@@ -383,7 +397,7 @@ def report(args, cfg, inp, world, steps, elapsed_ms, clk, kern, e2e_ms, blk):
         "e2e": {"value": round(T / (e2e_ms / 1e3), 2), "unit": "tokens/s",
                 "ms_per_step": round(e2e_ms, 5),
                 "h2d_bytes_per_step": T * cfg.H * elem, "d2h_bytes_per_step": T * cfg.H * elem},
-        "gpu_launches": 11 * steps if cfg.n_shared_experts else 9 * steps,
+        "gpu_launches": launches_per_step(cfg) * steps,
         "clocks": clk,
         "peaks": {"kind": pk_kind, "hbm_gbs": pk["hbm_gbs"], "bf16_tflops": pk["bf16_tflops"],
                   "bf16_tflops_sustained": pk.get("bf16_tflops_sustained")},

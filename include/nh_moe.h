@@ -86,7 +86,7 @@ typedef struct {
 /* Byte offsets of the regions inside the routed-path workspace `ws`. */
 typedef struct {
     size_t total_bytes;
-    size_t status;        /* int32[4]: status word, first bad index, spare      */
+    size_t status;        /* int32[16]: status, site, value, scheduler counters */
     size_t logits;        /* float [T, E] router logits                         */
     size_t router_w;      /* bf16 [E, 3H] router weight as three bf16 planes    */
     size_t counts;        /* int32 [E] assignments per expert                   */
@@ -99,6 +99,7 @@ typedef struct {
     size_t num_tiles;     /* int32 [1] number of valid tile entries             */
     size_t x_perm;        /* dtype [rows_alloc, H] x gathered in permuted order */
     size_t h;             /* dtype [rows_alloc, I] relu^2(up) in permuted order */
+    size_t y_part;        /* dtype [rows_alloc, H] weighted routed partial rows */
     int64_t rows_alloc;   /* T * k rounded up to the tile height                */
     int32_t tile_rows;    /* rows per tile entry of this (cfg, T)               */
     int32_t max_tiles;
@@ -177,28 +178,25 @@ nh_status nh_moe_permute(const nh_moe_config *cfg, int64_t T, const void *x,
 
 /*
  * Routed experts: h = relu(x_perm W_up[e]^T)^2 (float32 accumulate, h stored
- * in dtype), then y_acc[perm_token[r]] += perm_w[r] * (h[r] W_down[e]^T).
- * y_acc is zero-filled first by this call.
- *   w_up [E, I, H] dtype; w_down [E, H, I] dtype; y_acc [T, H] float32 (out).
+ * in dtype), then the weighted partial rows
+ *   y_part[r] = perm_w[r] * (h[r] W_down[e]^T)     (dtype, permuted row order)
+ * which nh_moe_finalize sums per token.  Both live in the workspace.
+ *   w_up [E, I, H] dtype; w_down [E, H, I] dtype.
  * Needs nh_moe_permute's workspace contents.
  */
 nh_status nh_moe_forward(const nh_moe_config *cfg, int64_t T, const void *w_up, const void *w_down,
-                         float *y_acc, void *ws, size_t ws_bytes, void *stream);
+                         void *ws, size_t ws_bytes, void *stream);
 
 /*
  * The two phases of nh_moe_forward, for callers that schedule or time them
  * separately (same arguments and requirements):
  *   nh_moe_experts_up:   h = relu(x_perm W_up[e]^T)^2 into the workspace;
- *   nh_moe_experts_down: y_acc[perm_token[r]] += perm_w[r] * (h[r] W_down[e]^T)
- *                        (accumulates: y_acc must hold the running sum, e.g. zeros).
+ *   nh_moe_experts_down: y_part[r] = perm_w[r] * (h[r] W_down[e]^T).
  */
 nh_status nh_moe_experts_up(const nh_moe_config *cfg, int64_t T, const void *w_up, void *ws,
                             size_t ws_bytes, void *stream);
-nh_status nh_moe_experts_down(const nh_moe_config *cfg, int64_t T, const void *w_down,
-                              float *y_acc, void *ws, size_t ws_bytes, void *stream);
-
-/* Zero-fill n floats of device memory (n >= 0) on `stream`. */
-nh_status nh_moe_zero(float *buf, int64_t n, void *stream);
+nh_status nh_moe_experts_down(const nh_moe_config *cfg, int64_t T, const void *w_down, void *ws,
+                              size_t ws_bytes, void *stream);
 
 /*
  * Shared expert (NemotronHMLP up_proj / down_proj, always on, unscaled):
@@ -212,10 +210,12 @@ nh_status nh_moe_shared(const nh_moe_config *cfg, int64_t T, const void *x, cons
                         size_t ws_shared_bytes, void *stream);
 
 /*
- * y = dtype(y_acc + y_shared) (y_shared may be NULL when there is no shared
- * expert).  y [T, H] dtype.
+ * y[t] = dtype( y_shared[t] + sum_j y_part[inv_row[t, j]] ), summed in float32
+ * in that order (deterministic; no atomics anywhere on the path).
+ *   ws: the routed workspace after nh_moe_forward; y_shared [T, H] float32
+ *   (NULL when the config has no shared expert); y [T, H] dtype (out).
  */
-nh_status nh_moe_finalize(const nh_moe_config *cfg, int64_t T, const float *y_acc,
+nh_status nh_moe_finalize(const nh_moe_config *cfg, int64_t T, const void *ws, size_t ws_bytes,
                           const float *y_shared, void *y, void *stream);
 
 /*

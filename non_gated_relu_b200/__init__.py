@@ -22,8 +22,7 @@ import threading
 from . import build as _build
 
 __all__ = ["NHMoEError", "Config", "Layout", "config_from", "load", "validate", "workspace_size",
-           "workspace_layout", "shared_workspace_size", "route", "route_noalloc", "permute", "forward", "experts_up", "experts_down",
-           "zero", "shared",
+           "workspace_layout", "shared_workspace_size", "route", "route_noalloc", "permute", "forward", "experts_up", "experts_down", "shared",
            "finalize", "check_device", "selftest_timeout", "library_path", "NemotronHMoE"]
 
 NH_OK, NH_ERR_INVALID_ARG, NH_ERR_UNSUPPORTED, NH_ERR_CUDA, NH_ERR_TIMEOUT, NH_ERR_DEVICE_CHECK = range(6)
@@ -53,7 +52,7 @@ class Layout(ctypes.Structure):
     """nh_moe_ws_layout: byte offsets of the routed-path workspace regions."""
     _fields_ = [(n, ctypes.c_size_t) for n in (
         "total_bytes", "status", "logits", "router_w", "counts", "offsets", "chunk_counts", "perm_token",
-        "perm_w", "inv_row", "tiles", "num_tiles", "x_perm", "h")] + [
+        "perm_w", "inv_row", "tiles", "num_tiles", "x_perm", "h", "y_part")] + [
         ("rows_alloc", ctypes.c_int64), ("tile_rows", ctypes.c_int32),
         ("max_tiles", ctypes.c_int32), ("n_chunks", ctypes.c_int32), ("swap_ab", ctypes.c_int32)]
 
@@ -77,7 +76,7 @@ _lib = None
 
 _EXPORTS = ["nh_moe_validate", "nh_moe_workspace_size", "nh_moe_workspace_layout",
             "nh_moe_shared_workspace_size", "nh_moe_route", "nh_moe_route_noalloc",
-            "nh_moe_permute", "nh_moe_forward", "nh_moe_experts_up", "nh_moe_experts_down", "nh_moe_zero",
+            "nh_moe_permute", "nh_moe_forward", "nh_moe_experts_up", "nh_moe_experts_down",
             "nh_moe_shared", "nh_moe_finalize", "nh_moe_check_device", "nh_moe_selftest_timeout",
             "nh_last_error", "nh_version"]
 
@@ -104,12 +103,11 @@ def load():
             "nh_moe_route": [C, I64, P, P, P, P, P, P, S, P],
             "nh_moe_route_noalloc": [C, I64, P, P, P, P, P, P],
             "nh_moe_permute": [C, I64, P, P, P, P, S, P],
-            "nh_moe_forward": [C, I64, P, P, P, P, S, P],
+            "nh_moe_forward": [C, I64, P, P, P, S, P],
             "nh_moe_experts_up": [C, I64, P, P, S, P],
-            "nh_moe_experts_down": [C, I64, P, P, P, S, P],
-            "nh_moe_zero": [P, I64, P],
+            "nh_moe_experts_down": [C, I64, P, P, S, P],
             "nh_moe_shared": [C, I64, P, P, P, P, P, S, P],
-            "nh_moe_finalize": [C, I64, P, P, P, P],
+            "nh_moe_finalize": [C, I64, P, S, P, P, P],
             "nh_moe_check_device": [P, P],
             "nh_moe_selftest_timeout": [P, ctypes.c_uint64, P],
         }
@@ -195,10 +193,10 @@ def permute(cfg, x, topk_idx, topk_w, ws, stream=None):
                                  _p(ws), _nbytes(ws), _stream(stream)))
 
 
-def forward(cfg, T: int, w_up, w_down, y_acc, ws, stream=None):
+def forward(cfg, T: int, w_up, w_down, ws, stream=None):
     c = config_from(cfg)
-    _check(load().nh_moe_forward(ctypes.byref(c), T, _p(w_up), _p(w_down), _p(y_acc), _p(ws),
-                                 _nbytes(ws), _stream(stream)))
+    _check(load().nh_moe_forward(ctypes.byref(c), T, _p(w_up), _p(w_down), _p(ws), _nbytes(ws),
+                                 _stream(stream)))
 
 
 def experts_up(cfg, T: int, w_up, ws, stream=None):
@@ -207,14 +205,10 @@ def experts_up(cfg, T: int, w_up, ws, stream=None):
                                     _stream(stream)))
 
 
-def experts_down(cfg, T: int, w_down, y_acc, ws, stream=None):
+def experts_down(cfg, T: int, w_down, ws, stream=None):
     c = config_from(cfg)
-    _check(load().nh_moe_experts_down(ctypes.byref(c), T, _p(w_down), _p(y_acc), _p(ws),
-                                      _nbytes(ws), _stream(stream)))
-
-
-def zero(buf, stream=None):
-    _check(load().nh_moe_zero(_p(buf), buf.numel(), _stream(stream)))
+    _check(load().nh_moe_experts_down(ctypes.byref(c), T, _p(w_down), _p(ws), _nbytes(ws),
+                                      _stream(stream)))
 
 
 def shared(cfg, x, w_shared_up, w_shared_down, y_shared, ws_shared, stream=None):
@@ -224,9 +218,9 @@ def shared(cfg, x, w_shared_up, w_shared_down, y_shared, ws_shared, stream=None)
                                 _nbytes(ws_shared), _stream(stream)))
 
 
-def finalize(cfg, T: int, y_acc, y_shared, y, stream=None):
+def finalize(cfg, T: int, ws, y_shared, y, stream=None):
     c = config_from(cfg)
-    _check(load().nh_moe_finalize(ctypes.byref(c), T, _p(y_acc), _p(y_shared), _p(y),
+    _check(load().nh_moe_finalize(ctypes.byref(c), T, _p(ws), _nbytes(ws), _p(y_shared), _p(y),
                                   _stream(stream)))
 
 

@@ -44,7 +44,6 @@ class Buffers:
     ws_shared: Optional[torch.Tensor]
     topk_idx: torch.Tensor
     topk_w: torch.Tensor
-    y_acc: torch.Tensor
     y_shared: Optional[torch.Tensor]
     y: torch.Tensor
 
@@ -97,8 +96,7 @@ class NemotronHMoE:
                 ys = torch.empty((T, self.H), dtype=torch.float32, device=dev)
             b = Buffers(T, ws, wss,
                         torch.empty((T, self.k), dtype=torch.int32, device=dev),
-                        torch.empty((T, self.k), dtype=torch.float32, device=dev),
-                        torch.empty((T, self.H), dtype=torch.float32, device=dev), ys,
+                        torch.empty((T, self.k), dtype=torch.float32, device=dev), ys,
                         torch.empty((T, self.H), dtype=self.dtype, device=dev))
             self._bufs[T] = b
         return b
@@ -130,12 +128,12 @@ class NemotronHMoE:
         permute(self.c, x, b.topk_idx, b.topk_w, b.ws, stream=main)
         pop()
         push("forward")
-        forward(self.c, T, self.w_up, self.w_down, b.y_acc, b.ws, stream=main)
+        forward(self.c, T, self.w_up, self.w_down, b.ws, stream=main)
         pop()
         if self.has_shared:
             main.wait_event(join)
         push("finalize")
-        finalize(self.c, T, b.y_acc, b.y_shared, b.y, stream=main)
+        finalize(self.c, T, b.ws, b.y_shared, b.y, stream=main)
         pop()
         return b.y
 

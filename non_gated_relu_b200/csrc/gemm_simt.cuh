@@ -11,7 +11,7 @@ namespace nh {
 
 enum Epilogue : int {
   EPI_UP_RELU2 = 0,      // out (dtype) [rows, N] = relu(acc)^2
-  EPI_DOWN_SCATTER = 1,  // y_acc[perm_token[r], n] += perm_w[r] * acc  (float32 atomics)
+  EPI_DOWN_WEIGHTED = 1, // out (dtype) [rows, N] = perm_w[r] * acc   (routed partial rows)
   EPI_STORE_F32 = 2,     // out (float32) [rows, N] = acc
 };
 
@@ -26,7 +26,6 @@ struct GemmArgs {
   int epi;
   void* out;
   int64_t ldo;            // row stride of out, elements
-  const int32_t* perm_token;
   const float* perm_w;
 };
 
@@ -94,8 +93,8 @@ __global__ void __launch_bounds__(256) simt_grouped_gemm(GemmArgs g) {
       const float v = acc[i][j];
       if (g.epi == EPI_UP_RELU2) {
         static_cast<Tin*>(g.out)[(size_t)r * g.ldo + n] = from_f32<Tin>(relu2(v));
-      } else if (g.epi == EPI_DOWN_SCATTER) {
-        atomicAdd(static_cast<float*>(g.out) + (size_t)g.perm_token[r] * g.ldo + n, g.perm_w[r] * v);
+      } else if (g.epi == EPI_DOWN_WEIGHTED) {
+        static_cast<Tin*>(g.out)[(size_t)r * g.ldo + n] = from_f32<Tin>(g.perm_w[r] * v);
       } else {
         static_cast<float*>(g.out)[(size_t)r * g.ldo + n] = v;
       }

@@ -7,7 +7,8 @@
 // and a fused epilogue turns it into
 //   up_proj:   h = relu(D)^2 stored in bf16              (non-gated expert,
 //              "up_proj -> relu^2 -> down_proj", vllm.cpp PR #518)
-//   down_proj: y_acc[token] += routing weight * D          (weighted combine)
+//   down_proj: y_part[row] = routing weight * D in bf16     (per-(token, expert)
+//              partial rows, summed per token by the finalize kernel)
 //   shared:    y_shared = D                                 (always-on expert)
 //
 // Two orientations:
@@ -47,11 +48,13 @@ struct TcArgs {
   int epi;                    // Epilogue
   void* out;
   int64_t ldo;                // row stride of out, elements
-  const int32_t* perm_token;
   const float* perm_w;
   int* status;
   uint64_t timeout_ns;
+  unsigned int* sched;        // [2]: next tile, CTAs finished; zero on entry, reset on exit
 };
+
+constexpr int TQ = 4;         // depth of the tile-id ring between the roles
 
 template <bool SWAP, int NT, int STAGES>
 struct Shape {
@@ -63,7 +66,7 @@ struct Shape {
   static constexpr int ACC_COLS = NT;
   static constexpr int TMEM_COLS = (2 * NT < 32) ? 32 : 2 * NT;
   static_assert((TMEM_COLS & (TMEM_COLS - 1)) == 0 && TMEM_COLS <= 512, "TMEM alloc");
-  static constexpr int BAR_BYTES = (2 * STAGES + 5) * 8 + 16;
+  static constexpr int BAR_BYTES = (2 * STAGES + 5 + 2 * TQ) * 8 + 16 + 4 * TQ;
   static constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + BAR_BYTES;
 };
 
@@ -87,29 +90,26 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, uint64
 
 // epilogue of 32 consecutive output features of one row (prefill orientation)
 __device__ __forceinline__ void epi_row32(const TcArgs& g, int r, int n, const float* v) {
-  if (g.epi == EPI_UP_RELU2) {
-    uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) + (size_t)r * g.ldo + n);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      uint4 p;
-      p.x = pack_bf16x2(relu2(v[8 * i + 0]), relu2(v[8 * i + 1]));
-      p.y = pack_bf16x2(relu2(v[8 * i + 2]), relu2(v[8 * i + 3]));
-      p.z = pack_bf16x2(relu2(v[8 * i + 4]), relu2(v[8 * i + 5]));
-      p.w = pack_bf16x2(relu2(v[8 * i + 6]), relu2(v[8 * i + 7]));
-      dst[i] = p;
-    }
-  } else if (g.epi == EPI_DOWN_SCATTER) {
-    const float w = g.perm_w[r];
-    float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.out) +
-                                            (size_t)g.perm_token[r] * g.ldo + n);
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      atomicAdd(dst + i, make_float4(w * v[4 * i], w * v[4 * i + 1], w * v[4 * i + 2],
-                                     w * v[4 * i + 3]));
-  } else {
+  if (g.epi == EPI_STORE_F32) {
     float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.out) + (size_t)r * g.ldo + n);
 #pragma unroll
     for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    return;
+  }
+  const bool up = g.epi == EPI_UP_RELU2;
+  const float w = up ? 1.f : g.perm_w[r];
+  float o[32];
+#pragma unroll
+  for (int i = 0; i < 32; ++i) o[i] = up ? relu2(v[i]) : w * v[i];
+  uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) + (size_t)r * g.ldo + n);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint4 p;
+    p.x = pack_bf16x2(o[8 * i + 0], o[8 * i + 1]);
+    p.y = pack_bf16x2(o[8 * i + 2], o[8 * i + 3]);
+    p.z = pack_bf16x2(o[8 * i + 4], o[8 * i + 5]);
+    p.w = pack_bf16x2(o[8 * i + 6], o[8 * i + 7]);
+    dst[i] = p;
   }
 }
 
@@ -117,8 +117,8 @@ __device__ __forceinline__ void epi_row32(const TcArgs& g, int r, int n, const f
 __device__ __forceinline__ void epi_elem(const TcArgs& g, int r, int f, float v) {
   if (g.epi == EPI_UP_RELU2) {
     static_cast<__nv_bfloat16*>(g.out)[(size_t)r * g.ldo + f] = __float2bfloat16_rn(relu2(v));
-  } else if (g.epi == EPI_DOWN_SCATTER) {
-    atomicAdd(static_cast<float*>(g.out) + (size_t)g.perm_token[r] * g.ldo + f, g.perm_w[r] * v);
+  } else if (g.epi == EPI_DOWN_WEIGHTED) {
+    static_cast<__nv_bfloat16*>(g.out)[(size_t)r * g.ldo + f] = __float2bfloat16_rn(g.perm_w[r] * v);
   } else {
     static_cast<float*>(g.out)[(size_t)r * g.ldo + f] = v;
   }
@@ -139,9 +139,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   auto tfull_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + a); };
   auto tempty_bar = [&](int a) { return bar0 + 8u * (2 * STAGES + 2 + a); };
   const uint32_t drain_bar = bar0 + 8u * (2 * STAGES + 4);
-  uint32_t* const tmem_slot =
-      reinterpret_cast<uint32_t*>(base_ptr + STAGES * S::STAGE_BYTES + (2 * STAGES + 5) * 8);
+  auto tq_full_bar = [&](int i) { return bar0 + 8u * (2 * STAGES + 5 + i); };
+  auto tq_empty_bar = [&](int i) { return bar0 + 8u * (2 * STAGES + 5 + TQ + i); };
+  uint32_t* const tmem_slot = reinterpret_cast<uint32_t*>(base_ptr + STAGES * S::STAGE_BYTES +
+                                                          (2 * STAGES + 5 + 2 * TQ) * 8);
   volatile int* const abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* const tile_q = reinterpret_cast<volatile int*>(tmem_slot + 4);
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   if (threadIdx.x == 0) {
@@ -154,6 +157,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_init(tempty_bar(a), 128);
     }
     mbar_init(drain_bar, 1);
+    for (int i = 0; i < TQ; ++i) {
+      mbar_init(tq_full_bar(i), 1);
+      mbar_init(tq_empty_bar(i), 1 + 4);   // MMA issuer + one lane per epilogue warp
+    }
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_map(&map_act);
@@ -175,12 +182,22 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int nk = g.K / BK;
 
   if (warp == 0 && lane == 0) {
-    // ---------------- TMA producer ----------------
+    // ---------------- TMA producer + tile scheduler ----------------
     int stage = 0;
     uint32_t phase = 0;
     long issued = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+    for (int i = 0; ok; ++i) {
+      const int q = i % TQ;
+      if (!mbar_wait(tq_empty_bar(q), ((i / TQ) & 1) ^ 1u, wc, SITE_TC_PRODUCER)) {
+        ok = false;
+        break;
+      }
+      int tile = (int)atomicAdd(g.sched, 1u);
+      if (tile >= total) tile = -1;
+      tile_q[q] = tile;
+      mbar_arrive(tq_full_bar(q));
+      if (tile < 0) break;
       const int m = tile / n_blocks, nb = tile - m * n_blocks;
       const int4 ent = tile_entry_of(g, m);
       for (int kb = 0; kb < nk; ++kb) {
@@ -218,7 +235,15 @@ __global__ void __launch_bounds__(THREADS, 1)
     uint32_t phase = 0;
     int it = 0;
     bool ok = true, any = false;
-    for (int tile = blockIdx.x; tile < total && ok; tile += gridDim.x) {
+    for (int i = 0; ok; ++i) {
+      const int q = i % TQ;
+      if (!mbar_wait(tq_full_bar(q), (i / TQ) & 1, wc, SITE_TC_MMA)) {
+        ok = false;
+        break;
+      }
+      const int tile = tile_q[q];
+      mbar_arrive(tq_empty_bar(q));
+      if (tile < 0) break;
       const int m = tile / n_blocks, nb = tile - m * n_blocks;
       const int acc = it & 1;
       const uint32_t aph = (uint32_t)((it >> 1) & 1);
@@ -263,11 +288,23 @@ __global__ void __launch_bounds__(THREADS, 1)
     // ---------------- epilogue: 4 warps, one TMEM lane quarter each ----------------
     const int q = warp & 3;
     int it = 0;
-    for (int tile = blockIdx.x; tile < total; tile += gridDim.x) {
+    for (int i = 0;; ++i) {
+      int tile = -1;
+      int ok = 1;
+      if (lane == 0) {
+        const int slot = i % TQ;
+        ok = mbar_wait(tq_full_bar(slot), (i / TQ) & 1, wc, SITE_TC_EPILOGUE) ? 1 : 0;
+        if (ok) {
+          tile = tile_q[slot];
+          mbar_arrive(tq_empty_bar(slot));
+        }
+      }
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      tile = __shfl_sync(0xffffffffu, tile, 0);
+      if (!ok || tile < 0) break;
       const int m = tile / n_blocks, nb = tile - m * n_blocks;
       const int acc = it & 1;
       const uint32_t aph = (uint32_t)((it >> 1) & 1);
-      int ok = 1;
       if (lane == 0) ok = mbar_wait(tfull_bar(acc), aph, wc, SITE_TC_EPILOGUE) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
@@ -306,6 +343,14 @@ __global__ void __launch_bounds__(THREADS, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, S::TMEM_COLS);
+  }
+  if (threadIdx.x == 0) {
+    // the last CTA to finish resets the scheduler for the next launch
+    __threadfence();
+    if (atomicAdd(g.sched + 1, 1u) == gridDim.x - 1) {
+      atomicExch(g.sched, 0u);
+      atomicExch(g.sched + 1, 0u);
+    }
   }
 }
 

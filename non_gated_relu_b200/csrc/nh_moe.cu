@@ -62,6 +62,12 @@ constexpr int MAX_E = 512;
 constexpr int MAX_G = 64;
 constexpr int MAX_K = 32;
 constexpr size_t ALIGN = 256;
+// status region of a workspace: int32[16]
+//   [0..2] status code, site, value   [3] router completion counter
+//   [4..5] router GEMM tile scheduler  [6..7] up GEMM  [8..9] down GEMM
+// (shared workspace: [4..5] shared up GEMM, [6..7] shared down GEMM)
+constexpr size_t STATUS_BYTES = 64;
+constexpr int SCHED_ROUTER = 4, SCHED_UP = 6, SCHED_DOWN = 8;
 
 static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -166,7 +172,7 @@ static nh_status make_plan(const nh_moe_config* c, int64_t T, Plan* p) {
     o = align_up(o + (bytes ? bytes : 1), ALIGN);
     return at;
   };
-  L.status = take(16);
+  L.status = take(STATUS_BYTES);
   L.logits = take((size_t)T * p->E * 4);
   L.router_w = take(p->bf16 ? (size_t)p->E * 3 * p->H * 2 : 0);
   L.counts = take((size_t)p->E * 4);
@@ -179,6 +185,7 @@ static nh_status make_plan(const nh_moe_config* c, int64_t T, Plan* p) {
   L.num_tiles = take(4);
   L.x_perm = take((size_t)rows * p->H * p->elem);
   L.h = take((size_t)rows * p->I * p->elem);
+  L.y_part = take((size_t)rows * p->H * p->elem);
   L.total_bytes = o;
   return NH_OK;
 }
@@ -319,9 +326,9 @@ struct GemmCall {
   int epi;
   void* out;
   int64_t ldo;
-  const int32_t* perm_token;
   const float* perm_w;
   int* status;
+  unsigned int* sched;  // tile scheduler counters (tensor-core path)
 };
 
 template <bool SWAP, int NT, int STAGES>
@@ -341,10 +348,11 @@ static nh_status launch_tc(const GemmCall& c, int dev, cudaStream_t st) {
   g.epi = c.epi;
   g.out = c.out;
   g.ldo = c.ldo;
-  g.perm_token = c.perm_token;
   g.perm_w = c.perm_w;
   g.status = c.status;
   g.timeout_ns = timeout_ns();
+  g.sched = c.sched;
+  if (!g.sched) return fail(NH_ERR_INVALID_ARG, "internal: no tile scheduler counters");
   const int n_blocks = SWAP ? (c.N + tc::M - 1) / tc::M : (c.N + NT - 1) / NT;
   const int64_t m_max = c.tiles ? c.max_tiles : (c.rows + c.tile_rows - 1) / c.tile_rows;
   const int64_t work = m_max * n_blocks;
@@ -369,7 +377,6 @@ static nh_status run_gemm(const Plan& p, const GemmCall& c, int dev, cudaStream_
     g.epi = c.epi;
     g.out = c.out;
     g.ldo = c.ldo;
-    g.perm_token = c.perm_token;
     g.perm_w = c.perm_w;
     const int64_t m_max = c.tiles ? c.max_tiles : (c.rows + c.tile_rows - 1) / c.tile_rows;
     if (m_max > 65535) return fail(NH_ERR_UNSUPPORTED, "float32 path: too many row tiles");
@@ -389,36 +396,58 @@ static nh_status run_gemm(const Plan& p, const GemmCall& c, int dev, cudaStream_
 // ----------------------------------------------------------------------------
 // small kernels
 // ----------------------------------------------------------------------------
-__global__ void zero_f32(float4* __restrict__ p, int64_t n4) {
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4;
-       i += (int64_t)gridDim.x * blockDim.x)
-    p[i] = make_float4(0.f, 0.f, 0.f, 0.f);
-}
-
-template <typename Tout>
-__global__ void finalize_kernel(const float* __restrict__ y_acc, const float* __restrict__ y_sh,
-                                Tout* __restrict__ y, int64_t n) {
+// y[t] = y_shared[t] + sum_j y_part[inv_row[t, j]], summed in fp32 in that
+// order (deterministic), rounded once to the output dtype.
+template <typename Tio>
+__global__ void finalize_gather(const Tio* __restrict__ y_part, const int32_t* __restrict__ inv_row,
+                                const float* __restrict__ y_sh, Tio* __restrict__ y, int64_t T,
+                                int k, int H) {
+  const int64_t n = T * H;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {
-    float v = y_acc[i];
-    if (y_sh) v += y_sh[i];
-    y[i] = from_f32<Tout>(v);
+    const int64_t t = i / H;
+    const int h = (int)(i - t * H);
+    float v = y_sh ? y_sh[i] : 0.f;
+    for (int j = 0; j < k; ++j) {
+      const int r = inv_row[t * k + j];
+      if (r >= 0) v += to_f32(y_part[(size_t)r * H + h]);
+    }
+    y[i] = from_f32<Tio>(v);
   }
 }
 
-__global__ void finalize_bf16_vec(const float4* __restrict__ y_acc, const float4* __restrict__ y_sh,
-                                  uint2* __restrict__ y, int64_t n4) {
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n4;
+// bf16, eight consecutive features per thread (16-byte loads and stores)
+__global__ void finalize_gather_bf16x8(const uint4* __restrict__ y_part,
+                                       const int32_t* __restrict__ inv_row,
+                                       const float4* __restrict__ y_sh, uint4* __restrict__ y,
+                                       int64_t T, int k, int H8) {
+  const int64_t n = T * H8;
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {
-    float4 a = y_acc[i];
+    const int64_t t = i / H8;
+    const int c = (int)(i - t * H8);
+    float a[8];
     if (y_sh) {
-      const float4 b = y_sh[i];
-      a.x += b.x;
-      a.y += b.y;
-      a.z += b.z;
-      a.w += b.w;
+      const float4 s0 = y_sh[2 * i], s1 = y_sh[2 * i + 1];
+      a[0] = s0.x; a[1] = s0.y; a[2] = s0.z; a[3] = s0.w;
+      a[4] = s1.x; a[5] = s1.y; a[6] = s1.z; a[7] = s1.w;
+    } else {
+#pragma unroll
+      for (int q = 0; q < 8; ++q) a[q] = 0.f;
     }
-    y[i] = make_uint2(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w));
+    for (int j = 0; j < k; ++j) {
+      const int r = inv_row[t * k + j];
+      if (r < 0) continue;
+      const uint4 u = y_part[(size_t)r * H8 + c];
+      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        a[2 * q] += __uint_as_float(w[q] << 16);
+        a[2 * q + 1] += __uint_as_float(w[q] & 0xffff0000u);
+      }
+    }
+    y[i] = make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]), pack_bf16x2(a[4], a[5]),
+                      pack_bf16x2(a[6], a[7]));
   }
 }
 
@@ -537,7 +566,7 @@ nh_status nh_moe_route(const nh_moe_config* cfg, int64_t T, const void* x, const
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int* status = at<int>(ws, p.lay.status);
   float* logits = at<float>(ws, p.lay.logits);
-  NH_CUDA(cudaMemsetAsync(status, 0, 16, st));
+  NH_CUDA(cudaMemsetAsync(status, 0, STATUS_BYTES, st));
   SelectArgs a;
   a.logits = logits;
   a.bias = bias;
@@ -556,8 +585,7 @@ nh_status nh_moe_route(const nh_moe_config* cfg, int64_t T, const void* x, const
   const size_t sel_smem = (size_t)8 * p.E * sizeof(float);
   if (T <= 32) {
     // decode: logits and selection in one launch (last block selects)
-    const int warps = (int)(p.E * ((T + 7) / 8));
-    const int blocks = (warps + 7) / 8;
+    const int blocks = p.E;
     unsigned int* done = reinterpret_cast<unsigned int*>(status + 3);
     if (p.bf16)
       router_fused_small<__nv_bfloat16><<<blocks, 256, sel_smem, st>>>(
@@ -589,6 +617,7 @@ nh_status nh_moe_route(const nh_moe_config* cfg, int64_t T, const void* x, const
     c.out = logits;
     c.ldo = p.E;
     c.status = status;
+    c.sched = reinterpret_cast<unsigned int*>(status + SCHED_ROUTER);
     NH_TRY((launch_tc<false, 256, 4>(c, dev, st)));
   } else {
     dim3 grid((unsigned)((T + RT_BT - 1) / RT_BT), (unsigned)((p.E + RT_BE - 1) / RT_BE));
@@ -632,7 +661,7 @@ nh_status nh_moe_route_noalloc(const nh_moe_config* cfg, int64_t T, const void* 
   int* status = static_cast<int*>(scratch);
   float* logits = reinterpret_cast<float*>(static_cast<char*>(scratch) + NOALLOC_HEADER);
   // the status word and the completion counter must start at zero each call
-  NH_CUDA(cudaMemsetAsync(status, 0, 16, st));
+  NH_CUDA(cudaMemsetAsync(status, 0, STATUS_BYTES, st));
   SelectArgs a;
   a.logits = logits;
   a.bias = bias;
@@ -649,8 +678,7 @@ nh_status nh_moe_route_noalloc(const nh_moe_config* cfg, int64_t T, const void* 
   a.group_score = cfg->group_score;
   a.use_sigma = (bias != nullptr) || cfg->group_score == NH_GROUP_SCORE_TOP2;
   const size_t sel_smem = (size_t)8 * a.E * sizeof(float);
-  const int warps = (int)(a.E * ((T + 7) / 8));
-  const int blocks = (warps + 7) / 8;
+  const int blocks = a.E;
   unsigned int* done = reinterpret_cast<unsigned int*>(status + 3);
   if (cfg->dtype == NH_BF16)
     router_fused_small<__nv_bfloat16><<<blocks, 256, sel_smem, st>>>(
@@ -688,13 +716,14 @@ nh_status nh_moe_permute(const nh_moe_config* cfg, int64_t T, const void* x,
           L.tile_rows, L.max_tiles, at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets),
           at<int4>(ws, L.tiles), at<int32_t>(ws, L.num_tiles), at<int32_t>(ws, L.perm_token),
           at<float>(ws, L.perm_w), at<int32_t>(ws, L.inv_row), at<__nv_bfloat16>(ws, L.x_perm),
-          status);
+          status, reinterpret_cast<unsigned int*>(status + SCHED_UP));
     else
       permute_small<float><<<1, 512, smem, st>>>(
           topk_idx, topk_w, static_cast<const float*>(x), (int)T, p.k, p.E, p.H, L.tile_rows,
           L.max_tiles, at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets),
           at<int4>(ws, L.tiles), at<int32_t>(ws, L.num_tiles), at<int32_t>(ws, L.perm_token),
-          at<float>(ws, L.perm_w), at<int32_t>(ws, L.inv_row), at<float>(ws, L.x_perm), status);
+          at<float>(ws, L.perm_w), at<int32_t>(ws, L.inv_row), at<float>(ws, L.x_perm), status,
+          reinterpret_cast<unsigned int*>(status + SCHED_UP));
     return launch_check("permute_small");
   }
   int32_t* chunk = at<int32_t>(ws, L.chunk_counts);
@@ -704,7 +733,8 @@ nh_status nh_moe_permute(const nh_moe_config* cfg, int64_t T, const void* x,
   permute_scan<<<1, scan_threads, 0, st>>>(chunk, L.n_chunks, p.E, L.tile_rows,
                                             at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets),
                                             at<int4>(ws, L.tiles), at<int32_t>(ws, L.num_tiles),
-                                            L.max_tiles);
+                                            L.max_tiles,
+                                            reinterpret_cast<unsigned int*>(status + SCHED_UP));
   NH_TRY(launch_check("permute_scan"));
   const size_t smem = (size_t)(p.E + PERM_CHUNK * p.k) * sizeof(int);
   const int gather_blocks = g_sm_count[dev] * 4;
@@ -730,14 +760,13 @@ nh_status nh_moe_permute(const nh_moe_config* cfg, int64_t T, const void* x,
   return launch_check("permute_gather");
 }
 
-static nh_status experts_phase(const nh_moe_config* cfg, int64_t T, const void* w, float* y_acc,
-                               void* ws, size_t ws_bytes, void* stream, bool up_phase) {
+static nh_status experts_phase(const nh_moe_config* cfg, int64_t T, const void* w, void* ws,
+                               size_t ws_bytes, void* stream, bool up_phase) {
   Plan p;
   NH_TRY(make_plan(cfg, T, &p));
   NH_TRY(check_ws(p, ws, ws_bytes));
   if (T == 0) return NH_OK;
   NH_TRY(check_ptr(w, up_phase ? "w_up" : "w_down"));
-  if (!up_phase) NH_TRY(check_ptr(y_acc, "y_acc"));
   int dev;
   NH_TRY(device_setup(&dev));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -751,9 +780,10 @@ static nh_status experts_phase(const nh_moe_config* cfg, int64_t T, const void* 
   c.tile_rows = L.tile_rows;
   c.swap = L.swap_ab;
   c.status = at<int>(ws, L.status);
+  c.sched = reinterpret_cast<unsigned int*>(c.status + (up_phase ? SCHED_UP : SCHED_DOWN));
+  c.W = w;
   if (up_phase) {
     c.A = at<void>(ws, L.x_perm);
-    c.W = w;
     c.N = p.I;
     c.K = p.H;
     c.epi = EPI_UP_RELU2;
@@ -761,13 +791,11 @@ static nh_status experts_phase(const nh_moe_config* cfg, int64_t T, const void* 
     c.ldo = p.I;
   } else {
     c.A = at<void>(ws, L.h);
-    c.W = w;
     c.N = p.H;
     c.K = p.I;
-    c.epi = EPI_DOWN_SCATTER;
-    c.out = y_acc;
+    c.epi = EPI_DOWN_WEIGHTED;
+    c.out = at<void>(ws, L.y_part);
     c.ldo = p.H;
-    c.perm_token = at<int32_t>(ws, L.perm_token);
     c.perm_w = at<float>(ws, L.perm_w);
   }
   return run_gemm(p, c, dev, st);
@@ -775,41 +803,24 @@ static nh_status experts_phase(const nh_moe_config* cfg, int64_t T, const void* 
 
 nh_status nh_moe_experts_up(const nh_moe_config* cfg, int64_t T, const void* w_up, void* ws,
                             size_t ws_bytes, void* stream) {
-  return experts_phase(cfg, T, w_up, nullptr, ws, ws_bytes, stream, true);
+  return experts_phase(cfg, T, w_up, ws, ws_bytes, stream, true);
 }
 
-nh_status nh_moe_experts_down(const nh_moe_config* cfg, int64_t T, const void* w_down,
-                              float* y_acc, void* ws, size_t ws_bytes, void* stream) {
-  return experts_phase(cfg, T, w_down, y_acc, ws, ws_bytes, stream, false);
-}
-
-nh_status nh_moe_zero(float* buf, int64_t n, void* stream) {
-  if (n < 0) return fail(NH_ERR_INVALID_ARG, "n must be >= 0");
-  if (n == 0) return NH_OK;
-  NH_TRY(check_ptr(buf, "buf"));
-  int dev;
-  NH_TRY(device_setup(&dev));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  if (n % 4 == 0) {
-    zero_f32<<<grid_for(n / 4, 256, dev), 256, 0, st>>>(reinterpret_cast<float4*>(buf), n / 4);
-    return launch_check("zero_f32");
-  }
-  NH_CUDA(cudaMemsetAsync(buf, 0, (size_t)n * 4, st));
-  return NH_OK;
+nh_status nh_moe_experts_down(const nh_moe_config* cfg, int64_t T, const void* w_down, void* ws,
+                              size_t ws_bytes, void* stream) {
+  return experts_phase(cfg, T, w_down, ws, ws_bytes, stream, false);
 }
 
 nh_status nh_moe_forward(const nh_moe_config* cfg, int64_t T, const void* w_up, const void* w_down,
-                         float* y_acc, void* ws, size_t ws_bytes, void* stream) {
+                         void* ws, size_t ws_bytes, void* stream) {
   Plan p;
   NH_TRY(make_plan(cfg, T, &p));
   NH_TRY(check_ws(p, ws, ws_bytes));
   if (T == 0) return NH_OK;
   NH_TRY(check_ptr(w_up, "w_up"));
   NH_TRY(check_ptr(w_down, "w_down"));
-  NH_TRY(check_ptr(y_acc, "y_acc"));
-  NH_TRY(nh_moe_zero(y_acc, T * p.H, stream));
   NH_TRY(nh_moe_experts_up(cfg, T, w_up, ws, ws_bytes, stream));
-  return nh_moe_experts_down(cfg, T, w_down, y_acc, ws, ws_bytes, stream);
+  return nh_moe_experts_down(cfg, T, w_down, ws, ws_bytes, stream);
 }
 
 nh_status nh_moe_shared(const nh_moe_config* cfg, int64_t T, const void* x, const void* w_su,
@@ -832,7 +843,7 @@ nh_status nh_moe_shared(const nh_moe_config* cfg, int64_t T, const void* x, cons
   cudaStream_t st = static_cast<cudaStream_t>(stream);
   int* status = static_cast<int*>(ws_shared);
   void* h = static_cast<char*>(ws_shared) + ALIGN;
-  NH_CUDA(cudaMemsetAsync(status, 0, 16, st));
+  NH_CUDA(cudaMemsetAsync(status, 0, STATUS_BYTES, st));
   GemmCall up{};
   up.A = x;
   up.rows = T;
@@ -847,6 +858,7 @@ nh_status nh_moe_shared(const nh_moe_config* cfg, int64_t T, const void* x, cons
   up.out = h;
   up.ldo = p.S;
   up.status = status;
+  up.sched = reinterpret_cast<unsigned int*>(status + 4);
   NH_TRY(run_gemm(p, up, dev, st));
   GemmCall dn = up;
   dn.A = h;
@@ -856,15 +868,16 @@ nh_status nh_moe_shared(const nh_moe_config* cfg, int64_t T, const void* x, cons
   dn.epi = EPI_STORE_F32;
   dn.out = y_shared;
   dn.ldo = p.H;
+  dn.sched = reinterpret_cast<unsigned int*>(status + 6);
   return run_gemm(p, dn, dev, st);
 }
 
-nh_status nh_moe_finalize(const nh_moe_config* cfg, int64_t T, const float* y_acc,
+nh_status nh_moe_finalize(const nh_moe_config* cfg, int64_t T, const void* ws, size_t ws_bytes,
                           const float* y_shared, void* y, void* stream) {
   Plan p;
   NH_TRY(make_plan(cfg, T, &p));
+  NH_TRY(check_ws(p, const_cast<void*>(ws), ws_bytes));
   if (T == 0) return NH_OK;
-  NH_TRY(check_ptr(y_acc, "y_acc"));
   NH_TRY(check_ptr(y, "y"));
   if (y_shared) NH_TRY(check_ptr(y_shared, "y_shared"));
   if (cfg->n_shared_experts && !y_shared)
@@ -872,17 +885,21 @@ nh_status nh_moe_finalize(const nh_moe_config* cfg, int64_t T, const float* y_ac
   int dev;
   NH_TRY(device_setup(&dev));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const int64_t n = T * p.H;
-  if (p.bf16 && n % 4 == 0) {
-    finalize_bf16_vec<<<grid_for(n / 4, 256, dev), 256, 0, st>>>(
-        reinterpret_cast<const float4*>(y_acc), reinterpret_cast<const float4*>(y_shared),
-        static_cast<uint2*>(y), n / 4);
+  const nh_moe_ws_layout& L = p.lay;
+  void* ws_nc = const_cast<void*>(ws);
+  const int32_t* inv = at<int32_t>(ws_nc, L.inv_row);
+  if (p.bf16 && p.H % 8 == 0) {
+    const int H8 = p.H / 8;
+    finalize_gather_bf16x8<<<grid_for(T * H8, 256, dev), 256, 0, st>>>(
+        at<uint4>(ws_nc, L.y_part), inv, reinterpret_cast<const float4*>(y_shared),
+        static_cast<uint4*>(y), T, p.k, H8);
   } else if (p.bf16) {
-    finalize_kernel<__nv_bfloat16><<<grid_for(n, 256, dev), 256, 0, st>>>(
-        y_acc, y_shared, static_cast<__nv_bfloat16*>(y), n);
+    finalize_gather<__nv_bfloat16><<<grid_for(T * p.H, 256, dev), 256, 0, st>>>(
+        at<__nv_bfloat16>(ws_nc, L.y_part), inv, y_shared, static_cast<__nv_bfloat16*>(y), T, p.k,
+        p.H);
   } else {
-    finalize_kernel<float><<<grid_for(n, 256, dev), 256, 0, st>>>(y_acc, y_shared,
-                                                                   static_cast<float*>(y), n);
+    finalize_gather<float><<<grid_for(T * p.H, 256, dev), 256, 0, st>>>(
+        at<float>(ws_nc, L.y_part), inv, y_shared, static_cast<float*>(y), T, p.k, p.H);
   }
   return launch_check("finalize");
 }

@@ -75,8 +75,10 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* smem_warp, int* 
 __global__ void permute_scan(int32_t* __restrict__ chunk_counts, int n_chunks, int E,
                              int tile_rows, int32_t* __restrict__ counts,
                              int32_t* __restrict__ offsets, int4* __restrict__ tiles,
-                             int32_t* __restrict__ num_tiles, int max_tiles) {
+                             int32_t* __restrict__ num_tiles, int max_tiles,
+                             unsigned int* sched_zero) {
   __shared__ int warp_sums[33];
+  if (threadIdx.x < 4) sched_zero[threadIdx.x] = 0u;  // up/down GEMM tile schedulers
   const int e = threadIdx.x;
   int total = 0;
   if (e < E)
@@ -213,9 +215,10 @@ __global__ void __launch_bounds__(512) permute_small(
     int T, int k, int E, int H, int tile_rows, int max_tiles, int32_t* __restrict__ counts,
     int32_t* __restrict__ offsets, int4* __restrict__ tiles, int32_t* __restrict__ num_tiles,
     int32_t* __restrict__ perm_token, float* __restrict__ perm_w, int32_t* __restrict__ inv_row,
-    Tin* __restrict__ x_perm, int* status) {
+    Tin* __restrict__ x_perm, int* status, unsigned int* sched_zero) {
   extern __shared__ int sm[];
   __shared__ int warp_sums[33];
+  if (threadIdx.x < 4) sched_zero[threadIdx.x] = 0u;  // up/down GEMM tile schedulers
   int* cnt = sm;
   int* pos = sm + E;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;

@@ -232,42 +232,69 @@ __global__ void __launch_bounds__(256) router_select(SelectArgs a) {
   select_token(a, t, a.logits + (size_t)t * a.E, sel_smem + (size_t)warp * a.E, lane);
 }
 
-// Decode-sized T (<= 32): logits by one warp per (expert, 8-token block), then
-// the last block to finish selects every token.  `done` is a zeroed counter
-// in the workspace; the last block resets it for the next call.
+// x[t, h .. h+3] as floats (h a multiple of 4, rows 8-byte aligned for bf16)
+__device__ __forceinline__ float4 load4(const __nv_bfloat16* p) {
+  const uint2 u = *reinterpret_cast<const uint2*>(p);
+  return make_float4(__uint_as_float(u.x << 16), __uint_as_float(u.x & 0xffff0000u),
+                     __uint_as_float(u.y << 16), __uint_as_float(u.y & 0xffff0000u));
+}
+__device__ __forceinline__ float4 load4(const float* p) {
+  return *reinterpret_cast<const float4*>(p);
+}
+
+// Decode-sized T (<= 32): block e computes expert e's logits for every token
+// (its 256 threads split H four elements at a time, then reduce), and the
+// last block to finish selects every token.  `done` is a counter that is
+// zero on entry; the last block resets it.
 template <typename Tin>
 __global__ void __launch_bounds__(256) router_fused_small(const Tin* __restrict__ x,
                                                           const float* __restrict__ wr,
                                                           SelectArgs a, int H,
                                                           unsigned int* done) {
   extern __shared__ float sel_smem[];
+  __shared__ float red[8][32];
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
   const int T = a.T, E = a.E;
-  const int warp = blockIdx.x * 8 + wib;
-  const int tblocks = (T + 7) >> 3;
-  const int e = warp / tblocks, tb = warp - e * tblocks;
+  const int e = blockIdx.x;
   float* logits = const_cast<float*>(a.logits);
-  if (e < E) {
-    const int t0 = tb * 8, nt = min(8, T - t0);
-    float acc[8];
+  float acc[32];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-    const float* w = wr + (size_t)e * H;
-    const Tin* xb = x + (size_t)t0 * H;
-#pragma unroll 4
-    for (int h = lane; h < H; h += 32) {
-      const float wv = __ldg(w + h);
+  for (int t = 0; t < 32; ++t) acc[t] = 0.f;
+  const float* w = wr + (size_t)e * H;
+  if ((H & 3) == 0) {
+    for (int h = threadIdx.x * 4; h < H; h += 1024) {
+      const float4 wv = __ldg(reinterpret_cast<const float4*>(w + h));
 #pragma unroll
-      for (int i = 0; i < 8; ++i)
-        if (i < nt) acc[i] = fmaf(to_f32(xb[(size_t)i * H + h]), wv, acc[i]);
+      for (int t = 0; t < 32; ++t) {
+        if (t < T) {
+          const float4 xv = load4(x + (size_t)t * H + h);
+          acc[t] = fmaf(xv.x, wv.x, fmaf(xv.y, wv.y, fmaf(xv.z, wv.z, fmaf(xv.w, wv.w, acc[t]))));
+        }
+      }
     }
+  } else {
+    for (int h = threadIdx.x; h < H; h += 256) {
+      const float wv = w[h];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-      float v = acc[i];
+      for (int t = 0; t < 32; ++t)
+        if (t < T) acc[t] = fmaf(to_f32(x[(size_t)t * H + h]), wv, acc[t]);
+    }
+  }
+#pragma unroll
+  for (int t = 0; t < 32; ++t) {
+    if (t < T) {
+      float v = acc[t];
 #pragma unroll
       for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0 && i < nt) logits[(size_t)(t0 + i) * E + e] = v;
+      if (lane == 0) red[wib][t] = v;
     }
+  }
+  __syncthreads();
+  if (wib == 0 && lane < T) {
+    float v = 0.f;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) v += red[i][lane];
+    logits[(size_t)lane * E + e] = v;
   }
   // last-block-done: the block that finishes last sees every logit
   __shared__ unsigned int ticket;
