@@ -14,6 +14,7 @@
 #include "common.cuh"
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
+#include "gemm_tc2.cuh"
 #include "permute.cuh"
 #include "route.cuh"
 
@@ -136,7 +137,7 @@ static void tile_plan(const nh_moe_config* c, int64_t T, int* tile_rows, int* sw
     *tile_rows = 64;
     *swap = 1;
   } else {
-    *tile_rows = tc::M;
+    *tile_rows = tc2::MP;   // 256-row tiles computed by CTA pairs
     *swap = 0;
   }
 }
@@ -217,6 +218,7 @@ static T* at(void* ws, size_t off) {
 constexpr int MAX_DEVICES = 64;
 static std::once_flag g_attr_once[MAX_DEVICES];
 static int g_sm_count[MAX_DEVICES];
+static int g_pair_clusters[MAX_DEVICES];  // co-resident 2-CTA clusters of tc2_grouped_gemm
 static nh_status g_attr_status[MAX_DEVICES];
 
 using TcPrefill = tc::Shape<false, 256, 4>;
@@ -239,6 +241,25 @@ static nh_status set_attrs(int dev) {
                                cudaFuncAttributeMaxDynamicSharedMemorySize, TcSwap32::SMEM));
   NH_CUDA(cudaFuncSetAttribute(tc::tc_grouped_gemm<true, 64, 6>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, TcSwap64::SMEM));
+  NH_CUDA(cudaFuncSetAttribute(tc2::tc2_grouped_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               tc2::SMEM));
+  {
+    cudaLaunchConfig_t lc = {};
+    lc.gridDim = dim3(2 * (prop.multiProcessorCount / 2), 1, 1);
+    lc.blockDim = dim3(tc2::THREADS, 1, 1);
+    lc.dynamicSmemBytes = tc2::SMEM;
+    cudaLaunchAttribute at[1];
+    at[0].id = cudaLaunchAttributeClusterDimension;
+    at[0].val.clusterDim.x = 2;
+    at[0].val.clusterDim.y = 1;
+    at[0].val.clusterDim.z = 1;
+    lc.attrs = at;
+    lc.numAttrs = 1;
+    int n = 0;
+    NH_CUDA(cudaOccupancyMaxActiveClusters(&n, tc2::tc2_grouped_gemm, &lc));
+    if (n < 1) return fail(NH_ERR_UNSUPPORTED, "no 2-CTA cluster of the pair GEMM fits on device %d", dev);
+    g_pair_clusters[dev] = n;
+  }
   return NH_OK;
 }
 
@@ -362,6 +383,49 @@ static nh_status launch_tc(const GemmCall& c, int dev, cudaStream_t st) {
   return launch_check("tc_grouped_gemm");
 }
 
+// prefill orientation on CTA pairs: 256-row tiles, each CTA stages 128 rows of
+// the activations and half of the weight rows
+static nh_status launch_tc2(const GemmCall& c, int dev, cudaStream_t st) {
+  CUtensorMap ma, mw;
+  NH_TRY(map_2d(&ma, c.A, c.a_kwrap ? c.a_kwrap : c.K, c.rows, tc2::HALF));
+  NH_TRY(map_3d(&mw, c.W, c.K, c.N, c.n_exp, tc2::HALF));
+  tc::TcArgs g;
+  g.tiles = c.tiles;
+  g.num_tiles = c.num_tiles;
+  g.dense_rows = (int)c.rows;
+  g.tile_rows = c.tile_rows;
+  g.N = c.N;
+  g.K = c.K;
+  g.a_kwrap = c.a_kwrap;
+  g.epi = c.epi;
+  g.out = c.out;
+  g.ldo = c.ldo;
+  g.perm_w = c.perm_w;
+  g.status = c.status;
+  g.timeout_ns = timeout_ns();
+  g.sched = c.sched;
+  if (!g.sched) return fail(NH_ERR_INVALID_ARG, "internal: no tile scheduler counters");
+  if (c.tile_rows != tc2::MP) return fail(NH_ERR_INVALID_ARG, "internal: pair tiles are 256 rows");
+  const int n_blocks = (c.N + tc2::NT - 1) / tc2::NT;
+  const int64_t m_max = c.tiles ? c.max_tiles : (c.rows + c.tile_rows - 1) / c.tile_rows;
+  const int64_t pairs = std::min<int64_t>(m_max * n_blocks, g_pair_clusters[dev]);
+  if (pairs <= 0) return NH_OK;
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = dim3((unsigned)(2 * pairs), 1, 1);
+  lc.blockDim = dim3(tc2::THREADS, 1, 1);
+  lc.dynamicSmemBytes = tc2::SMEM;
+  lc.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeClusterDimension;
+  at[0].val.clusterDim.x = 2;
+  at[0].val.clusterDim.y = 1;
+  at[0].val.clusterDim.z = 1;
+  lc.attrs = at;
+  lc.numAttrs = 1;
+  NH_CUDA(cudaLaunchKernelEx(&lc, tc2::tc2_grouped_gemm, ma, mw, g));
+  return launch_check("tc2_grouped_gemm");
+}
+
 static nh_status run_gemm(const Plan& p, const GemmCall& c, int dev, cudaStream_t st) {
   if (c.rows == 0) return NH_OK;
   if (!p.bf16) {
@@ -384,7 +448,7 @@ static nh_status run_gemm(const Plan& p, const GemmCall& c, int dev, cudaStream_
     simt_grouped_gemm<float><<<grid, 256, 0, st>>>(g);
     return launch_check("simt_grouped_gemm");
   }
-  if (!c.swap) return launch_tc<false, 256, 4>(c, dev, st);
+  if (!c.swap) return launch_tc2(c, dev, st);
   switch (c.tile_rows) {
     case 16: return launch_tc<true, 16, 8>(c, dev, st);
     case 32: return launch_tc<true, 32, 8>(c, dev, st);

@@ -91,7 +91,7 @@ def test_workspace_layout(name):
     elif T <= 64:
         assert L.swap_ab == 1 and L.tile_rows >= T and L.tile_rows % 16 == 0
     else:
-        assert L.swap_ab == 0 and L.tile_rows == 128
+        assert L.swap_ab == 0 and L.tile_rows == 256     # CTA-pair tiles
     assert L.max_tiles >= -(-rows // L.tile_rows) + cfg.E - 1
 
 
