@@ -9,6 +9,12 @@
 // this halves the B operand that has to be staged and read for the same
 // number of MMA cycles, which is what limits the one-CTA 128 x 256 tile.
 //
+// An expert's last, partial tile (fewer than 256 rows) is computed swapped:
+// 256 weight rows (128 per CTA) on the MMA M side and the remaining token rows
+// (rounded up to 16) on N, so the tensor cores do not multiply padding rows.
+// Both tile kinds use the same tensor maps and the same accumulator layout;
+// only the operand roles, the MMA shape and the epilogue's indexing change.
+//
 // Roles per CTA (192 threads), as in the one-CTA kernel:
 //   warp 0 lane 0  TMA producer (both CTAs; the leader also runs the tile
 //                  scheduler and forwards each tile id to the peer);
@@ -31,7 +37,7 @@ constexpr int UMMA_K = 16;
 constexpr int MP = 256;       // tile rows (MMA M across the pair)
 constexpr int NT = 256;       // tile features (MMA N)
 constexpr int HALF = 128;     // rows of A and of B staged per CTA
-constexpr int STAGES = 6;
+constexpr int STAGES = 7;
 constexpr int THREADS = 192;
 constexpr int A_BYTES = HALF * BK * 2;
 constexpr int B_BYTES = HALF * BK * 2;
@@ -41,6 +47,17 @@ constexpr int TQ = 4;
 constexpr int NBAR = 2 * STAGES + 5 + 2 * TQ;
 constexpr int SMEM = STAGES * STAGE_BYTES + 1024 + NBAR * 8 + 16 + 4 * TQ;
 static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
+
+// MMA N of a swapped remainder tile of `rows` token rows
+__device__ __forceinline__ int swap_n(int rows) { return (rows + 15) & ~15; }
+
+// tile entry (expert, first row, rows, kind); kind 1 = swapped remainder tile
+__device__ __forceinline__ int4 pair_entry(const tc::TcArgs& g, int m) {
+  if (g.tiles) return g.tiles[m];
+  const int r0 = m * g.tile_rows;
+  const int rows = min(g.tile_rows, g.dense_rows - r0);
+  return make_int4(0, r0, rows, rows < g.tile_rows ? 1 : 0);
+}
 
 __global__ void __launch_bounds__(THREADS, 1)
     tc2_grouped_gemm(const __grid_constant__ CUtensorMap map_act,
@@ -130,11 +147,17 @@ __global__ void __launch_bounds__(THREADS, 1)
       }
       if (tile < 0) break;
       const int m = tile / n_blocks, nb = tile - m * n_blocks;
-      const int4 ent = tc::tile_entry_of(g, m);
+      const int4 ent = pair_entry(g, m);
       const int n0 = nb * NT;
-      const int half_n = min(NT, g.N - n0) / 2;
-      const int a_row = ent.y + (int)rank * HALF;
-      const int b_row = n0 + (int)rank * half_n;
+      // operand rows staged by this CTA: slot A (M side) and slot B (N side)
+      int a_row, b_row;
+      if (ent.w == 0) {                                     // activations x weights
+        a_row = ent.y + (int)rank * HALF;
+        b_row = n0 + (int)rank * (min(NT, g.N - n0) / 2);
+      } else {                                              // weights x remainder rows
+        a_row = n0 + (int)rank * HALF;
+        b_row = ent.y + (int)rank * (swap_n(ent.z) / 2);
+      }
       for (int kb = 0; kb < nk; ++kb) {
         if (!mbar_wait_cluster(empty_bar(stage), phase ^ 1u, wc, SITE_TC_PRODUCER)) {
           ok = false;
@@ -144,8 +167,13 @@ __global__ void __launch_bounds__(THREADS, 1)
         const uint32_t fb = map_to_rank(full_bar(stage), 0);
         const int ka = g.a_kwrap ? (kb * BK) % g.a_kwrap : kb * BK;
         if (leader) mbar_arrive_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
-        tma_load_2d_pair(sa, &map_act, fb, ka, a_row);
-        tma_load_3d_pair(sb, &map_w, fb, kb * BK, b_row, ent.x);
+        if (ent.w == 0) {
+          tma_load_2d_pair(sa, &map_act, fb, ka, a_row);
+          tma_load_3d_pair(sb, &map_w, fb, kb * BK, b_row, ent.x);
+        } else {
+          tma_load_3d_pair(sa, &map_w, fb, kb * BK, a_row, ent.x);
+          tma_load_2d_pair(sb, &map_act, fb, ka, b_row);
+        }
         ++issued;
         if (++stage == STAGES) {
           stage = 0;
@@ -176,6 +204,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       mbar_arrive(tq_empty_bar(q));
       if (tile < 0) break;
       const int nb = tile % n_blocks;
+      const int4 ent = pair_entry(g, tile / n_blocks);
       const int acc = it & 1;
       const uint32_t aph = (uint32_t)((it >> 1) & 1);
       if (!mbar_wait_cluster(tempty_bar(acc), aph ^ 1u, wc, SITE_TC_MMA)) {
@@ -183,7 +212,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         break;
       }
       tc_fence_after();
-      const int n_mma = min(NT, g.N - nb * NT);
+      const int n_mma = ent.w == 0 ? min(NT, g.N - nb * NT) : swap_n(ent.z);
       const uint32_t idesc = make_idesc_bf16(MP, n_mma);
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * NT);
       for (int kb = 0; kb < nk; ++kb) {
@@ -243,16 +272,31 @@ __global__ void __launch_bounds__(THREADS, 1)
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      const int4 ent = tc::tile_entry_of(g, m);
-      const int row = (int)rank * HALF + qw * 32 + lane;
-      const bool valid = row < ent.z;
+      const int4 ent = pair_entry(g, m);
       const int n0 = nb * NT;
-      const int n_eff = min(NT, g.N - n0);
       const uint32_t tq = tmem_base + ((uint32_t)(qw * 32) << 16) + (uint32_t)(acc * NT);
-      for (int c = 0; c < n_eff; c += 32) {
-        float v[32];
-        tmem_ld_x32(tq + (uint32_t)c, v);
-        if (valid) tc::epi_row32(g, ent.y + row, n0 + c, v);
+      if (ent.w == 0) {
+        // accumulator lane = token row, column = output feature
+        const int row = (int)rank * HALF + qw * 32 + lane;
+        const bool valid = row < ent.z;
+        const int n_eff = min(NT, g.N - n0);
+        for (int c = 0; c < n_eff; c += 32) {
+          float v[32];
+          tmem_ld_x32(tq + (uint32_t)c, v);
+          if (valid) tc::epi_row32(g, ent.y + row, n0 + c, v);
+        }
+      } else {
+        // accumulator lane = output feature, column = token row of the remainder
+        const int f = n0 + (int)rank * HALF + qw * 32 + lane;
+        const bool valid = f < g.N;
+        const int n_mma = swap_n(ent.z);
+        for (int c = 0; c < n_mma; c += 16) {
+          float v[16];
+          tmem_ld_x16(tq + (uint32_t)c, v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (valid && c + j < ent.z) tc::epi_elem(g, ent.y + c + j, f, v[j]);
+        }
       }
       tc_fence_before();
       __syncwarp();

@@ -14,6 +14,13 @@
 namespace nh {
 
 constexpr int PERM_CHUNK = 256;  // tokens per histogram chunk
+constexpr int PAIR_TILE_ROWS = 256;
+
+// kind of a tile entry: 1 marks the partial last tile of an expert in the
+// CTA-pair GEMM (256-row tiles), which that GEMM computes swapped
+__device__ __forceinline__ int tile_kind(int rows, int tile_rows) {
+  return (tile_rows == PAIR_TILE_ROWS && rows < tile_rows) ? 1 : 0;
+}
 
 // per-chunk expert histogram: chunk_counts[c][e]
 __global__ void __launch_bounds__(256) permute_hist(const int32_t* __restrict__ idx, int T, int k,
@@ -99,7 +106,8 @@ __global__ void permute_scan(int32_t* __restrict__ chunk_counts, int n_chunks, i
     }
     for (int i = 0; i < nt && toff + i < max_tiles; ++i) {
       const int r0 = i * tile_rows;
-      tiles[toff + i] = make_int4(e, off + r0, min(tile_rows, total - r0), 0);
+      const int rows = min(tile_rows, total - r0);
+      tiles[toff + i] = make_int4(e, off + r0, rows, tile_kind(rows, tile_rows));
     }
   }
   if (e == 0) {
@@ -243,8 +251,10 @@ __global__ void __launch_bounds__(512) permute_small(
   if (e < E) {
     counts[e] = total;
     offsets[e] = off;
-    for (int i = 0; i < nt && toff + i < max_tiles; ++i)
-      tiles[toff + i] = make_int4(e, off + i * tile_rows, min(tile_rows, total - i * tile_rows), 0);
+    for (int i = 0; i < nt && toff + i < max_tiles; ++i) {
+      const int rows = min(tile_rows, total - i * tile_rows);
+      tiles[toff + i] = make_int4(e, off + i * tile_rows, rows, tile_kind(rows, tile_rows));
+    }
     cnt[e] = off;  // running position for the ranking
   }
   if (e == 0) {
