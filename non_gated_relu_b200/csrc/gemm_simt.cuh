@@ -47,6 +47,8 @@ template <typename Tin>
 __global__ void __launch_bounds__(256) simt_grouped_gemm(GemmArgs g) {
   __shared__ __align__(16) float As[SG_BK][SG_PAD];
   __shared__ __align__(16) float Bs[SG_BK][SG_PAD];
+  pdl_wait();
+  pdl_trigger();
   int4 ent;
   if (!tile_entry(g, blockIdx.y, ent)) return;
   const int e = ent.x, r0 = ent.y, nrows = ent.z;

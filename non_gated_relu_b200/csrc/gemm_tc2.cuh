@@ -109,6 +109,9 @@ __global__ void __launch_bounds__(THREADS, 1)
   cluster_sync_all();   // peers' barriers are initialised before any remote arrive
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  // everything above overlaps the previous kernel; inputs are read from here on
+  pdl_wait();
+  pdl_trigger();
   const WaitCtl wc{abort_flag, g.status, g.timeout_ns};
 
   const int num_m = g.tiles ? *g.num_tiles : (g.dense_rows + g.tile_rows - 1) / g.tile_rows;

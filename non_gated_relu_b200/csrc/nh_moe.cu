@@ -283,6 +283,28 @@ static uint64_t timeout_ns() {
   return v;
 }
 
+// Launch with programmatic dependent launch allowed: the kernel may start its
+// prologue while the previous kernel in the stream finishes; every kernel of
+// this library executes griddepcontrol.wait before it reads its inputs.
+template <typename Kern, typename... Args>
+static nh_status launch_k(const char* what, Kern kernel, dim3 grid, dim3 block, size_t smem,
+                          cudaStream_t st, Args... args) {
+  cudaLaunchConfig_t lc = {};
+  lc.gridDim = grid;
+  lc.blockDim = block;
+  lc.dynamicSmemBytes = smem;
+  lc.stream = st;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  lc.attrs = at;
+  lc.numAttrs = 1;
+  const cudaError_t e = cudaLaunchKernelEx(&lc, kernel, args...);
+  if (e != cudaSuccess)
+    return fail(NH_ERR_CUDA, "launch of %s failed: %s", what, cudaGetErrorString(e));
+  return NH_OK;
+}
+
 // ----------------------------------------------------------------------------
 // TMA tensor maps (driver entry point fetched through the runtime)
 // ----------------------------------------------------------------------------
@@ -379,7 +401,7 @@ static nh_status launch_tc(const GemmCall& c, int dev, cudaStream_t st) {
   const int64_t work = m_max * n_blocks;
   const int grid = (int)std::min<int64_t>(work, g_sm_count[dev]);
   if (grid <= 0) return NH_OK;
-  tc::tc_grouped_gemm<SWAP, NT, STAGES><<<grid, tc::THREADS, S::SMEM, st>>>(ma, mw, g);
+  NH_TRY((launch_k("tc_grouped_gemm", tc::tc_grouped_gemm<SWAP, NT, STAGES>, dim3(grid), dim3(tc::THREADS), S::SMEM, st, ma, mw, g)));
   return launch_check("tc_grouped_gemm");
 }
 
@@ -415,13 +437,15 @@ static nh_status launch_tc2(const GemmCall& c, int dev, cudaStream_t st) {
   lc.blockDim = dim3(tc2::THREADS, 1, 1);
   lc.dynamicSmemBytes = tc2::SMEM;
   lc.stream = st;
-  cudaLaunchAttribute at[1];
+  cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = 2;
   at[0].val.clusterDim.y = 1;
   at[0].val.clusterDim.z = 1;
+  at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[1].val.programmaticStreamSerializationAllowed = 1;
   lc.attrs = at;
-  lc.numAttrs = 1;
+  lc.numAttrs = 2;
   NH_CUDA(cudaLaunchKernelEx(&lc, tc2::tc2_grouped_gemm, ma, mw, g));
   return launch_check("tc2_grouped_gemm");
 }
@@ -445,7 +469,7 @@ static nh_status run_gemm(const Plan& p, const GemmCall& c, int dev, cudaStream_
     const int64_t m_max = c.tiles ? c.max_tiles : (c.rows + c.tile_rows - 1) / c.tile_rows;
     if (m_max > 65535) return fail(NH_ERR_UNSUPPORTED, "float32 path: too many row tiles");
     dim3 grid((c.N + SG_BN - 1) / SG_BN, (unsigned)m_max);
-    simt_grouped_gemm<float><<<grid, 256, 0, st>>>(g);
+    NH_TRY((launch_k("simt_grouped_gemm", simt_grouped_gemm<float>, dim3(grid), dim3(256), 0, st, g)));
     return launch_check("simt_grouped_gemm");
   }
   if (!c.swap) return launch_tc2(c, dev, st);
@@ -466,6 +490,8 @@ template <typename Tio>
 __global__ void finalize_gather(const Tio* __restrict__ y_part, const int32_t* __restrict__ inv_row,
                                 const float* __restrict__ y_sh, Tio* __restrict__ y, int64_t T,
                                 int k, int H) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t n = T * H;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -485,6 +511,8 @@ __global__ void finalize_gather_bf16x8(const uint4* __restrict__ y_part,
                                        const int32_t* __restrict__ inv_row,
                                        const float4* __restrict__ y_sh, uint4* __restrict__ y,
                                        int64_t T, int k, int H8) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t n = T * H8;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {
@@ -652,19 +680,19 @@ nh_status nh_moe_route(const nh_moe_config* cfg, int64_t T, const void* x, const
     const int blocks = p.E;
     unsigned int* done = reinterpret_cast<unsigned int*>(status + 3);
     if (p.bf16)
-      router_fused_small<__nv_bfloat16><<<blocks, 256, sel_smem, st>>>(
-          static_cast<const __nv_bfloat16*>(x), w_router, a, p.H, done);
+      NH_TRY((launch_k("router_fused_small", router_fused_small<__nv_bfloat16>, dim3(blocks), dim3(256), sel_smem, st, 
+          static_cast<const __nv_bfloat16*>(x), w_router, a, p.H, done)));
     else
-      router_fused_small<float><<<blocks, 256, sel_smem, st>>>(static_cast<const float*>(x),
-                                                                w_router, a, p.H, done);
+      NH_TRY((launch_k("router_fused_small", router_fused_small<float>, dim3(blocks), dim3(256), sel_smem, st, static_cast<const float*>(x),
+                                                                w_router, a, p.H, done)));
     return launch_check("router_fused_small");
   }
   if (p.bf16 && p.E % 32 == 0) {
     // logits on the tensor cores: x (bf16) against the fp32 router weight split
     // into three bf16 planes, accumulated over K = 3H in fp32
     __nv_bfloat16* wsplit = at<__nv_bfloat16>(ws, p.lay.router_w);
-    router_split<<<grid_for((int64_t)p.E * p.H, 256, dev), 256, 0, st>>>(w_router, wsplit, p.E,
-                                                                          p.H);
+    NH_TRY((launch_k("router_split", router_split, dim3(grid_for((int64_t)p.E * p.H, 256, dev)), dim3(256), 0, st, w_router, wsplit, p.E,
+                                                                          p.H)));
     NH_TRY(launch_check("router_split"));
     GemmCall c{};
     c.A = x;
@@ -686,14 +714,14 @@ nh_status nh_moe_route(const nh_moe_config* cfg, int64_t T, const void* x, const
   } else {
     dim3 grid((unsigned)((T + RT_BT - 1) / RT_BT), (unsigned)((p.E + RT_BE - 1) / RT_BE));
     if (p.bf16)
-      router_logits_tiled<__nv_bfloat16><<<grid, 256, 0, st>>>(
-          static_cast<const __nv_bfloat16*>(x), w_router, logits, (int)T, p.H, p.E);
+      NH_TRY((launch_k("router_logits_tiled", router_logits_tiled<__nv_bfloat16>, dim3(grid), dim3(256), 0, st, 
+          static_cast<const __nv_bfloat16*>(x), w_router, logits, (int)T, p.H, p.E)));
     else
-      router_logits_tiled<float><<<grid, 256, 0, st>>>(static_cast<const float*>(x), w_router,
-                                                       logits, (int)T, p.H, p.E);
+      NH_TRY((launch_k("router_logits_tiled", router_logits_tiled<float>, dim3(grid), dim3(256), 0, st, static_cast<const float*>(x), w_router,
+                                                       logits, (int)T, p.H, p.E)));
     NH_TRY(launch_check("router_logits_tiled"));
   }
-  router_select<<<(unsigned)((T + 7) / 8), 256, sel_smem, st>>>(a);
+  NH_TRY((launch_k("router_select", router_select, dim3((unsigned)((T + 7) / 8)), dim3(256), sel_smem, st, a)));
   return launch_check("router_select");
 }
 
@@ -775,51 +803,51 @@ nh_status nh_moe_permute(const nh_moe_config* cfg, int64_t T, const void* x,
     // decode-sized: the whole permute in one block
     const size_t smem = (size_t)(p.E + T * p.k) * sizeof(int);
     if (p.bf16)
-      permute_small<__nv_bfloat16><<<1, 512, smem, st>>>(
+      NH_TRY((launch_k("permute_small", permute_small<__nv_bfloat16>, dim3(1), dim3(512), smem, st, 
           topk_idx, topk_w, static_cast<const __nv_bfloat16*>(x), (int)T, p.k, p.E, p.H,
           L.tile_rows, L.max_tiles, at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets),
           at<int4>(ws, L.tiles), at<int32_t>(ws, L.num_tiles), at<int32_t>(ws, L.perm_token),
           at<float>(ws, L.perm_w), at<int32_t>(ws, L.inv_row), at<__nv_bfloat16>(ws, L.x_perm),
-          status, reinterpret_cast<unsigned int*>(status + SCHED_UP));
+          status, reinterpret_cast<unsigned int*>(status + SCHED_UP))));
     else
-      permute_small<float><<<1, 512, smem, st>>>(
+      NH_TRY((launch_k("permute_small", permute_small<float>, dim3(1), dim3(512), smem, st, 
           topk_idx, topk_w, static_cast<const float*>(x), (int)T, p.k, p.E, p.H, L.tile_rows,
           L.max_tiles, at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets),
           at<int4>(ws, L.tiles), at<int32_t>(ws, L.num_tiles), at<int32_t>(ws, L.perm_token),
           at<float>(ws, L.perm_w), at<int32_t>(ws, L.inv_row), at<float>(ws, L.x_perm), status,
-          reinterpret_cast<unsigned int*>(status + SCHED_UP));
+          reinterpret_cast<unsigned int*>(status + SCHED_UP))));
     return launch_check("permute_small");
   }
   int32_t* chunk = at<int32_t>(ws, L.chunk_counts);
-  permute_hist<<<L.n_chunks, 256, p.E * sizeof(int), st>>>(topk_idx, (int)T, p.k, p.E, chunk, status);
+  NH_TRY((launch_k("permute_hist", permute_hist, dim3(L.n_chunks), dim3(256), p.E * sizeof(int), st, topk_idx, (int)T, p.k, p.E, chunk, status)));
   NH_TRY(launch_check("permute_hist"));
   const int scan_threads = ((p.E + 31) / 32) * 32;
-  permute_scan<<<1, scan_threads, 0, st>>>(chunk, L.n_chunks, p.E, L.tile_rows,
+  NH_TRY((launch_k("permute_scan", permute_scan, dim3(1), dim3(scan_threads), 0, st, chunk, L.n_chunks, p.E, L.tile_rows,
                                             at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets),
                                             at<int4>(ws, L.tiles), at<int32_t>(ws, L.num_tiles),
                                             L.max_tiles,
-                                            reinterpret_cast<unsigned int*>(status + SCHED_UP));
+                                            reinterpret_cast<unsigned int*>(status + SCHED_UP))));
   NH_TRY(launch_check("permute_scan"));
   const size_t smem = (size_t)(p.E + PERM_CHUNK * p.k) * sizeof(int);
   const int gather_blocks = g_sm_count[dev] * 4;
   if (p.bf16) {
-    permute_scatter<__nv_bfloat16><<<L.n_chunks, 32, smem, st>>>(
+    NH_TRY((launch_k("permute_scatter", permute_scatter<__nv_bfloat16>, dim3(L.n_chunks), dim3(32), smem, st, 
         topk_idx, topk_w, static_cast<const __nv_bfloat16*>(x), (int)T, p.k, p.E, p.H, chunk,
         at<int32_t>(ws, L.perm_token), at<float>(ws, L.perm_w), at<int32_t>(ws, L.inv_row),
-        at<__nv_bfloat16>(ws, L.x_perm), status, 0);
+        at<__nv_bfloat16>(ws, L.x_perm), status, 0)));
     NH_TRY(launch_check("permute_scatter"));
-    permute_gather<__nv_bfloat16><<<gather_blocks, 256, 0, st>>>(
+    NH_TRY((launch_k("permute_gather", permute_gather<__nv_bfloat16>, dim3(gather_blocks), dim3(256), 0, st, 
         static_cast<const __nv_bfloat16*>(x), at<int32_t>(ws, L.perm_token),
-        at<int32_t>(ws, L.offsets), p.E, p.H, at<__nv_bfloat16>(ws, L.x_perm));
+        at<int32_t>(ws, L.offsets), p.E, p.H, at<__nv_bfloat16>(ws, L.x_perm))));
   } else {
-    permute_scatter<float><<<L.n_chunks, 32, smem, st>>>(
+    NH_TRY((launch_k("permute_scatter", permute_scatter<float>, dim3(L.n_chunks), dim3(32), smem, st, 
         topk_idx, topk_w, static_cast<const float*>(x), (int)T, p.k, p.E, p.H, chunk,
         at<int32_t>(ws, L.perm_token), at<float>(ws, L.perm_w), at<int32_t>(ws, L.inv_row),
-        at<float>(ws, L.x_perm), status, 0);
+        at<float>(ws, L.x_perm), status, 0)));
     NH_TRY(launch_check("permute_scatter"));
-    permute_gather<float><<<gather_blocks, 256, 0, st>>>(
+    NH_TRY((launch_k("permute_gather", permute_gather<float>, dim3(gather_blocks), dim3(256), 0, st, 
         static_cast<const float*>(x), at<int32_t>(ws, L.perm_token), at<int32_t>(ws, L.offsets),
-        p.E, p.H, at<float>(ws, L.x_perm));
+        p.E, p.H, at<float>(ws, L.x_perm))));
   }
   return launch_check("permute_gather");
 }
@@ -954,16 +982,16 @@ nh_status nh_moe_finalize(const nh_moe_config* cfg, int64_t T, const void* ws, s
   const int32_t* inv = at<int32_t>(ws_nc, L.inv_row);
   if (p.bf16 && p.H % 8 == 0) {
     const int H8 = p.H / 8;
-    finalize_gather_bf16x8<<<grid_for(T * H8, 256, dev), 256, 0, st>>>(
+    NH_TRY((launch_k("finalize_gather_bf16x8", finalize_gather_bf16x8, dim3(grid_for(T * H8, 256, dev)), dim3(256), 0, st, 
         at<uint4>(ws_nc, L.y_part), inv, reinterpret_cast<const float4*>(y_shared),
-        static_cast<uint4*>(y), T, p.k, H8);
+        static_cast<uint4*>(y), T, p.k, H8)));
   } else if (p.bf16) {
-    finalize_gather<__nv_bfloat16><<<grid_for(T * p.H, 256, dev), 256, 0, st>>>(
+    NH_TRY((launch_k("finalize_gather", finalize_gather<__nv_bfloat16>, dim3(grid_for(T * p.H, 256, dev)), dim3(256), 0, st, 
         at<__nv_bfloat16>(ws_nc, L.y_part), inv, y_shared, static_cast<__nv_bfloat16*>(y), T, p.k,
-        p.H);
+        p.H)));
   } else {
-    finalize_gather<float><<<grid_for(T * p.H, 256, dev), 256, 0, st>>>(
-        at<float>(ws_nc, L.y_part), inv, y_shared, static_cast<float*>(y), T, p.k, p.H);
+    NH_TRY((launch_k("finalize_gather", finalize_gather<float>, dim3(grid_for(T * p.H, 256, dev)), dim3(256), 0, st, 
+        at<float>(ws_nc, L.y_part), inv, y_shared, static_cast<float*>(y), T, p.k, p.H)));
   }
   return launch_check("finalize");
 }

@@ -27,6 +27,8 @@ __global__ void __launch_bounds__(256) permute_hist(const int32_t* __restrict__ 
                                                     int E, int32_t* __restrict__ chunk_counts,
                                                     int* status) {
   extern __shared__ int hist[];
+  pdl_wait();
+  pdl_trigger();
   for (int e = threadIdx.x; e < E; e += blockDim.x) hist[e] = 0;
   __syncthreads();
   const int t0 = blockIdx.x * PERM_CHUNK;
@@ -85,6 +87,8 @@ __global__ void permute_scan(int32_t* __restrict__ chunk_counts, int n_chunks, i
                              int32_t* __restrict__ num_tiles, int max_tiles,
                              unsigned int* sched_zero) {
   __shared__ int warp_sums[33];
+  pdl_wait();
+  pdl_trigger();
   if (threadIdx.x < 4) sched_zero[threadIdx.x] = 0u;  // up/down GEMM tile schedulers
   const int e = threadIdx.x;
   int total = 0;
@@ -126,6 +130,8 @@ __global__ void __launch_bounds__(256) permute_scatter(
     int32_t* __restrict__ perm_token, float* __restrict__ perm_w, int32_t* __restrict__ inv_row,
     Tin* __restrict__ x_perm, int* status, int do_gather) {
   extern __shared__ int sm[];
+  pdl_wait();
+  pdl_trigger();
   int* run = sm;
   int* pos = sm + E;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
@@ -207,6 +213,8 @@ __global__ void __launch_bounds__(256) permute_gather(const Tin* __restrict__ x,
                                                       const int32_t* __restrict__ perm_token,
                                                       const int32_t* __restrict__ offsets, int E,
                                                       int H, Tin* __restrict__ x_perm) {
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int rows = offsets[E];
   const int nw = (gridDim.x * blockDim.x) >> 5;
@@ -226,6 +234,8 @@ __global__ void __launch_bounds__(512) permute_small(
     Tin* __restrict__ x_perm, int* status, unsigned int* sched_zero) {
   extern __shared__ int sm[];
   __shared__ int warp_sums[33];
+  pdl_wait();
+  pdl_trigger();
   if (threadIdx.x < 4) sched_zero[threadIdx.x] = 0u;  // up/down GEMM tile schedulers
   int* cnt = sm;
   int* pos = sm + E;

@@ -14,39 +14,6 @@
 
 namespace nh {
 
-// ----- logits, small T: one warp per (expert, block of up to 8 tokens) ------
-template <typename Tin>
-__global__ void __launch_bounds__(256) router_logits_warp(const Tin* __restrict__ x,
-                                                          const float* __restrict__ wr,
-                                                          float* __restrict__ logits, int T, int H,
-                                                          int E) {
-  const int warp = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  const int lane = threadIdx.x & 31;
-  const int tblocks = (T + 7) >> 3;
-  const int e = warp / tblocks, tb = warp - e * tblocks;
-  if (e >= E) return;
-  const int t0 = tb * 8;
-  const int nt = min(8, T - t0);
-  float acc[8];
-#pragma unroll
-  for (int i = 0; i < 8; ++i) acc[i] = 0.f;
-  const float* w = wr + (size_t)e * H;
-  const Tin* xb = x + (size_t)t0 * H;
-  for (int h = lane; h < H; h += 32) {
-    const float wv = w[h];
-#pragma unroll
-    for (int i = 0; i < 8; ++i)
-      if (i < nt) acc[i] = fmaf(to_f32(xb[(size_t)i * H + h]), wv, acc[i]);
-  }
-#pragma unroll
-  for (int i = 0; i < 8; ++i) {
-    float v = acc[i];
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (lane == 0 && i < nt) logits[(size_t)(t0 + i) * E + e] = v;
-  }
-}
-
 // ----- logits, large T: 64 tokens x 64 experts per block, 4x4 per thread ----
 constexpr int RT_BT = 64, RT_BE = 64, RT_BK = 32, RT_PAD = 68;
 
@@ -57,6 +24,8 @@ __global__ void __launch_bounds__(256) router_logits_tiled(const Tin* __restrict
                                                            int H, int E) {
   __shared__ __align__(16) float xs[RT_BK][RT_PAD];
   __shared__ __align__(16) float ws[RT_BK][RT_PAD];
+  pdl_wait();
+  pdl_trigger();
   const int t0 = blockIdx.x * RT_BT, e0 = blockIdx.y * RT_BE;
   const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
   float acc[4][4];
@@ -226,6 +195,8 @@ __device__ __forceinline__ void select_token(const SelectArgs& a, int t, const f
 // one warp per token; dynamic smem: warps_per_block * E floats
 __global__ void __launch_bounds__(256) router_select(SelectArgs a) {
   extern __shared__ float sel_smem[];
+  pdl_wait();
+  pdl_trigger();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int t = blockIdx.x * (blockDim.x >> 5) + warp;
   if (t >= a.T) return;
@@ -257,6 +228,8 @@ __global__ void __launch_bounds__(256) router_fused_small(const Tin* __restrict_
   const int T = a.T, E = a.E;
   const int e = blockIdx.x;
   float* logits = const_cast<float*>(a.logits);
+  pdl_wait();
+  pdl_trigger();
   float acc[32];
 #pragma unroll
   for (int t = 0; t < 32; ++t) acc[t] = 0.f;
@@ -314,6 +287,8 @@ __global__ void __launch_bounds__(256) router_fused_small(const Tin* __restrict_
 // over K = 3H reproduces the fp32-weight logits.
 __global__ void router_split(const float* __restrict__ wr, __nv_bfloat16* __restrict__ out, int E,
                              int H) {
+  pdl_wait();
+  pdl_trigger();
   const int64_t n = (int64_t)E * H;
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x) {
