@@ -95,6 +95,28 @@ def batch_x(cfg, i):
     return x
 
 
+def rank_batch_ids(nb, rank):
+    """Input batches of one rank: every rank gets its own nb batches (token data
+    parallelism: ranks never share a batch); rank 0's first batch is the
+    workload's own x."""
+    return [rank * nb + i for i in range(nb)]
+
+
+def max_over_ranks(elapsed_ms, dist, device):
+    """Timed-region length of the whole job: the slowest rank's (all-reduce MAX)."""
+    if dist is None:
+        return float(elapsed_ms)
+    import torch
+    t = torch.tensor([float(elapsed_ms)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def job_throughput(tokens_per_rank_step, world, steps, elapsed_ms):
+    """Whole-job tokens/s: the tokens all ranks processed over the max-over-ranks time."""
+    return tokens_per_rank_step * world * steps / (elapsed_ms / 1e3)
+
+
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
     FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
@@ -180,8 +202,8 @@ def run_ours(args, rank, world, local_rank):
     T = cfg.T
     nb = max(1, args.batches)
     xs = []
-    for i in range(nb):
-        xi = inp.x if (i == 0 and rank == 0) else batch_x(cfg, i + nb * rank)
+    for i in rank_batch_ids(nb, rank):
+        xi = inp.x if i == 0 else batch_x(cfg, i)
         t = torch.from_numpy(xi)
         t = t.view(torch.bfloat16) if xi.dtype == np.uint16 else t
         xs.append(t.to(dev))
@@ -244,10 +266,7 @@ def run_ours(args, rank, world, local_rank):
         dist.barrier()
     elapsed_ms = t_start.elapsed_time(t_end)
     clk = clocks.stop() if rank == 0 else None
-    if dist:
-        tt = torch.tensor([elapsed_ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        elapsed_ms = float(tt.item())
+    elapsed_ms = max_over_ranks(elapsed_ms, dist, dev)
     rc = blk.check(T)
     if rc != 0:
         raise RuntimeError(f"device status {rc} after the timed region")
@@ -272,7 +291,8 @@ def run_ours(args, rank, world, local_rank):
         blk(xh[i % nb])
     h1.record(main)
     torch.cuda.synchronize(dev)
-    e2e_ms = h0.elapsed_time(h1) / e2e_steps
+    e2e_total_ms = max_over_ranks(h0.elapsed_time(h1), dist, dev)
+    e2e_ms = e2e_total_ms / e2e_steps
 
     result = None
     if rank == 0:
@@ -341,8 +361,7 @@ def report(args, cfg, inp, world, steps, elapsed_ms, clk, kern, e2e_ms, blk):
     pk, pk_kind = peaks()
     T = cfg.T
     ms = elapsed_ms / steps
-    tokens = T * world * steps
-    value = tokens / (elapsed_ms / 1e3)
+    value = job_throughput(T, world, steps, elapsed_ms)
     flops_tok = cfg.flops_per_token()
     tflops = flops_tok * T * world / (ms / 1e3) / 1e12
     elem = 2 if cfg.dtype == "bf16" else 4
@@ -394,7 +413,7 @@ def report(args, cfg, inp, world, steps, elapsed_ms, clk, kern, e2e_ms, blk):
         "hbm_gbs_step": round(hbm_step, 1), "hbm_frac_step": round(hbm_step / pk["hbm_gbs"], 4),
         "roofline": roof,
         "kernel_ms": {k: round(v, 5) for k, v in kern.items()},
-        "e2e": {"value": round(T / (e2e_ms / 1e3), 2), "unit": "tokens/s",
+        "e2e": {"value": round(job_throughput(T, world, 1, e2e_ms), 2), "unit": "tokens/s",
                 "ms_per_step": round(e2e_ms, 5),
                 "h2d_bytes_per_step": T * cfg.H * elem, "d2h_bytes_per_step": T * cfg.H * elem},
         "gpu_launches": launches_per_step(cfg) * steps,
