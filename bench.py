@@ -124,7 +124,16 @@ class ClockSampler:
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
     def __init__(self, gpu_index):
-        self.idx = gpu_index
+        # nvidia-smi numbers GPUs physically; under CUDA_VISIBLE_DEVICES the
+        # torch index differs, so address the device by its UUID when known
+        self.idx = str(gpu_index)
+        try:
+            import torch
+            uuid = str(torch.cuda.get_device_properties(gpu_index).uuid)
+            if uuid:
+                self.idx = uuid if uuid.startswith("GPU-") else "GPU-" + uuid
+        except Exception:
+            pass
         self.proc = None
         self.lines = []
 
@@ -325,7 +334,7 @@ def kernel_times(blk, xs, b, nb, steps):
         timed("route", lambda: nh.route(blk.c, x, blk.w_router, blk.bias, b.topk_idx, b.topk_w,
                                          b.ws, stream=main))
         timed("permute", lambda: nh.permute(blk.c, x, b.topk_idx, b.topk_w, b.ws, stream=main))
-        timed("experts_up", lambda: nh.experts_up(blk.c, T, blk.w_up, b.ws, stream=main))
+        timed("experts_up", lambda: nh.experts_up(blk.c, x, blk.w_up, b.ws, stream=main))
         timed("experts_down", lambda: nh.experts_down(blk.c, T, blk.w_down, b.ws, stream=main))
         timed("finalize", lambda: nh.finalize(blk.c, T, b.ws, b.y_shared, b.y, stream=main))
         torch.cuda.synchronize(blk.device)

@@ -97,7 +97,8 @@ typedef struct {
     size_t inv_row;       /* int32 [T, k] permuted row of assignment (t, j)     */
     size_t tiles;         /* int32 [max_tiles, 4] (expert, first row, rows, 0)  */
     size_t num_tiles;     /* int32 [1] number of valid tile entries             */
-    size_t x_perm;        /* dtype [rows_alloc, H] x gathered in permuted order */
+    size_t x_perm;        /* dtype [rows_alloc, H] x gathered in permuted order
+                             (empty when swap_ab: decode reads x directly)    */
     size_t h;             /* dtype [rows_alloc, I] relu^2(up) in permuted order */
     size_t y_part;        /* dtype [rows_alloc, H] weighted routed partial rows */
     int64_t rows_alloc;   /* T * k rounded up to the tile height                */
@@ -139,6 +140,19 @@ nh_status nh_moe_route(const nh_moe_config *cfg, int64_t T, const void *x, const
                        void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * nh_moe_route followed by nh_moe_permute, as one call with the same
+ * arguments and results (topk_idx / topk_w written, workspace filled for
+ * nh_moe_forward).  For T <= 32 and n_routed_experts <= 256 both run in a
+ * single kernel: the block that finishes the router logits last selects every
+ * token and then permutes the routing it produced; otherwise it makes the two
+ * calls.
+ */
+nh_status nh_moe_route_permute(const nh_moe_config *cfg, int64_t T, const void *x,
+                               const float *w_router, const float *e_score_correction_bias,
+                               int32_t *topk_idx, float *topk_w, void *ws, size_t ws_bytes,
+                               void *stream);
+
+/*
  * nh_moe_route_noalloc: the router of nh_moe_route for decode-sized batches,
  * for callers that cannot allocate device memory or pass a workspace (for
  * example code running under a CUDA graph capture where allocation is not
@@ -177,24 +191,25 @@ nh_status nh_moe_permute(const nh_moe_config *cfg, int64_t T, const void *x,
                          void *stream);
 
 /*
- * Routed experts: h = relu(x_perm W_up[e]^T)^2 (float32 accumulate, h stored
- * in dtype), then the weighted partial rows
+ * Routed experts: h[r] = relu(x[perm_token[r]] W_up[e]^T)^2 (float32
+ * accumulate, h stored in dtype), then the weighted partial rows
  *   y_part[r] = perm_w[r] * (h[r] W_down[e]^T)     (dtype, permuted row order)
  * which nh_moe_finalize sums per token.  Both live in the workspace.
- *   w_up [E, I, H] dtype; w_down [E, H, I] dtype.
+ *   x [T, H] dtype (the same x that nh_moe_permute saw); w_up [E, I, H] dtype;
+ *   w_down [E, H, I] dtype.
  * Needs nh_moe_permute's workspace contents.
  */
-nh_status nh_moe_forward(const nh_moe_config *cfg, int64_t T, const void *w_up, const void *w_down,
-                         void *ws, size_t ws_bytes, void *stream);
+nh_status nh_moe_forward(const nh_moe_config *cfg, int64_t T, const void *x, const void *w_up,
+                         const void *w_down, void *ws, size_t ws_bytes, void *stream);
 
 /*
  * The two phases of nh_moe_forward, for callers that schedule or time them
  * separately (same arguments and requirements):
- *   nh_moe_experts_up:   h = relu(x_perm W_up[e]^T)^2 into the workspace;
+ *   nh_moe_experts_up:   h = relu(x[perm_token] W_up[e]^T)^2 into the workspace;
  *   nh_moe_experts_down: y_part[r] = perm_w[r] * (h[r] W_down[e]^T).
  */
-nh_status nh_moe_experts_up(const nh_moe_config *cfg, int64_t T, const void *w_up, void *ws,
-                            size_t ws_bytes, void *stream);
+nh_status nh_moe_experts_up(const nh_moe_config *cfg, int64_t T, const void *x, const void *w_up,
+                            void *ws, size_t ws_bytes, void *stream);
 nh_status nh_moe_experts_down(const nh_moe_config *cfg, int64_t T, const void *w_down, void *ws,
                               size_t ws_bytes, void *stream);
 

@@ -22,7 +22,7 @@ import threading
 from . import build as _build
 
 __all__ = ["NHMoEError", "Config", "Layout", "config_from", "load", "validate", "workspace_size",
-           "workspace_layout", "shared_workspace_size", "route", "route_noalloc", "permute", "forward", "experts_up", "experts_down", "shared",
+           "workspace_layout", "shared_workspace_size", "route", "route_noalloc", "route_permute", "permute", "forward", "experts_up", "experts_down", "shared",
            "finalize", "check_device", "selftest_timeout", "library_path", "NemotronHMoE"]
 
 NH_OK, NH_ERR_INVALID_ARG, NH_ERR_UNSUPPORTED, NH_ERR_CUDA, NH_ERR_TIMEOUT, NH_ERR_DEVICE_CHECK = range(6)
@@ -75,7 +75,7 @@ _lock = threading.Lock()
 _lib = None
 
 _EXPORTS = ["nh_moe_validate", "nh_moe_workspace_size", "nh_moe_workspace_layout",
-            "nh_moe_shared_workspace_size", "nh_moe_route", "nh_moe_route_noalloc",
+            "nh_moe_shared_workspace_size", "nh_moe_route", "nh_moe_route_noalloc", "nh_moe_route_permute",
             "nh_moe_permute", "nh_moe_forward", "nh_moe_experts_up", "nh_moe_experts_down",
             "nh_moe_shared", "nh_moe_finalize", "nh_moe_check_device", "nh_moe_selftest_timeout",
             "nh_last_error", "nh_version"]
@@ -102,9 +102,10 @@ def load():
             "nh_moe_shared_workspace_size": [C, I64, ctypes.POINTER(S)],
             "nh_moe_route": [C, I64, P, P, P, P, P, P, S, P],
             "nh_moe_route_noalloc": [C, I64, P, P, P, P, P, P],
+            "nh_moe_route_permute": [C, I64, P, P, P, P, P, P, S, P],
             "nh_moe_permute": [C, I64, P, P, P, P, S, P],
-            "nh_moe_forward": [C, I64, P, P, P, S, P],
-            "nh_moe_experts_up": [C, I64, P, P, S, P],
+            "nh_moe_forward": [C, I64, P, P, P, P, S, P],
+            "nh_moe_experts_up": [C, I64, P, P, P, S, P],
             "nh_moe_experts_down": [C, I64, P, P, S, P],
             "nh_moe_shared": [C, I64, P, P, P, P, P, S, P],
             "nh_moe_finalize": [C, I64, P, S, P, P, P],
@@ -187,22 +188,30 @@ def route_noalloc(cfg, x, w_router, bias, topk_idx, topk_w, stream=None):
                                        _p(bias), _p(topk_idx), _p(topk_w), _stream(stream)))
 
 
+def route_permute(cfg, x, w_router, bias, topk_idx, topk_w, ws, stream=None):
+    """route + permute in one call (one kernel for T <= 32)."""
+    c = config_from(cfg)
+    _check(load().nh_moe_route_permute(ctypes.byref(c), x.shape[0], _p(x), _p(w_router), _p(bias),
+                                       _p(topk_idx), _p(topk_w), _p(ws), _nbytes(ws),
+                                       _stream(stream)))
+
+
 def permute(cfg, x, topk_idx, topk_w, ws, stream=None):
     c = config_from(cfg)
     _check(load().nh_moe_permute(ctypes.byref(c), x.shape[0], _p(x), _p(topk_idx), _p(topk_w),
                                  _p(ws), _nbytes(ws), _stream(stream)))
 
 
-def forward(cfg, T: int, w_up, w_down, ws, stream=None):
+def forward(cfg, x, w_up, w_down, ws, stream=None):
     c = config_from(cfg)
-    _check(load().nh_moe_forward(ctypes.byref(c), T, _p(w_up), _p(w_down), _p(ws), _nbytes(ws),
-                                 _stream(stream)))
+    _check(load().nh_moe_forward(ctypes.byref(c), x.shape[0], _p(x), _p(w_up), _p(w_down), _p(ws),
+                                 _nbytes(ws), _stream(stream)))
 
 
-def experts_up(cfg, T: int, w_up, ws, stream=None):
+def experts_up(cfg, x, w_up, ws, stream=None):
     c = config_from(cfg)
-    _check(load().nh_moe_experts_up(ctypes.byref(c), T, _p(w_up), _p(ws), _nbytes(ws),
-                                    _stream(stream)))
+    _check(load().nh_moe_experts_up(ctypes.byref(c), x.shape[0], _p(x), _p(w_up), _p(ws),
+                                    _nbytes(ws), _stream(stream)))
 
 
 def experts_down(cfg, T: int, w_down, ws, stream=None):

@@ -5,7 +5,7 @@ The Nemotron-H MoE block (``NemotronHMoE.__call__(x) -> y`` with a
 commit "Add support for Nemotron sharding", nemotron_h.pyi) on one GPU.  One
 call runs, on the caller's stream and a side stream:
 
-    main: route -> permute -> forward (routed experts) --+
+    main: route + permute -> forward (routed experts) --+
     side: shared expert ----------------------------------+-> finalize
 
 All arithmetic happens in libnhmoe's kernels; this class only owns buffers,
@@ -19,7 +19,7 @@ from typing import Dict, Optional
 import numpy as np
 import torch
 
-from . import (check_device, config_from, finalize, forward, permute, route, shared,
+from . import (check_device, config_from, finalize, forward, route_permute, shared,
                shared_workspace_size, validate, workspace_size, NH_BF16)
 
 
@@ -121,14 +121,11 @@ class NemotronHMoE:
             pop()
             join = torch.cuda.Event()
             join.record(self.side)
-        push("route")
-        route(self.c, x, self.w_router, self.bias, b.topk_idx, b.topk_w, b.ws, stream=main)
-        pop()
-        push("permute")
-        permute(self.c, x, b.topk_idx, b.topk_w, b.ws, stream=main)
+        push("route_permute")
+        route_permute(self.c, x, self.w_router, self.bias, b.topk_idx, b.topk_w, b.ws, stream=main)
         pop()
         push("forward")
-        forward(self.c, T, self.w_up, self.w_down, b.ws, stream=main)
+        forward(self.c, x, self.w_up, self.w_down, b.ws, stream=main)
         pop()
         if self.has_shared:
             main.wait_event(join)

@@ -49,6 +49,9 @@ struct TcArgs {
   void* out;
   int64_t ldo;                // row stride of out, elements
   const float* perm_w;
+  const int32_t* row_token;   // decode up projection: activations are x itself (rows
+                              // 0..NT-1) and permuted row r takes accumulator column
+                              // row_token[r]; null otherwise
   int* status;
   uint64_t timeout_ns;
   unsigned int* sched;        // [2]: next tile, CTAs finished; zero on entry, reset on exit
@@ -216,7 +219,7 @@ __global__ void __launch_bounds__(THREADS, 1)
           tma_load_3d(sb, &map_w, full_bar(stage), kb * BK, nb * NT, ent.x);
         } else {
           tma_load_3d(sa, &map_w, full_bar(stage), kb * BK, nb * M, ent.x);
-          tma_load_2d(sb, &map_act, full_bar(stage), ka, ent.y);
+          tma_load_2d(sb, &map_act, full_bar(stage), ka, g.row_token ? 0 : ent.y);
         }
         ++issued;
         if (++stage == STAGES) {
@@ -331,9 +334,21 @@ __global__ void __launch_bounds__(THREADS, 1)
         for (int c = 0; c < NT; c += 16) {
           float v[16];
           tmem_ld_x16(tq + (uint32_t)c, v);
+          if (g.row_token) {
+            // accumulator columns are tokens: row r of the expert takes column row_token[r]
+            for (int j = 0; j < ent.z; ++j) {
+              const int t = g.row_token[ent.y + j] - c;
+              if (t < 0 || t >= 16) continue;
+              float val = 0.f;
 #pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (valid && c + j < ent.z) epi_elem(g, ent.y + c + j, f, v[j]);
+              for (int u = 0; u < 16; ++u) val = (u == t) ? v[u] : val;
+              if (valid) epi_elem(g, ent.y + j, f, val);
+            }
+          } else {
+#pragma unroll
+            for (int j = 0; j < 16; ++j)
+              if (valid && c + j < ent.z) epi_elem(g, ent.y + c + j, f, v[j]);
+          }
         }
       }
       tc_fence_before();

@@ -17,6 +17,7 @@
 #include "gemm_tc2.cuh"
 #include "permute.cuh"
 #include "route.cuh"
+#include "route_permute.cuh"
 
 namespace nh {
 
@@ -69,6 +70,10 @@ constexpr size_t ALIGN = 256;
 // (shared workspace: [4..5] shared up GEMM, [6..7] shared down GEMM)
 constexpr size_t STATUS_BYTES = 64;
 constexpr int SCHED_ROUTER = 4, SCHED_UP = 6, SCHED_DOWN = 8;
+constexpr int ROUTE_PERMUTE_MAX_T = 32;
+constexpr int ROUTE_PERMUTE_MAX_E = 256;
+// fused decode router + permute: 8 warps x 2E selection floats + E + 3 T k
+constexpr int ROUTE_PERMUTE_SMEM_MAX = (16 * 256 + 256 + 3 * 32 * 32) * 4;
 
 static size_t align_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
 
@@ -184,7 +189,7 @@ static nh_status make_plan(const nh_moe_config* c, int64_t T, Plan* p) {
   L.inv_row = take((size_t)rows * 4);
   L.tiles = take((size_t)L.max_tiles * 16);
   L.num_tiles = take(4);
-  L.x_perm = take((size_t)rows * p->H * p->elem);
+  L.x_perm = take(L.swap_ab ? 0 : (size_t)rows * p->H * p->elem);
   L.h = take((size_t)rows * p->I * p->elem);
   L.y_part = take((size_t)rows * p->H * p->elem);
   L.total_bytes = o;
@@ -210,6 +215,24 @@ static nh_status check_ws(const Plan& p, void* ws, size_t ws_bytes) {
 template <typename T>
 static T* at(void* ws, size_t off) {
   return reinterpret_cast<T*>(static_cast<char*>(ws) + off);
+}
+
+static PermuteOut permute_out(void* ws, const nh_moe_ws_layout& L, int* status) {
+  PermuteOut o;
+  o.tile_rows = L.tile_rows;
+  o.max_tiles = L.max_tiles;
+  o.counts = at<int32_t>(ws, L.counts);
+  o.offsets = at<int32_t>(ws, L.offsets);
+  o.tiles = at<int4>(ws, L.tiles);
+  o.num_tiles = at<int32_t>(ws, L.num_tiles);
+  o.perm_token = at<int32_t>(ws, L.perm_token);
+  o.perm_w = at<float>(ws, L.perm_w);
+  o.inv_row = at<int32_t>(ws, L.inv_row);
+  o.x_perm = at<void>(ws, L.x_perm);
+  o.status = status;
+  o.sched_zero = reinterpret_cast<unsigned int*>(status + SCHED_UP);
+  o.gather = L.swap_ab ? 0 : 1;
+  return o;
 }
 
 // ----------------------------------------------------------------------------
@@ -243,6 +266,10 @@ static nh_status set_attrs(int dev) {
                                cudaFuncAttributeMaxDynamicSharedMemorySize, TcSwap64::SMEM));
   NH_CUDA(cudaFuncSetAttribute(tc2::tc2_grouped_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                tc2::SMEM));
+  NH_CUDA(cudaFuncSetAttribute(route_permute_small<__nv_bfloat16>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, ROUTE_PERMUTE_SMEM_MAX));
+  NH_CUDA(cudaFuncSetAttribute(route_permute_small<float>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, ROUTE_PERMUTE_SMEM_MAX));
   {
     cudaLaunchConfig_t lc = {};
     lc.gridDim = dim3(2 * (prop.multiProcessorCount / 2), 1, 1);
@@ -370,6 +397,7 @@ struct GemmCall {
   void* out;
   int64_t ldo;
   const float* perm_w;
+  const int32_t* row_token;  // decode up projection reads x directly
   int* status;
   unsigned int* sched;  // tile scheduler counters (tensor-core path)
 };
@@ -392,6 +420,7 @@ static nh_status launch_tc(const GemmCall& c, int dev, cudaStream_t st) {
   g.out = c.out;
   g.ldo = c.ldo;
   g.perm_w = c.perm_w;
+  g.row_token = c.row_token;
   g.status = c.status;
   g.timeout_ns = timeout_ns();
   g.sched = c.sched;
@@ -423,6 +452,7 @@ static nh_status launch_tc2(const GemmCall& c, int dev, cudaStream_t st) {
   g.out = c.out;
   g.ldo = c.ldo;
   g.perm_w = c.perm_w;
+  g.row_token = nullptr;
   g.status = c.status;
   g.timeout_ns = timeout_ns();
   g.sched = c.sched;
@@ -674,7 +704,7 @@ nh_status nh_moe_route(const nh_moe_config* cfg, int64_t T, const void* x, const
   a.alpha = cfg->routed_scaling_factor;
   a.group_score = cfg->group_score;
   a.use_sigma = (bias != nullptr) || cfg->group_score == NH_GROUP_SCORE_TOP2;
-  const size_t sel_smem = (size_t)8 * p.E * sizeof(float);
+  const size_t sel_smem = (size_t)8 * 2 * p.E * sizeof(float);
   if (T <= 32) {
     // decode: logits and selection in one launch (last block selects)
     const int blocks = p.E;
@@ -769,7 +799,7 @@ nh_status nh_moe_route_noalloc(const nh_moe_config* cfg, int64_t T, const void* 
   a.alpha = cfg->routed_scaling_factor;
   a.group_score = cfg->group_score;
   a.use_sigma = (bias != nullptr) || cfg->group_score == NH_GROUP_SCORE_TOP2;
-  const size_t sel_smem = (size_t)8 * a.E * sizeof(float);
+  const size_t sel_smem = (size_t)8 * 2 * a.E * sizeof(float);
   const int blocks = a.E;
   unsigned int* done = reinterpret_cast<unsigned int*>(status + 3);
   if (cfg->dtype == NH_BF16)
@@ -801,22 +831,16 @@ nh_status nh_moe_permute(const nh_moe_config* cfg, int64_t T, const void* x,
   int* status = at<int>(ws, L.status);
   if (T <= PERM_CHUNK) {
     // decode-sized: the whole permute in one block
+    const PermuteOut o = permute_out(ws, L, status);
     const size_t smem = (size_t)(p.E + T * p.k) * sizeof(int);
     if (p.bf16)
-      NH_TRY((launch_k("permute_small", permute_small<__nv_bfloat16>, dim3(1), dim3(512), smem, st, 
-          topk_idx, topk_w, static_cast<const __nv_bfloat16*>(x), (int)T, p.k, p.E, p.H,
-          L.tile_rows, L.max_tiles, at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets),
-          at<int4>(ws, L.tiles), at<int32_t>(ws, L.num_tiles), at<int32_t>(ws, L.perm_token),
-          at<float>(ws, L.perm_w), at<int32_t>(ws, L.inv_row), at<__nv_bfloat16>(ws, L.x_perm),
-          status, reinterpret_cast<unsigned int*>(status + SCHED_UP))));
+      NH_TRY((launch_k("permute_small", permute_small<__nv_bfloat16>, dim3(1), dim3(512), smem, st,
+                       topk_idx, topk_w, static_cast<const __nv_bfloat16*>(x), (int)T, p.k, p.E,
+                       p.H, o)));
     else
-      NH_TRY((launch_k("permute_small", permute_small<float>, dim3(1), dim3(512), smem, st, 
-          topk_idx, topk_w, static_cast<const float*>(x), (int)T, p.k, p.E, p.H, L.tile_rows,
-          L.max_tiles, at<int32_t>(ws, L.counts), at<int32_t>(ws, L.offsets),
-          at<int4>(ws, L.tiles), at<int32_t>(ws, L.num_tiles), at<int32_t>(ws, L.perm_token),
-          at<float>(ws, L.perm_w), at<int32_t>(ws, L.inv_row), at<float>(ws, L.x_perm), status,
-          reinterpret_cast<unsigned int*>(status + SCHED_UP))));
-    return launch_check("permute_small");
+      NH_TRY((launch_k("permute_small", permute_small<float>, dim3(1), dim3(512), smem, st,
+                       topk_idx, topk_w, static_cast<const float*>(x), (int)T, p.k, p.E, p.H, o)));
+    return NH_OK;
   }
   int32_t* chunk = at<int32_t>(ws, L.chunk_counts);
   NH_TRY((launch_k("permute_hist", permute_hist, dim3(L.n_chunks), dim3(256), p.E * sizeof(int), st, topk_idx, (int)T, p.k, p.E, chunk, status)));
@@ -852,13 +876,61 @@ nh_status nh_moe_permute(const nh_moe_config* cfg, int64_t T, const void* x,
   return launch_check("permute_gather");
 }
 
-static nh_status experts_phase(const nh_moe_config* cfg, int64_t T, const void* w, void* ws,
-                               size_t ws_bytes, void* stream, bool up_phase) {
+nh_status nh_moe_route_permute(const nh_moe_config* cfg, int64_t T, const void* x,
+                               const float* w_router, const float* bias, int32_t* topk_idx,
+                               float* topk_w, void* ws, size_t ws_bytes, void* stream) {
+  Plan p;
+  NH_TRY(make_plan(cfg, T, &p));
+  NH_TRY(check_ws(p, ws, ws_bytes));
+  if (T > ROUTE_PERMUTE_MAX_T || p.E > ROUTE_PERMUTE_MAX_E) {
+    NH_TRY(nh_moe_route(cfg, T, x, w_router, bias, topk_idx, topk_w, ws, ws_bytes, stream));
+    return nh_moe_permute(cfg, T, x, topk_idx, topk_w, ws, ws_bytes, stream);
+  }
+  if (T == 0) return nh_moe_permute(cfg, T, x, topk_idx, topk_w, ws, ws_bytes, stream);
+  NH_TRY(check_ptr(x, "x"));
+  NH_TRY(check_ptr(w_router, "w_router"));
+  NH_TRY(check_ptr(topk_idx, "topk_idx"));
+  NH_TRY(check_ptr(topk_w, "topk_w"));
+  if (bias) NH_TRY(check_ptr(bias, "e_score_correction_bias"));
+  int dev;
+  NH_TRY(device_setup(&dev));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const nh_moe_ws_layout& L = p.lay;
+  int* status = at<int>(ws, L.status);
+  NH_CUDA(cudaMemsetAsync(status, 0, STATUS_BYTES, st));
+  SelectArgs a;
+  a.logits = at<float>(ws, L.logits);
+  a.bias = bias;
+  a.topk_idx = topk_idx;
+  a.topk_w = topk_w;
+  a.status = status;
+  a.T = (int)T;
+  a.E = p.E;
+  a.G = p.G;
+  a.tg = p.tg;
+  a.k = p.k;
+  a.norm = cfg->norm_topk_prob;
+  a.alpha = cfg->routed_scaling_factor;
+  a.group_score = cfg->group_score;
+  a.use_sigma = (bias != nullptr) || cfg->group_score == NH_GROUP_SCORE_TOP2;
+  const PermuteOut o = permute_out(ws, L, status);
+  const size_t smem = (size_t)(16 * p.E + p.E + 3 * T * p.k) * sizeof(float);
+  unsigned int* done = reinterpret_cast<unsigned int*>(status + 3);
+  if (p.bf16)
+    return launch_k("route_permute_small", route_permute_small<__nv_bfloat16>, dim3(p.E), dim3(256),
+                    smem, st, static_cast<const __nv_bfloat16*>(x), w_router, a, p.H, done, o);
+  return launch_k("route_permute_small", route_permute_small<float>, dim3(p.E), dim3(256), smem, st,
+                  static_cast<const float*>(x), w_router, a, p.H, done, o);
+}
+
+static nh_status experts_phase(const nh_moe_config* cfg, int64_t T, const void* x, const void* w,
+                               void* ws, size_t ws_bytes, void* stream, bool up_phase) {
   Plan p;
   NH_TRY(make_plan(cfg, T, &p));
   NH_TRY(check_ws(p, ws, ws_bytes));
   if (T == 0) return NH_OK;
   NH_TRY(check_ptr(w, up_phase ? "w_up" : "w_down"));
+  if (up_phase) NH_TRY(check_ptr(x, "x"));
   int dev;
   NH_TRY(device_setup(&dev));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -875,7 +947,14 @@ static nh_status experts_phase(const nh_moe_config* cfg, int64_t T, const void* 
   c.sched = reinterpret_cast<unsigned int*>(c.status + (up_phase ? SCHED_UP : SCHED_DOWN));
   c.W = w;
   if (up_phase) {
-    c.A = at<void>(ws, L.x_perm);
+    if (L.swap_ab) {
+      // decode: the activation tile is x itself; rows map to tokens by perm_token
+      c.A = x;
+      c.rows = T;
+      c.row_token = at<int32_t>(ws, L.perm_token);
+    } else {
+      c.A = at<void>(ws, L.x_perm);
+    }
     c.N = p.I;
     c.K = p.H;
     c.epi = EPI_UP_RELU2;
@@ -893,25 +972,26 @@ static nh_status experts_phase(const nh_moe_config* cfg, int64_t T, const void* 
   return run_gemm(p, c, dev, st);
 }
 
-nh_status nh_moe_experts_up(const nh_moe_config* cfg, int64_t T, const void* w_up, void* ws,
-                            size_t ws_bytes, void* stream) {
-  return experts_phase(cfg, T, w_up, ws, ws_bytes, stream, true);
+nh_status nh_moe_experts_up(const nh_moe_config* cfg, int64_t T, const void* x, const void* w_up,
+                            void* ws, size_t ws_bytes, void* stream) {
+  return experts_phase(cfg, T, x, w_up, ws, ws_bytes, stream, true);
 }
 
 nh_status nh_moe_experts_down(const nh_moe_config* cfg, int64_t T, const void* w_down, void* ws,
                               size_t ws_bytes, void* stream) {
-  return experts_phase(cfg, T, w_down, ws, ws_bytes, stream, false);
+  return experts_phase(cfg, T, nullptr, w_down, ws, ws_bytes, stream, false);
 }
 
-nh_status nh_moe_forward(const nh_moe_config* cfg, int64_t T, const void* w_up, const void* w_down,
-                         void* ws, size_t ws_bytes, void* stream) {
+nh_status nh_moe_forward(const nh_moe_config* cfg, int64_t T, const void* x, const void* w_up,
+                         const void* w_down, void* ws, size_t ws_bytes, void* stream) {
   Plan p;
   NH_TRY(make_plan(cfg, T, &p));
   NH_TRY(check_ws(p, ws, ws_bytes));
   if (T == 0) return NH_OK;
+  NH_TRY(check_ptr(x, "x"));
   NH_TRY(check_ptr(w_up, "w_up"));
   NH_TRY(check_ptr(w_down, "w_down"));
-  NH_TRY(nh_moe_experts_up(cfg, T, w_up, ws, ws_bytes, stream));
+  NH_TRY(nh_moe_experts_up(cfg, T, x, w_up, ws, ws_bytes, stream));
   return nh_moe_experts_down(cfg, T, w_down, ws, ws_bytes, stream);
 }
 

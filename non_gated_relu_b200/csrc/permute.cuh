@@ -222,25 +222,20 @@ __global__ void __launch_bounds__(256) permute_gather(const Tin* __restrict__ x,
     copy_row(x + (size_t)perm_token[p] * H, x_perm + (size_t)p * H, H, lane);
 }
 
-// Whole permute in one block for T <= PERM_CHUNK tokens (decode): histogram,
-// scan, tile table, stable ranking and gather.  blockDim.x = 512 (>= E).
-// Dynamic smem: int cnt[E] + int pos[T * k].
+// Whole permute of T <= PERM_CHUNK tokens by one block of blockDim.x >= E
+// threads: histogram, scan, tile table, stable ranking and gather.  idx / w
+// may live in global or shared memory; cnt [E] and pos [T * k] are shared
+// memory; warp_sums [33] is shared memory.
 template <typename Tin>
-__global__ void __launch_bounds__(512) permute_small(
-    const int32_t* __restrict__ idx, const float* __restrict__ w, const Tin* __restrict__ x,
-    int T, int k, int E, int H, int tile_rows, int max_tiles, int32_t* __restrict__ counts,
-    int32_t* __restrict__ offsets, int4* __restrict__ tiles, int32_t* __restrict__ num_tiles,
-    int32_t* __restrict__ perm_token, float* __restrict__ perm_w, int32_t* __restrict__ inv_row,
-    Tin* __restrict__ x_perm, int* status, unsigned int* sched_zero) {
-  extern __shared__ int sm[];
-  __shared__ int warp_sums[33];
-  pdl_wait();
-  pdl_trigger();
-  if (threadIdx.x < 4) sched_zero[threadIdx.x] = 0u;  // up/down GEMM tile schedulers
-  int* cnt = sm;
-  int* pos = sm + E;
+__device__ __forceinline__ void permute_block(
+    const int32_t* idx, const float* w, const Tin* __restrict__ x, int T, int k, int E, int H,
+    int tile_rows, int max_tiles, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
+    int4* __restrict__ tiles, int32_t* __restrict__ num_tiles, int32_t* __restrict__ perm_token,
+    float* __restrict__ perm_w, int32_t* __restrict__ inv_row, Tin* __restrict__ x_perm,
+    int* status, unsigned int* sched_zero, int* cnt, int* pos, int* warp_sums, bool gather) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int n = T * k;
+  if (threadIdx.x < 4) sched_zero[threadIdx.x] = 0u;  // up/down GEMM tile schedulers
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
   for (int a = threadIdx.x; a < n; a += blockDim.x) {
@@ -294,12 +289,42 @@ __global__ void __launch_bounds__(512) permute_small(
       }
     }
   }
+  if (!gather) return;  // decode: the up projection reads x itself
   __syncthreads();
   const int nw = blockDim.x >> 5;
   for (int a = warp; a < n; a += nw) {
     const int p = pos[a];
     if (p >= 0) copy_row(x + (size_t)(a / k) * H, x_perm + (size_t)p * H, H, lane);
   }
+}
+
+struct PermuteOut {
+  int tile_rows, max_tiles;
+  int32_t *counts, *offsets;
+  int4* tiles;
+  int32_t *num_tiles, *perm_token;
+  float* perm_w;
+  int32_t* inv_row;
+  void* x_perm;
+  int* status;
+  unsigned int* sched_zero;
+  int gather;   // 0: no x_perm (decode orientation reads x directly)
+};
+
+// Whole permute in one block for T <= PERM_CHUNK tokens (decode).
+// blockDim.x = 512 (>= E).  Dynamic smem: int cnt[E] + int pos[T * k].
+template <typename Tin>
+__global__ void __launch_bounds__(512) permute_small(const int32_t* __restrict__ idx,
+                                                     const float* __restrict__ w,
+                                                     const Tin* __restrict__ x, int T, int k, int E,
+                                                     int H, PermuteOut o) {
+  extern __shared__ int sm[];
+  __shared__ int warp_sums[33];
+  pdl_wait();
+  pdl_trigger();
+  permute_block(idx, w, x, T, k, E, H, o.tile_rows, o.max_tiles, o.counts, o.offsets, o.tiles,
+                o.num_tiles, o.perm_token, o.perm_w, o.inv_row, static_cast<Tin*>(o.x_perm),
+                o.status, o.sched_zero, sm, sm + E, warp_sums, o.gather != 0);
 }
 
 }  // namespace nh

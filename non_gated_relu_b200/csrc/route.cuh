@@ -104,10 +104,13 @@ __device__ __forceinline__ void warp_best(float& v, int& i) {
 // Selection of one token by one warp; `sel` holds the token's E selection
 // scores in shared memory (written by the caller).
 __device__ __forceinline__ void select_token(const SelectArgs& a, int t, const float* l,
-                                             float* sel, int lane) {
+                                             float* sel, int lane, int32_t* idx_out = nullptr,
+                                             float* w_out = nullptr) {
   const int E = a.E, G = a.G, g = E / G;
+  float* lraw = sel + E;  // the token's logits, staged next to its selection scores
   for (int e = lane; e < E; e += 32) {
     const float le = __ldcg(l + e);  // produced by another block or kernel: read at L2
+    lraw[e] = le;
     sel[e] = a.use_sigma ? sigmoid_f32(le) + (a.bias ? a.bias[e] : 0.f) : le;
   }
   __syncwarp();
@@ -156,6 +159,10 @@ __device__ __forceinline__ void select_token(const SelectArgs& a, int t, const f
     pq = bq;
     pv = bv;
   }
+  // which of this lane's experts (e = lane + 32 i, E <= 512) lie in kept groups
+  uint32_t mine = 0;
+  for (int i = 0, e = lane; e < E; ++i, e += 32)
+    if ((keep >> (e / g)) & 1ull) mine |= 1u << i;
   // top-k experts of the kept groups in (score desc, id asc) order
   int pe = -1;
   float pev = 0.f, ssum = 0.f, my_s = 0.f;
@@ -163,8 +170,8 @@ __device__ __forceinline__ void select_token(const SelectArgs& a, int t, const f
   for (int j = 0; j < a.k; ++j) {
     float bv = 0.f;
     int be = -1;
-    for (int e = lane; e < E; e += 32) {
-      if (!((keep >> (e / g)) & 1ull)) continue;
+    for (int i = 0, e = lane; e < E; ++i, e += 32) {
+      if (!((mine >> i) & 1u)) continue;
       const float v = sel[e];
       if (pe >= 0 && !ranks_before(pev, pe, v, e)) continue;
       if (be < 0 || ranks_before(v, e, bv, be)) {
@@ -177,7 +184,7 @@ __device__ __forceinline__ void select_token(const SelectArgs& a, int t, const f
       if (lane == 0) record_status(a.status, NH_ERR_DEVICE_CHECK, SITE_ROUTE_SELECT, t);
       be = 0;
     }
-    const float sj = sigmoid_f32(__ldcg(l + be));
+    const float sj = sigmoid_f32(lraw[be]);
     ssum += sj;
     if (lane == j) {
       my_e = be;
@@ -187,12 +194,17 @@ __device__ __forceinline__ void select_token(const SelectArgs& a, int t, const f
     pev = bv;
   }
   if (lane < a.k) {
+    const float wj = a.norm ? a.alpha * my_s / ssum : a.alpha * my_s;
     a.topk_idx[(size_t)t * a.k + lane] = my_e;
-    a.topk_w[(size_t)t * a.k + lane] = a.norm ? a.alpha * my_s / ssum : a.alpha * my_s;
+    a.topk_w[(size_t)t * a.k + lane] = wj;
+    if (idx_out) {
+      idx_out[t * a.k + lane] = my_e;
+      w_out[t * a.k + lane] = wj;
+    }
   }
 }
 
-// one warp per token; dynamic smem: warps_per_block * E floats
+// one warp per token; dynamic smem: warps_per_block * 2E floats
 __global__ void __launch_bounds__(256) router_select(SelectArgs a) {
   extern __shared__ float sel_smem[];
   pdl_wait();
@@ -200,7 +212,7 @@ __global__ void __launch_bounds__(256) router_select(SelectArgs a) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int t = blockIdx.x * (blockDim.x >> 5) + warp;
   if (t >= a.T) return;
-  select_token(a, t, a.logits + (size_t)t * a.E, sel_smem + (size_t)warp * a.E, lane);
+  select_token(a, t, a.logits + (size_t)t * a.E, sel_smem + (size_t)warp * 2 * a.E, lane);
 }
 
 // x[t, h .. h+3] as floats (h a multiple of 4, rows 8-byte aligned for bf16)
@@ -213,40 +225,45 @@ __device__ __forceinline__ float4 load4(const float* p) {
   return *reinterpret_cast<const float4*>(p);
 }
 
-// Decode-sized T (<= 32): block e computes expert e's logits for every token
-// (its 256 threads split H four elements at a time, then reduce), and the
-// last block to finish selects every token.  `done` is a counter that is
-// zero on entry; the last block resets it.
+// Logits of expert e for the T <= 32 tokens, by one block: threads split H
+// four elements at a time with all weight loads of a thread issued first,
+// then a block reduction.  red: [blockDim/32][32] floats of shared memory.
 template <typename Tin>
-__global__ void __launch_bounds__(256) router_fused_small(const Tin* __restrict__ x,
-                                                          const float* __restrict__ wr,
-                                                          SelectArgs a, int H,
-                                                          unsigned int* done) {
-  extern __shared__ float sel_smem[];
-  __shared__ float red[8][32];
-  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
-  const int T = a.T, E = a.E;
-  const int e = blockIdx.x;
-  float* logits = const_cast<float*>(a.logits);
-  pdl_wait();
-  pdl_trigger();
+__device__ __forceinline__ void router_block_logits(const Tin* __restrict__ x,
+                                                    const float* __restrict__ wr, int e, int T,
+                                                    int E, int H, float* logits,
+                                                    float (*red)[32]) {
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  const int step = blockDim.x * 4;
   float acc[32];
 #pragma unroll
   for (int t = 0; t < 32; ++t) acc[t] = 0.f;
   const float* w = wr + (size_t)e * H;
   if ((H & 3) == 0) {
-    for (int h = threadIdx.x * 4; h < H; h += 1024) {
-      const float4 wv = __ldg(reinterpret_cast<const float4*>(w + h));
+    constexpr int U = 2;
+    for (int h0 = threadIdx.x * 4; h0 < H; h0 += U * step) {
+      float4 wv[U];
 #pragma unroll
-      for (int t = 0; t < 32; ++t) {
-        if (t < T) {
-          const float4 xv = load4(x + (size_t)t * H + h);
-          acc[t] = fmaf(xv.x, wv.x, fmaf(xv.y, wv.y, fmaf(xv.z, wv.z, fmaf(xv.w, wv.w, acc[t]))));
+      for (int u = 0; u < U; ++u) {
+        const int h = h0 + u * step;
+        wv[u] = h < H ? __ldg(reinterpret_cast<const float4*>(w + h)) : make_float4(0.f, 0.f, 0.f, 0.f);
+      }
+#pragma unroll
+      for (int u = 0; u < U; ++u) {
+        const int h = h0 + u * step;
+        if (h >= H) break;
+#pragma unroll
+        for (int t = 0; t < 32; ++t) {
+          if (t < T) {
+            const float4 xv = load4(x + (size_t)t * H + h);
+            acc[t] = fmaf(xv.x, wv[u].x,
+                          fmaf(xv.y, wv[u].y, fmaf(xv.z, wv[u].z, fmaf(xv.w, wv[u].w, acc[t]))));
+          }
         }
       }
     }
   } else {
-    for (int h = threadIdx.x; h < H; h += 256) {
+    for (int h = threadIdx.x; h < H; h += blockDim.x) {
       const float wv = w[h];
 #pragma unroll
       for (int t = 0; t < 32; ++t)
@@ -265,10 +282,29 @@ __global__ void __launch_bounds__(256) router_fused_small(const Tin* __restrict_
   __syncthreads();
   if (wib == 0 && lane < T) {
     float v = 0.f;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) v += red[i][lane];
+    for (int i = 0; i < nw; ++i) v += red[i][lane];
     logits[(size_t)lane * E + e] = v;
   }
+}
+
+// Decode-sized T (<= 32): block e computes expert e's logits for every token
+// (its 256 threads split H four elements at a time, then reduce), and the
+// last block to finish selects every token.  `done` is a counter that is
+// zero on entry; the last block resets it.
+template <typename Tin>
+__global__ void __launch_bounds__(256) router_fused_small(const Tin* __restrict__ x,
+                                                          const float* __restrict__ wr,
+                                                          SelectArgs a, int H,
+                                                          unsigned int* done) {
+  extern __shared__ float sel_smem[];
+  __shared__ float red[16][32];
+  const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5;
+  const int T = a.T, E = a.E;
+  const int e = blockIdx.x;
+  float* logits = const_cast<float*>(a.logits);
+  pdl_wait();
+  pdl_trigger();
+  router_block_logits(x, wr, e, T, E, H, logits, red);
   // last-block-done: the block that finishes last sees every logit
   __shared__ unsigned int ticket;
   __threadfence();
@@ -278,7 +314,7 @@ __global__ void __launch_bounds__(256) router_fused_small(const Tin* __restrict_
   if (ticket != gridDim.x - 1) return;
   __threadfence();
   for (int t = wib; t < T; t += 8)
-    select_token(a, t, logits + (size_t)t * E, sel_smem + (size_t)wib * E, lane);
+    select_token(a, t, logits + (size_t)t * E, sel_smem + (size_t)wib * 2 * E, lane);
   if (threadIdx.x == 0) *done = 0u;
 }
 

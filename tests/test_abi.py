@@ -78,7 +78,7 @@ def test_workspace_layout(name):
                ("counts", cfg.E * 4),
                ("offsets", (cfg.E + 1) * 4), ("chunk_counts", L.n_chunks * cfg.E * 4),
                ("perm_token", rows * 4), ("perm_w", rows * 4), ("inv_row", rows * 4),
-               ("tiles", L.max_tiles * 16), ("num_tiles", 4), ("x_perm", rows * cfg.H * elem),
+               ("tiles", L.max_tiles * 16), ("num_tiles", 4), ("x_perm", 0 if L.swap_ab else rows * cfg.H * elem),
                ("h", rows * cfg.I * elem), ("y_part", rows * cfg.H * elem)]
     spans = sorted((getattr(L, n), getattr(L, n) + sz, n) for n, sz in regions)
     for (a0, a1, an), (b0, b1, bn) in zip(spans, spans[1:]):
@@ -107,7 +107,7 @@ def test_argument_checks_before_any_device_work():
     assert rc == nh.NH_ERR_INVALID_ARG and b"needed" in lib.nh_last_error()
     # misaligned pointer
     need = nh.workspace_size(c, 8)
-    rc = lib.nh_moe_forward(ctypes.byref(c), 8, P(18), P(16), P(256), need, None)
+    rc = lib.nh_moe_forward(ctypes.byref(c), 8, P(16), P(18), P(16), P(256), need, None)
     assert rc == nh.NH_ERR_INVALID_ARG and b"aligned" in lib.nh_last_error()
     # negative T
     rc = lib.nh_moe_workspace_size(ctypes.byref(c), -1, ctypes.byref(ctypes.c_size_t()))
