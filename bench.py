@@ -39,8 +39,7 @@ import synth  # noqa: E402
 METRIC = "MoE-block tokens/s and TFLOP/s (frac of bf16 peak / HBM roofline), 1×B200"
 DEFAULT_WORKLOAD = "decode_bf16_t8"
 FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
-KERNEL_SOURCES = ["non_gated_relu_b200/csrc/gemm_tc.cuh", "non_gated_relu_b200/csrc/common.cuh",
-                  "non_gated_relu_b200/csrc/nh_moe.cu"]
+KERNEL_SOURCE_DIR = "non_gated_relu_b200/csrc"
 
 
 def parse():
@@ -440,10 +439,15 @@ def report(args, cfg, inp, world, steps, elapsed_ms, clk, kern, e2e_ms, blk):
 
 
 def kernel_hash():
+    """Hash of every CUDA source of the library: profiler counters recorded for
+    one build are reported only while the sources are unchanged."""
     h = hashlib.sha256()
-    for p in KERNEL_SOURCES:
-        with open(os.path.join(ROOT, p), "rb") as f:
-            h.update(f.read())
+    d = os.path.join(ROOT, KERNEL_SOURCE_DIR)
+    for name in sorted(os.listdir(d)):
+        if name.endswith((".cu", ".cuh")):
+            with open(os.path.join(d, name), "rb") as f:
+                h.update(name.encode())
+                h.update(f.read())
     return h.hexdigest()[:16]
 
 
