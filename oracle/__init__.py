@@ -51,6 +51,14 @@ class _Cfg(ctypes.Structure):
                 ("group_score", ctypes.c_int64)]
 
 
+class _Wt(ctypes.Structure):
+    """nho_wt: one stacked weight tensor [n_mat][rows][cols] (float32, bf16 or NVFP4)."""
+    _fields_ = [("format", ctypes.c_int64), ("data", ctypes.c_void_p),
+                ("scales", ctypes.c_void_p), ("global_", ctypes.c_void_p),
+                ("rows", ctypes.c_int64), ("cols", ctypes.c_int64),
+                ("scale_pitch", ctypes.c_int64)]
+
+
 def _load():
     global _lib
     with _lock:
@@ -61,6 +69,10 @@ def _load():
             lib.nho_route.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int64, P, P, P, P, P, P, P]
             lib.nho_forward.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int64, P, P, P, P, P, P,
                                         P, P, P, P, ctypes.c_int64, P, P, P]
+            W = ctypes.POINTER(_Wt)
+            lib.nho_forward_wt.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int64, P, P, P, W, W, W,
+                                           W, P, P, P, ctypes.c_int64, P, P, P]
+            lib.nho_dequant.argtypes = [W, ctypes.c_int64, P]
             _lib = lib
     return _lib
 
@@ -72,7 +84,7 @@ def _swap_library(path):
     global _lib
     prev = _load()
     lib = ctypes.CDLL(path)
-    for name in ("nho_check_config", "nho_route", "nho_forward"):
+    for name in ("nho_check_config", "nho_route", "nho_forward", "nho_forward_wt", "nho_dequant"):
         getattr(lib, name).argtypes = getattr(prev, name).argtypes
     with _lock:
         _lib = lib
@@ -145,6 +157,54 @@ def route_parallel(cfg, x, w_router, bias=None, threads: int = 8, group_score: i
     return tuple(np.concatenate([p[i] for p in parts]) for i in range(4))
 
 
+def _wt_nvfp4(q, rows, cols):
+    codes, scales, g = (np.ascontiguousarray(q[0], np.uint8), np.ascontiguousarray(q[1], np.uint8),
+                        np.ascontiguousarray(q[2], np.float32))
+    keep = (codes, scales, g)
+    return _Wt(2, codes.ctypes.data, scales.ctypes.data, g.ctypes.data, rows, cols,
+               scales.shape[-1]), keep
+
+
+def dequant_nvfp4(q, rows, cols, mat=0):
+    """Dense float64 [rows, cols] of matrix `mat` of an NVFP4 tensor (codes, scales, global)."""
+    w, keep = _wt_nvfp4(q, rows, cols)
+    out = np.zeros((rows, cols), np.float64)
+    rc = _load().nho_dequant(ctypes.byref(w), mat, _ptr(out))
+    if rc:
+        raise OracleError(f"nho_dequant failed ({rc})")
+    return out
+
+
+def _forward_nvfp4(inp, tok, oi, ow, group_score):
+    cfg = inp.cfg
+    lib = _load()
+    c = _cfg(cfg, group_score)
+    n = tok.shape[0]
+    y = np.zeros((n, cfg.H), np.float64)
+    idx = np.zeros((n, cfg.k), np.int32)
+    w = np.zeros((n, cfg.k), np.float64)
+    q = inp.nvfp4
+    up, k1 = _wt_nvfp4(q["up"], cfg.I, cfg.H)
+    dn, k2 = _wt_nvfp4(q["down"], cfg.H, cfg.I)
+    su = sd = None
+    keep = [k1, k2]
+    if cfg.n_shared_experts:
+        su, k3 = _wt_nvfp4(q["shared_up"], cfg.S, cfg.H)
+        sd, k4 = _wt_nvfp4(q["shared_down"], cfg.H, cfg.S)
+        keep += [k3, k4]
+    x = _stored(inp.x, cfg.dtype)
+    wr = np.ascontiguousarray(inp.w_router, np.float32)
+    b = None if inp.bias is None else np.ascontiguousarray(inp.bias, np.float32)
+    rc = lib.nho_forward_wt(ctypes.byref(c), inp.x.shape[0], _ptr(x), _ptr(wr), _ptr(b),
+                            ctypes.byref(up), ctypes.byref(dn),
+                            ctypes.byref(su) if su is not None else None,
+                            ctypes.byref(sd) if sd is not None else None,
+                            _ptr(oi), _ptr(ow), _ptr(tok), n, _ptr(y), _ptr(idx), _ptr(w))
+    if rc:
+        raise OracleError(f"nho_forward_wt failed ({rc})")
+    return y, idx, w
+
+
 def forward(inp, tokens=None, override_idx=None, override_w=None, group_score: int = 0):
     """Block output y (float64 [n_tok, H]) for the listed tokens (default: all).
 
@@ -165,6 +225,8 @@ def forward(inp, tokens=None, override_idx=None, override_w=None, group_score: i
     if override_idx is not None:
         oi = np.ascontiguousarray(override_idx, np.int32).reshape(n, cfg.k)
         ow = np.ascontiguousarray(override_w, np.float64).reshape(n, cfg.k)
+    if getattr(inp, "nvfp4", None) is not None:
+        return _forward_nvfp4(inp, tok, oi, ow, group_score)
     x = _stored(inp.x, cfg.dtype)
     args = [_stored(a, cfg.dtype) if a is not None else None
             for a in (inp.w_up, inp.w_down, inp.w_shared_up, inp.w_shared_down)]

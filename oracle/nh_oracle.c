@@ -37,6 +37,17 @@
  * Wu [E][I][H], Wd [E][H][I], Wsu [S][H], Wsd [H][S]; x [T][H].  Activations
  * and expert weights are float32 (dtype 0) or bf16 bit patterns (dtype 1).
  *
+ * Expert and shared weights may instead be NVFP4 (W4A16 with group size 16:
+ * "NVFP4 W4A16 group_size 16 on the experts, shared experts", vllm.cpp PR
+ * #518).  Reading of that format (the pages give no more): every element is
+ * an E2M1 code (sign, 2 exponent bits with bias 1, 1 mantissa bit; values
+ * 0, 0.5, 1, 1.5, 2, 3, 4, 6), two per byte with the even column in the low
+ * nibble; every 16 consecutive columns of a row share one E4M3 scale byte
+ * (sign, 4 exponent bits with bias 7, 3 mantissa bits, no infinities,
+ * S.1111.111 is NaN), rows of scale bytes padded to a multiple of 16 bytes;
+ * and each matrix has one float32 global scale.  The weight is
+ *   w = e2m1(code) * e4m3(scale) * global.
+ *
  * Single-threaded, plain loops, built -O2 without fast-math.
  */
 #include <math.h>
@@ -66,6 +77,50 @@ static double load(const void *p, int64_t i, int64_t dtype) {
         return (double)f;
     }
     return (double)((const float *)p)[i];
+}
+
+/* One stacked weight tensor [n_mat][rows][cols] in one of three formats. */
+typedef struct {
+    int64_t format;          /* 0 float32, 1 bf16, 2 NVFP4 */
+    const void *data;        /* elements; NVFP4: codes [n_mat][rows][cols / 2] */
+    const uint8_t *scales;   /* NVFP4: E4M3 [n_mat][rows][scale_pitch] */
+    const float *global;     /* NVFP4: [n_mat] */
+    int64_t rows, cols, scale_pitch;
+} nho_wt;
+
+/* E2M1 value of a 4-bit code, from its bit fields */
+static double e2m1_value(unsigned code) {
+    const unsigned sign = (code >> 3) & 1u, e = (code >> 1) & 3u, m = code & 1u;
+    const double mag = (e == 0) ? 0.5 * m : ldexp(1.0 + 0.5 * m, (int)e - 1);
+    return sign ? -mag : mag;
+}
+
+/* E4M3 value of a byte, from its bit fields (S.1111.111 is NaN) */
+static double e4m3_value(unsigned byte) {
+    const unsigned sign = (byte >> 7) & 1u, e = (byte >> 3) & 15u, m = byte & 7u;
+    if (e == 15u && m == 7u) return NAN;
+    const double mag = (e == 0) ? ldexp(m / 8.0, -6) : ldexp(1.0 + m / 8.0, (int)e - 7);
+    return sign ? -mag : mag;
+}
+
+/* element idx = row * cols + col of matrix `mat`, exactly as a double */
+static double wt_get(const nho_wt *w, int64_t mat, int64_t idx) {
+    const int64_t per = w->rows * w->cols;
+    if (w->format != 2) return load(w->data, mat * per + idx, w->format);
+    const int64_t r = idx / w->cols, col = idx - r * w->cols;
+    const uint8_t byte = ((const uint8_t *)w->data)[mat * per / 2 + r * (w->cols / 2) + col / 2];
+    const unsigned code = (col & 1) ? (byte >> 4) : (byte & 15u);
+    const uint8_t sb = w->scales[(mat * w->rows + r) * w->scale_pitch + col / 16];
+    return e2m1_value(code) * e4m3_value(sb) * (double)w->global[mat];
+}
+
+/* dense float64 copy of matrix `mat` of a weight tensor (for the tests' pins) */
+int nho_dequant(const nho_wt *w, int64_t mat, double *out) {
+    if (!w || !out || w->rows < 1 || w->cols < 1) return -2;
+    if (w->format == 2 && (w->cols % 2 || !w->scales || !w->global ||
+                           w->scale_pitch * 16 < w->cols)) return -2;
+    for (int64_t i = 0; i < w->rows * w->cols; ++i) out[i] = wt_get(w, mat, i);
+    return 0;
 }
 
 int nho_check_config(const nho_cfg *c) {
@@ -185,21 +240,20 @@ int nho_route(const nho_cfg *c, int64_t T, const void *x, const float *wr, const
     return NHO_OK;
 }
 
-/* out[H] += scale * Wd relu(Wu xt)^2 for one expert MLP (Wu [n][H], Wd [H][n]);
- * u is scratch of n doubles.  wd_stride is the row stride of Wd. */
-static void mlp_relu2(const nho_cfg *c, const double *xt, const void *wu, int64_t wu_off,
-                      const void *wd, int64_t wd_off, int64_t n, int64_t wd_stride,
-                      double scale, double *u, double *out) {
+/* out[H] += scale * Wd relu(Wu xt)^2 for matrix `mat` of the up tensor (rows n,
+ * cols H) and the down tensor (rows H, cols n); u is scratch of n doubles. */
+static void mlp_relu2(const nho_cfg *c, const double *xt, const nho_wt *up, const nho_wt *down,
+                      int64_t mat, int64_t n, double scale, double *u, double *out) {
     const int64_t H = c->H;
     for (int64_t i = 0; i < n; ++i) {
         double a = 0.0;
-        for (int64_t h = 0; h < H; ++h) a += load(wu, wu_off + i * H + h, c->dtype) * xt[h];
+        for (int64_t h = 0; h < H; ++h) a += wt_get(up, mat, i * H + h) * xt[h];
         double r = a > 0.0 ? a : 0.0;
         u[i] = r * r;
     }
     for (int64_t h = 0; h < H; ++h) {
         double a = 0.0;
-        for (int64_t i = 0; i < n; ++i) a += load(wd, wd_off + h * wd_stride + i, c->dtype) * u[i];
+        for (int64_t i = 0; i < n; ++i) a += wt_get(down, mat, h * down->cols + i) * u[i];
         out[h] += scale * a;
     }
 }
@@ -210,17 +264,21 @@ static void mlp_relu2(const nho_cfg *c, const double *xt, const void *wu, int64_
  *   ovr_idx/ovr_w [n_tok][k]: when non-NULL, this routing replaces the
  *     oracle's own (to check expert maths under another side's routing);
  *   idx_out/w_out [n_tok][k]: the routing used (may be NULL).
+ * up [E][I][H], down [E][H][I], su [1][S][H], sd [1][H][S] in any format.
  */
-int nho_forward(const nho_cfg *c, int64_t T, const void *x, const float *wr, const float *bias,
-                const void *w_up, const void *w_down, const void *w_su, const void *w_sd,
-                const int32_t *ovr_idx, const double *ovr_w, const int64_t *tokens,
-                int64_t n_tok, double *y, int32_t *idx_out, double *w_out) {
+int nho_forward_wt(const nho_cfg *c, int64_t T, const void *x, const float *wr, const float *bias,
+                   const nho_wt *up, const nho_wt *down, const nho_wt *su, const nho_wt *sd,
+                   const int32_t *ovr_idx, const double *ovr_w, const int64_t *tokens,
+                   int64_t n_tok, double *y, int32_t *idx_out, double *w_out) {
     int rc = nho_check_config(c);
     if (rc) return rc;
-    if (n_tok < 0 || (n_tok > 0 && (!x || !tokens || !y || !w_up || !w_down))) return NHO_BAD_ARG;
+    if (n_tok < 0 || (n_tok > 0 && (!x || !tokens || !y || !up || !down))) return NHO_BAD_ARG;
     if (!ovr_idx && !wr) return NHO_BAD_ARG;
-    if (c->n_shared && (!w_su || !w_sd)) return NHO_BAD_ARG;
+    if (c->n_shared && (!su || !sd)) return NHO_BAD_ARG;
     const int64_t H = c->H, I = c->I, S = c->S, k = c->k;
+    if (up->rows != I || up->cols != H || down->rows != H || down->cols != I) return NHO_BAD_ARG;
+    if (c->n_shared && (su->rows != S || su->cols != H || sd->rows != H || sd->cols != S))
+        return NHO_BAD_ARG;
     int64_t nmax = I > S ? I : S;
     double *xt = (double *)malloc(sizeof(double) * (size_t)H);
     double *u = (double *)malloc(sizeof(double) * (size_t)nmax);
@@ -250,11 +308,8 @@ int nho_forward(const nho_cfg *c, int64_t T, const void *x, const float *wr, con
         }
         double *yt = y + n * H;
         for (int64_t h = 0; h < H; ++h) yt[h] = 0.0;
-        for (int64_t j = 0; j < k; ++j) {
-            int64_t e = idx[j];
-            mlp_relu2(c, xt, w_up, e * I * H, w_down, e * H * I, I, I, w[j], u, yt);
-        }
-        if (c->n_shared) mlp_relu2(c, xt, w_su, 0, w_sd, 0, S, S, 1.0, u, yt);
+        for (int64_t j = 0; j < k; ++j) mlp_relu2(c, xt, up, down, idx[j], I, w[j], u, yt);
+        if (c->n_shared) mlp_relu2(c, xt, su, sd, 0, S, 1.0, u, yt);
         if (idx_out)
             for (int64_t j = 0; j < k; ++j) idx_out[n * k + j] = idx[j];
         if (w_out)
@@ -262,4 +317,22 @@ int nho_forward(const nho_cfg *c, int64_t T, const void *x, const float *wr, con
     }
     free(xt); free(u); free(scr); free(iscr); free(idx); free(w);
     return rc;
+}
+
+/* nho_forward_wt with float32 / bf16 weights given as plain arrays in c->dtype */
+int nho_forward(const nho_cfg *c, int64_t T, const void *x, const float *wr, const float *bias,
+                const void *w_up, const void *w_down, const void *w_su, const void *w_sd,
+                const int32_t *ovr_idx, const double *ovr_w, const int64_t *tokens,
+                int64_t n_tok, double *y, int32_t *idx_out, double *w_out) {
+    int rc = nho_check_config(c);
+    if (rc) return rc;
+    const nho_wt up = {c->dtype, w_up, NULL, NULL, c->I, c->H, 0};
+    const nho_wt down = {c->dtype, w_down, NULL, NULL, c->H, c->I, 0};
+    const nho_wt su = {c->dtype, w_su, NULL, NULL, c->S, c->H, 0};
+    const nho_wt sd = {c->dtype, w_sd, NULL, NULL, c->H, c->S, 0};
+    if (n_tok > 0 && (!w_up || !w_down)) return NHO_BAD_ARG;
+    if (c->n_shared && (!w_su || !w_sd)) return NHO_BAD_ARG;
+    return nho_forward_wt(c, T, x, wr, bias, &up, &down, c->n_shared ? &su : NULL,
+                          c->n_shared ? &sd : NULL, ovr_idx, ovr_w, tokens, n_tok, y, idx_out,
+                          w_out);
 }

@@ -53,6 +53,7 @@ class MoEConfig:
     norm_topk_prob: bool = True
     routed_scaling_factor: float = 2.5
     dtype: str = "bf16"          # activations and expert weights; router is fp32
+    weight_format: str = "native"  # expert / shared weights: "native" (= dtype) or "nvfp4"
     seed: int = 0
     x_std: float = 1.0
     w_std: float = 0.02
@@ -110,6 +111,10 @@ CONFIGS = {
         n_group=8, topk_group=1, num_experts_per_tok=6, moe_intermediate_size=1856,
         moe_shared_expert_intermediate_size=3712, seed=3,
         wr_std=float(1.0 / np.sqrt(2688))),
+    "decode_nvfp4_t8": MoEConfig(
+        "decode_nvfp4_t8", T=8, hidden_size=2688, n_routed_experts=128, n_group=8,
+        topk_group=1, num_experts_per_tok=6, moe_intermediate_size=1856,
+        moe_shared_expert_intermediate_size=3712, seed=5, weight_format="nvfp4"),
     "stress_bf16_t4096": MoEConfig(
         "stress_bf16_t4096", T=4096, hidden_size=4096, n_routed_experts=256, n_group=8,
         topk_group=2, num_experts_per_tok=8, moe_intermediate_size=2048,
@@ -147,6 +152,79 @@ def _store(a: np.ndarray, dtype: str) -> np.ndarray:
     return f32_to_bf16_bits(a) if dtype == "bf16" else np.ascontiguousarray(a, np.float32)
 
 
+# ---------------------------------------------------------------------------
+# NVFP4 weight encoding (input generation: the weights of an "nvfp4" workload
+# are drawn as float32, then encoded; the oracle and the CUDA library each
+# decode them with their own code)
+# ---------------------------------------------------------------------------
+_E2M1_MAG = np.array([0.0, 0.5, 1.0, 1.5, 2.0, 3.0, 4.0, 6.0])
+# decision boundaries between neighbouring magnitudes; a value on a boundary
+# goes to the magnitude with an even code (round to nearest even)
+_E2M1_EDGE = np.array([0.25, 0.75, 1.25, 1.75, 2.5, 3.5, 5.0])
+_E2M1_TIE_UP = np.array([False, True, False, True, False, True, False])
+
+
+def _e4m3_positive_table():
+    codes = np.arange(0, 0x7F, dtype=np.int64)             # 0x7F is NaN
+    e, m = codes >> 3, codes & 7
+    val = np.where(e == 0, m / 8.0 * 2.0 ** -6, (1 + m / 8.0) * 2.0 ** (e - 7))
+    return codes, val
+
+
+_E4M3_CODES, _E4M3_VALS = _e4m3_positive_table()
+
+
+def _e4m3_encode_positive(v):
+    """Nearest E4M3 code of non-negative values (ties to even code), saturating at 448."""
+    v = np.minimum(np.asarray(v, np.float64), _E4M3_VALS[-1])
+    hi = np.clip(np.searchsorted(_E4M3_VALS, v), 1, len(_E4M3_VALS) - 1)
+    lo = hi - 1
+    dlo, dhi = v - _E4M3_VALS[lo], _E4M3_VALS[hi] - v
+    pick_hi = (dhi < dlo) | ((dhi == dlo) & (_E4M3_CODES[hi] % 2 == 0))
+    return np.where(pick_hi, _E4M3_CODES[hi], _E4M3_CODES[lo]).astype(np.uint8)
+
+
+def _e2m1_encode(q):
+    a = np.abs(q)
+    idx = np.searchsorted(_E2M1_EDGE, a, side="left")      # a <= edge -> lower magnitude
+    on_edge = np.zeros(a.shape, bool)
+    for i, edge in enumerate(_E2M1_EDGE):
+        on_edge |= (a == edge) & _E2M1_TIE_UP[i] & (idx == i)
+    idx = np.minimum(idx + on_edge, 7)
+    sign = (q < 0) & (idx > 0)
+    return (idx | (sign.astype(np.int64) << 3)).astype(np.uint8)
+
+
+def nvfp4_scale_pitch(cols: int) -> int:
+    """Bytes per row of scale factors: one per 16 columns, padded to 16 bytes."""
+    return ((cols // 16 + 15) // 16) * 16
+
+
+def quantize_nvfp4(w: np.ndarray):
+    """Encode float weights [n_mat, rows, cols] (cols % 16 == 0) as NVFP4.
+
+    Returns (codes uint8 [n_mat, rows, cols/2], scales uint8 [n_mat, rows,
+    pitch], global float32 [n_mat]): per matrix a global scale amax/(6*448),
+    per 16 columns an E4M3 scale nearest to block_amax/6/global, per element
+    the E2M1 code nearest to w / (scale * global) (ties to even)."""
+    w = np.asarray(w, np.float32)
+    n, r, c = w.shape
+    assert c % 16 == 0
+    amax = np.abs(w).reshape(n, -1).max(axis=1).astype(np.float64)
+    g = np.where(amax > 0, amax / (6.0 * 448.0), 1.0).astype(np.float32)
+    blocks = w.reshape(n, r, c // 16, 16).astype(np.float64)
+    bmax = np.abs(blocks).max(axis=-1)
+    scode = _e4m3_encode_positive(bmax / 6.0 / g[:, None, None].astype(np.float64))
+    sval = _E4M3_VALS[scode.astype(np.int64)] * g[:, None, None].astype(np.float64)
+    q = np.where(sval[..., None] > 0, blocks / np.where(sval > 0, sval, 1.0)[..., None], 0.0)
+    codes = _e2m1_encode(q).reshape(n, r, c)
+    packed = (codes[..., 0::2] | (codes[..., 1::2] << 4)).astype(np.uint8)
+    pitch = nvfp4_scale_pitch(c)
+    scales = np.zeros((n, r, pitch), np.uint8)
+    scales[..., : c // 16] = scode
+    return packed, scales, g
+
+
 @dataclasses.dataclass
 class MoEInputs:
     """Host arrays of one workload.  bf16 tensors are uint16 bit patterns.
@@ -167,6 +245,9 @@ class MoEInputs:
     tie_tokens: Optional[np.ndarray] = None
     tie_cols: Optional[np.ndarray] = None
     skew_b: Optional[float] = None
+    # NVFP4 workloads: {"up", "down", "shared_up", "shared_down"} ->
+    # (codes, scales, global) as returned by quantize_nvfp4
+    nvfp4: Optional[dict] = None
 
 
 def default_threads() -> int:
@@ -222,6 +303,8 @@ def make_inputs(cfg: MoEConfig, skew_b: Optional[float] = None,
                 threads: Optional[int] = None, with_bias: bool = False) -> MoEInputs:
     """All inputs of a workload (expert weights drawn in parallel threads)."""
     x, wr, hot, ties, tcols = make_router_and_x(cfg, skew_b)
+    if cfg.weight_format == "nvfp4":
+        return _make_nvfp4_inputs(cfg, x, wr, hot, ties, tcols, skew_b, threads, with_bias)
     sdt = np.uint16 if cfg.dtype == "bf16" else np.float32
     w_up = np.empty((cfg.E, cfg.I, cfg.H), sdt)
     w_down = np.empty((cfg.E, cfg.H, cfg.I), sdt)
@@ -239,6 +322,31 @@ def make_inputs(cfg: MoEConfig, skew_b: Optional[float] = None,
     if with_bias:
         bias = _normal(cfg.seed, _BIAS, 0, (cfg.E,), 0.1).astype(np.float32)
     return MoEInputs(cfg, x, wr, w_up, w_down, wsu, wsd, bias, hot, ties, tcols, skew_b)
+
+
+def _make_nvfp4_inputs(cfg, x, wr, hot, ties, tcols, skew_b, threads, with_bias):
+    """Weights drawn as float32 (same streams as the native format) and encoded
+    as NVFP4, one matrix per thread task."""
+    E, H, I, S = cfg.E, cfg.H, cfg.I, cfg.S
+    pu, pd = nvfp4_scale_pitch(H), nvfp4_scale_pitch(I)
+    up = (np.empty((E, I, H // 2), np.uint8), np.empty((E, I, pu), np.uint8), np.empty(E, np.float32))
+    dn = (np.empty((E, H, I // 2), np.uint8), np.empty((E, H, pd), np.uint8), np.empty(E, np.float32))
+
+    def fill(e):
+        u = _normal(cfg.seed, _WUP, e, (I, H), cfg.w_std)
+        d = _normal(cfg.seed, _WDOWN, e, (H, I), cfg.w_std)
+        for dst, w in ((up, u), (dn, d)):
+            c, sc, g = quantize_nvfp4(w[None])
+            dst[0][e], dst[1][e], dst[2][e] = c[0], sc[0], g[0]
+
+    with ThreadPoolExecutor(threads or default_threads()) as ex:
+        list(ex.map(fill, range(E)))
+    q = {"up": up, "down": dn}
+    if cfg.n_shared_experts:
+        q["shared_up"] = quantize_nvfp4(_normal(cfg.seed, _WSU, 0, (S, H), cfg.w_std)[None])
+        q["shared_down"] = quantize_nvfp4(_normal(cfg.seed, _WSD, 0, (H, S), cfg.w_std)[None])
+    bias = _normal(cfg.seed, _BIAS, 0, (E,), 0.1).astype(np.float32) if with_bias else None
+    return MoEInputs(cfg, x, wr, None, None, None, None, bias, hot, ties, tcols, skew_b, q)
 
 
 def to_f64(a: np.ndarray, dtype: str) -> np.ndarray:

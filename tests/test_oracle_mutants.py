@@ -21,12 +21,18 @@ MUTANTS = {
     "relu_not_squared": ("u[i] = r * r;", "u[i] = r;"),
     "relu_dropped": ("double r = a > 0.0 ? a : 0.0;", "double r = a;"),
     "shared_dropped": ("if (c->n_shared) mlp_relu2", "if (0) mlp_relu2"),
+    "e2m1_mantissa_weight": ("1.0 + 0.5 * m, (int)e - 1", "1.0 + 0.25 * m, (int)e - 1"),
+    "e2m1_subnormal_wrong": ("(e == 0) ? 0.5 * m :", "(e == 0) ? 1.0 * m :"),
+    "e4m3_bias_off_by_one": ("ldexp(1.0 + m / 8.0, (int)e - 7)", "ldexp(1.0 + m / 8.0, (int)e - 8)"),
+    "nvfp4_nibble_order": ("(col & 1) ? (byte >> 4) : (byte & 15u)", "(col & 1) ? (byte & 15u) : (byte >> 4)"),
+    "nvfp4_scale_group_of_8": ("* w->scale_pitch + col / 16]", "* w->scale_pitch + col / 8]"),
+    "nvfp4_global_ignored": ("* (double)w->global[mat];", ";"),
     "norm_ignored": ("w[j] = c->norm ? c->alpha * s[cand[j]] / sum : c->alpha * s[cand[j]];",
                      "w[j] = c->alpha * s[cand[j]];"),
     "alpha_dropped": ("w[j] = c->norm ? c->alpha * s[cand[j]] / sum : c->alpha * s[cand[j]];",
                       "w[j] = c->norm ? s[cand[j]] / sum : s[cand[j]];"),
-    "down_transposed": ("load(wd, wd_off + h * wd_stride + i, c->dtype)",
-                        "load(wd, wd_off + i * c->H + h, c->dtype)"),
+    "down_transposed": ("wt_get(down, mat, h * down->cols + i)",
+                        "wt_get(down, mat, i * down->rows + h)"),
     "weights_from_biased_score": ("for (int64_t j = 0; j < c->k; ++j) sum += s[cand[j]];",
                                   "for (int64_t j = 0; j < c->k; ++j) sum += sel[cand[j]];"),
     "norm_over_k_minus_1": ("for (int64_t j = 0; j < c->k; ++j) sum += s[cand[j]];",
@@ -34,7 +40,8 @@ MUTANTS = {
     "bf16_widen_wrong_shift": ("<< 16;", "<< 15;"),
 }
 
-PINS = ["tests/test_oracle_route.py", "tests/test_oracle_forward.py"]
+PINS = ["tests/test_oracle_route.py", "tests/test_oracle_forward.py",
+        "tests/test_oracle_nvfp4.py"]
 
 
 @pytest.mark.parametrize("name", sorted(MUTANTS))
