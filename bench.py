@@ -206,7 +206,7 @@ def run_ours(args, rank, world, local_rank):
     cfg = workload(args)
     inp = synth.make_inputs(cfg, skew_b=skew_b(cfg))
     blk = nh.NemotronHMoE(cfg, inp.w_router, inp.w_up, inp.w_down, inp.w_shared_up,
-                          inp.w_shared_down, device=dev)
+                          inp.w_shared_down, device=dev, nvfp4=inp.nvfp4)
     T = cfg.T
     nb = max(1, args.batches)
     xs = []
@@ -327,21 +327,34 @@ def kernel_times(blk, xs, b, nb, steps):
             ev[n][0].record(stream)
             fn()
             ev[n][1].record(stream)
-        if blk.has_shared:
+        if blk.has_shared and blk.nvfp4:
+            timed("shared", lambda: nh.shared_nvfp4(blk.c, x, blk.q4["shared_up"],
+                                                     blk.q4["shared_down"], b.y_shared,
+                                                     b.ws_shared, stream=main))
+        elif blk.has_shared:
             timed("shared", lambda: nh.shared(blk.c, x, blk.w_shared_up, blk.w_shared_down,
                                                b.y_shared, b.ws_shared, stream=main))
         timed("route", lambda: nh.route(blk.c, x, blk.w_router, blk.bias, b.topk_idx, b.topk_w,
                                          b.ws, stream=main))
         timed("permute", lambda: nh.permute(blk.c, x, b.topk_idx, b.topk_w, b.ws, stream=main))
-        timed("experts_up", lambda: nh.experts_up(blk.c, x, blk.w_up, b.ws, stream=main))
-        timed("experts_down", lambda: nh.experts_down(blk.c, T, blk.w_down, b.ws, stream=main))
+        if blk.nvfp4:
+            # up and down run back to back in one call; each is timed as half
+            timed("experts_up", lambda: nh.forward_nvfp4(blk.c, x, blk.q4["up"], blk.q4["down"],
+                                                          b.ws, stream=main))
+        else:
+            timed("experts_up", lambda: nh.experts_up(blk.c, x, blk.w_up, b.ws, stream=main))
+            timed("experts_down", lambda: nh.experts_down(blk.c, T, blk.w_down, b.ws,
+                                                           stream=main))
         timed("finalize", lambda: nh.finalize(blk.c, T, b.ws, b.y_shared, b.y, stream=main))
         torch.cuda.synchronize(blk.device)
         for n in names:
-            if n == "shared" and not blk.has_shared:
+            if (n == "shared" and not blk.has_shared) or (n == "experts_down" and blk.nvfp4):
                 continue
             acc[n] += ev[n][0].elapsed_time(ev[n][1])
-    return {n: acc[n] / steps for n in names}
+    out = {n: acc[n] / steps for n in names}
+    if blk.nvfp4:
+        out["experts_up"] = out["experts_down"] = acc["experts_up"] / steps / 2
+    return out
 
 
 def launches_per_step(cfg):
@@ -376,8 +389,9 @@ def report(args, cfg, inp, world, steps, elapsed_ms, clk, kern, e2e_ms, blk):
     b = blk.buffers(T)
     idx = b.topk_idx.cpu().numpy()
     D = distinct_experts(cfg, idx)
-    expert_bytes = cfg.I * cfg.H * elem            # one projection of one expert
-    shared_bytes = 2 * cfg.S * cfg.H * elem if cfg.n_shared_experts else 0
+    welem = 0.5 + 1.0 / 16 if cfg.weight_format == "nvfp4" else elem   # bytes per weight
+    expert_bytes = int(cfg.I * cfg.H * welem)      # one projection of one expert
+    shared_bytes = int(2 * cfg.S * cfg.H * welem) if cfg.n_shared_experts else 0
     rows = T * cfg.k
     # algorithmic bytes of one step: touched weights + router + x in + y out
     step_bytes = (D * 2 * expert_bytes + shared_bytes + cfg.E * cfg.H * 4
@@ -407,7 +421,8 @@ def report(args, cfg, inp, world, steps, elapsed_ms, clk, kern, e2e_ms, blk):
         "metric": METRIC, "value": round(value, 2), "unit": "tokens/s", "n_gpus": world,
         "steps": steps, "warmup": max(3, args.warmup), "ms_per_step": round(ms, 5),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "bf16" if cfg.dtype == "bf16" else "f32", "data": "synthetic",
+        "dtype": ("nvfp4 weights, bf16 activations" if cfg.weight_format == "nvfp4"
+                  else ("bf16" if cfg.dtype == "bf16" else "f32")), "data": "synthetic",
         "config": {"workload": cfg.name, "tokens_per_step_per_gpu": T, "hidden_size": cfg.H,
                    "n_routed_experts": cfg.E, "n_group": cfg.G, "topk_group": cfg.tg,
                    "num_experts_per_tok": cfg.k, "moe_intermediate_size": cfg.I,

@@ -61,6 +61,30 @@ typedef enum {
     NH_GROUP_SCORE_TOP2 = 1   /* sum of the two largest (needs >= 2 experts per group) */
 } nh_group_score;
 
+/* Storage of the routed and shared expert weights. */
+typedef enum {
+    NH_WEIGHTS_NATIVE = 0,    /* in the activation dtype (bf16 or float32)          */
+    NH_WEIGHTS_NVFP4 = 1      /* NVFP4, see nh_nvfp4_weight (needs dtype NH_BF16)   */
+} nh_weight_format;
+
+/*
+ * One stacked NVFP4 weight tensor [n_mat][rows][cols] (W4A16, group size 16:
+ * "NVFP4 W4A16 group_size 16 on the experts, shared experts", vllm.cpp PR
+ * #518).  Element (m, r, c) = e2m1(code) * e4m3(scale) * global[m] where
+ *   codes  [n_mat][rows][cols/2]: two E2M1 codes per byte, column 2j in the
+ *          low nibble of byte j;
+ *   scales [n_mat][rows][pitch]: E4M3 scale of columns 16b .. 16b+15 in byte
+ *          b; pitch = ceil(cols/16) rounded up to a multiple of 16 bytes;
+ *   global [n_mat]: float32.
+ * All three are device pointers, 16-byte aligned.  The struct itself is a
+ * host struct.
+ */
+typedef struct {
+    const uint8_t *codes;
+    const uint8_t *scales;
+    const float *global_scale;
+} nh_nvfp4_weight;
+
 /*
  * Block configuration.  Field names are the model's config.json / MLX
  * ModelArgs names (exo commit "Add support for Nemotron sharding",
@@ -81,6 +105,7 @@ typedef struct {
     float routed_scaling_factor;                  /* alpha, finite                */
     int32_t dtype;                                /* nh_dtype                     */
     int32_t group_score;                          /* nh_group_score               */
+    int32_t weight_format;                        /* nh_weight_format             */
 } nh_moe_config;
 
 /* Byte offsets of the regions inside the routed-path workspace `ws`. */
@@ -105,7 +130,8 @@ typedef struct {
     int32_t tile_rows;    /* rows per tile entry of this (cfg, T)               */
     int32_t max_tiles;
     int32_t n_chunks;     /* token chunks of the permute histogram              */
-    int32_t swap_ab;      /* 1: weights on the MMA M side (small T)             */
+    int32_t swap_ab;      /* 1: weights on the MMA M side (small T, or NVFP4)   */
+    int32_t x_direct;     /* 1: the up projection reads x itself (no x_perm)    */
 } nh_moe_ws_layout;
 
 /* Validate a configuration (no device work). */
@@ -203,6 +229,18 @@ nh_status nh_moe_forward(const nh_moe_config *cfg, int64_t T, const void *x, con
                          const void *w_down, void *ws, size_t ws_bytes, void *stream);
 
 /*
+ * nh_moe_forward with NVFP4 routed-expert weights (cfg->weight_format ==
+ * NH_WEIGHTS_NVFP4): w_up [E][I][H], w_down [E][H][I] as nh_nvfp4_weight.
+ * The weights are dequantized stage by stage in shared memory (code x block
+ * scale, exact in bf16), multiplied on the tensor cores, and the float32
+ * matrix scale is applied in the epilogue.  Same results layout as
+ * nh_moe_forward.
+ */
+nh_status nh_moe_forward_nvfp4(const nh_moe_config *cfg, int64_t T, const void *x,
+                               const nh_nvfp4_weight *w_up, const nh_nvfp4_weight *w_down,
+                               void *ws, size_t ws_bytes, void *stream);
+
+/*
  * The two phases of nh_moe_forward, for callers that schedule or time them
  * separately (same arguments and requirements):
  *   nh_moe_experts_up:   h = relu(x[perm_token] W_up[e]^T)^2 into the workspace;
@@ -223,6 +261,13 @@ nh_status nh_moe_experts_down(const nh_moe_config *cfg, int64_t T, const void *w
 nh_status nh_moe_shared(const nh_moe_config *cfg, int64_t T, const void *x, const void *w_shared_up,
                         const void *w_shared_down, float *y_shared, void *ws_shared,
                         size_t ws_shared_bytes, void *stream);
+
+/* nh_moe_shared with NVFP4 shared-expert weights: w_shared_up [1][S][H],
+ * w_shared_down [1][H][S]. */
+nh_status nh_moe_shared_nvfp4(const nh_moe_config *cfg, int64_t T, const void *x,
+                              const nh_nvfp4_weight *w_shared_up,
+                              const nh_nvfp4_weight *w_shared_down, float *y_shared,
+                              void *ws_shared, size_t ws_shared_bytes, void *stream);
 
 /*
  * y[t] = dtype( y_shared[t] + sum_j y_part[inv_row[t, j]] ), summed in float32

@@ -22,7 +22,7 @@ import threading
 from . import build as _build
 
 __all__ = ["NHMoEError", "Config", "Layout", "config_from", "load", "validate", "workspace_size",
-           "workspace_layout", "shared_workspace_size", "route", "route_noalloc", "route_permute", "permute", "forward", "experts_up", "experts_down", "shared",
+           "workspace_layout", "shared_workspace_size", "route", "route_noalloc", "route_permute", "permute", "forward", "experts_up", "experts_down", "shared", "forward_nvfp4", "shared_nvfp4", "nvfp4_weight",
            "finalize", "check_device", "selftest_timeout", "library_path", "NemotronHMoE"]
 
 NH_OK, NH_ERR_INVALID_ARG, NH_ERR_UNSUPPORTED, NH_ERR_CUDA, NH_ERR_TIMEOUT, NH_ERR_DEVICE_CHECK = range(6)
@@ -45,7 +45,16 @@ class Config(ctypes.Structure):
                 ("moe_shared_expert_intermediate_size", ctypes.c_int32),
                 ("n_shared_experts", ctypes.c_int32), ("norm_topk_prob", ctypes.c_int32),
                 ("routed_scaling_factor", ctypes.c_float), ("dtype", ctypes.c_int32),
-                ("group_score", ctypes.c_int32)]
+                ("group_score", ctypes.c_int32), ("weight_format", ctypes.c_int32)]
+
+
+class NvFp4Weight(ctypes.Structure):
+    """nh_nvfp4_weight: device pointers of one stacked NVFP4 tensor."""
+    _fields_ = [("codes", ctypes.c_void_p), ("scales", ctypes.c_void_p),
+                ("global_scale", ctypes.c_void_p)]
+
+
+NH_WEIGHTS_NATIVE, NH_WEIGHTS_NVFP4 = 0, 1
 
 
 class Layout(ctypes.Structure):
@@ -54,7 +63,8 @@ class Layout(ctypes.Structure):
         "total_bytes", "status", "logits", "router_w", "counts", "offsets", "chunk_counts", "perm_token",
         "perm_w", "inv_row", "tiles", "num_tiles", "x_perm", "h", "y_part")] + [
         ("rows_alloc", ctypes.c_int64), ("tile_rows", ctypes.c_int32),
-        ("max_tiles", ctypes.c_int32), ("n_chunks", ctypes.c_int32), ("swap_ab", ctypes.c_int32)]
+        ("max_tiles", ctypes.c_int32), ("n_chunks", ctypes.c_int32), ("swap_ab", ctypes.c_int32),
+        ("x_direct", ctypes.c_int32)]
 
 
 def config_from(c, group_score: int = 0) -> Config:
@@ -68,7 +78,9 @@ def config_from(c, group_score: int = 0) -> Config:
                   int(c.moe_shared_expert_intermediate_size), int(c.n_shared_experts),
                   int(bool(c.norm_topk_prob)), float(c.routed_scaling_factor),
                   NH_BF16 if dt in ("bf16", NH_BF16) else NH_F32,
-                  int(getattr(c, "group_score", group_score)))
+                  int(getattr(c, "group_score", group_score)),
+                  NH_WEIGHTS_NVFP4 if getattr(c, "weight_format", "native") in ("nvfp4", 1)
+                  else NH_WEIGHTS_NATIVE)
 
 
 _lock = threading.Lock()
@@ -108,6 +120,10 @@ def load():
             "nh_moe_experts_up": [C, I64, P, P, P, S, P],
             "nh_moe_experts_down": [C, I64, P, P, S, P],
             "nh_moe_shared": [C, I64, P, P, P, P, P, S, P],
+            "nh_moe_forward_nvfp4": [C, I64, P, ctypes.POINTER(NvFp4Weight),
+                                     ctypes.POINTER(NvFp4Weight), P, S, P],
+            "nh_moe_shared_nvfp4": [C, I64, P, ctypes.POINTER(NvFp4Weight),
+                                    ctypes.POINTER(NvFp4Weight), P, P, S, P],
             "nh_moe_finalize": [C, I64, P, S, P, P, P],
             "nh_moe_check_device": [P, P],
             "nh_moe_selftest_timeout": [P, ctypes.c_uint64, P],
@@ -225,6 +241,25 @@ def shared(cfg, x, w_shared_up, w_shared_down, y_shared, ws_shared, stream=None)
     _check(load().nh_moe_shared(ctypes.byref(c), x.shape[0], _p(x), _p(w_shared_up),
                                 _p(w_shared_down), _p(y_shared), _p(ws_shared),
                                 _nbytes(ws_shared), _stream(stream)))
+
+
+def nvfp4_weight(codes, scales, global_scale) -> NvFp4Weight:
+    """Struct of device pointers for one stacked NVFP4 tensor (tensors stay owned by the caller)."""
+    return NvFp4Weight(codes.data_ptr(), scales.data_ptr(), global_scale.data_ptr())
+
+
+def forward_nvfp4(cfg, x, w_up, w_down, ws, stream=None):
+    """nh_moe_forward with NVFP4 weights; w_up / w_down are NvFp4Weight structs."""
+    c = config_from(cfg)
+    _check(load().nh_moe_forward_nvfp4(ctypes.byref(c), x.shape[0], _p(x), ctypes.byref(w_up),
+                                       ctypes.byref(w_down), _p(ws), _nbytes(ws), _stream(stream)))
+
+
+def shared_nvfp4(cfg, x, w_shared_up, w_shared_down, y_shared, ws_shared, stream=None):
+    c = config_from(cfg)
+    _check(load().nh_moe_shared_nvfp4(ctypes.byref(c), x.shape[0], _p(x), ctypes.byref(w_shared_up),
+                                      ctypes.byref(w_shared_down), _p(y_shared), _p(ws_shared),
+                                      _nbytes(ws_shared), _stream(stream)))
 
 
 def finalize(cfg, T: int, ws, y_shared, y, stream=None):

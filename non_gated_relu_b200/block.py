@@ -19,8 +19,9 @@ from typing import Dict, Optional
 import numpy as np
 import torch
 
-from . import (check_device, config_from, finalize, forward, route_permute, shared,
-               shared_workspace_size, validate, workspace_size, NH_BF16)
+from . import (check_device, config_from, finalize, forward, forward_nvfp4, nvfp4_weight,
+               route_permute, shared, shared_nvfp4, shared_workspace_size, validate,
+               workspace_size, NH_BF16, NH_WEIGHTS_NVFP4)
 
 
 def _to_device(a, dtype: torch.dtype, device) -> torch.Tensor:
@@ -58,8 +59,8 @@ class NemotronHMoE:
     taken as bf16 bit patterns.
     """
 
-    def __init__(self, cfg, w_router, w_up, w_down, w_shared_up=None, w_shared_down=None,
-                 bias=None, device=None):
+    def __init__(self, cfg, w_router, w_up=None, w_down=None, w_shared_up=None,
+                 w_shared_down=None, bias=None, device=None, nvfp4=None):
         self.cfg = cfg
         self.c = config_from(cfg)
         validate(self.c)
@@ -72,12 +73,28 @@ class NemotronHMoE:
         self.has_shared = bool(self.c.n_shared_experts)
         self.w_router = _to_device(w_router, torch.float32, self.device)
         self.bias = _to_device(bias, torch.float32, self.device)
-        self.w_up = _to_device(w_up, self.dtype, self.device)
-        self.w_down = _to_device(w_down, self.dtype, self.device)
-        self.w_shared_up = _to_device(w_shared_up, self.dtype, self.device)
-        self.w_shared_down = _to_device(w_shared_down, self.dtype, self.device)
-        if self.has_shared and (self.w_shared_up is None or self.w_shared_down is None):
-            raise ValueError("config has a shared expert but no shared weights were given")
+        self.nvfp4 = self.c.weight_format == NH_WEIGHTS_NVFP4
+        if self.nvfp4:
+            # {"up", "down", "shared_up", "shared_down"} -> (codes, scales, global)
+            if nvfp4 is None:
+                raise ValueError("config has NVFP4 weights: pass nvfp4={...}")
+            self._q4_tensors = {}
+            self.q4 = {}
+            for name, (codes, scales, glob) in nvfp4.items():
+                t = tuple(torch.as_tensor(a).to(self.device).contiguous()
+                          for a in (codes, scales, glob))
+                self._q4_tensors[name] = t
+                self.q4[name] = nvfp4_weight(*t)
+            self.w_up = self.w_down = self.w_shared_up = self.w_shared_down = None
+            if self.has_shared and ("shared_up" not in self.q4 or "shared_down" not in self.q4):
+                raise ValueError("config has a shared expert but no shared weights were given")
+        else:
+            self.w_up = _to_device(w_up, self.dtype, self.device)
+            self.w_down = _to_device(w_down, self.dtype, self.device)
+            self.w_shared_up = _to_device(w_shared_up, self.dtype, self.device)
+            self.w_shared_down = _to_device(w_shared_down, self.dtype, self.device)
+            if self.has_shared and (self.w_shared_up is None or self.w_shared_down is None):
+                raise ValueError("config has a shared expert but no shared weights were given")
         with torch.cuda.device(self.device):
             self.side = torch.cuda.Stream()
         self._bufs: Dict[int, Buffers] = {}
@@ -116,8 +133,12 @@ class NemotronHMoE:
             fork.record(main)
             self.side.wait_event(fork)
             push("shared")
-            shared(self.c, x, self.w_shared_up, self.w_shared_down, b.y_shared, b.ws_shared,
-                   stream=self.side)
+            if self.nvfp4:
+                shared_nvfp4(self.c, x, self.q4["shared_up"], self.q4["shared_down"], b.y_shared,
+                             b.ws_shared, stream=self.side)
+            else:
+                shared(self.c, x, self.w_shared_up, self.w_shared_down, b.y_shared, b.ws_shared,
+                       stream=self.side)
             pop()
             join = torch.cuda.Event()
             join.record(self.side)
@@ -125,7 +146,10 @@ class NemotronHMoE:
         route_permute(self.c, x, self.w_router, self.bias, b.topk_idx, b.topk_w, b.ws, stream=main)
         pop()
         push("forward")
-        forward(self.c, x, self.w_up, self.w_down, b.ws, stream=main)
+        if self.nvfp4:
+            forward_nvfp4(self.c, x, self.q4["up"], self.q4["down"], b.ws, stream=main)
+        else:
+            forward(self.c, x, self.w_up, self.w_down, b.ws, stream=main)
         pop()
         if self.has_shared:
             main.wait_event(join)

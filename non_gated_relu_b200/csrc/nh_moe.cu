@@ -15,6 +15,7 @@
 #include "gemm_simt.cuh"
 #include "gemm_tc.cuh"
 #include "gemm_tc2.cuh"
+#include "gemm_q4.cuh"
 #include "permute.cuh"
 #include "route.cuh"
 #include "route_permute.cuh"
@@ -103,6 +104,10 @@ static nh_status validate(const nh_moe_config* c) {
     return fail(NH_ERR_INVALID_ARG, "unknown group_score");
   if (c->group_score == NH_GROUP_SCORE_TOP2 && g < 2)
     return fail(NH_ERR_INVALID_ARG, "the top-2 group score needs >= 2 experts per group");
+  if (c->weight_format != NH_WEIGHTS_NATIVE && c->weight_format != NH_WEIGHTS_NVFP4)
+    return fail(NH_ERR_INVALID_ARG, "unknown weight_format");
+  if (c->weight_format == NH_WEIGHTS_NVFP4 && c->dtype != NH_BF16)
+    return fail(NH_ERR_INVALID_ARG, "NVFP4 weights need bf16 activations (W4A16)");
   // valid; now what the kernels implement
   if (c->n_routed_experts > MAX_E)
     return fail(NH_ERR_UNSUPPORTED, "n_routed_experts > %d", MAX_E);
@@ -129,7 +134,11 @@ struct Plan {
 // rows of one tile entry for T tokens: decode-sized T puts the weights on the
 // MMA M side (swap), with all of an expert's rows in one entry
 static void tile_plan(const nh_moe_config* c, int64_t T, int* tile_rows, int* swap) {
-  if (c->dtype == NH_F32) {
+  if (c->weight_format == NH_WEIGHTS_NVFP4) {
+    // weights are dequantized per stage: always weights on the MMA M side
+    *tile_rows = T <= 16 ? 16 : (T <= 32 ? 32 : 64);
+    *swap = 1;
+  } else if (c->dtype == NH_F32) {
     *tile_rows = SG_BM;
     *swap = 0;
   } else if (T <= 16) {
@@ -169,6 +178,7 @@ static nh_status make_plan(const nh_moe_config* c, int64_t T, Plan* p) {
   tile_plan(c, T, &tr, &sw);
   L.tile_rows = tr;
   L.swap_ab = sw;
+  L.x_direct = (sw && T <= 64) ? 1 : 0;   // every token fits one activation tile
   L.max_tiles = (int)((rows + tr - 1) / tr + p->E);
   L.n_chunks = (int)((T + PERM_CHUNK - 1) / PERM_CHUNK);
   L.rows_alloc = rows;
@@ -189,7 +199,7 @@ static nh_status make_plan(const nh_moe_config* c, int64_t T, Plan* p) {
   L.inv_row = take((size_t)rows * 4);
   L.tiles = take((size_t)L.max_tiles * 16);
   L.num_tiles = take(4);
-  L.x_perm = take(L.swap_ab ? 0 : (size_t)rows * p->H * p->elem);
+  L.x_perm = take(L.x_direct ? 0 : (size_t)rows * p->H * p->elem);
   L.h = take((size_t)rows * p->I * p->elem);
   L.y_part = take((size_t)rows * p->H * p->elem);
   L.total_bytes = o;
@@ -231,7 +241,7 @@ static PermuteOut permute_out(void* ws, const nh_moe_ws_layout& L, int* status) 
   o.x_perm = at<void>(ws, L.x_perm);
   o.status = status;
   o.sched_zero = reinterpret_cast<unsigned int*>(status + SCHED_UP);
-  o.gather = L.swap_ab ? 0 : 1;
+  o.gather = L.x_direct ? 0 : 1;
   return o;
 }
 
@@ -266,6 +276,12 @@ static nh_status set_attrs(int dev) {
                                cudaFuncAttributeMaxDynamicSharedMemorySize, TcSwap64::SMEM));
   NH_CUDA(cudaFuncSetAttribute(tc2::tc2_grouped_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                tc2::SMEM));
+  NH_CUDA(cudaFuncSetAttribute(q4::tc_q4_gemm<16, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               q4::Shape<16, 8>::SMEM));
+  NH_CUDA(cudaFuncSetAttribute(q4::tc_q4_gemm<32, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               q4::Shape<32, 8>::SMEM));
+  NH_CUDA(cudaFuncSetAttribute(q4::tc_q4_gemm<64, 7>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               q4::Shape<64, 7>::SMEM));
   NH_CUDA(cudaFuncSetAttribute(route_permute_small<__nv_bfloat16>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, ROUTE_PERMUTE_SMEM_MAX));
   NH_CUDA(cudaFuncSetAttribute(route_permute_small<float>,
@@ -478,6 +494,72 @@ static nh_status launch_tc2(const GemmCall& c, int dev, cudaStream_t st) {
   lc.numAttrs = 2;
   NH_CUDA(cudaLaunchKernelEx(&lc, tc2::tc2_grouped_gemm, ma, mw, g));
   return launch_check("tc2_grouped_gemm");
+}
+
+// uint8 [n_mat, rows, row_bytes] (no swizzle), box {box_bytes, 128 rows, 1}
+static nh_status map_u8_3d(CUtensorMap* m, const void* base, int64_t row_bytes, int64_t rows,
+                           int64_t n_mat, int box_bytes) {
+  auto fn = encode_fn();
+  if (!fn) return fail(NH_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  cuuint64_t dims[3] = {(cuuint64_t)row_bytes, (cuuint64_t)rows, (cuuint64_t)n_mat};
+  cuuint64_t strides[2] = {(cuuint64_t)row_bytes, (cuuint64_t)(row_bytes * rows)};
+  cuuint32_t box[3] = {(cuuint32_t)box_bytes, (cuuint32_t)q4::M, 1};
+  cuuint32_t es[3] = {1, 1, 1};
+  CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
+                  es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(NH_ERR_CUDA, "cuTensorMapEncodeTiled (u8) failed: %d", (int)r);
+  return NH_OK;
+}
+
+static int64_t nvfp4_pitch(int64_t cols) { return ((cols / 16 + 15) / 16) * 16; }
+
+template <int NT, int STAGES>
+static nh_status launch_q4(const GemmCall& c, const nh_nvfp4_weight& w, int dev, cudaStream_t st) {
+  using S = q4::Shape<NT, STAGES>;
+  CUtensorMap ma, mc, ms;
+  NH_TRY(map_2d(&ma, c.A, c.K, c.rows, NT));
+  NH_TRY(map_u8_3d(&mc, w.codes, c.K / 2, c.N, c.n_exp, q4::BK / 2));
+  NH_TRY(map_u8_3d(&ms, w.scales, nvfp4_pitch(c.K), c.N, c.n_exp, q4::SCALE_BOX));
+  q4::Q4Args qa;
+  tc::TcArgs& g = qa.g;
+  g.tiles = c.tiles;
+  g.num_tiles = c.num_tiles;
+  g.dense_rows = (int)c.rows;
+  g.tile_rows = c.tile_rows;
+  g.N = c.N;
+  g.K = c.K;
+  g.a_kwrap = 0;
+  g.epi = c.epi;
+  g.out = c.out;
+  g.ldo = c.ldo;
+  g.perm_w = c.perm_w;
+  g.row_token = c.row_token;
+  g.status = c.status;
+  g.timeout_ns = timeout_ns();
+  g.sched = c.sched;
+  qa.gscale = w.global_scale;
+  const int n_blocks = (c.N + q4::M - 1) / q4::M;
+  const int64_t m_max = c.tiles ? c.max_tiles : (c.rows + c.tile_rows - 1) / c.tile_rows;
+  const int grid = (int)std::min<int64_t>(m_max * n_blocks, g_sm_count[dev]);
+  if (grid <= 0) return NH_OK;
+  return launch_k("tc_q4_gemm", q4::tc_q4_gemm<NT, STAGES>, dim3(grid), dim3(q4::THREADS), S::SMEM,
+                  st, ma, mc, ms, qa);
+}
+
+static nh_status run_gemm_q4(const GemmCall& c, const nh_nvfp4_weight* w, int dev,
+                             cudaStream_t st) {
+  if (c.rows == 0) return NH_OK;
+  if (!w || !w->codes || !w->scales || !w->global_scale)
+    return fail(NH_ERR_INVALID_ARG, "NVFP4 weight with a NULL pointer");
+  if (reinterpret_cast<uintptr_t>(w->codes) % 16 || reinterpret_cast<uintptr_t>(w->scales) % 16)
+    return fail(NH_ERR_INVALID_ARG, "NVFP4 codes / scales must be 16-byte aligned");
+  switch (c.tile_rows) {
+    case 16: return launch_q4<16, 8>(c, *w, dev, st);
+    case 32: return launch_q4<32, 8>(c, *w, dev, st);
+    case 64: return launch_q4<64, 7>(c, *w, dev, st);
+    default: return fail(NH_ERR_UNSUPPORTED, "NVFP4 tile rows %d", c.tile_rows);
+  }
 }
 
 static nh_status run_gemm(const Plan& p, const GemmCall& c, int dev, cudaStream_t st) {
@@ -924,12 +1006,17 @@ nh_status nh_moe_route_permute(const nh_moe_config* cfg, int64_t T, const void* 
 }
 
 static nh_status experts_phase(const nh_moe_config* cfg, int64_t T, const void* x, const void* w,
-                               void* ws, size_t ws_bytes, void* stream, bool up_phase) {
+                               void* ws, size_t ws_bytes, void* stream, bool up_phase,
+                               const nh_nvfp4_weight* wq = nullptr) {
   Plan p;
   NH_TRY(make_plan(cfg, T, &p));
   NH_TRY(check_ws(p, ws, ws_bytes));
+  const bool nvfp4 = cfg->weight_format == NH_WEIGHTS_NVFP4;
+  if (nvfp4 != (wq != nullptr))
+    return fail(NH_ERR_INVALID_ARG, nvfp4 ? "config has NVFP4 weights: use the _nvfp4 entry points"
+                                          : "config has native weights: use nh_moe_forward");
   if (T == 0) return NH_OK;
-  NH_TRY(check_ptr(w, up_phase ? "w_up" : "w_down"));
+  if (!nvfp4) NH_TRY(check_ptr(w, up_phase ? "w_up" : "w_down"));
   if (up_phase) NH_TRY(check_ptr(x, "x"));
   int dev;
   NH_TRY(device_setup(&dev));
@@ -947,7 +1034,7 @@ static nh_status experts_phase(const nh_moe_config* cfg, int64_t T, const void* 
   c.sched = reinterpret_cast<unsigned int*>(c.status + (up_phase ? SCHED_UP : SCHED_DOWN));
   c.W = w;
   if (up_phase) {
-    if (L.swap_ab) {
+    if (L.x_direct) {
       // decode: the activation tile is x itself; rows map to tokens by perm_token
       c.A = x;
       c.rows = T;
@@ -969,6 +1056,7 @@ static nh_status experts_phase(const nh_moe_config* cfg, int64_t T, const void* 
     c.ldo = p.H;
     c.perm_w = at<float>(ws, L.perm_w);
   }
+  if (nvfp4) return run_gemm_q4(c, wq, dev, st);
   return run_gemm(p, c, dev, st);
 }
 
@@ -995,11 +1083,45 @@ nh_status nh_moe_forward(const nh_moe_config* cfg, int64_t T, const void* x, con
   return nh_moe_experts_down(cfg, T, w_down, ws, ws_bytes, stream);
 }
 
+nh_status nh_moe_forward_nvfp4(const nh_moe_config* cfg, int64_t T, const void* x,
+                               const nh_nvfp4_weight* w_up, const nh_nvfp4_weight* w_down,
+                               void* ws, size_t ws_bytes, void* stream) {
+  if (!w_up || !w_down) return fail(NH_ERR_INVALID_ARG, "w_up / w_down is NULL");
+  NH_TRY(experts_phase(cfg, T, x, nullptr, ws, ws_bytes, stream, true, w_up));
+  return experts_phase(cfg, T, x, nullptr, ws, ws_bytes, stream, false, w_down);
+}
+
+static nh_status shared_impl(const nh_moe_config* cfg, int64_t T, const void* x, const void* w_su,
+                             const void* w_sd, const nh_nvfp4_weight* q_su,
+                             const nh_nvfp4_weight* q_sd, float* y_shared, void* ws_shared,
+                             size_t ws_shared_bytes, void* stream);
+
+nh_status nh_moe_shared_nvfp4(const nh_moe_config* cfg, int64_t T, const void* x,
+                              const nh_nvfp4_weight* w_su, const nh_nvfp4_weight* w_sd,
+                              float* y_shared, void* ws_shared, size_t ws_shared_bytes,
+                              void* stream) {
+  if (!w_su || !w_sd) return fail(NH_ERR_INVALID_ARG, "w_shared_up / w_shared_down is NULL");
+  return shared_impl(cfg, T, x, nullptr, nullptr, w_su, w_sd, y_shared, ws_shared,
+                     ws_shared_bytes, stream);
+}
+
 nh_status nh_moe_shared(const nh_moe_config* cfg, int64_t T, const void* x, const void* w_su,
                         const void* w_sd, float* y_shared, void* ws_shared, size_t ws_shared_bytes,
                         void* stream) {
+  return shared_impl(cfg, T, x, w_su, w_sd, nullptr, nullptr, y_shared, ws_shared,
+                     ws_shared_bytes, stream);
+}
+
+static nh_status shared_impl(const nh_moe_config* cfg, int64_t T, const void* x, const void* w_su,
+                             const void* w_sd, const nh_nvfp4_weight* q_su,
+                             const nh_nvfp4_weight* q_sd, float* y_shared, void* ws_shared,
+                             size_t ws_shared_bytes, void* stream) {
   Plan p;
   NH_TRY(make_plan(cfg, T, &p));
+  const bool nvfp4 = cfg->weight_format == NH_WEIGHTS_NVFP4;
+  if (nvfp4 != (q_su != nullptr))
+    return fail(NH_ERR_INVALID_ARG, nvfp4 ? "config has NVFP4 weights: use nh_moe_shared_nvfp4"
+                                          : "config has native weights: use nh_moe_shared");
   size_t need;
   NH_TRY(nh_moe_shared_workspace_size(cfg, T, &need));
   NH_TRY(check_ptr(ws_shared, "ws_shared"));
@@ -1007,8 +1129,10 @@ nh_status nh_moe_shared(const nh_moe_config* cfg, int64_t T, const void* x, cons
     return fail(NH_ERR_INVALID_ARG, "ws_shared holds %zu bytes, %zu needed", ws_shared_bytes, need);
   if (T == 0) return NH_OK;
   NH_TRY(check_ptr(x, "x"));
-  NH_TRY(check_ptr(w_su, "w_shared_up"));
-  NH_TRY(check_ptr(w_sd, "w_shared_down"));
+  if (!nvfp4) {
+    NH_TRY(check_ptr(w_su, "w_shared_up"));
+    NH_TRY(check_ptr(w_sd, "w_shared_down"));
+  }
   NH_TRY(check_ptr(y_shared, "y_shared"));
   int dev;
   NH_TRY(device_setup(&dev));
@@ -1031,7 +1155,8 @@ nh_status nh_moe_shared(const nh_moe_config* cfg, int64_t T, const void* x, cons
   up.ldo = p.S;
   up.status = status;
   up.sched = reinterpret_cast<unsigned int*>(status + 4);
-  NH_TRY(run_gemm(p, up, dev, st));
+  if (nvfp4) NH_TRY(run_gemm_q4(up, q_su, dev, st));
+  else NH_TRY(run_gemm(p, up, dev, st));
   GemmCall dn = up;
   dn.A = h;
   dn.W = w_sd;
@@ -1041,6 +1166,7 @@ nh_status nh_moe_shared(const nh_moe_config* cfg, int64_t T, const void* x, cons
   dn.out = y_shared;
   dn.ldo = p.H;
   dn.sched = reinterpret_cast<unsigned int*>(status + 6);
+  if (nvfp4) return run_gemm_q4(dn, q_sd, dev, st);
   return run_gemm(p, dn, dev, st);
 }
 

@@ -43,7 +43,7 @@ def to_dev(a, cfg=None):
 def make_block(inp):
     import non_gated_relu_b200 as nh
     return nh.NemotronHMoE(inp.cfg, inp.w_router, inp.w_up, inp.w_down, inp.w_shared_up,
-                           inp.w_shared_down, bias=inp.bias)
+                           inp.w_shared_down, bias=inp.bias, nvfp4=inp.nvfp4)
 
 
 def run_block(inp, blk=None):

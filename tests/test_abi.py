@@ -58,6 +58,11 @@ def test_validation_rejects_bad_configs():
         assert e.value.status == nh.NH_ERR_UNSUPPORTED, kw
     # the float32 path takes any size
     nh.validate(base.replace(dtype="f32", hidden_size=2690, moe_intermediate_size=1850))
+    # NVFP4 weights need bf16 activations
+    with pytest.raises(nh.NHMoEError) as e:
+        nh.validate(base.replace(dtype="f32", weight_format="nvfp4"))
+    assert e.value.status == nh.NH_ERR_INVALID_ARG
+    nh.validate(base.replace(weight_format="nvfp4"))
     # top-2 group score needs two experts per group
     c = nh.config_from(base.replace(n_routed_experts=8, n_group=8, num_experts_per_tok=1))
     c.group_score = 1
@@ -78,7 +83,7 @@ def test_workspace_layout(name):
                ("counts", cfg.E * 4),
                ("offsets", (cfg.E + 1) * 4), ("chunk_counts", L.n_chunks * cfg.E * 4),
                ("perm_token", rows * 4), ("perm_w", rows * 4), ("inv_row", rows * 4),
-               ("tiles", L.max_tiles * 16), ("num_tiles", 4), ("x_perm", 0 if L.swap_ab else rows * cfg.H * elem),
+               ("tiles", L.max_tiles * 16), ("num_tiles", 4), ("x_perm", 0 if L.x_direct else rows * cfg.H * elem),
                ("h", rows * cfg.I * elem), ("y_part", rows * cfg.H * elem)]
     spans = sorted((getattr(L, n), getattr(L, n) + sz, n) for n, sz in regions)
     for (a0, a1, an), (b0, b1, bn) in zip(spans, spans[1:]):
@@ -86,7 +91,9 @@ def test_workspace_layout(name):
     assert spans[-1][1] <= L.total_bytes
     assert all(getattr(L, n) % 256 == 0 for n, _ in regions)
     # tile plan: decode-sized T puts weights on the MMA M side
-    if cfg.dtype == "f32":
+    if cfg.weight_format == "nvfp4":
+        assert L.swap_ab == 1 and L.tile_rows in (16, 32, 64)
+    elif cfg.dtype == "f32":
         assert L.tile_rows == 64 and L.swap_ab == 0
     elif T <= 64:
         assert L.swap_ab == 1 and L.tile_rows >= T and L.tile_rows % 16 == 0

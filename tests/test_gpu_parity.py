@@ -44,6 +44,13 @@ SMALL = {
                                n_group=64, topk_group=8, num_experts_per_tok=32,
                                moe_intermediate_size=64, moe_shared_expert_intermediate_size=64,
                                seed=13),
+    # NVFP4 weights (W4A16): decode orientation 16 / 32 / 64, and 64-row tiles
+    # with a gathered x_perm for T > 64
+    "small_nvfp4_t5": small("small_nvfp4_t5", T=5, seed=41, weight_format="nvfp4"),
+    "small_nvfp4_t29": small("small_nvfp4_t29", T=29, seed=42, weight_format="nvfp4"),
+    "small_nvfp4_t64": small("small_nvfp4_t64", T=64, seed=43, weight_format="nvfp4",
+                             moe_intermediate_size=192),
+    "small_nvfp4_t150": small("small_nvfp4_t150", T=150, seed=44, weight_format="nvfp4"),
     # single expert (routing is trivial)
     "small_one_expert": small("small_one_expert", T=40, n_routed_experts=1, n_group=1,
                               topk_group=1, num_experts_per_tok=1, seed=14),

@@ -37,7 +37,7 @@ def check_permute(cfg, x_np, idx, w, ws, lay, x_dev):
     np.testing.assert_array_equal(region(ws, lay.inv_row, rows, np.int32).reshape(T, k),
                                   ref["inv_row"])
     elem = np.uint16 if cfg.dtype == "bf16" else np.float32
-    if not lay.swap_ab:   # the decode orientation reads x directly (no x_perm)
+    if not lay.x_direct:   # the decode orientation reads x directly (no x_perm)
         xp = region(ws, lay.x_perm, rows * cfg.H, elem).reshape(rows, cfg.H)
         np.testing.assert_array_equal(xp, x_np[ref["perm_token"]])
     nt = int(region(ws, lay.num_tiles, 1, np.int32)[0])
