@@ -69,8 +69,8 @@ typedef enum {
 
 /*
  * One stacked NVFP4 weight tensor [n_mat][rows][cols] (W4A16, group size 16:
- * "NVFP4 W4A16 group_size 16 on the experts, shared experts", vllm.cpp PR
- * #518).  Element (m, r, c) = e2m1(code) * e4m3(scale) * global[m] where
+ * vllm.cpp PR #518 names this storage for the checkpoint's routed and shared
+ * expert weights).  Element (m, r, c) = e2m1(code) * e4m3(scale) * global[m] where
  *   codes  [n_mat][rows][cols/2]: two E2M1 codes per byte, column 2j in the
  *          low nibble of byte j;
  *   scales [n_mat][rows][pitch]: E4M3 scale of columns 16b .. 16b+15 in byte
@@ -183,8 +183,8 @@ nh_status nh_moe_route_permute(const nh_moe_config *cfg, int64_t T, const void *
  * for callers that cannot allocate device memory or pass a workspace (for
  * example code running under a CUDA graph capture where allocation is not
  * allowed, serving stacks whose memory pool has already claimed the device,
- * or plugin hosts that give an op no scratch buffer).  It has no counterpart
- * on the pages: it is a packaging choice of this library.
+ * or plugin hosts that give an op no scratch buffer).  None of the cited
+ * sources has such a call: it is a packaging choice of this library.
  *   Same arguments and results as nh_moe_route, without ws / ws_bytes.
  *   Limits: T <= 32 and T * n_routed_experts <= 16384; larger sizes return
  *   NH_ERR_INVALID_ARG with a message naming the limit (use nh_moe_route).

@@ -5,8 +5,9 @@
 // is accumulated in tensor memory by tcgen05.mma (bf16 in, f32 accumulate)
 // from operand tiles that TMA stages in shared memory with 128-byte swizzle,
 // and a fused epilogue turns it into
-//   up_proj:   h = relu(D)^2 stored in bf16              (non-gated expert,
-//              "up_proj -> relu^2 -> down_proj", vllm.cpp PR #518)
+//   up_proj:   h = relu(D)^2 stored in bf16              (non-gated expert:
+//              no gate projection, squared relu between the two
+//              projections; vllm.cpp PR #518)
 //   down_proj: y_part[row] = routing weight * D in bf16     (per-(token, expert)
 //              partial rows, summed per token by the finalize kernel)
 //   shared:    y_shared = D                                 (always-on expert)

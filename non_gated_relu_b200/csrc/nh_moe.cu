@@ -278,10 +278,10 @@ static nh_status set_attrs(int dev) {
                                tc2::SMEM));
   NH_CUDA(cudaFuncSetAttribute(q4::tc_q4_gemm<16, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                q4::Shape<16, 8>::SMEM));
-  NH_CUDA(cudaFuncSetAttribute(q4::tc_q4_gemm<32, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               q4::Shape<32, 8>::SMEM));
-  NH_CUDA(cudaFuncSetAttribute(q4::tc_q4_gemm<64, 7>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               q4::Shape<64, 7>::SMEM));
+  NH_CUDA(cudaFuncSetAttribute(q4::tc_q4_gemm<32, 6>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               q4::Shape<32, 6>::SMEM));
+  NH_CUDA(cudaFuncSetAttribute(q4::tc_q4_gemm<64, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                               q4::Shape<64, 4>::SMEM));
   NH_CUDA(cudaFuncSetAttribute(route_permute_small<__nv_bfloat16>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, ROUTE_PERMUTE_SMEM_MAX));
   NH_CUDA(cudaFuncSetAttribute(route_permute_small<float>,
@@ -496,9 +496,10 @@ static nh_status launch_tc2(const GemmCall& c, int dev, cudaStream_t st) {
   return launch_check("tc2_grouped_gemm");
 }
 
-// uint8 [n_mat, rows, row_bytes] (no swizzle), box {box_bytes, 128 rows, 1}
+// uint8 [n_mat, rows, row_bytes], box {box_bytes, 128 rows, 1}; with `swizzle`
+// the box is 128 bytes wide and lands with the 128-byte swizzle
 static nh_status map_u8_3d(CUtensorMap* m, const void* base, int64_t row_bytes, int64_t rows,
-                           int64_t n_mat, int box_bytes) {
+                           int64_t n_mat, int box_bytes, bool swizzle) {
   auto fn = encode_fn();
   if (!fn) return fail(NH_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
   cuuint64_t dims[3] = {(cuuint64_t)row_bytes, (cuuint64_t)rows, (cuuint64_t)n_mat};
@@ -506,7 +507,8 @@ static nh_status map_u8_3d(CUtensorMap* m, const void* base, int64_t row_bytes, 
   cuuint32_t box[3] = {(cuuint32_t)box_bytes, (cuuint32_t)q4::M, 1};
   cuuint32_t es[3] = {1, 1, 1};
   CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 3, const_cast<void*>(base), dims, strides, box,
-                  es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE,
+                  es, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                  swizzle ? CU_TENSOR_MAP_SWIZZLE_128B : CU_TENSOR_MAP_SWIZZLE_NONE,
                   CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   if (r != CUDA_SUCCESS) return fail(NH_ERR_CUDA, "cuTensorMapEncodeTiled (u8) failed: %d", (int)r);
   return NH_OK;
@@ -519,8 +521,8 @@ static nh_status launch_q4(const GemmCall& c, const nh_nvfp4_weight& w, int dev,
   using S = q4::Shape<NT, STAGES>;
   CUtensorMap ma, mc, ms;
   NH_TRY(map_2d(&ma, c.A, c.K, c.rows, NT));
-  NH_TRY(map_u8_3d(&mc, w.codes, c.K / 2, c.N, c.n_exp, q4::BK / 2));
-  NH_TRY(map_u8_3d(&ms, w.scales, nvfp4_pitch(c.K), c.N, c.n_exp, q4::SCALE_BOX));
+  NH_TRY(map_u8_3d(&mc, w.codes, c.K / 2, c.N, c.n_exp, q4::CODE_ROW, true));
+  NH_TRY(map_u8_3d(&ms, w.scales, nvfp4_pitch(c.K), c.N, c.n_exp, q4::SCALE_BOX, false));
   q4::Q4Args qa;
   tc::TcArgs& g = qa.g;
   g.tiles = c.tiles;
@@ -556,8 +558,8 @@ static nh_status run_gemm_q4(const GemmCall& c, const nh_nvfp4_weight* w, int de
     return fail(NH_ERR_INVALID_ARG, "NVFP4 codes / scales must be 16-byte aligned");
   switch (c.tile_rows) {
     case 16: return launch_q4<16, 8>(c, *w, dev, st);
-    case 32: return launch_q4<32, 8>(c, *w, dev, st);
-    case 64: return launch_q4<64, 7>(c, *w, dev, st);
+    case 32: return launch_q4<32, 6>(c, *w, dev, st);
+    case 64: return launch_q4<64, 4>(c, *w, dev, st);
     default: return fail(NH_ERR_UNSUPPORTED, "NVFP4 tile rows %d", c.tile_rows);
   }
 }

@@ -37,9 +37,10 @@
  * Wu [E][I][H], Wd [E][H][I], Wsu [S][H], Wsd [H][S]; x [T][H].  Activations
  * and expert weights are float32 (dtype 0) or bf16 bit patterns (dtype 1).
  *
- * Expert and shared weights may instead be NVFP4 (W4A16 with group size 16:
- * "NVFP4 W4A16 group_size 16 on the experts, shared experts", vllm.cpp PR
- * #518).  Reading of that format (the pages give no more): every element is
+ * Expert and shared weights may instead be NVFP4 (vllm.cpp PR #518: the
+ * checkpoint keeps routed and shared expert weights in 4-bit NVFP4 with one
+ * scale per 16 inputs, activations in 16 bits).  Reading of that format (the
+ * PR names it and no more): every element is
  * an E2M1 code (sign, 2 exponent bits with bias 1, 1 mantissa bit; values
  * 0, 0.5, 1, 1.5, 2, 3, 4, 6), two per byte with the even column in the low
  * nibble; every 16 consecutive columns of a row share one E4M3 scale byte

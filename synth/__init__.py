@@ -4,7 +4,7 @@ This module is shared by the CPU oracle, the tests and the benchmark.  It
 holds only workload definitions and random-number recipes: no step of the
 MoE arithmetic (no routing, no matmul, no activation) lives here.
 
-Workloads follow the MoE layer printed on the pages:
+Workloads follow the Nemotron-H MoE layer as these sources give it:
   * baseRT issue #46, "Architecture (config.json)": 128 routed experts, 6 per
     token, n_groups=8, topk_group=1, routed_scaling_factor=2.5,
     norm_topk_prob, 1 shared expert 3712 wide, relu2, no gate_proj;
@@ -37,7 +37,7 @@ class MoEConfig:
 
     Field names are the config.json names of the Nemotron-H model (MLX
     ``ModelArgs`` in the exo commit "Add support for Nemotron sharding").
-    ``n_group`` is the router's group count (the pages' MoE summary also
+    ``n_group`` is the router's group count (the baseRT MoE summary also
     spells it "n_groups", which in ``ModelArgs`` is the Mamba-2 field).
     """
     name: str
