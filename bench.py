@@ -50,6 +50,10 @@ def parse():
     ap.add_argument("--workload", default=DEFAULT_WORKLOAD, choices=synth.CONFIG_ORDER)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--parallel", default="dp", choices=["dp", "tp"],
+                    help="dp: disjoint token batches per GPU, replicated weights (weak "
+                         "scaling); tp: I and S sharded over the GPUs, same tokens, one "
+                         "all-reduce of y per step (strong scaling)")
     ap.add_argument("--batches", type=int, default=4, help="distinct input batches cycled")
     ap.add_argument("--eager", action="store_true",
                     help="timed loop calls the block eagerly (NVTX range per call) instead of "
@@ -453,6 +457,138 @@ def report(args, cfg, inp, world, steps, elapsed_ms, clk, kern, e2e_ms, blk):
     return out
 
 
+def run_tp(args, rank, world, local_rank):
+    """Tensor parallel: every rank holds its 64-feature blocks of I and S, all
+    ranks process the same T tokens, and one NCCL all-reduce sums the float32
+    block output per step (non_gated_relu_b200.tp).  The rank's own path runs
+    as a CUDA graph; the all-reduce and the final rounding follow it on the
+    same stream.  value = T / step time (strong scaling)."""
+    import torch
+    from non_gated_relu_b200 import tp
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    cfg = workload(args)
+    inp = synth.make_inputs(cfg, skew_b=skew_b(cfg))
+    blk = tp.TPNemotronHMoE(cfg, inp.w_router, inp.w_up, inp.w_down, inp.w_shared_up,
+                            inp.w_shared_down, nvfp4=inp.nvfp4, world=world, rank=rank,
+                            device=dev)
+    T = cfg.T
+    nb = max(1, args.batches)
+    xs = []
+    for i in range(nb):                          # the same batches on every rank
+        xi = inp.x if i == 0 else batch_x(cfg, i)
+        t = torch.from_numpy(xi)
+        t = t.view(torch.bfloat16) if xi.dtype == np.uint16 else t
+        xs.append(t.to(dev))
+    b = blk.block.buffers(T)
+    graphs = []
+    for i in range(nb):
+        s = torch.cuda.Stream(dev)
+        s.wait_stream(torch.cuda.current_stream(dev))
+        with torch.cuda.stream(s):
+            blk.partial(xs[i])
+        torch.cuda.current_stream(dev).wait_stream(s)
+        torch.cuda.synchronize(dev)
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g):
+            blk.partial(xs[i])
+        graphs.append(g)
+
+    def step(i):
+        graphs[i % nb].replay()
+        tp.all_reduce_sum(b.y_f32)
+        return blk.output(b.y_f32)
+
+    main = torch.cuda.current_stream(dev)
+    for i in range(max(3, args.warmup)):
+        step(i)
+    torch.cuda.synchronize(dev)
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(main)
+    for i in range(20):
+        step(i)
+    e1.record(main)
+    e1.synchronize()
+    est = e0.elapsed_time(e1) / 20.0
+    steps = args.steps if args.steps > 0 else int(max(20, min(20000, 2000.0 / max(est, 1e-3))))
+    if world > 1:
+        import torch.distributed as dist
+        dist_mod = dist
+        # every rank runs the same number of steps (and so the same collectives)
+        st = torch.tensor([steps], device=dev)
+        dist.broadcast(st, 0)
+        steps = int(st.item())
+    else:
+        dist_mod = None
+    clocks = ClockSampler(local_rank)
+    if rank == 0:
+        clocks.start()
+        time.sleep(0.3)
+    if dist_mod:
+        dist_mod.barrier()
+    torch.cuda.synchronize(dev)
+    t0, t1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    t0.record(main)
+    for i in range(steps):
+        step(i)
+    t1.record(main)
+    torch.cuda.synchronize(dev)
+    if dist_mod:
+        dist_mod.barrier()
+    elapsed_ms = max_over_ranks(t0.elapsed_time(t1), dist_mod, dev)
+    clk = clocks.stop() if rank == 0 else None
+    rc = blk.block.check(T)
+    if rc != 0:
+        raise RuntimeError(f"device status {rc} after the timed region")
+    # end to end: pinned host x -> device -> step -> host y, every step
+    xh = [x.cpu().pin_memory() for x in xs]
+    xd = torch.empty_like(xs[0])
+    yh = torch.empty((T, cfg.H), dtype=xs[0].dtype).pin_memory()
+    e2e_steps = min(steps, 2000)
+
+    def e2e_step(i):
+        xd.copy_(xh[i % nb], non_blocking=True)
+        blk.partial(xd)
+        tp.all_reduce_sum(b.y_f32)
+        yh.copy_(blk.output(b.y_f32), non_blocking=True)
+        main.synchronize()
+    for i in range(3):
+        e2e_step(i)
+    h0, h1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    h0.record(main)
+    for i in range(e2e_steps):
+        e2e_step(i)
+    h1.record(main)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(h0.elapsed_time(h1), dist_mod, dev) / e2e_steps
+    del graphs
+    if rank != 0:
+        return None
+    ms = elapsed_ms / steps
+    elem = 2 if cfg.dtype == "bf16" else 4
+    return {
+        "metric": METRIC, "value": round(T / (ms / 1e3), 2), "unit": "tokens/s",
+        "n_gpus": world, "steps": steps, "warmup": max(3, args.warmup),
+        "ms_per_step": round(ms, 5), "higher_is_better": True, "scaling": "strong",
+        "vs_baseline": None,
+        "dtype": ("nvfp4 weights, bf16 activations" if cfg.weight_format == "nvfp4"
+                  else ("bf16" if cfg.dtype == "bf16" else "f32")), "data": "synthetic",
+        "config": {"workload": cfg.name, "tokens_per_step": T,
+                   "parallelism": f"tp{world} (I and S in 64-feature blocks per GPU, one "
+                                  f"all-reduce of the float32 block output per step)",
+                   "moe_intermediate_size_per_gpu": blk.cfg_rank.moe_intermediate_size,
+                   "moe_shared_expert_intermediate_size_per_gpu":
+                       blk.cfg_rank.moe_shared_expert_intermediate_size,
+                   "l2": "inputs larger than L2 (the expert weights touched per step)"},
+        "e2e": {"value": round(T / (e2e_ms / 1e3), 2), "unit": "tokens/s",
+                "ms_per_step": round(e2e_ms, 5),
+                "h2d_bytes_per_step": T * cfg.H * elem, "d2h_bytes_per_step": T * cfg.H * elem},
+        "gpu_launches": (launches_per_step(blk.cfg_rank) + 1) * steps,
+        "clocks": clk,
+    }
+
+
 def kernel_hash():
     """Hash of every CUDA source of the library: profiler counters recorded for
     one build are reported only while the sources are unchanged."""
@@ -529,7 +665,7 @@ def main():
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        out = run_ours(args, rank, world, local_rank)
+        out = (run_tp if args.parallel == "tp" else run_ours)(args, rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

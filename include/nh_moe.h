@@ -279,6 +279,29 @@ nh_status nh_moe_finalize(const nh_moe_config *cfg, int64_t T, const void *ws, s
                           const float *y_shared, void *y, void *stream);
 
 /*
+ * Tensor-parallel shards (exo commit "Add support for Nemotron sharding",
+ * the NemotronHMoE branch of the sharding strategy: the routed fc1 and the
+ * shared up_proj are split over their output features, the routed fc2 and the
+ * shared down_proj over their input features, the router is replicated, and
+ * one all-reduce sums the block output).
+ * A rank runs the whole path with the config of its shard
+ * (moe_intermediate_size and moe_shared_expert_intermediate_size set to its
+ * share of I and S, each a multiple of 64) and its slices of the weights,
+ * then calls nh_moe_finalize_partial instead of nh_moe_finalize:
+ *   y_f32[t] = y_shared[t] + sum_j y_part[inv_row[t, j]]     (float32, no rounding)
+ * The caller sums y_f32 over the ranks (an all-reduce) and rounds the sum once
+ * with nh_moe_cast_output:
+ *   y[t] = dtype(y_f32[t])
+ * y_f32 [T, H] float32 and y [T, H] dtype are device buffers, 16-byte aligned.
+ * Errors as nh_moe_finalize.
+ */
+nh_status nh_moe_finalize_partial(const nh_moe_config *cfg, int64_t T, const void *ws,
+                                  size_t ws_bytes, const float *y_shared, float *y_f32,
+                                  void *stream);
+nh_status nh_moe_cast_output(const nh_moe_config *cfg, int64_t T, const float *y_f32, void *y,
+                             void *stream);
+
+/*
  * Synchronises `stream`, reads the workspace status word and returns it
  * (NH_OK, NH_ERR_TIMEOUT or NH_ERR_DEVICE_CHECK); a pending CUDA error is
  * returned as NH_ERR_CUDA.  `ws` is a routed-path workspace.

@@ -23,7 +23,7 @@ from . import build as _build
 
 __all__ = ["NHMoEError", "Config", "Layout", "config_from", "load", "validate", "workspace_size",
            "workspace_layout", "shared_workspace_size", "route", "route_noalloc", "route_permute", "permute", "forward", "experts_up", "experts_down", "shared", "forward_nvfp4", "shared_nvfp4", "nvfp4_weight",
-           "finalize", "check_device", "selftest_timeout", "library_path", "NemotronHMoE"]
+           "finalize", "finalize_partial", "cast_output", "check_device", "selftest_timeout", "library_path", "NemotronHMoE"]
 
 NH_OK, NH_ERR_INVALID_ARG, NH_ERR_UNSUPPORTED, NH_ERR_CUDA, NH_ERR_TIMEOUT, NH_ERR_DEVICE_CHECK = range(6)
 STATUS_NAMES = {0: "NH_OK", 1: "NH_ERR_INVALID_ARG", 2: "NH_ERR_UNSUPPORTED", 3: "NH_ERR_CUDA",
@@ -89,7 +89,8 @@ _lib = None
 _EXPORTS = ["nh_moe_validate", "nh_moe_workspace_size", "nh_moe_workspace_layout",
             "nh_moe_shared_workspace_size", "nh_moe_route", "nh_moe_route_noalloc", "nh_moe_route_permute",
             "nh_moe_permute", "nh_moe_forward", "nh_moe_experts_up", "nh_moe_experts_down",
-            "nh_moe_shared", "nh_moe_finalize", "nh_moe_check_device", "nh_moe_selftest_timeout",
+            "nh_moe_shared", "nh_moe_finalize", "nh_moe_finalize_partial", "nh_moe_cast_output",
+            "nh_moe_check_device", "nh_moe_selftest_timeout",
             "nh_last_error", "nh_version"]
 
 
@@ -125,6 +126,8 @@ def load():
             "nh_moe_shared_nvfp4": [C, I64, P, ctypes.POINTER(NvFp4Weight),
                                     ctypes.POINTER(NvFp4Weight), P, P, S, P],
             "nh_moe_finalize": [C, I64, P, S, P, P, P],
+            "nh_moe_finalize_partial": [C, I64, P, S, P, P, P],
+            "nh_moe_cast_output": [C, I64, P, P, P],
             "nh_moe_check_device": [P, P],
             "nh_moe_selftest_timeout": [P, ctypes.c_uint64, P],
         }
@@ -266,6 +269,20 @@ def finalize(cfg, T: int, ws, y_shared, y, stream=None):
     c = config_from(cfg)
     _check(load().nh_moe_finalize(ctypes.byref(c), T, _p(ws), _nbytes(ws), _p(y_shared), _p(y),
                                   _stream(stream)))
+
+
+def finalize_partial(cfg, T: int, ws, y_shared, y_f32, stream=None):
+    """Tensor-parallel rank: y_f32 = the float32 sum of this rank's partial
+    rows and shared output, without the final rounding."""
+    c = config_from(cfg)
+    _check(load().nh_moe_finalize_partial(ctypes.byref(c), T, _p(ws), _nbytes(ws), _p(y_shared),
+                                          _p(y_f32), _stream(stream)))
+
+
+def cast_output(cfg, T: int, y_f32, y, stream=None):
+    """y = dtype(y_f32), the one rounding of an all-reduced block output."""
+    c = config_from(cfg)
+    _check(load().nh_moe_cast_output(ctypes.byref(c), T, _p(y_f32), _p(y), _stream(stream)))
 
 
 def check_device(ws, stream=None) -> int:

@@ -19,8 +19,8 @@ from typing import Dict, Optional
 import numpy as np
 import torch
 
-from . import (check_device, config_from, finalize, forward, forward_nvfp4, nvfp4_weight,
-               route_permute, shared, shared_nvfp4, shared_workspace_size, validate,
+from . import (check_device, config_from, finalize, finalize_partial, forward, forward_nvfp4,
+               nvfp4_weight, route_permute, shared, shared_nvfp4, shared_workspace_size, validate,
                workspace_size, NH_BF16, NH_WEIGHTS_NVFP4)
 
 
@@ -47,6 +47,7 @@ class Buffers:
     topk_w: torch.Tensor
     y_shared: Optional[torch.Tensor]
     y: torch.Tensor
+    y_f32: Optional[torch.Tensor] = None     # tensor-parallel partial sum (float32)
 
 
 class NemotronHMoE:
@@ -120,11 +121,15 @@ class NemotronHMoE:
 
     # ------------------------------------------------------------------ compute
     def forward(self, x: torch.Tensor, bufs: Optional[Buffers] = None,
-                nvtx: bool = False) -> torch.Tensor:
+                nvtx: bool = False, partial: bool = False) -> torch.Tensor:
         """y for a device tensor x [T, H]; returns the buffer-owned y [T, H].
-        ``nvtx`` wraps each call in an NVTX range of its name (for profilers)."""
+        ``nvtx`` wraps each call in an NVTX range of its name (for profilers).
+        ``partial`` (a tensor-parallel shard) returns instead the float32
+        sum of this shard's contributions, unrounded, for an all-reduce."""
         T = x.shape[0]
         b = bufs or self.buffers(T)
+        if partial and b.y_f32 is None:
+            b.y_f32 = torch.empty((T, self.H), dtype=torch.float32, device=self.device)
         main = torch.cuda.current_stream(self.device)
         push = torch.cuda.nvtx.range_push if nvtx else (lambda name: None)
         pop = torch.cuda.nvtx.range_pop if nvtx else (lambda: None)
@@ -154,9 +159,12 @@ class NemotronHMoE:
         if self.has_shared:
             main.wait_event(join)
         push("finalize")
-        finalize(self.c, T, b.ws, b.y_shared, b.y, stream=main)
+        if partial:
+            finalize_partial(self.c, T, b.ws, b.y_shared, b.y_f32, stream=main)
+        else:
+            finalize(self.c, T, b.ws, b.y_shared, b.y, stream=main)
         pop()
-        return b.y
+        return b.y_f32 if partial else b.y
 
     def capture(self, T: int):
         """Capture the call sequence for T tokens in a CUDA graph.

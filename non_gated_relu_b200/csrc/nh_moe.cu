@@ -599,10 +599,11 @@ static nh_status run_gemm(const Plan& p, const GemmCall& c, int dev, cudaStream_
 // small kernels
 // ----------------------------------------------------------------------------
 // y[t] = y_shared[t] + sum_j y_part[inv_row[t, j]], summed in fp32 in that
-// order (deterministic), rounded once to the output dtype.
-template <typename Tio>
-__global__ void finalize_gather(const Tio* __restrict__ y_part, const int32_t* __restrict__ inv_row,
-                                const float* __restrict__ y_sh, Tio* __restrict__ y, int64_t T,
+// order (deterministic), rounded once to the output type (float32 output:
+// no rounding, for the tensor-parallel partial sums).
+template <typename Tin, typename Tout>
+__global__ void finalize_gather(const Tin* __restrict__ y_part, const int32_t* __restrict__ inv_row,
+                                const float* __restrict__ y_sh, Tout* __restrict__ y, int64_t T,
                                 int k, int H) {
   pdl_wait();
   pdl_trigger();
@@ -616,14 +617,16 @@ __global__ void finalize_gather(const Tio* __restrict__ y_part, const int32_t* _
       const int r = inv_row[t * k + j];
       if (r >= 0) v += to_f32(y_part[(size_t)r * H + h]);
     }
-    y[i] = from_f32<Tio>(v);
+    y[i] = from_f32<Tout>(v);
   }
 }
 
-// bf16, eight consecutive features per thread (16-byte loads and stores)
+// bf16, eight consecutive features per thread (16-byte loads and stores);
+// output bf16 (uint4 per thread) or, with OUT_F32, float32 (two float4)
+template <bool OUT_F32>
 __global__ void finalize_gather_bf16x8(const uint4* __restrict__ y_part,
                                        const int32_t* __restrict__ inv_row,
-                                       const float4* __restrict__ y_sh, uint4* __restrict__ y,
+                                       const float4* __restrict__ y_sh, void* __restrict__ y,
                                        int64_t T, int k, int H8) {
   pdl_wait();
   pdl_trigger();
@@ -652,9 +655,38 @@ __global__ void finalize_gather_bf16x8(const uint4* __restrict__ y_part,
         a[2 * q + 1] += __uint_as_float(w[q] & 0xffff0000u);
       }
     }
-    y[i] = make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]), pack_bf16x2(a[4], a[5]),
-                      pack_bf16x2(a[6], a[7]));
+    if (OUT_F32) {
+      float4* yf = static_cast<float4*>(y);
+      yf[2 * i] = make_float4(a[0], a[1], a[2], a[3]);
+      yf[2 * i + 1] = make_float4(a[4], a[5], a[6], a[7]);
+    } else {
+      static_cast<uint4*>(y)[i] =
+          make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]), pack_bf16x2(a[4], a[5]),
+                     pack_bf16x2(a[6], a[7]));
+    }
   }
+}
+
+// y = dtype(y_f32): the one rounding of a tensor-parallel block output
+__global__ void cast_output_bf16x8(const float4* __restrict__ y_f32, uint4* __restrict__ y,
+                                   int64_t n8) {
+  pdl_wait();
+  pdl_trigger();
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8;
+       i += (int64_t)gridDim.x * blockDim.x) {
+    const float4 a = y_f32[2 * i], b = y_f32[2 * i + 1];
+    y[i] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
+                      pack_bf16x2(b.z, b.w));
+  }
+}
+
+template <typename Tout>
+__global__ void cast_output(const float* __restrict__ y_f32, Tout* __restrict__ y, int64_t n) {
+  pdl_wait();
+  pdl_trigger();
+  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+       i += (int64_t)gridDim.x * blockDim.x)
+    y[i] = from_f32<Tout>(y_f32[i]);
 }
 
 __global__ void selftest_timeout_kernel(int* status, uint64_t timeout_ns) {
@@ -1172,13 +1204,15 @@ static nh_status shared_impl(const nh_moe_config* cfg, int64_t T, const void* x,
   return run_gemm(p, dn, dev, st);
 }
 
-nh_status nh_moe_finalize(const nh_moe_config* cfg, int64_t T, const void* ws, size_t ws_bytes,
-                          const float* y_shared, void* y, void* stream) {
+// y (dtype, rounded once) or, with out_f32, the float32 sum without rounding
+static nh_status finalize_impl(const nh_moe_config* cfg, int64_t T, const void* ws,
+                               size_t ws_bytes, const float* y_shared, void* y, bool out_f32,
+                               void* stream) {
   Plan p;
   NH_TRY(make_plan(cfg, T, &p));
   NH_TRY(check_ws(p, const_cast<void*>(ws), ws_bytes));
   if (T == 0) return NH_OK;
-  NH_TRY(check_ptr(y, "y"));
+  NH_TRY(check_ptr(y, out_f32 ? "y_f32" : "y"));
   if (y_shared) NH_TRY(check_ptr(y_shared, "y_shared"));
   if (cfg->n_shared_experts && !y_shared)
     return fail(NH_ERR_INVALID_ARG, "y_shared is NULL but the config has a shared expert");
@@ -1188,20 +1222,70 @@ nh_status nh_moe_finalize(const nh_moe_config* cfg, int64_t T, const void* ws, s
   const nh_moe_ws_layout& L = p.lay;
   void* ws_nc = const_cast<void*>(ws);
   const int32_t* inv = at<int32_t>(ws_nc, L.inv_row);
+  const dim3 blk(256);
   if (p.bf16 && p.H % 8 == 0) {
     const int H8 = p.H / 8;
-    NH_TRY((launch_k("finalize_gather_bf16x8", finalize_gather_bf16x8, dim3(grid_for(T * H8, 256, dev)), dim3(256), 0, st, 
-        at<uint4>(ws_nc, L.y_part), inv, reinterpret_cast<const float4*>(y_shared),
-        static_cast<uint4*>(y), T, p.k, H8)));
+    const dim3 grid(grid_for(T * H8, 256, dev));
+    const uint4* yp = at<uint4>(ws_nc, L.y_part);
+    const float4* ys = reinterpret_cast<const float4*>(y_shared);
+    if (out_f32)
+      NH_TRY((launch_k("finalize_gather_bf16x8", finalize_gather_bf16x8<true>, grid, blk, 0, st,
+                       yp, inv, ys, y, T, p.k, H8)));
+    else
+      NH_TRY((launch_k("finalize_gather_bf16x8", finalize_gather_bf16x8<false>, grid, blk, 0, st,
+                       yp, inv, ys, y, T, p.k, H8)));
   } else if (p.bf16) {
-    NH_TRY((launch_k("finalize_gather", finalize_gather<__nv_bfloat16>, dim3(grid_for(T * p.H, 256, dev)), dim3(256), 0, st, 
-        at<__nv_bfloat16>(ws_nc, L.y_part), inv, y_shared, static_cast<__nv_bfloat16*>(y), T, p.k,
-        p.H)));
+    const dim3 grid(grid_for(T * p.H, 256, dev));
+    const __nv_bfloat16* yp = at<__nv_bfloat16>(ws_nc, L.y_part);
+    if (out_f32)
+      NH_TRY((launch_k("finalize_gather", finalize_gather<__nv_bfloat16, float>, grid, blk, 0, st,
+                       yp, inv, y_shared, static_cast<float*>(y), T, p.k, p.H)));
+    else
+      NH_TRY((launch_k("finalize_gather", finalize_gather<__nv_bfloat16, __nv_bfloat16>, grid,
+                       blk, 0, st, yp, inv, y_shared, static_cast<__nv_bfloat16*>(y), T, p.k,
+                       p.H)));
   } else {
-    NH_TRY((launch_k("finalize_gather", finalize_gather<float>, dim3(grid_for(T * p.H, 256, dev)), dim3(256), 0, st, 
-        at<float>(ws_nc, L.y_part), inv, y_shared, static_cast<float*>(y), T, p.k, p.H)));
+    NH_TRY((launch_k("finalize_gather", finalize_gather<float, float>,
+                     dim3(grid_for(T * p.H, 256, dev)), blk, 0, st, at<float>(ws_nc, L.y_part),
+                     inv, y_shared, static_cast<float*>(y), T, p.k, p.H)));
   }
   return launch_check("finalize");
+}
+
+nh_status nh_moe_finalize(const nh_moe_config* cfg, int64_t T, const void* ws, size_t ws_bytes,
+                          const float* y_shared, void* y, void* stream) {
+  return finalize_impl(cfg, T, ws, ws_bytes, y_shared, y, false, stream);
+}
+
+nh_status nh_moe_finalize_partial(const nh_moe_config* cfg, int64_t T, const void* ws,
+                                  size_t ws_bytes, const float* y_shared, float* y_f32,
+                                  void* stream) {
+  return finalize_impl(cfg, T, ws, ws_bytes, y_shared, y_f32, true, stream);
+}
+
+nh_status nh_moe_cast_output(const nh_moe_config* cfg, int64_t T, const float* y_f32, void* y,
+                             void* stream) {
+  NH_TRY(nh_moe_validate(cfg));
+  if (T < 0) return fail(NH_ERR_INVALID_ARG, "T must be >= 0");
+  if (T == 0) return NH_OK;
+  NH_TRY(check_ptr(y_f32, "y_f32"));
+  NH_TRY(check_ptr(y, "y"));
+  int dev;
+  NH_TRY(device_setup(&dev));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const int64_t n = T * (int64_t)cfg->hidden_size;
+  if (cfg->dtype == NH_BF16 && n % 8 == 0) {
+    NH_TRY((launch_k("cast_output_bf16x8", cast_output_bf16x8, dim3(grid_for(n / 8, 256, dev)),
+                     dim3(256), 0, st, reinterpret_cast<const float4*>(y_f32),
+                     static_cast<uint4*>(y), n / 8)));
+  } else if (cfg->dtype == NH_BF16) {
+    NH_TRY((launch_k("cast_output", cast_output<__nv_bfloat16>, dim3(grid_for(n, 256, dev)),
+                     dim3(256), 0, st, y_f32, static_cast<__nv_bfloat16*>(y), n)));
+  } else {
+    NH_TRY((launch_k("cast_output", cast_output<float>, dim3(grid_for(n, 256, dev)), dim3(256), 0,
+                     st, y_f32, static_cast<float*>(y), n)));
+  }
+  return launch_check("cast_output");
 }
 
 nh_status nh_moe_check_device(void* ws, void* stream) {
