@@ -210,7 +210,8 @@ def run_ours(args, rank, world, local_rank):
     cfg = workload(args)
     inp = synth.make_inputs(cfg, skew_b=skew_b(cfg))
     blk = nh.NemotronHMoE(cfg, inp.w_router, inp.w_up, inp.w_down, inp.w_shared_up,
-                          inp.w_shared_down, device=dev, nvfp4=inp.nvfp4)
+                          inp.w_shared_down, device=dev, nvfp4=inp.nvfp4,
+                          w_latent_fc1=inp.w_latent_fc1, w_latent_fc2=inp.w_latent_fc2)
     T = cfg.T
     nb = max(1, args.batches)
     xs = []
@@ -338,18 +339,39 @@ def kernel_times(blk, xs, b, nb, steps):
         elif blk.has_shared:
             timed("shared", lambda: nh.shared(blk.c, x, blk.w_shared_up, blk.w_shared_down,
                                                b.y_shared, b.ws_shared, stream=main))
-        timed("route", lambda: nh.route(blk.c, x, blk.w_router, blk.bias, b.topk_idx, b.topk_w,
-                                         b.ws, stream=main))
-        timed("permute", lambda: nh.permute(blk.c, x, b.topk_idx, b.topk_w, b.ws, stream=main))
-        if blk.nvfp4:
+        if blk.latent:
+            # routing on x, fc1 (counted with the permute), experts in width L
+            ce = blk.c_exp
+            timed("route", lambda: nh.route(blk.c, x, blk.w_router, blk.bias, b.topk_idx,
+                                             b.topk_w, b.ws_route, stream=main))
+            timed("permute", lambda: (nh.latent_in(blk.c, x, blk.w_latent_fc1, b.x_lat, b.ws_lat,
+                                                   stream=main),
+                                      nh.reset_status(b.ws, stream=main),
+                                      nh.permute(ce, b.x_lat, b.topk_idx, b.topk_w, b.ws,
+                                                 stream=main)))
+            xe = b.x_lat
+        else:
+            ce = blk.c
+            timed("route", lambda: nh.route(blk.c, x, blk.w_router, blk.bias, b.topk_idx,
+                                             b.topk_w, b.ws, stream=main))
+            timed("permute", lambda: nh.permute(blk.c, x, b.topk_idx, b.topk_w, b.ws, stream=main))
+            xe = x
+        if blk.nvfp4 and not blk.latent:
             # up and down run back to back in one call; each is timed as half
             timed("experts_up", lambda: nh.forward_nvfp4(blk.c, x, blk.q4["up"], blk.q4["down"],
                                                           b.ws, stream=main))
         else:
-            timed("experts_up", lambda: nh.experts_up(blk.c, x, blk.w_up, b.ws, stream=main))
-            timed("experts_down", lambda: nh.experts_down(blk.c, T, blk.w_down, b.ws,
+            timed("experts_up", lambda: nh.experts_up(ce, xe, blk.w_up, b.ws, stream=main))
+            timed("experts_down", lambda: nh.experts_down(ce, T, blk.w_down, b.ws,
                                                            stream=main))
-        timed("finalize", lambda: nh.finalize(blk.c, T, b.ws, b.y_shared, b.y, stream=main))
+        if blk.latent:
+            # finalize in width L, fc2 onto the shared output, the one rounding
+            timed("finalize", lambda: (nh.finalize(ce, T, b.ws, None, b.y_lat, stream=main),
+                                       nh.latent_out(blk.c, T, b.y_lat, blk.w_latent_fc2,
+                                                     b.y_acc, b.ws_lat, stream=main),
+                                       nh.cast_output(blk.c, T, b.y_acc, b.y, stream=main)))
+        else:
+            timed("finalize", lambda: nh.finalize(blk.c, T, b.ws, b.y_shared, b.y, stream=main))
         torch.cuda.synchronize(blk.device)
         for n in names:
             if (n == "shared" and not blk.has_shared) or (n == "experts_down" and blk.nvfp4):
@@ -364,6 +386,11 @@ def kernel_times(blk, xs, b, nb, steps):
 def launches_per_step(cfg):
     """Kernels of one block call (memsets excluded), as nh_moe.cu launches them."""
     T = cfg.T
+    if getattr(cfg, "latent_size", 0):
+        # route (no fused permute), fc1, permute, up, down, finalize, fc2, cast, shared
+        n = 1 if T <= 32 else (3 if cfg.dtype == "bf16" and cfg.E % 32 == 0 else 2)
+        n += 1 + (1 if T <= 256 else 4) + 2 + 1 + 1 + 1
+        return n + (2 if cfg.n_shared_experts else 0)
     if T <= 32:
         n = 1                                   # fused router
     elif cfg.dtype == "bf16" and cfg.E % 32 == 0:
@@ -394,18 +421,19 @@ def report(args, cfg, inp, world, steps, elapsed_ms, clk, kern, e2e_ms, blk):
     idx = b.topk_idx.cpu().numpy()
     D = distinct_experts(cfg, idx)
     welem = 0.5 + 1.0 / 16 if cfg.weight_format == "nvfp4" else elem   # bytes per weight
-    expert_bytes = int(cfg.I * cfg.H * welem)      # one projection of one expert
+    expert_bytes = int(cfg.I * cfg.HE * welem)     # one projection of one expert
     shared_bytes = int(2 * cfg.S * cfg.H * welem) if cfg.n_shared_experts else 0
     rows = T * cfg.k
     # algorithmic bytes of one step: touched weights + router + x in + y out
-    step_bytes = (D * 2 * expert_bytes + shared_bytes + cfg.E * cfg.H * 4
+    latent_bytes = 2 * cfg.latent_size * cfg.H * elem if cfg.latent_size else 0
+    step_bytes = (D * 2 * expert_bytes + shared_bytes + latent_bytes + cfg.E * cfg.H * 4
                   + 2 * T * cfg.H * elem)
     hbm_step = step_bytes / (ms / 1e3) / 1e9
     # dominant kernel roofline
     decode = T <= 64
     if decode:
         dom = "experts_up" if kern["experts_up"] >= kern["experts_down"] else "experts_down"
-        kb = D * expert_bytes + rows * (cfg.H + cfg.I) * elem
+        kb = D * expert_bytes + rows * (cfg.HE + cfg.I) * elem
         ach = kb / (kern[dom] / 1e3) / 1e9
         peak = pk["hbm_gbs"]
         roof = {"bound": "hbm", "kernel": dom, "achieved": round(ach, 1), "peak": peak,
@@ -413,7 +441,7 @@ def report(args, cfg, inp, world, steps, elapsed_ms, clk, kern, e2e_ms, blk):
                 "algorithmic_bytes_per_launch": kb, "ms_per_launch": round(kern[dom], 5)}
     else:
         dom = "experts_up" if kern["experts_up"] >= kern["experts_down"] else "experts_down"
-        kf = 2.0 * rows * cfg.H * cfg.I
+        kf = 2.0 * rows * cfg.HE * cfg.I
         ach = kf / (kern[dom] / 1e3) / 1e12
         peak = pk.get("bf16_tflops_sustained", pk["bf16_tflops"]) if pk_kind == "measured" else pk["bf16_tflops"]
         roof = {"bound": "tensor", "kernel": dom, "achieved": round(ach, 1), "peak": peak,

@@ -106,6 +106,10 @@ typedef struct {
     int32_t dtype;                                /* nh_dtype                     */
     int32_t group_score;                          /* nh_group_score               */
     int32_t weight_format;                        /* nh_weight_format             */
+    int32_t latent_size;                          /* L: 0, or the routed experts'
+                                                     width between the latent
+                                                     projections (see
+                                                     nh_moe_latent_in)           */
 } nh_moe_config;
 
 /* Byte offsets of the regions inside the routed-path workspace `ws`. */
@@ -300,6 +304,48 @@ nh_status nh_moe_finalize_partial(const nh_moe_config *cfg, int64_t T, const voi
                                   void *stream);
 nh_status nh_moe_cast_output(const nh_moe_config *cfg, int64_t T, const float *y_f32, void *y,
                              void *stream);
+
+/*
+ * Latent MoE projections (ModelOpt descriptor NemotronHMoELayerDescriptor:
+ * latent_fc1_name='fc1_latent_proj', latent_fc2_name='fc2_latent_proj'; the
+ * descriptor names the two modules and gives no formula).  Reading used, with
+ * L = cfg->latent_size > 0:
+ *   x_lat = dtype(x W_fc1^T)                     W_fc1 [L, H]   (nh_moe_latent_in)
+ *   routed experts on x_lat, in width L: W_up [E, I, L], W_down [E, L, I],
+ *     routing on x (nh_moe_route with cfg), combined as usual into
+ *     y_lat [T, L] (nh_moe_finalize, rounded to dtype)
+ *   y_acc += y_lat W_fc2^T                       W_fc2 [H, L]   (nh_moe_latent_out)
+ *     where y_acc holds the shared expert's y_shared; without a shared
+ *     expert nh_moe_latent_out writes y_acc = y_lat W_fc2^T instead
+ *   y = dtype(y_acc)                                            (nh_moe_cast_output)
+ * The routed-expert calls (nh_moe_permute, nh_moe_forward[_nvfp4],
+ * nh_moe_experts_*, nh_moe_finalize[_partial]) take the expert-width config
+ * that nh_moe_latent_config writes (hidden_size = L, latent_size = 0,
+ * n_shared_experts = 0) and return NH_ERR_INVALID_ARG for a config with
+ * latent_size > 0; nh_moe_route and nh_moe_shared take cfg itself.
+ * nh_moe_route needs only the first `counts` bytes of its workspace layout.
+ *   x [T, H], x_lat [T, L], y_lat [T, L]: dtype; W_fc1, W_fc2: dtype (also
+ *   with NVFP4 expert weights); y_acc [T, H] float32 (read and written; each
+ *   element by one thread, deterministic); ws_latent:
+ *   nh_moe_latent_workspace_size bytes.  Device pointers, 16-byte aligned.
+ */
+nh_status nh_moe_latent_config(const nh_moe_config *cfg, nh_moe_config *expert_cfg);
+nh_status nh_moe_latent_workspace_size(const nh_moe_config *cfg, int64_t T, size_t *bytes);
+nh_status nh_moe_latent_in(const nh_moe_config *cfg, int64_t T, const void *x,
+                           const void *w_latent_fc1, void *x_lat, void *ws_latent,
+                           size_t ws_latent_bytes, void *stream);
+nh_status nh_moe_latent_out(const nh_moe_config *cfg, int64_t T, const void *y_lat,
+                            const void *w_latent_fc2, float *y_acc, void *ws_latent,
+                            size_t ws_latent_bytes, void *stream);
+
+/*
+ * Clear the status word at the start of workspace `ws` (any of the
+ * library's workspaces), asynchronously on `stream`.  nh_moe_route,
+ * nh_moe_route_permute, nh_moe_shared and the latent projections clear their
+ * own workspace; a sequence that starts on a routed workspace with
+ * nh_moe_permute (the experts of a latent block) calls this first.
+ */
+nh_status nh_moe_reset_status(void *ws, void *stream);
 
 /*
  * Synchronises `stream`, reads the workspace status word and returns it

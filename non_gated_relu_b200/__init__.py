@@ -23,7 +23,8 @@ from . import build as _build
 
 __all__ = ["NHMoEError", "Config", "Layout", "config_from", "load", "validate", "workspace_size",
            "workspace_layout", "shared_workspace_size", "route", "route_noalloc", "route_permute", "permute", "forward", "experts_up", "experts_down", "shared", "forward_nvfp4", "shared_nvfp4", "nvfp4_weight",
-           "finalize", "finalize_partial", "cast_output", "check_device", "selftest_timeout", "library_path", "NemotronHMoE"]
+           "finalize", "finalize_partial", "cast_output", "latent_config", "latent_workspace_size",
+           "latent_in", "latent_out", "reset_status", "check_device", "selftest_timeout", "library_path", "NemotronHMoE"]
 
 NH_OK, NH_ERR_INVALID_ARG, NH_ERR_UNSUPPORTED, NH_ERR_CUDA, NH_ERR_TIMEOUT, NH_ERR_DEVICE_CHECK = range(6)
 STATUS_NAMES = {0: "NH_OK", 1: "NH_ERR_INVALID_ARG", 2: "NH_ERR_UNSUPPORTED", 3: "NH_ERR_CUDA",
@@ -45,7 +46,8 @@ class Config(ctypes.Structure):
                 ("moe_shared_expert_intermediate_size", ctypes.c_int32),
                 ("n_shared_experts", ctypes.c_int32), ("norm_topk_prob", ctypes.c_int32),
                 ("routed_scaling_factor", ctypes.c_float), ("dtype", ctypes.c_int32),
-                ("group_score", ctypes.c_int32), ("weight_format", ctypes.c_int32)]
+                ("group_score", ctypes.c_int32), ("weight_format", ctypes.c_int32),
+                ("latent_size", ctypes.c_int32)]
 
 
 class NvFp4Weight(ctypes.Structure):
@@ -80,7 +82,7 @@ def config_from(c, group_score: int = 0) -> Config:
                   NH_BF16 if dt in ("bf16", NH_BF16) else NH_F32,
                   int(getattr(c, "group_score", group_score)),
                   NH_WEIGHTS_NVFP4 if getattr(c, "weight_format", "native") in ("nvfp4", 1)
-                  else NH_WEIGHTS_NATIVE)
+                  else NH_WEIGHTS_NATIVE, int(getattr(c, "latent_size", 0) or 0))
 
 
 _lock = threading.Lock()
@@ -90,7 +92,9 @@ _EXPORTS = ["nh_moe_validate", "nh_moe_workspace_size", "nh_moe_workspace_layout
             "nh_moe_shared_workspace_size", "nh_moe_route", "nh_moe_route_noalloc", "nh_moe_route_permute",
             "nh_moe_permute", "nh_moe_forward", "nh_moe_experts_up", "nh_moe_experts_down",
             "nh_moe_shared", "nh_moe_finalize", "nh_moe_finalize_partial", "nh_moe_cast_output",
-            "nh_moe_check_device", "nh_moe_selftest_timeout",
+            "nh_moe_latent_config", "nh_moe_latent_workspace_size", "nh_moe_latent_in",
+            "nh_moe_latent_out", "nh_moe_reset_status", "nh_moe_check_device",
+            "nh_moe_selftest_timeout",
             "nh_last_error", "nh_version"]
 
 
@@ -128,7 +132,12 @@ def load():
             "nh_moe_finalize": [C, I64, P, S, P, P, P],
             "nh_moe_finalize_partial": [C, I64, P, S, P, P, P],
             "nh_moe_cast_output": [C, I64, P, P, P],
+            "nh_moe_latent_config": [C, C],
+            "nh_moe_latent_workspace_size": [C, I64, ctypes.POINTER(S)],
+            "nh_moe_latent_in": [C, I64, P, P, P, P, S, P],
+            "nh_moe_latent_out": [C, I64, P, P, P, P, S, P],
             "nh_moe_check_device": [P, P],
+            "nh_moe_reset_status": [P, P],
             "nh_moe_selftest_timeout": [P, ctypes.c_uint64, P],
         }
         for name, args in sig.items():
@@ -283,6 +292,41 @@ def cast_output(cfg, T: int, y_f32, y, stream=None):
     """y = dtype(y_f32), the one rounding of an all-reduced block output."""
     c = config_from(cfg)
     _check(load().nh_moe_cast_output(ctypes.byref(c), T, _p(y_f32), _p(y), _stream(stream)))
+
+
+def latent_config(cfg) -> Config:
+    """The expert-width config the routed-expert calls of a latent block take
+    (hidden_size = latent_size, no latent projections, no shared expert)."""
+    c = config_from(cfg)
+    out = Config()
+    _check(load().nh_moe_latent_config(ctypes.byref(c), ctypes.byref(out)))
+    return out
+
+
+def latent_workspace_size(cfg, T: int) -> int:
+    c = config_from(cfg)
+    n = ctypes.c_size_t()
+    _check(load().nh_moe_latent_workspace_size(ctypes.byref(c), T, ctypes.byref(n)))
+    return n.value
+
+
+def latent_in(cfg, x, w_latent_fc1, x_lat, ws_latent, stream=None):
+    """x_lat = dtype(x W_fc1^T)."""
+    c = config_from(cfg)
+    _check(load().nh_moe_latent_in(ctypes.byref(c), x.shape[0], _p(x), _p(w_latent_fc1),
+                                   _p(x_lat), _p(ws_latent), _nbytes(ws_latent), _stream(stream)))
+
+
+def latent_out(cfg, T: int, y_lat, w_latent_fc2, y_acc, ws_latent, stream=None):
+    """y_acc += y_lat W_fc2^T (y_acc = ... without a shared expert), float32."""
+    c = config_from(cfg)
+    _check(load().nh_moe_latent_out(ctypes.byref(c), T, _p(y_lat), _p(w_latent_fc2), _p(y_acc),
+                                    _p(ws_latent), _nbytes(ws_latent), _stream(stream)))
+
+
+def reset_status(ws, stream=None):
+    """Clear a workspace's status word (asynchronously, on `stream`)."""
+    _check(load().nh_moe_reset_status(_p(ws), _stream(stream)))
 
 
 def check_device(ws, stream=None) -> int:

@@ -8,6 +8,14 @@ call runs, on the caller's stream and a side stream:
     main: route + permute -> forward (routed experts) --+
     side: shared expert ----------------------------------+-> finalize
 
+With latent projections (config ``latent_size`` L > 0; the modules
+fc1_latent_proj / fc2_latent_proj of the ModelOpt descriptor
+NemotronHMoELayerDescriptor) the routed experts run in width L:
+
+    main: route(x) -> fc1: x_lat -> permute + forward + finalize in width L
+          -> y_lat --+-> fc2: y_shared += y_lat W_fc2^T -> cast -> y
+    side: shared expert(x) -> y_shared
+
 All arithmetic happens in libnhmoe's kernels; this class only owns buffers,
 streams, events and (optionally) a CUDA graph of the call sequence.
 """
@@ -19,9 +27,11 @@ from typing import Dict, Optional
 import numpy as np
 import torch
 
-from . import (check_device, config_from, finalize, finalize_partial, forward, forward_nvfp4,
-               nvfp4_weight, route_permute, shared, shared_nvfp4, shared_workspace_size, validate,
-               workspace_size, NH_BF16, NH_WEIGHTS_NVFP4)
+from . import (cast_output, check_device, config_from, finalize, finalize_partial, forward,
+               forward_nvfp4, latent_config, latent_in, latent_out, latent_workspace_size,
+               nvfp4_weight, permute, reset_status, route, route_permute, shared, shared_nvfp4,
+               shared_workspace_size, validate, workspace_layout, workspace_size, NH_BF16,
+               NH_WEIGHTS_NVFP4)
 
 
 def _to_device(a, dtype: torch.dtype, device) -> torch.Tensor:
@@ -48,6 +58,13 @@ class Buffers:
     y_shared: Optional[torch.Tensor]
     y: torch.Tensor
     y_f32: Optional[torch.Tensor] = None     # tensor-parallel partial sum (float32)
+    # latent blocks: routing workspace (full width), projection workspace,
+    # x_lat / y_lat [T, L], float32 accumulator [T, H] (y_shared when present)
+    ws_route: Optional[torch.Tensor] = None
+    ws_lat: Optional[torch.Tensor] = None
+    x_lat: Optional[torch.Tensor] = None
+    y_lat: Optional[torch.Tensor] = None
+    y_acc: Optional[torch.Tensor] = None
 
 
 class NemotronHMoE:
@@ -61,7 +78,8 @@ class NemotronHMoE:
     """
 
     def __init__(self, cfg, w_router, w_up=None, w_down=None, w_shared_up=None,
-                 w_shared_down=None, bias=None, device=None, nvfp4=None):
+                 w_shared_down=None, bias=None, device=None, nvfp4=None, w_latent_fc1=None,
+                 w_latent_fc2=None):
         self.cfg = cfg
         self.c = config_from(cfg)
         validate(self.c)
@@ -96,6 +114,17 @@ class NemotronHMoE:
             self.w_shared_down = _to_device(w_shared_down, self.dtype, self.device)
             if self.has_shared and (self.w_shared_up is None or self.w_shared_down is None):
                 raise ValueError("config has a shared expert but no shared weights were given")
+        self.latent = bool(self.c.latent_size)
+        if self.latent:
+            # routed-expert calls take the expert-width config
+            self.c_exp = latent_config(self.c)
+            self.L = self.c.latent_size
+            self.w_latent_fc1 = _to_device(w_latent_fc1, self.dtype, self.device)
+            self.w_latent_fc2 = _to_device(w_latent_fc2, self.dtype, self.device)
+            if self.w_latent_fc1 is None or self.w_latent_fc2 is None:
+                raise ValueError("config has latent_size > 0: pass w_latent_fc1 / w_latent_fc2")
+        else:
+            self.c_exp = self.c
         with torch.cuda.device(self.device):
             self.side = torch.cuda.Stream()
         self._bufs: Dict[int, Buffers] = {}
@@ -107,7 +136,7 @@ class NemotronHMoE:
         b = self._bufs.get(T)
         if b is None:
             dev = self.device
-            ws = torch.empty(workspace_size(self.c, T), dtype=torch.uint8, device=dev)
+            ws = torch.empty(workspace_size(self.c_exp, T), dtype=torch.uint8, device=dev)
             wss = ys = None
             if self.has_shared:
                 wss = torch.empty(shared_workspace_size(self.c, T), dtype=torch.uint8, device=dev)
@@ -116,6 +145,15 @@ class NemotronHMoE:
                         torch.empty((T, self.k), dtype=torch.int32, device=dev),
                         torch.empty((T, self.k), dtype=torch.float32, device=dev), ys,
                         torch.empty((T, self.H), dtype=self.dtype, device=dev))
+            if self.latent:
+                b.ws_route = torch.empty(max(256, workspace_layout(self.c, T).counts),
+                                         dtype=torch.uint8, device=dev)
+                b.ws_lat = torch.empty(latent_workspace_size(self.c, T), dtype=torch.uint8,
+                                       device=dev)
+                b.x_lat = torch.empty((T, self.L), dtype=self.dtype, device=dev)
+                b.y_lat = torch.empty((T, self.L), dtype=self.dtype, device=dev)
+                b.y_acc = (b.y_shared if self.has_shared else
+                           torch.empty((T, self.H), dtype=torch.float32, device=dev))
             self._bufs[T] = b
         return b
 
@@ -147,6 +185,9 @@ class NemotronHMoE:
             pop()
             join = torch.cuda.Event()
             join.record(self.side)
+        if self.latent:
+            return self._forward_latent(x, b, main, join if self.has_shared else None, partial,
+                                        push, pop)
         push("route_permute")
         route_permute(self.c, x, self.w_router, self.bias, b.topk_idx, b.topk_w, b.ws, stream=main)
         pop()
@@ -165,6 +206,36 @@ class NemotronHMoE:
             finalize(self.c, T, b.ws, b.y_shared, b.y, stream=main)
         pop()
         return b.y_f32 if partial else b.y
+
+    def _forward_latent(self, x, b, main, join, partial, push, pop):
+        T = x.shape[0]
+        push("route")
+        route(self.c, x, self.w_router, self.bias, b.topk_idx, b.topk_w, b.ws_route, stream=main)
+        pop()
+        push("latent_in")
+        latent_in(self.c, x, self.w_latent_fc1, b.x_lat, b.ws_lat, stream=main)
+        pop()
+        push("experts")
+        ce = self.c_exp
+        reset_status(b.ws, stream=main)
+        permute(ce, b.x_lat, b.topk_idx, b.topk_w, b.ws, stream=main)
+        if self.nvfp4:
+            forward_nvfp4(ce, b.x_lat, self.q4["up"], self.q4["down"], b.ws, stream=main)
+        else:
+            forward(ce, b.x_lat, self.w_up, self.w_down, b.ws, stream=main)
+        finalize(ce, T, b.ws, None, b.y_lat, stream=main)
+        pop()
+        if join is not None:
+            main.wait_event(join)
+        push("latent_out")
+        latent_out(self.c, T, b.y_lat, self.w_latent_fc2, b.y_acc, b.ws_lat, stream=main)
+        pop()
+        if partial:
+            return b.y_acc
+        push("cast")
+        cast_output(self.c, T, b.y_acc, b.y, stream=main)
+        pop()
+        return b.y
 
     def capture(self, T: int):
         """Capture the call sequence for T tokens in a CUDA graph.
@@ -192,8 +263,9 @@ class NemotronHMoE:
         """Status word of the last call for T tokens (synchronises)."""
         b = self.buffers(T)
         rc = check_device(b.ws)
-        if rc == 0 and b.ws_shared is not None:
-            rc = check_device(b.ws_shared)
+        for extra in (b.ws_shared, b.ws_route, b.ws_lat):
+            if rc == 0 and extra is not None:
+                rc = check_device(extra)
         return rc
 
     def __call__(self, x, use_graph: bool = True):

@@ -13,6 +13,9 @@ enum Epilogue : int {
   EPI_UP_RELU2 = 0,      // out (dtype) [rows, N] = relu(acc)^2
   EPI_DOWN_WEIGHTED = 1, // out (dtype) [rows, N] = perm_w[r] * acc   (routed partial rows)
   EPI_STORE_F32 = 2,     // out (float32) [rows, N] = acc
+  EPI_STORE = 3,         // out (dtype) [rows, N] = acc             (latent fc1 projection)
+  EPI_ADD_F32 = 4,       // out (float32) [rows, N] += acc          (latent fc2 projection;
+                         //   each element has one owner tile: no atomics)
 };
 
 struct GemmArgs {
@@ -97,6 +100,10 @@ __global__ void __launch_bounds__(256) simt_grouped_gemm(GemmArgs g) {
         static_cast<Tin*>(g.out)[(size_t)r * g.ldo + n] = from_f32<Tin>(relu2(v));
       } else if (g.epi == EPI_DOWN_WEIGHTED) {
         static_cast<Tin*>(g.out)[(size_t)r * g.ldo + n] = from_f32<Tin>(g.perm_w[r] * v);
+      } else if (g.epi == EPI_STORE) {
+        static_cast<Tin*>(g.out)[(size_t)r * g.ldo + n] = from_f32<Tin>(v);
+      } else if (g.epi == EPI_ADD_F32) {
+        static_cast<float*>(g.out)[(size_t)r * g.ldo + n] += v;
       } else {
         static_cast<float*>(g.out)[(size_t)r * g.ldo + n] = v;
       }

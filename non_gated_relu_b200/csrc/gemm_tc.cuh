@@ -94,14 +94,22 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, uint64
 
 // epilogue of 32 consecutive output features of one row (prefill orientation)
 __device__ __forceinline__ void epi_row32(const TcArgs& g, int r, int n, const float* v) {
-  if (g.epi == EPI_STORE_F32) {
+  if (g.epi == EPI_STORE_F32 || g.epi == EPI_ADD_F32) {
     float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.out) + (size_t)r * g.ldo + n);
+    const bool add = g.epi == EPI_ADD_F32;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) dst[i] = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+    for (int i = 0; i < 8; ++i) {
+      float4 o = make_float4(v[4 * i], v[4 * i + 1], v[4 * i + 2], v[4 * i + 3]);
+      if (add) {
+        const float4 a = dst[i];
+        o.x += a.x; o.y += a.y; o.z += a.z; o.w += a.w;
+      }
+      dst[i] = o;
+    }
     return;
   }
   const bool up = g.epi == EPI_UP_RELU2;
-  const float w = up ? 1.f : g.perm_w[r];
+  const float w = (up || g.epi == EPI_STORE) ? 1.f : g.perm_w[r];
   float o[32];
 #pragma unroll
   for (int i = 0; i < 32; ++i) o[i] = up ? relu2(v[i]) : w * v[i];
@@ -123,6 +131,10 @@ __device__ __forceinline__ void epi_elem(const TcArgs& g, int r, int f, float v)
     static_cast<__nv_bfloat16*>(g.out)[(size_t)r * g.ldo + f] = __float2bfloat16_rn(relu2(v));
   } else if (g.epi == EPI_DOWN_WEIGHTED) {
     static_cast<__nv_bfloat16*>(g.out)[(size_t)r * g.ldo + f] = __float2bfloat16_rn(g.perm_w[r] * v);
+  } else if (g.epi == EPI_STORE) {
+    static_cast<__nv_bfloat16*>(g.out)[(size_t)r * g.ldo + f] = __float2bfloat16_rn(v);
+  } else if (g.epi == EPI_ADD_F32) {
+    static_cast<float*>(g.out)[(size_t)r * g.ldo + f] += v;
   } else {
     static_cast<float*>(g.out)[(size_t)r * g.ldo + f] = v;
   }

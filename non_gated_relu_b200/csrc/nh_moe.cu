@@ -108,6 +108,7 @@ static nh_status validate(const nh_moe_config* c) {
     return fail(NH_ERR_INVALID_ARG, "unknown weight_format");
   if (c->weight_format == NH_WEIGHTS_NVFP4 && c->dtype != NH_BF16)
     return fail(NH_ERR_INVALID_ARG, "NVFP4 weights need bf16 activations (W4A16)");
+  if (c->latent_size < 0) return fail(NH_ERR_INVALID_ARG, "latent_size must be >= 0");
   // valid; now what the kernels implement
   if (c->n_routed_experts > MAX_E)
     return fail(NH_ERR_UNSUPPORTED, "n_routed_experts > %d", MAX_E);
@@ -115,10 +116,11 @@ static nh_status validate(const nh_moe_config* c) {
   if (c->num_experts_per_tok > MAX_K) return fail(NH_ERR_UNSUPPORTED, "num_experts_per_tok > %d", MAX_K);
   if (c->dtype == NH_BF16) {
     if (c->hidden_size % 64 || c->moe_intermediate_size % 64 ||
-        (c->n_shared_experts && c->moe_shared_expert_intermediate_size % 64))
+        (c->n_shared_experts && c->moe_shared_expert_intermediate_size % 64) ||
+        c->latent_size % 64)
       return fail(NH_ERR_UNSUPPORTED,
-                  "bf16 tensor-core path needs hidden, intermediate and shared sizes that are "
-                  "multiples of 64");
+                  "bf16 tensor-core path needs hidden, intermediate, shared and latent sizes "
+                  "that are multiples of 64");
   }
   return NH_OK;
 }
@@ -219,6 +221,15 @@ static nh_status check_ws(const Plan& p, void* ws, size_t ws_bytes) {
     return fail(NH_ERR_INVALID_ARG, "ws must be %zu-byte aligned", ALIGN);
   if (ws_bytes < p.lay.total_bytes)
     return fail(NH_ERR_INVALID_ARG, "ws holds %zu bytes, %zu needed", ws_bytes, p.lay.total_bytes);
+  return NH_OK;
+}
+
+// the routed-expert calls take the expert-width config of a latent block
+static nh_status no_latent(const nh_moe_config* c, const char* what) {
+  if (c && c->latent_size)
+    return fail(NH_ERR_INVALID_ARG,
+                "%s: config has latent_size %d; pass the expert-width config of "
+                "nh_moe_latent_config", what, c->latent_size);
   return NH_OK;
 }
 
@@ -792,7 +803,13 @@ nh_status nh_moe_route(const nh_moe_config* cfg, int64_t T, const void* x, const
                        size_t ws_bytes, void* stream) {
   Plan p;
   NH_TRY(make_plan(cfg, T, &p));
-  NH_TRY(check_ws(p, ws, ws_bytes));
+  // routing touches only the regions before `counts` (status, logits, router_w)
+  NH_TRY(check_ptr(ws, "ws"));
+  if (reinterpret_cast<uintptr_t>(ws) % ALIGN)
+    return fail(NH_ERR_INVALID_ARG, "ws must be %zu-byte aligned", ALIGN);
+  if (ws_bytes < p.lay.counts)
+    return fail(NH_ERR_INVALID_ARG, "ws holds %zu bytes, %zu needed for routing", ws_bytes,
+                p.lay.counts);
   if (T == 0) return NH_OK;
   NH_TRY(check_ptr(x, "x"));
   NH_TRY(check_ptr(w_router, "w_router"));
@@ -930,6 +947,7 @@ nh_status nh_moe_route_noalloc(const nh_moe_config* cfg, int64_t T, const void* 
 nh_status nh_moe_permute(const nh_moe_config* cfg, int64_t T, const void* x,
                          const int32_t* topk_idx, const float* topk_w, void* ws, size_t ws_bytes,
                          void* stream) {
+  NH_TRY(no_latent(cfg, "nh_moe_permute"));
   Plan p;
   NH_TRY(make_plan(cfg, T, &p));
   NH_TRY(check_ws(p, ws, ws_bytes));
@@ -995,6 +1013,7 @@ nh_status nh_moe_permute(const nh_moe_config* cfg, int64_t T, const void* x,
 nh_status nh_moe_route_permute(const nh_moe_config* cfg, int64_t T, const void* x,
                                const float* w_router, const float* bias, int32_t* topk_idx,
                                float* topk_w, void* ws, size_t ws_bytes, void* stream) {
+  NH_TRY(no_latent(cfg, "nh_moe_route_permute"));
   Plan p;
   NH_TRY(make_plan(cfg, T, &p));
   NH_TRY(check_ws(p, ws, ws_bytes));
@@ -1042,6 +1061,7 @@ nh_status nh_moe_route_permute(const nh_moe_config* cfg, int64_t T, const void* 
 static nh_status experts_phase(const nh_moe_config* cfg, int64_t T, const void* x, const void* w,
                                void* ws, size_t ws_bytes, void* stream, bool up_phase,
                                const nh_nvfp4_weight* wq = nullptr) {
+  NH_TRY(no_latent(cfg, "routed experts"));
   Plan p;
   NH_TRY(make_plan(cfg, T, &p));
   NH_TRY(check_ws(p, ws, ws_bytes));
@@ -1208,6 +1228,7 @@ static nh_status shared_impl(const nh_moe_config* cfg, int64_t T, const void* x,
 static nh_status finalize_impl(const nh_moe_config* cfg, int64_t T, const void* ws,
                                size_t ws_bytes, const float* y_shared, void* y, bool out_f32,
                                void* stream) {
+  NH_TRY(no_latent(cfg, "finalize"));
   Plan p;
   NH_TRY(make_plan(cfg, T, &p));
   NH_TRY(check_ws(p, const_cast<void*>(ws), ws_bytes));
@@ -1286,6 +1307,92 @@ nh_status nh_moe_cast_output(const nh_moe_config* cfg, int64_t T, const float* y
                      st, y_f32, static_cast<float*>(y), n)));
   }
   return launch_check("cast_output");
+}
+
+// ---------------------------------------------------------------------------
+// latent projections around the routed experts
+// ---------------------------------------------------------------------------
+nh_status nh_moe_latent_config(const nh_moe_config* cfg, nh_moe_config* expert_cfg) {
+  NH_TRY(validate(cfg));
+  if (!expert_cfg) return fail(NH_ERR_INVALID_ARG, "expert_cfg is NULL");
+  if (cfg->latent_size < 1) return fail(NH_ERR_INVALID_ARG, "config has no latent projections");
+  *expert_cfg = *cfg;
+  expert_cfg->hidden_size = cfg->latent_size;
+  expert_cfg->latent_size = 0;
+  expert_cfg->n_shared_experts = 0;
+  return validate(expert_cfg);
+}
+
+nh_status nh_moe_latent_workspace_size(const nh_moe_config* cfg, int64_t T, size_t* bytes) {
+  if (!bytes) return fail(NH_ERR_INVALID_ARG, "bytes is NULL");
+  Plan p;
+  NH_TRY(make_plan(cfg, T, &p));
+  if (cfg->latent_size < 1) return fail(NH_ERR_INVALID_ARG, "config has no latent projections");
+  *bytes = ALIGN;   // status word and tile scheduler counters
+  return NH_OK;
+}
+
+// out = x W^T for one projection: fc1 (H -> L, EPI_STORE) or fc2 (L -> H, EPI_ADD_F32)
+static nh_status latent_gemm(const nh_moe_config* cfg, int64_t T, const void* a, const void* w,
+                             void* out, bool fc1, void* ws, size_t ws_bytes, void* stream) {
+  Plan p;
+  NH_TRY(make_plan(cfg, T, &p));
+  if (cfg->latent_size < 1) return fail(NH_ERR_INVALID_ARG, "config has no latent projections");
+  NH_TRY(check_ptr(ws, "ws_latent"));
+  if (ws_bytes < ALIGN)
+    return fail(NH_ERR_INVALID_ARG, "ws_latent holds %zu bytes, %zu needed", ws_bytes, ALIGN);
+  if (T == 0) return NH_OK;
+  NH_TRY(check_ptr(a, fc1 ? "x" : "y_lat"));
+  NH_TRY(check_ptr(w, fc1 ? "w_latent_fc1" : "w_latent_fc2"));
+  NH_TRY(check_ptr(out, fc1 ? "x_lat" : "y_acc"));
+  int dev;
+  NH_TRY(device_setup(&dev));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  int* status = static_cast<int*>(ws);
+  NH_CUDA(cudaMemsetAsync(status, 0, STATUS_BYTES, st));
+  // the projections are dense layers in the activation dtype: plan their tiles
+  // as native-format weights
+  nh_moe_config cn = *cfg;
+  cn.weight_format = NH_WEIGHTS_NATIVE;
+  int tr, sw;
+  tile_plan(&cn, T, &tr, &sw);
+  const int L = cfg->latent_size;
+  GemmCall g{};
+  g.A = a;
+  g.rows = T;
+  g.W = w;
+  g.n_exp = 1;
+  g.N = fc1 ? L : p.H;
+  g.K = fc1 ? p.H : L;
+  g.tiles = nullptr;
+  g.tile_rows = tr;
+  g.swap = sw;
+  // fc2 adds onto the shared expert's output; without a shared expert it writes
+  g.epi = fc1 ? EPI_STORE : (cfg->n_shared_experts ? EPI_ADD_F32 : EPI_STORE_F32);
+  g.out = out;
+  g.ldo = g.N;
+  g.status = status;
+  g.sched = reinterpret_cast<unsigned int*>(status + 4);
+  return run_gemm(p, g, dev, st);
+}
+
+nh_status nh_moe_latent_in(const nh_moe_config* cfg, int64_t T, const void* x,
+                           const void* w_latent_fc1, void* x_lat, void* ws_latent,
+                           size_t ws_latent_bytes, void* stream) {
+  return latent_gemm(cfg, T, x, w_latent_fc1, x_lat, true, ws_latent, ws_latent_bytes, stream);
+}
+
+nh_status nh_moe_latent_out(const nh_moe_config* cfg, int64_t T, const void* y_lat,
+                            const void* w_latent_fc2, float* y_acc, void* ws_latent,
+                            size_t ws_latent_bytes, void* stream) {
+  return latent_gemm(cfg, T, y_lat, w_latent_fc2, y_acc, false, ws_latent, ws_latent_bytes,
+                     stream);
+}
+
+nh_status nh_moe_reset_status(void* ws, void* stream) {
+  NH_TRY(check_ptr(ws, "ws"));
+  NH_CUDA(cudaMemsetAsync(ws, 0, STATUS_BYTES, static_cast<cudaStream_t>(stream)));
+  return NH_OK;
 }
 
 nh_status nh_moe_check_device(void* ws, void* stream) {

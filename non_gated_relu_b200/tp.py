@@ -144,6 +144,8 @@ class TPNemotronHMoE:
         self.rank = rank if rank is not None else (dist.get_rank(group) if dist_on else 0)
         self.group = group
         self.cfg = cfg
+        if getattr(cfg, "latent_size", 0):
+            raise NotImplementedError("tensor parallelism of a latent block is not built")
         self.cfg_rank = shard_config(cfg, self.world, self.rank)
         q = None
         if config_from(cfg).weight_format == NH_WEIGHTS_NVFP4:

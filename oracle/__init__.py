@@ -73,6 +73,9 @@ def _load():
             lib.nho_forward_wt.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int64, P, P, P, W, W, W,
                                            W, P, P, P, ctypes.c_int64, P, P, P]
             lib.nho_dequant.argtypes = [W, ctypes.c_int64, P]
+            lib.nho_forward_latent.argtypes = [ctypes.POINTER(_Cfg), ctypes.c_int64,
+                                               ctypes.c_int64, P, P, P, W, W, W, W, P, P, P, P,
+                                               P, ctypes.c_int64, P, P, P]
             _lib = lib
     return _lib
 
@@ -205,6 +208,58 @@ def _forward_nvfp4(inp, tok, oi, ow, group_score):
     return y, idx, w
 
 
+def _wt_native(a, dtype, rows, cols):
+    a = _stored(a, dtype)
+    return _Wt(1 if dtype == "bf16" else 0, a.ctypes.data, None, None, rows, cols, 0), a
+
+
+def _forward_latent(inp, tok, oi, ow, group_score):
+    """Latent block (nho_forward_latent): routed experts between
+    fc1_latent_proj and fc2_latent_proj; parity of this reading is unpinned."""
+    cfg = inp.cfg
+    lib = _load()
+    c = _cfg(cfg, group_score)
+    n = tok.shape[0]
+    L = cfg.latent_size
+    y = np.zeros((n, cfg.H), np.float64)
+    idx = np.zeros((n, cfg.k), np.int32)
+    w = np.zeros((n, cfg.k), np.float64)
+    keep = []
+    if getattr(inp, "nvfp4", None) is not None:
+        q = inp.nvfp4
+        up, k1 = _wt_nvfp4(q["up"], cfg.I, L)
+        dn, k2 = _wt_nvfp4(q["down"], L, cfg.I)
+        su = sd = None
+        keep += [k1, k2]
+        if cfg.n_shared_experts:
+            su, k3 = _wt_nvfp4(q["shared_up"], cfg.S, cfg.H)
+            sd, k4 = _wt_nvfp4(q["shared_down"], cfg.H, cfg.S)
+            keep += [k3, k4]
+    else:
+        up, k1 = _wt_native(inp.w_up, cfg.dtype, cfg.I, L)
+        dn, k2 = _wt_native(inp.w_down, cfg.dtype, L, cfg.I)
+        su = sd = None
+        keep += [k1, k2]
+        if cfg.n_shared_experts:
+            su, k3 = _wt_native(inp.w_shared_up, cfg.dtype, cfg.S, cfg.H)
+            sd, k4 = _wt_native(inp.w_shared_down, cfg.dtype, cfg.H, cfg.S)
+            keep += [k3, k4]
+    x = _stored(inp.x, cfg.dtype)
+    wl1 = _stored(inp.w_latent_fc1, cfg.dtype)
+    wl2 = _stored(inp.w_latent_fc2, cfg.dtype)
+    wr = np.ascontiguousarray(inp.w_router, np.float32)
+    b = None if inp.bias is None else np.ascontiguousarray(inp.bias, np.float32)
+    rc = lib.nho_forward_latent(ctypes.byref(c), L, inp.x.shape[0], _ptr(x), _ptr(wr), _ptr(b),
+                                ctypes.byref(up), ctypes.byref(dn),
+                                ctypes.byref(su) if su is not None else None,
+                                ctypes.byref(sd) if sd is not None else None,
+                                _ptr(wl1), _ptr(wl2), _ptr(oi), _ptr(ow), _ptr(tok), n, _ptr(y),
+                                _ptr(idx), _ptr(w))
+    if rc:
+        raise OracleError(f"nho_forward_latent failed ({rc})")
+    return y, idx, w
+
+
 def forward(inp, tokens=None, override_idx=None, override_w=None, group_score: int = 0):
     """Block output y (float64 [n_tok, H]) for the listed tokens (default: all).
 
@@ -225,6 +280,8 @@ def forward(inp, tokens=None, override_idx=None, override_w=None, group_score: i
     if override_idx is not None:
         oi = np.ascontiguousarray(override_idx, np.int32).reshape(n, cfg.k)
         ow = np.ascontiguousarray(override_w, np.float64).reshape(n, cfg.k)
+    if getattr(cfg, "latent_size", 0):
+        return _forward_latent(inp, tok, oi, ow, group_score)
     if getattr(inp, "nvfp4", None) is not None:
         return _forward_nvfp4(inp, tok, oi, ow, group_score)
     x = _stored(inp.x, cfg.dtype)

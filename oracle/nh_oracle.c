@@ -242,10 +242,10 @@ int nho_route(const nho_cfg *c, int64_t T, const void *x, const float *wr, const
 }
 
 /* out[H] += scale * Wd relu(Wu xt)^2 for matrix `mat` of the up tensor (rows n,
- * cols H) and the down tensor (rows H, cols n); u is scratch of n doubles. */
-static void mlp_relu2(const nho_cfg *c, const double *xt, const nho_wt *up, const nho_wt *down,
+ * cols H) and the down tensor (rows H, cols n); u is scratch of n doubles.
+ * H is the width of xt and out (the hidden size, or the latent size). */
+static void mlp_relu2(int64_t H, const double *xt, const nho_wt *up, const nho_wt *down,
                       int64_t mat, int64_t n, double scale, double *u, double *out) {
-    const int64_t H = c->H;
     for (int64_t i = 0; i < n; ++i) {
         double a = 0.0;
         for (int64_t h = 0; h < H; ++h) a += wt_get(up, mat, i * H + h) * xt[h];
@@ -309,8 +309,8 @@ int nho_forward_wt(const nho_cfg *c, int64_t T, const void *x, const float *wr, 
         }
         double *yt = y + n * H;
         for (int64_t h = 0; h < H; ++h) yt[h] = 0.0;
-        for (int64_t j = 0; j < k; ++j) mlp_relu2(c, xt, up, down, idx[j], I, w[j], u, yt);
-        if (c->n_shared) mlp_relu2(c, xt, su, sd, 0, S, 1.0, u, yt);
+        for (int64_t j = 0; j < k; ++j) mlp_relu2(H, xt, up, down, idx[j], I, w[j], u, yt);
+        if (c->n_shared) mlp_relu2(H, xt, su, sd, 0, S, 1.0, u, yt);
         if (idx_out)
             for (int64_t j = 0; j < k; ++j) idx_out[n * k + j] = idx[j];
         if (w_out)
@@ -336,4 +336,87 @@ int nho_forward(const nho_cfg *c, int64_t T, const void *x, const float *wr, con
     return nho_forward_wt(c, T, x, wr, bias, &up, &down, c->n_shared ? &su : NULL,
                           c->n_shared ? &sd : NULL, ovr_idx, ovr_w, tokens, n_tok, y, idx_out,
                           w_out);
+}
+
+/*
+ * Latent MoE: the routed experts work in a latent width L between two
+ * projections (ModelOpt descriptor "NemotronHMoELayerDescriptor", parameters
+ * latent_fc1_name='fc1_latent_proj' and latent_fc2_name='fc2_latent_proj';
+ * the descriptor names the two modules and no more).  Reading used:
+ *   xl = Wl1 x                           (fc1_latent_proj, [L][H])
+ *   yl = sum_j w_j * Wd[e_j] relu(Wu[e_j] xl)^2   (experts in width L:
+ *                                         Wu [E][I][L], Wd [E][L][I])
+ *   y  = Wl2 yl + Wsd relu(Wsu x)^2      (fc2_latent_proj, [H][L]; the
+ *                                         router and the shared expert see
+ *                                         the full-width x)
+ * with the routing of steps 1-6 on x.  No intermediate rounding.
+ * PARITY UNPINNED as a reading of the pages (they give no formula); the
+ * tests pin this function to the plain block at identity projections.
+ * wl1, wl2 are in c->dtype.  Other arguments as nho_forward_wt.
+ */
+int nho_forward_latent(const nho_cfg *c, int64_t L, int64_t T, const void *x, const float *wr,
+                       const float *bias, const nho_wt *up, const nho_wt *down,
+                       const nho_wt *su, const nho_wt *sd, const void *wl1, const void *wl2,
+                       const int32_t *ovr_idx, const double *ovr_w, const int64_t *tokens,
+                       int64_t n_tok, double *y, int32_t *idx_out, double *w_out) {
+    int rc = nho_check_config(c);
+    if (rc) return rc;
+    if (L < 1 || n_tok < 0 || (n_tok > 0 && (!x || !tokens || !y || !up || !down || !wl1 || !wl2)))
+        return NHO_BAD_ARG;
+    if (!ovr_idx && !wr) return NHO_BAD_ARG;
+    if (c->n_shared && (!su || !sd)) return NHO_BAD_ARG;
+    const int64_t H = c->H, I = c->I, S = c->S, k = c->k;
+    if (up->rows != I || up->cols != L || down->rows != L || down->cols != I) return NHO_BAD_ARG;
+    if (c->n_shared && (su->rows != S || su->cols != H || sd->rows != H || sd->cols != S))
+        return NHO_BAD_ARG;
+    int64_t nmax = I > S ? I : S;
+    double *xt = (double *)malloc(sizeof(double) * (size_t)H);
+    double *xl = (double *)malloc(sizeof(double) * (size_t)L);
+    double *yl = (double *)malloc(sizeof(double) * (size_t)L);
+    double *u = (double *)malloc(sizeof(double) * (size_t)nmax);
+    double *scr = (double *)malloc(sizeof(double) * (size_t)(3 * c->E));
+    int64_t *iscr = (int64_t *)malloc(sizeof(int64_t) * (size_t)(2 * c->E));
+    int32_t *idx = (int32_t *)malloc(sizeof(int32_t) * (size_t)k);
+    double *w = (double *)malloc(sizeof(double) * (size_t)k);
+    if (!xt || !xl || !yl || !u || !scr || !iscr || !idx || !w) {
+        free(xt); free(xl); free(yl); free(u); free(scr); free(iscr); free(idx); free(w);
+        return NHO_NOMEM;
+    }
+    rc = NHO_OK;
+    for (int64_t n = 0; n < n_tok; ++n) {
+        int64_t t = tokens[n];
+        if (t < 0 || t >= T) { rc = NHO_BAD_ARG; break; }
+        for (int64_t h = 0; h < H; ++h) xt[h] = load(x, t * H + h, c->dtype);
+        if (ovr_idx) {
+            for (int64_t j = 0; j < k; ++j) {
+                idx[j] = ovr_idx[n * k + j];
+                w[j] = ovr_w[n * k + j];
+                if (idx[j] < 0 || idx[j] >= c->E) rc = NHO_BAD_ARG;
+            }
+            if (rc) break;
+        } else {
+            double gg, ge;
+            route_one(c, x, t, wr, bias, idx, w, &gg, &ge, scr, iscr);
+        }
+        for (int64_t l = 0; l < L; ++l) {
+            double a = 0.0;
+            for (int64_t h = 0; h < H; ++h) a += load(wl1, l * H + h, c->dtype) * xt[h];
+            xl[l] = a;
+            yl[l] = 0.0;
+        }
+        for (int64_t j = 0; j < k; ++j) mlp_relu2(L, xl, up, down, idx[j], I, w[j], u, yl);
+        double *yt = y + n * H;
+        for (int64_t h = 0; h < H; ++h) {
+            double a = 0.0;
+            for (int64_t l = 0; l < L; ++l) a += load(wl2, h * L + l, c->dtype) * yl[l];
+            yt[h] = a;
+        }
+        if (c->n_shared) mlp_relu2(H, xt, su, sd, 0, S, 1.0, u, yt);
+        if (idx_out)
+            for (int64_t j = 0; j < k; ++j) idx_out[n * k + j] = idx[j];
+        if (w_out)
+            for (int64_t j = 0; j < k; ++j) w_out[n * k + j] = w[j];
+    }
+    free(xt); free(xl); free(yl); free(u); free(scr); free(iscr); free(idx); free(w);
+    return rc;
 }

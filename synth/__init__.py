@@ -28,7 +28,7 @@ from typing import Optional
 import numpy as np
 
 # tensor ids of the independent streams
-_X, _WR, _WUP, _WDOWN, _WSU, _WSD, _SKEW, _TIE, _BIAS = range(1, 10)
+_X, _WR, _WUP, _WDOWN, _WSU, _WSD, _SKEW, _TIE, _BIAS, _WL1, _WL2 = range(1, 12)
 
 
 @dataclasses.dataclass(frozen=True)
@@ -62,6 +62,8 @@ class MoEConfig:
     skew_hot_per_group: int = 0
     tie_fraction: float = 0.0    # fraction of tokens built to tie exactly
     tie_columns: int = 0
+    latent_size: int = 0         # >0: routed experts in this width between
+                                 # fc1_latent_proj [L, H] and fc2_latent_proj [H, L]
 
     # short aliases used by the kernels' notation
     @property
@@ -78,15 +80,23 @@ class MoEConfig:
     def I(self): return self.moe_intermediate_size
     @property
     def S(self): return self.moe_shared_expert_intermediate_size
+    @property
+    def L(self): return self.latent_size
+    @property
+    def HE(self):
+        """Width of the routed experts' input and output (hidden or latent)."""
+        return self.latent_size or self.hidden_size
 
     def replace(self, **kw) -> "MoEConfig":
         return dataclasses.replace(self, **kw)
 
     def flops_per_token(self) -> int:
         """Algorithmic flops per token: router GEMV + k routed MLPs + shared MLP."""
-        f = 2 * self.H * self.E + self.k * 4 * self.H * self.I
+        f = 2 * self.H * self.E + self.k * 4 * self.HE * self.I
         if self.n_shared_experts:
             f += 4 * self.H * self.S
+        if self.latent_size:
+            f += 4 * self.H * self.latent_size
         return f
 
 
@@ -120,6 +130,11 @@ CONFIGS = {
         topk_group=2, num_experts_per_tok=8, moe_intermediate_size=2048,
         moe_shared_expert_intermediate_size=4096, seed=4,
         tie_fraction=0.05, tie_columns=8),
+    # latent projections around the routed experts (width 1024), decode shape
+    "decode_latent_bf16_t8": MoEConfig(
+        "decode_latent_bf16_t8", T=8, hidden_size=2688, n_routed_experts=128, n_group=8,
+        topk_group=1, num_experts_per_tok=6, moe_intermediate_size=1856,
+        moe_shared_expert_intermediate_size=3712, seed=6, latent_size=1024),
 }
 
 CONFIG_ORDER = list(CONFIGS)
@@ -248,6 +263,10 @@ class MoEInputs:
     # NVFP4 workloads: {"up", "down", "shared_up", "shared_down"} ->
     # (codes, scales, global) as returned by quantize_nvfp4
     nvfp4: Optional[dict] = None
+    # latent workloads: fc1_latent_proj [L, H], fc2_latent_proj [H, L] (dtype);
+    # w_up is then [E, I, L] and w_down [E, L, I]
+    w_latent_fc1: Optional[np.ndarray] = None
+    w_latent_fc2: Optional[np.ndarray] = None
 
 
 def default_threads() -> int:
@@ -293,10 +312,23 @@ def make_router_and_x(cfg: MoEConfig, skew_b: Optional[float] = None):
 
 
 def make_expert(cfg: MoEConfig, e: int):
-    """(w_up[e] [I, H], w_down[e] [H, I]) of routed expert e, in the storage dtype."""
-    up = _store(_normal(cfg.seed, _WUP, e, (cfg.I, cfg.H), cfg.w_std), cfg.dtype)
-    down = _store(_normal(cfg.seed, _WDOWN, e, (cfg.H, cfg.I), cfg.w_std), cfg.dtype)
+    """(w_up[e] [I, HE], w_down[e] [HE, I]) of routed expert e, in the storage
+    dtype (HE = hidden size, or the latent size of a latent workload)."""
+    up = _store(_normal(cfg.seed, _WUP, e, (cfg.I, cfg.HE), cfg.w_std), cfg.dtype)
+    down = _store(_normal(cfg.seed, _WDOWN, e, (cfg.HE, cfg.I), cfg.w_std), cfg.dtype)
     return up, down
+
+
+def make_latent(cfg: MoEConfig):
+    """(fc1_latent_proj [L, H], fc2_latent_proj [H, L]) in the storage dtype,
+    drawn with standard deviations 1/sqrt(H) and 1/sqrt(L) (unit-variance
+    latent activations for unit-variance x), or (None, None)."""
+    if not cfg.latent_size:
+        return None, None
+    L, H = cfg.latent_size, cfg.H
+    w1 = _store(_normal(cfg.seed, _WL1, 0, (L, H), H ** -0.5), cfg.dtype)
+    w2 = _store(_normal(cfg.seed, _WL2, 0, (H, L), L ** -0.5), cfg.dtype)
+    return w1, w2
 
 
 def make_inputs(cfg: MoEConfig, skew_b: Optional[float] = None,
@@ -306,8 +338,8 @@ def make_inputs(cfg: MoEConfig, skew_b: Optional[float] = None,
     if cfg.weight_format == "nvfp4":
         return _make_nvfp4_inputs(cfg, x, wr, hot, ties, tcols, skew_b, threads, with_bias)
     sdt = np.uint16 if cfg.dtype == "bf16" else np.float32
-    w_up = np.empty((cfg.E, cfg.I, cfg.H), sdt)
-    w_down = np.empty((cfg.E, cfg.H, cfg.I), sdt)
+    w_up = np.empty((cfg.E, cfg.I, cfg.HE), sdt)
+    w_down = np.empty((cfg.E, cfg.HE, cfg.I), sdt)
 
     def fill(e):
         w_up[e], w_down[e] = make_expert(cfg, e)
@@ -321,13 +353,15 @@ def make_inputs(cfg: MoEConfig, skew_b: Optional[float] = None,
     bias = None
     if with_bias:
         bias = _normal(cfg.seed, _BIAS, 0, (cfg.E,), 0.1).astype(np.float32)
-    return MoEInputs(cfg, x, wr, w_up, w_down, wsu, wsd, bias, hot, ties, tcols, skew_b)
+    wl1, wl2 = make_latent(cfg)
+    return MoEInputs(cfg, x, wr, w_up, w_down, wsu, wsd, bias, hot, ties, tcols, skew_b,
+                     w_latent_fc1=wl1, w_latent_fc2=wl2)
 
 
 def _make_nvfp4_inputs(cfg, x, wr, hot, ties, tcols, skew_b, threads, with_bias):
     """Weights drawn as float32 (same streams as the native format) and encoded
     as NVFP4, one matrix per thread task."""
-    E, H, I, S = cfg.E, cfg.H, cfg.I, cfg.S
+    E, H, I, S = cfg.E, cfg.HE, cfg.I, cfg.S
     pu, pd = nvfp4_scale_pitch(H), nvfp4_scale_pitch(I)
     up = (np.empty((E, I, H // 2), np.uint8), np.empty((E, I, pu), np.uint8), np.empty(E, np.float32))
     dn = (np.empty((E, H, I // 2), np.uint8), np.empty((E, H, pd), np.uint8), np.empty(E, np.float32))
@@ -343,10 +377,13 @@ def _make_nvfp4_inputs(cfg, x, wr, hot, ties, tcols, skew_b, threads, with_bias)
         list(ex.map(fill, range(E)))
     q = {"up": up, "down": dn}
     if cfg.n_shared_experts:
-        q["shared_up"] = quantize_nvfp4(_normal(cfg.seed, _WSU, 0, (S, H), cfg.w_std)[None])
-        q["shared_down"] = quantize_nvfp4(_normal(cfg.seed, _WSD, 0, (H, S), cfg.w_std)[None])
+        Hs = cfg.H
+        q["shared_up"] = quantize_nvfp4(_normal(cfg.seed, _WSU, 0, (S, Hs), cfg.w_std)[None])
+        q["shared_down"] = quantize_nvfp4(_normal(cfg.seed, _WSD, 0, (Hs, S), cfg.w_std)[None])
     bias = _normal(cfg.seed, _BIAS, 0, (E,), 0.1).astype(np.float32) if with_bias else None
-    return MoEInputs(cfg, x, wr, None, None, None, None, bias, hot, ties, tcols, skew_b, q)
+    wl1, wl2 = make_latent(cfg)
+    return MoEInputs(cfg, x, wr, None, None, None, None, bias, hot, ties, tcols, skew_b, q,
+                     w_latent_fc1=wl1, w_latent_fc2=wl2)
 
 
 def to_f64(a: np.ndarray, dtype: str) -> np.ndarray:

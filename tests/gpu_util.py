@@ -43,7 +43,8 @@ def to_dev(a, cfg=None):
 def make_block(inp):
     import non_gated_relu_b200 as nh
     return nh.NemotronHMoE(inp.cfg, inp.w_router, inp.w_up, inp.w_down, inp.w_shared_up,
-                           inp.w_shared_down, bias=inp.bias, nvfp4=inp.nvfp4)
+                           inp.w_shared_down, bias=inp.bias, nvfp4=inp.nvfp4,
+                           w_latent_fc1=inp.w_latent_fc1, w_latent_fc2=inp.w_latent_fc2)
 
 
 def run_block(inp, blk=None):
