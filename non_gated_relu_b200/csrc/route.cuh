@@ -108,10 +108,19 @@ __device__ __forceinline__ void select_token(const SelectArgs& a, int t, const f
                                              float* w_out = nullptr) {
   const int E = a.E, G = a.G, g = E / G;
   float* lraw = sel + E;  // the token's logits, staged next to its selection scores
-  for (int e = lane; e < E; e += 32) {
-    const float le = __ldcg(l + e);  // produced by another block or kernel: read at L2
-    lraw[e] = le;
-    sel[e] = a.use_sigma ? sigmoid_f32(le) + (a.bias ? a.bias[e] : 0.f) : le;
+  // produced by another block or kernel: read at L2, four loads in flight
+  for (int e0 = lane; e0 < E; e0 += 128) {
+    float le[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) le[i] = __ldcg(l + min(e0 + 32 * i, E - 1));
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int e = e0 + 32 * i;
+      if (e < E) {
+        lraw[e] = le[i];
+        sel[e] = a.use_sigma ? sigmoid_f32(le[i]) + (a.bias ? a.bias[e] : 0.f) : le[i];
+      }
+    }
   }
   __syncwarp();
   // group scores: lane q (and q + 32) reduces its group
@@ -159,14 +168,66 @@ __device__ __forceinline__ void select_token(const SelectArgs& a, int t, const f
     pq = bq;
     pv = bv;
   }
+  float ssum = 0.f, my_s = 0.f;
+  int my_e = 0;
+  const int n_cand = a.tg * g;   // experts of the kept groups
+  if (n_cand <= 128) {
+    // Rank every candidate against all candidates under the same total order
+    // (score desc, id asc): a candidate of rank r < k is the r-th pick.  All
+    // ranks are independent, so this is one pass instead of k argmax rounds.
+    int c_e[4], c_r[4];
+    float c_s[4];
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      const int j = lane + 32 * r;
+      c_r[r] = a.k;
+      c_e[r] = 0;
+      c_s[r] = 0.f;
+      if (j < n_cand) {
+        uint64_t kk = keep;          // j-th candidate: kept groups ascending, ids ascending
+        for (int m = j / g; m > 0; --m) kk &= kk - 1;
+        if (kk == 0) continue;       // fewer kept groups (a recorded selection error)
+        const int e = (__ffsll((long long)kk) - 1) * g + j % g;
+        const float v = sel[e];
+        int rank = 0;
+        for (uint64_t k2 = keep; k2; k2 &= k2 - 1) {
+          const int e0 = (__ffsll((long long)k2) - 1) * g;
+          for (int i = 0; i < g; ++i) rank += ranks_before(sel[e0 + i], e0 + i, v, e) ? 1 : 0;
+        }
+        c_e[r] = e;
+        c_r[r] = rank;
+        if (rank < a.k) c_s[r] = sigmoid_f32(lraw[e]);
+      }
+    }
+    __syncwarp();
+    // picks by rank into this warp's scratch (sel / lraw are no longer read);
+    // a slot no candidate fills (only after a selection error) keeps expert 0
+    if (lane < a.k) {
+      sel[lane] = 0.f;
+      lraw[lane] = __int_as_float(0);
+    }
+    __syncwarp();
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+      if (c_r[r] < a.k) {
+        sel[c_r[r]] = c_s[r];
+        lraw[c_r[r]] = __int_as_float(c_e[r]);
+      }
+    }
+    __syncwarp();
+    for (int j = 0; j < a.k; ++j) ssum += sel[j];   // pick order, as the scores are summed below
+    if (lane < a.k) {
+      my_s = sel[lane];
+      my_e = __float_as_int(lraw[lane]);
+    }
+  } else {
   // which of this lane's experts (e = lane + 32 i, E <= 512) lie in kept groups
   uint32_t mine = 0;
   for (int i = 0, e = lane; e < E; ++i, e += 32)
     if ((keep >> (e / g)) & 1ull) mine |= 1u << i;
   // top-k experts of the kept groups in (score desc, id asc) order
   int pe = -1;
-  float pev = 0.f, ssum = 0.f, my_s = 0.f;
-  int my_e = 0;
+  float pev = 0.f;
   for (int j = 0; j < a.k; ++j) {
     float bv = 0.f;
     int be = -1;
@@ -192,6 +253,7 @@ __device__ __forceinline__ void select_token(const SelectArgs& a, int t, const f
     }
     pe = be;
     pev = bv;
+  }
   }
   if (lane < a.k) {
     const float wj = a.norm ? a.alpha * my_s / ssum : a.alpha * my_s;
@@ -225,59 +287,55 @@ __device__ __forceinline__ float4 load4(const float* p) {
   return *reinterpret_cast<const float4*>(p);
 }
 
-// Logits of expert e for the T <= 32 tokens, by one block: threads split H
-// four elements at a time with all weight loads of a thread issued first,
-// then a block reduction.  red: [blockDim/32][32] floats of shared memory.
-template <typename Tin>
-__device__ __forceinline__ void router_block_logits(const Tin* __restrict__ x,
-                                                    const float* __restrict__ wr, int e, int T,
-                                                    int E, int H, float* logits,
-                                                    float (*red)[32]) {
+// Logits of expert e for T <= TB tokens, by one block: threads split H four
+// elements at a time.  The token loads are unconditional (rows past T re-read
+// row T - 1), so a thread issues its loads for eight tokens back to back
+// instead of one dependent round trip per token; then a block reduction.
+// red: [blockDim/32][32].
+template <int TB, typename Tin>
+__device__ __forceinline__ void router_block_logits_t(const Tin* __restrict__ x,
+                                                      const float* __restrict__ wr, int e, int T,
+                                                      int E, int H, float* logits,
+                                                      float (*red)[32]) {
   const int lane = threadIdx.x & 31, wib = threadIdx.x >> 5, nw = blockDim.x >> 5;
   const int step = blockDim.x * 4;
-  float acc[32];
+  float acc[TB];
 #pragma unroll
-  for (int t = 0; t < 32; ++t) acc[t] = 0.f;
+  for (int t = 0; t < TB; ++t) acc[t] = 0.f;
   const float* w = wr + (size_t)e * H;
   if ((H & 3) == 0) {
-    constexpr int U = 2;
-    for (int h0 = threadIdx.x * 4; h0 < H; h0 += U * step) {
-      float4 wv[U];
+#pragma unroll 2
+    for (int h = threadIdx.x * 4; h < H; h += step) {
+      const int hh = h;
+      const float4 wv = __ldg(reinterpret_cast<const float4*>(w + hh));
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int h = h0 + u * step;
-        wv[u] = h < H ? __ldg(reinterpret_cast<const float4*>(w + h)) : make_float4(0.f, 0.f, 0.f, 0.f);
-      }
+      for (int t0 = 0; t0 < TB; t0 += 8) {
+        float4 xv[8];
 #pragma unroll
-      for (int u = 0; u < U; ++u) {
-        const int h = h0 + u * step;
-        if (h >= H) break;
-#pragma unroll
-        for (int t = 0; t < 32; ++t) {
-          if (t < T) {
-            const float4 xv = load4(x + (size_t)t * H + h);
-            acc[t] = fmaf(xv.x, wv[u].x,
-                          fmaf(xv.y, wv[u].y, fmaf(xv.z, wv[u].z, fmaf(xv.w, wv[u].w, acc[t]))));
-          }
+        for (int i = 0; i < 8; ++i) {
+          const int tt = min(t0 + i, T - 1);
+          xv[i] = load4(x + (size_t)tt * H + hh);
         }
+#pragma unroll
+        for (int i = 0; i < 8; ++i)
+          acc[t0 + i] = fmaf(xv[i].x, wv.x,
+                             fmaf(xv[i].y, wv.y, fmaf(xv[i].z, wv.z, fmaf(xv[i].w, wv.w, acc[t0 + i]))));
       }
     }
   } else {
     for (int h = threadIdx.x; h < H; h += blockDim.x) {
       const float wv = w[h];
 #pragma unroll
-      for (int t = 0; t < 32; ++t)
-        if (t < T) acc[t] = fmaf(to_f32(x[(size_t)t * H + h]), wv, acc[t]);
+      for (int t = 0; t < TB; ++t)
+        acc[t] = fmaf(to_f32(x[(size_t)min(t, T - 1) * H + h]), wv, acc[t]);
     }
   }
 #pragma unroll
-  for (int t = 0; t < 32; ++t) {
-    if (t < T) {
-      float v = acc[t];
+  for (int t = 0; t < TB; ++t) {
+    float v = acc[t];
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-      if (lane == 0) red[wib][t] = v;
-    }
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (lane == 0) red[wib][t] = v;
   }
   __syncthreads();
   if (wib == 0 && lane < T) {
@@ -285,6 +343,16 @@ __device__ __forceinline__ void router_block_logits(const Tin* __restrict__ x,
     for (int i = 0; i < nw; ++i) v += red[i][lane];
     logits[(size_t)lane * E + e] = v;
   }
+}
+
+template <typename Tin>
+__device__ __forceinline__ void router_block_logits(const Tin* __restrict__ x,
+                                                    const float* __restrict__ wr, int e, int T,
+                                                    int E, int H, float* logits,
+                                                    float (*red)[32]) {
+  if (T <= 8) router_block_logits_t<8>(x, wr, e, T, E, H, logits, red);
+  else if (T <= 16) router_block_logits_t<16>(x, wr, e, T, E, H, logits, red);
+  else router_block_logits_t<32>(x, wr, e, T, E, H, logits, red);
 }
 
 // Decode-sized T (<= 32): block e computes expert e's logits for every token
