@@ -1,0 +1,244 @@
+// gemv_q4.cuh -- NVFP4 expert GEMM for decode-sized tiles (at most 32 tokens
+// per expert) with warp-level MMAs fed straight from registers.
+//
+// With one or two tokens per expert a 128-row tcgen05.mma pays a fixed cost per
+// 128 x 16 block of weights whatever N is (about 90 SM cycles, measured), which
+// caps the tensor-memory kernel (gemm_q4.cuh) near a quarter of HBM speed.
+// Here each warp owns 16 weight rows of one tile entry (one warp task): it
+// loads the rows' 4-bit codes with 16-byte global loads, turns them into bf16 in registers
+// (the exact bit construction of gemm_q4.cuh: code * scale * 2^-8) and issues
+// mma.sync m16n8k16 (bf16 in, f32 accumulate) with the tokens on N = 8; the
+// float32 matrix scale * 2^8 is applied in the epilogue.  Nothing goes
+// through shared or tensor memory.
+//
+// Feature order inside the MMA.  The MMA sums over its 16 k slots in any
+// order, so weights and activations may use one common permutation of the
+// features.  In a block of BK (128, or a 64-feature tail) features, k-tile kt
+// (of BK/16), slot kappa = 8h + 2 tq + p (tq = lane % 4, h, p in {0, 1}) holds
+// feature (BK/4) tq + 4 kt + 2h + p.  Thread tq's features are then the
+// contiguous run [(BK/4) tq, (BK/4)(tq + 1)) -- BK/8 bytes of codes per row,
+// one 16-byte (or 8-byte) load -- and its activation values come four
+// consecutive bf16 at a time.  The permutation is a bijection of the block,
+// so every product is summed exactly once.
+#pragma once
+
+#include "gemm_q4.cuh"
+
+namespace nh {
+namespace q4v {
+
+constexpr int WARPS = 8;   // per CTA
+constexpr int MT = 16;     // weight rows per warp task
+
+struct Args {
+  tc::TcArgs g;            // tiles / dense rows, N, K, epilogue, out, perm_w, row_token, status
+  const void* A;           // activations [*, K] bf16 (x, x_perm, h)
+  const uint8_t* codes;    // [n_mat, N, K / 2]
+  const uint8_t* scales;   // [n_mat, N, pitch]
+  const float* gscale;     // [n_mat]
+  int pitch;               // scale bytes per row
+};
+
+__device__ __forceinline__ void mma_bf16_16816(float* c, uint32_t a0, uint32_t a1, uint32_t a2,
+                                               uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, "
+      "{%8,%9}, {%0,%1,%2,%3};"
+      : "+f"(c[0]), "+f"(c[1]), "+f"(c[2]), "+f"(c[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// One block of BK features for one n-tile (8 tokens): codes of rows gq (ca)
+// and gq + 8 (cb) of this thread's run (BK/8 bytes = BK/32 words each), the
+// scale multipliers of the run's groups, and the activation row of token gq.
+// Word w of the run holds k-tiles 2w and 2w + 1; even and odd k-tiles go to
+// two accumulators (c0, c1) so consecutive MMAs do not wait on each other.
+template <int BK>
+__device__ __forceinline__ void block_mma(const uint32_t* ca, const uint32_t* cb,
+                                          const uint32_t* ma, const uint32_t* mb,
+                                          const __nv_bfloat16* act, float* c0, float* c1) {
+  constexpr int KT = BK / 16;
+  uint2 bv[KT];
+#pragma unroll
+  for (int kt = 0; kt < KT; ++kt) bv[kt] = __ldg(reinterpret_cast<const uint2*>(act + 4 * kt));
+#pragma unroll
+  for (int w = 0; w < KT / 2; ++w) {
+    uint32_t pa[4], pb[4];
+    // a 16-feature scale group is 8 bytes = 2 words of the run
+    q4::dq_word(ca[w], ma[w / 2], pa);
+    q4::dq_word(cb[w], mb[w / 2], pb);
+    // k-tile kt: slots 2tq + {0,1} = byte 2kt, slots 2tq + 8 + {0,1} = byte 2kt + 1
+    mma_bf16_16816(c0, pa[0], pb[0], pa[1], pb[1], bv[2 * w].x, bv[2 * w].y);
+    mma_bf16_16816(c1, pa[2], pb[2], pa[3], pb[3], bv[2 * w + 1].x, bv[2 * w + 1].y);
+  }
+}
+
+// Few tasks (dense rows: the shared expert, the latent projections).
+// NT: tokens per tile entry (16 or 32).  A CTA task is (tile entry, 16 weight
+// rows); its 8 warps split the 128-feature blocks of K round-robin (the
+// 64-feature tail goes to the next warp in turn) and their partial tiles are
+// added through shared memory in warp order (deterministic), then warp 0
+// applies the epilogue.  An entry with more than 8 tokens takes one pass per
+// 8 tokens.  Tasks are dealt round-robin over the grid.
+template <int NT>
+__global__ void __launch_bounds__(WARPS * 32, 3) q4_gemv_splitk(const Args a) {
+  __shared__ float red[WARPS][32][4];
+  const tc::TcArgs& g = a.g;
+  pdl_wait();
+  pdl_trigger();
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int gq = lane >> 2, tq = lane & 3;
+  const int num_m = g.tiles ? *g.num_tiles : (g.dense_rows + g.tile_rows - 1) / g.tile_rows;
+  const int n_rb = g.N / MT;                        // N is a multiple of 64
+  const int total = num_m * n_rb;
+  const int K = g.K;
+  const int nkb = K / 128, tail = K % 128;          // tail: 0 or 64 (K is a multiple of 64)
+  const size_t row_bytes = (size_t)K / 2;
+  const __nv_bfloat16* A = static_cast<const __nv_bfloat16*>(a.A);
+  for (int task = blockIdx.x; task < total; task += gridDim.x) {
+    const int m = task / n_rb, rb = task - m * n_rb;
+    const int r0 = rb * MT;
+    const int4 ent = tc::tile_entry_of(g, m);
+    const int count = ent.z;
+    const size_t wrow_a = (size_t)ent.x * g.N + r0 + gq;   // rows gq and gq + 8
+    const uint8_t* ca_p = a.codes + wrow_a * row_bytes;
+    const uint8_t* cb_p = ca_p + 8 * row_bytes;
+    const uint8_t* sa_p = a.scales + wrow_a * a.pitch;
+    const uint8_t* sb_p = sa_p + 8 * (size_t)a.pitch;
+    for (int n0 = 0; n0 < count; n0 += 8) {
+      // activation row of token n0 + gq (rows past count re-read the last
+      // token; their columns are never stored)
+      const int j = min(n0 + gq, count - 1);
+      const int arow = g.row_token ? g.row_token[ent.y + j] : ent.y + j;
+      const __nv_bfloat16* act = A + (size_t)arow * K;
+      float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+      int kb = warp;
+      uint4 qa = make_uint4(0, 0, 0, 0), qb = qa;
+      if (kb < nkb) {
+        qa = __ldg(reinterpret_cast<const uint4*>(ca_p + (size_t)kb * 64 + 16 * tq));
+        qb = __ldg(reinterpret_cast<const uint4*>(cb_p + (size_t)kb * 64 + 16 * tq));
+      }
+      for (; kb < nkb; kb += WARPS) {
+        // the warp's next block is in flight while this one is used
+        uint4 na = qa, nbq = qb;
+        if (kb + WARPS < nkb) {
+          na = __ldg(reinterpret_cast<const uint4*>(ca_p + (size_t)(kb + WARPS) * 64 + 16 * tq));
+          nbq = __ldg(reinterpret_cast<const uint4*>(cb_p + (size_t)(kb + WARPS) * 64 + 16 * tq));
+        }
+        // thread tq's 32 features are scale groups 8 kb + 2 tq and + 1
+        const uint32_t sa2 = *reinterpret_cast<const uint16_t*>(sa_p + kb * 8 + 2 * tq);
+        const uint32_t sb2 = *reinterpret_cast<const uint16_t*>(sb_p + kb * 8 + 2 * tq);
+        const uint32_t ma[2] = {q4::scale_mult(sa2 & 0xffu), q4::scale_mult(sa2 >> 8)};
+        const uint32_t mb[2] = {q4::scale_mult(sb2 & 0xffu), q4::scale_mult(sb2 >> 8)};
+        const uint32_t cwa[4] = {qa.x, qa.y, qa.z, qa.w}, cwb[4] = {qb.x, qb.y, qb.z, qb.w};
+        block_mma<128>(cwa, cwb, ma, mb, act + kb * 128 + 32 * tq, c0, c1);
+        qa = na;
+        qb = nbq;
+      }
+      if (tail && warp == nkb % WARPS) {
+        // 64-feature tail: thread tq's run is features [16 tq, 16 tq + 16), one group
+        const size_t off = (size_t)nkb * 64 + 8 * tq;
+        const uint2 ta = __ldg(reinterpret_cast<const uint2*>(ca_p + off));
+        const uint2 tb = __ldg(reinterpret_cast<const uint2*>(cb_p + off));
+        const uint32_t ma[1] = {q4::scale_mult(sa_p[nkb * 8 + tq])};
+        const uint32_t mb[1] = {q4::scale_mult(sb_p[nkb * 8 + tq])};
+        const uint32_t cwa[2] = {ta.x, ta.y}, cwb[2] = {tb.x, tb.y};
+        block_mma<64>(cwa, cwb, ma, mb, act + nkb * 128 + 16 * tq, c0, c1);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) red[warp][lane][i] = c0[i] + c1[i];
+      __syncthreads();
+      if (warp == 0) {
+        // c: rows (gq, gq + 8) x tokens (n0 + 2 tq, n0 + 2 tq + 1)
+        const float gs = a.gscale[ent.x] * q4::DQ_UNSCALE;
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          float v = 0.f;
+#pragma unroll
+          for (int w = 0; w < WARPS; ++w) v += red[w][lane][i];
+          const int jj = n0 + 2 * tq + (i & 1);
+          const int f = r0 + gq + (i >> 1) * 8;
+          if (jj < count) tc::epi_elem(g, ent.y + jj, f, v * gs);
+        }
+      }
+      __syncthreads();
+    }
+  }
+}
+
+// Many tasks (the routed experts).  Warp tasks (tile entry, 16 weight rows)
+// are dealt round-robin over all warps of the grid; each warp runs the whole
+// K with the next block's codes in flight.  An entry with more than 8 tokens
+// takes one pass per 8 tokens (the codes are re-read from L1/L2).
+template <int NT>
+__global__ void __launch_bounds__(WARPS * 32, 3) q4_gemv_rows(const Args a) {
+  const tc::TcArgs& g = a.g;
+  pdl_wait();
+  pdl_trigger();
+  const int lane = threadIdx.x & 31;
+  const int gq = lane >> 2, tq = lane & 3;
+  const int num_m = g.tiles ? *g.num_tiles : (g.dense_rows + g.tile_rows - 1) / g.tile_rows;
+  const int n_rb = g.N / MT;
+  const int total = num_m * n_rb;
+  const int K = g.K;
+  const int nkb = K / 128, tail = K % 128;
+  const size_t row_bytes = (size_t)K / 2;
+  const __nv_bfloat16* A = static_cast<const __nv_bfloat16*>(a.A);
+  const int nwarps = gridDim.x * WARPS;
+  for (int task = blockIdx.x * WARPS + (threadIdx.x >> 5); task < total; task += nwarps) {
+    const int m = task / n_rb, rb = task - m * n_rb;
+    const int r0 = rb * MT;
+    const int4 ent = tc::tile_entry_of(g, m);
+    const int count = ent.z;
+    const size_t wrow_a = (size_t)ent.x * g.N + r0 + gq;
+    const uint8_t* ca_p = a.codes + wrow_a * row_bytes;
+    const uint8_t* cb_p = ca_p + 8 * row_bytes;
+    const uint8_t* sa_p = a.scales + wrow_a * a.pitch;
+    const uint8_t* sb_p = sa_p + 8 * (size_t)a.pitch;
+    const float gs = a.gscale[ent.x] * q4::DQ_UNSCALE;
+    for (int n0 = 0; n0 < count; n0 += 8) {
+      const int j = min(n0 + gq, count - 1);
+      const int arow = g.row_token ? g.row_token[ent.y + j] : ent.y + j;
+      const __nv_bfloat16* act = A + (size_t)arow * K;
+      float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+      uint4 qa = make_uint4(0, 0, 0, 0), qb = qa;
+      if (nkb > 0) {
+        qa = __ldg(reinterpret_cast<const uint4*>(ca_p + 16 * tq));
+        qb = __ldg(reinterpret_cast<const uint4*>(cb_p + 16 * tq));
+      }
+      for (int kb = 0; kb < nkb; ++kb) {
+        uint4 na = qa, nbq = qb;
+        if (kb + 1 < nkb) {
+          na = __ldg(reinterpret_cast<const uint4*>(ca_p + (size_t)(kb + 1) * 64 + 16 * tq));
+          nbq = __ldg(reinterpret_cast<const uint4*>(cb_p + (size_t)(kb + 1) * 64 + 16 * tq));
+        }
+        const uint32_t sa2 = *reinterpret_cast<const uint16_t*>(sa_p + kb * 8 + 2 * tq);
+        const uint32_t sb2 = *reinterpret_cast<const uint16_t*>(sb_p + kb * 8 + 2 * tq);
+        const uint32_t ma[2] = {q4::scale_mult(sa2 & 0xffu), q4::scale_mult(sa2 >> 8)};
+        const uint32_t mb[2] = {q4::scale_mult(sb2 & 0xffu), q4::scale_mult(sb2 >> 8)};
+        const uint32_t cwa[4] = {qa.x, qa.y, qa.z, qa.w}, cwb[4] = {qb.x, qb.y, qb.z, qb.w};
+        block_mma<128>(cwa, cwb, ma, mb, act + kb * 128 + 32 * tq, c0, c1);
+        qa = na;
+        qb = nbq;
+      }
+      if (tail) {
+        const size_t off = (size_t)nkb * 64 + 8 * tq;
+        const uint2 ta = __ldg(reinterpret_cast<const uint2*>(ca_p + off));
+        const uint2 tb = __ldg(reinterpret_cast<const uint2*>(cb_p + off));
+        const uint32_t ma[1] = {q4::scale_mult(sa_p[nkb * 8 + tq])};
+        const uint32_t mb[1] = {q4::scale_mult(sb_p[nkb * 8 + tq])};
+        const uint32_t cwa[2] = {ta.x, ta.y}, cwb[2] = {tb.x, tb.y};
+        block_mma<64>(cwa, cwb, ma, mb, act + nkb * 128 + 16 * tq, c0, c1);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const int jj = n0 + 2 * tq + (i & 1);
+        const int f = r0 + gq + (i >> 1) * 8;
+        if (jj < count) tc::epi_elem(g, ent.y + jj, f, (c0[i] + c1[i]) * gs);
+      }
+    }
+  }
+}
+
+}  // namespace q4v
+}  // namespace nh

@@ -16,6 +16,7 @@
 #include "gemm_tc.cuh"
 #include "gemm_tc2.cuh"
 #include "gemm_q4.cuh"
+#include "gemv_q4.cuh"
 #include "permute.cuh"
 #include "route.cuh"
 #include "route_permute.cuh"
@@ -560,6 +561,48 @@ static nh_status launch_q4(const GemmCall& c, const nh_nvfp4_weight& w, int dev,
                   st, ma, mc, ms, qa);
 }
 
+// decode-sized tiles: warp-level MMAs from registers (gemv_q4.cuh)
+template <int NT>
+static nh_status launch_q4v(const GemmCall& c, const nh_nvfp4_weight& w, int dev,
+                            cudaStream_t st) {
+  q4v::Args a;
+  tc::TcArgs& g = a.g;
+  g.tiles = c.tiles;
+  g.num_tiles = c.num_tiles;
+  g.dense_rows = (int)c.rows;
+  g.tile_rows = c.tile_rows;
+  g.N = c.N;
+  g.K = c.K;
+  g.a_kwrap = 0;
+  g.epi = c.epi;
+  g.out = c.out;
+  g.ldo = c.ldo;
+  g.perm_w = c.perm_w;
+  g.row_token = c.row_token;
+  g.status = c.status;
+  g.timeout_ns = timeout_ns();
+  g.sched = c.sched;
+  a.A = c.A;
+  a.codes = w.codes;
+  a.scales = w.scales;
+  a.gscale = w.global_scale;
+  a.pitch = (int)nvfp4_pitch(c.K);
+  // tasks: (tile entry, 16 weight rows).  Few tasks (dense rows: shared
+  // expert, latent projections): one per CTA with K split over its warps;
+  // many (routed experts): one per warp.
+  const int64_t m_max = c.tiles ? c.max_tiles : (c.rows + c.tile_rows - 1) / c.tile_rows;
+  const int64_t tasks = m_max * (c.N / q4v::MT);
+  const int64_t slots = (int64_t)g_sm_count[dev] * 3;   // resident CTAs
+  if (tasks <= 0) return NH_OK;
+  if (!c.tiles && tasks < slots * q4v::WARPS / 2)
+    return launch_k("q4_gemv_splitk", q4v::q4_gemv_splitk<NT>,
+                    dim3((unsigned)std::min<int64_t>(tasks, slots)), dim3(q4v::WARPS * 32), 0, st,
+                    a);
+  const int64_t grid = std::min<int64_t>((tasks + q4v::WARPS - 1) / q4v::WARPS, slots);
+  return launch_k("q4_gemv_rows", q4v::q4_gemv_rows<NT>, dim3((unsigned)grid),
+                  dim3(q4v::WARPS * 32), 0, st, a);
+}
+
 static nh_status run_gemm_q4(const GemmCall& c, const nh_nvfp4_weight* w, int dev,
                              cudaStream_t st) {
   if (c.rows == 0) return NH_OK;
@@ -568,8 +611,8 @@ static nh_status run_gemm_q4(const GemmCall& c, const nh_nvfp4_weight* w, int de
   if (reinterpret_cast<uintptr_t>(w->codes) % 16 || reinterpret_cast<uintptr_t>(w->scales) % 16)
     return fail(NH_ERR_INVALID_ARG, "NVFP4 codes / scales must be 16-byte aligned");
   switch (c.tile_rows) {
-    case 16: return launch_q4<16, 8>(c, *w, dev, st);
-    case 32: return launch_q4<32, 6>(c, *w, dev, st);
+    case 16: return launch_q4v<16>(c, *w, dev, st);
+    case 32: return launch_q4v<32>(c, *w, dev, st);
     case 64: return launch_q4<64, 4>(c, *w, dev, st);
     default: return fail(NH_ERR_UNSUPPORTED, "NVFP4 tile rows %d", c.tile_rows);
   }
