@@ -126,6 +126,10 @@ class NemotronHMoE:
         else:
             self.c_exp = self.c
         with torch.cuda.device(self.device):
+            # the routed path (router -> experts -> finalize) is the critical
+            # path: its kernels run on the highest-priority stream, so pending
+            # CTAs start before those of the shared expert on `side`
+            self.hi = torch.cuda.Stream(priority=-5)
             self.side = torch.cuda.Stream()
         self._bufs: Dict[int, Buffers] = {}
         self._graphs: Dict[int, tuple] = {}
@@ -168,12 +172,14 @@ class NemotronHMoE:
         b = bufs or self.buffers(T)
         if partial and b.y_f32 is None:
             b.y_f32 = torch.empty((T, self.H), dtype=torch.float32, device=self.device)
-        main = torch.cuda.current_stream(self.device)
+        caller = torch.cuda.current_stream(self.device)
+        main = self.hi
         push = torch.cuda.nvtx.range_push if nvtx else (lambda name: None)
         pop = torch.cuda.nvtx.range_pop if nvtx else (lambda: None)
+        fork = torch.cuda.Event()
+        fork.record(caller)
+        main.wait_event(fork)
         if self.has_shared:
-            fork = torch.cuda.Event()
-            fork.record(main)
             self.side.wait_event(fork)
             push("shared")
             if self.nvfp4:
@@ -186,8 +192,10 @@ class NemotronHMoE:
             join = torch.cuda.Event()
             join.record(self.side)
         if self.latent:
-            return self._forward_latent(x, b, main, join if self.has_shared else None, partial,
-                                        push, pop)
+            out = self._forward_latent(x, b, main, join if self.has_shared else None, partial,
+                                       push, pop)
+            self._join(caller, main)
+            return out
         push("route_permute")
         route_permute(self.c, x, self.w_router, self.bias, b.topk_idx, b.topk_w, b.ws, stream=main)
         pop()
@@ -205,7 +213,14 @@ class NemotronHMoE:
         else:
             finalize(self.c, T, b.ws, b.y_shared, b.y, stream=main)
         pop()
+        self._join(caller, main)
         return b.y_f32 if partial else b.y
+
+    @staticmethod
+    def _join(caller, main):
+        done = torch.cuda.Event()
+        done.record(main)
+        caller.wait_event(done)
 
     def _forward_latent(self, x, b, main, join, partial, push, pop):
         T = x.shape[0]

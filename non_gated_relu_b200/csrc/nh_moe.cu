@@ -17,6 +17,7 @@
 #include "gemm_tc2.cuh"
 #include "gemm_q4.cuh"
 #include "gemv_q4.cuh"
+#include "gemv_bf16.cuh"
 #include "permute.cuh"
 #include "route.cuh"
 #include "route_permute.cuh"
@@ -341,6 +342,19 @@ static uint64_t timeout_ns() {
 // Launch with programmatic dependent launch allowed: the kernel may start its
 // prologue while the previous kernel in the stream finishes; every kernel of
 // this library executes griddepcontrol.wait before it reads its inputs.
+// The launching stream's priority, set again as a launch attribute so that a
+// CUDA graph captured from prioritised streams keeps it per kernel node: the
+// block scheduler then starts pending CTAs of the routed path (a high
+// priority stream) before those of the concurrent shared expert.
+static int stream_priority(cudaStream_t st) {
+  int p = 0;
+  if (cudaStreamGetPriority(st, &p) != cudaSuccess) {
+    cudaGetLastError();
+    p = 0;
+  }
+  return p;
+}
+
 template <typename Kern, typename... Args>
 static nh_status launch_k(const char* what, Kern kernel, dim3 grid, dim3 block, size_t smem,
                           cudaStream_t st, Args... args) {
@@ -349,11 +363,13 @@ static nh_status launch_k(const char* what, Kern kernel, dim3 grid, dim3 block, 
   lc.blockDim = block;
   lc.dynamicSmemBytes = smem;
   lc.stream = st;
-  cudaLaunchAttribute at[1];
+  cudaLaunchAttribute at[2];
   at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   at[0].val.programmaticStreamSerializationAllowed = 1;
+  at[1].id = cudaLaunchAttributePriority;
+  at[1].val.priority = stream_priority(st);
   lc.attrs = at;
-  lc.numAttrs = 1;
+  lc.numAttrs = 2;
   const cudaError_t e = cudaLaunchKernelEx(&lc, kernel, args...);
   if (e != cudaSuccess)
     return fail(NH_ERR_CUDA, "launch of %s failed: %s", what, cudaGetErrorString(e));
@@ -495,15 +511,17 @@ static nh_status launch_tc2(const GemmCall& c, int dev, cudaStream_t st) {
   lc.blockDim = dim3(tc2::THREADS, 1, 1);
   lc.dynamicSmemBytes = tc2::SMEM;
   lc.stream = st;
-  cudaLaunchAttribute at[2];
+  cudaLaunchAttribute at[3];
   at[0].id = cudaLaunchAttributeClusterDimension;
   at[0].val.clusterDim.x = 2;
   at[0].val.clusterDim.y = 1;
   at[0].val.clusterDim.z = 1;
   at[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
   at[1].val.programmaticStreamSerializationAllowed = 1;
+  at[2].id = cudaLaunchAttributePriority;
+  at[2].val.priority = stream_priority(st);
   lc.attrs = at;
-  lc.numAttrs = 2;
+  lc.numAttrs = 3;
   NH_CUDA(cudaLaunchKernelEx(&lc, tc2::tc2_grouped_gemm, ma, mw, g));
   return launch_check("tc2_grouped_gemm");
 }
@@ -618,8 +636,42 @@ static nh_status run_gemm_q4(const GemmCall& c, const nh_nvfp4_weight* w, int de
   }
 }
 
+// dense rows of decode size (shared expert, latent projections): CTA tasks of
+// 16 weight rows with K split over the warps (gemv_bf16.cuh)
+template <int NT>
+static nh_status launch_dgv(const GemmCall& c, int dev, cudaStream_t st) {
+  dgv::Args a;
+  tc::TcArgs& g = a.g;
+  g.tiles = nullptr;
+  g.num_tiles = nullptr;
+  g.dense_rows = (int)c.rows;
+  g.tile_rows = c.tile_rows;
+  g.N = c.N;
+  g.K = c.K;
+  g.a_kwrap = 0;
+  g.epi = c.epi;
+  g.out = c.out;
+  g.ldo = c.ldo;
+  g.perm_w = c.perm_w;
+  g.row_token = nullptr;
+  g.status = c.status;
+  g.timeout_ns = timeout_ns();
+  g.sched = c.sched;
+  a.A = c.A;
+  a.W = c.W;
+  const int64_t tasks = (c.rows + c.tile_rows - 1) / c.tile_rows * (c.N / dgv::MT);
+  const int64_t grid = std::min<int64_t>(tasks, (int64_t)g_sm_count[dev] * 2);
+  if (grid <= 0) return NH_OK;
+  return launch_k("bf16_gemv_splitk", dgv::bf16_gemv_splitk<NT>, dim3((unsigned)grid),
+                  dim3(dgv::WARPS * 32), 0, st, a);
+}
+
 static nh_status run_gemm(const Plan& p, const GemmCall& c, int dev, cudaStream_t st) {
   if (c.rows == 0) return NH_OK;
+  if (p.bf16 && !c.tiles && c.swap && c.a_kwrap == 0 && c.n_exp == 1 && !c.row_token) {
+    if (c.tile_rows == 16) return launch_dgv<16>(c, dev, st);
+    if (c.tile_rows == 32) return launch_dgv<32>(c, dev, st);
+  }
   if (!p.bf16) {
     GemmArgs g;
     g.A = c.A;
