@@ -74,6 +74,22 @@ __device__ __forceinline__ void block_mma(const uint32_t* ca, const uint32_t* cb
 }
 
 // Few tasks (dense rows: the shared expert, the latent projections).
+// block_mma with the activation run already in registers: run features
+// 8u .. 8u + 7 in bv[u] (.x: 8u + {0,1}, .y: {2,3}, .z: {4,5}, .w: {6,7}).
+__device__ __forceinline__ void block_mma_b(const uint32_t* ca, const uint32_t* cb,
+                                            const uint32_t* ma, const uint32_t* mb,
+                                            const uint4* bv, float* c0, float* c1) {
+#pragma unroll
+  for (int w = 0; w < 4; ++w) {
+    uint32_t pa[4], pb[4];
+    q4::dq_word(ca[w], ma[w / 2], pa);
+    q4::dq_word(cb[w], mb[w / 2], pb);
+    // word w = k-tiles 2w (features 8w + 0..3) and 2w + 1 (8w + 4..7)
+    mma_bf16_16816(c0, pa[0], pb[0], pa[1], pb[1], bv[w].x, bv[w].y);
+    mma_bf16_16816(c1, pa[2], pb[2], pa[3], pb[3], bv[w].z, bv[w].w);
+  }
+}
+
 // NT: tokens per tile entry (16 or 32).  A CTA task is (tile entry, 16 weight
 // rows); its 8 warps split the 128-feature blocks of K round-robin (the
 // 64-feature tail goes to the next warp in turn) and their partial tiles are
@@ -168,10 +184,10 @@ __global__ void __launch_bounds__(WARPS * 32, 3) q4_gemv_splitk(const Args a) {
 
 // Many tasks (the routed experts).  Warp tasks (tile entry, 16 weight rows)
 // are dealt round-robin over all warps of the grid; each warp runs the whole
-// K with the next block's codes in flight.  An entry with more than 8 tokens
+// K with the next block's codes, scale bytes and activation run in flight.  An entry with more than 8 tokens
 // takes one pass per 8 tokens (the codes are re-read from L1/L2).
 template <int NT>
-__global__ void __launch_bounds__(WARPS * 32, 3) q4_gemv_rows(const Args a) {
+__global__ void __launch_bounds__(WARPS * 32, 2) q4_gemv_rows(const Args a) {
   const tc::TcArgs& g = a.g;
   pdl_wait();
   pdl_trigger();
@@ -201,25 +217,34 @@ __global__ void __launch_bounds__(WARPS * 32, 3) q4_gemv_rows(const Args a) {
       const int arow = g.row_token ? g.row_token[ent.y + j] : ent.y + j;
       const __nv_bfloat16* act = A + (size_t)arow * K;
       float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
-      uint4 qa = make_uint4(0, 0, 0, 0), qb = qa;
-      if (nkb > 0) {
-        qa = __ldg(reinterpret_cast<const uint4*>(ca_p + 16 * tq));
-        qb = __ldg(reinterpret_cast<const uint4*>(cb_p + 16 * tq));
-      }
+      // block kb's codes, scale bytes and activation run, loaded one block ahead
+      uint4 qa = make_uint4(0, 0, 0, 0), qb = qa, xb[4] = {qa, qa, qa, qa};
+      uint32_t sa2 = 0, sb2 = 0;
+      auto fetch = [&](int kb, uint4& fa, uint4& fb, uint4* fx, uint32_t& fsa, uint32_t& fsb) {
+        fa = __ldg(reinterpret_cast<const uint4*>(ca_p + (size_t)kb * 64 + 16 * tq));
+        fb = __ldg(reinterpret_cast<const uint4*>(cb_p + (size_t)kb * 64 + 16 * tq));
+        const uint4* xr = reinterpret_cast<const uint4*>(act + kb * 128 + 32 * tq);
+#pragma unroll
+        for (int u = 0; u < 4; ++u) fx[u] = __ldg(xr + u);
+        // thread tq's 32 features are scale groups 8 kb + 2 tq and + 1
+        fsa = *reinterpret_cast<const uint16_t*>(sa_p + kb * 8 + 2 * tq);
+        fsb = *reinterpret_cast<const uint16_t*>(sb_p + kb * 8 + 2 * tq);
+      };
+      if (nkb > 0) fetch(0, qa, qb, xb, sa2, sb2);
       for (int kb = 0; kb < nkb; ++kb) {
-        uint4 na = qa, nbq = qb;
-        if (kb + 1 < nkb) {
-          na = __ldg(reinterpret_cast<const uint4*>(ca_p + (size_t)(kb + 1) * 64 + 16 * tq));
-          nbq = __ldg(reinterpret_cast<const uint4*>(cb_p + (size_t)(kb + 1) * 64 + 16 * tq));
-        }
-        const uint32_t sa2 = *reinterpret_cast<const uint16_t*>(sa_p + kb * 8 + 2 * tq);
-        const uint32_t sb2 = *reinterpret_cast<const uint16_t*>(sb_p + kb * 8 + 2 * tq);
+        uint4 na = qa, nbq = qb, nx[4] = {xb[0], xb[1], xb[2], xb[3]};
+        uint32_t nsa = sa2, nsb = sb2;
+        if (kb + 1 < nkb) fetch(kb + 1, na, nbq, nx, nsa, nsb);
         const uint32_t ma[2] = {q4::scale_mult(sa2 & 0xffu), q4::scale_mult(sa2 >> 8)};
         const uint32_t mb[2] = {q4::scale_mult(sb2 & 0xffu), q4::scale_mult(sb2 >> 8)};
         const uint32_t cwa[4] = {qa.x, qa.y, qa.z, qa.w}, cwb[4] = {qb.x, qb.y, qb.z, qb.w};
-        block_mma<128>(cwa, cwb, ma, mb, act + kb * 128 + 32 * tq, c0, c1);
+        block_mma_b(cwa, cwb, ma, mb, xb, c0, c1);
         qa = na;
         qb = nbq;
+#pragma unroll
+        for (int u = 0; u < 4; ++u) xb[u] = nx[u];
+        sa2 = nsa;
+        sb2 = nsb;
       }
       if (tail) {
         const size_t off = (size_t)nkb * 64 + 8 * tq;

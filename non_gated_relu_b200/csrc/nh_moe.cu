@@ -616,7 +616,9 @@ static nh_status launch_q4v(const GemmCall& c, const nh_nvfp4_weight& w, int dev
     return launch_k("q4_gemv_splitk", q4v::q4_gemv_splitk<NT>,
                     dim3((unsigned)std::min<int64_t>(tasks, slots)), dim3(q4v::WARPS * 32), 0, st,
                     a);
-  const int64_t grid = std::min<int64_t>((tasks + q4v::WARPS - 1) / q4v::WARPS, slots);
+  // the rows kernel keeps two CTAs per SM (its launch bounds): one wave
+  const int64_t grid = std::min<int64_t>((tasks + q4v::WARPS - 1) / q4v::WARPS,
+                                         (int64_t)g_sm_count[dev] * 2);
   return launch_k("q4_gemv_rows", q4v::q4_gemv_rows<NT>, dim3((unsigned)grid),
                   dim3(q4v::WARPS * 32), 0, st, a);
 }

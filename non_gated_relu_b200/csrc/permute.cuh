@@ -143,24 +143,37 @@ __global__ void __launch_bounds__(256) permute_scatter(
     for (int e = lane; e < E; e += 32) run[e] = chunk_base[(size_t)c * E + e];
     __syncwarp();
     const unsigned lt = (1u << lane) - 1u;
-    for (int b = 0; b < n; b += 32) {
-      const int a = b + lane;
-      int e = (a < n) ? idx[a0 + a] : -1;
-      if (e >= E) e = -1;  // already reported by the histogram
-      const unsigned peers = __match_any_sync(0xffffffffu, e);
-      const int start = (e >= 0) ? run[e] : 0;
-      __syncwarp();
-      const int p = start + __popc(peers & lt);
-      if (e >= 0 && lane == __ffs(peers) - 1) run[e] = start + __popc(peers);
-      __syncwarp();
-      if (a < n) {
-        pos[a] = (e >= 0) ? p : -1;
-        if (e >= 0) {
-          perm_token[p] = t0 + a / k;
-          perm_w[p] = w[a0 + a];
-          inv_row[a0 + a] = p;
-        } else {
-          inv_row[a0 + a] = -1;
+    // eight rounds of 32 assignments at a time: their loads are issued
+    // together, then the rounds rank in order (the ranking is sequential)
+    for (int b0 = 0; b0 < n; b0 += 8 * 32) {
+      int ev[8];
+      float wv[8];
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const int a = b0 + 32 * r + lane;
+        ev[r] = (a < n) ? idx[a0 + a] : -1;
+        wv[r] = (a < n) ? w[a0 + a] : 0.f;
+      }
+#pragma unroll
+      for (int r = 0; r < 8; ++r) {
+        const int a = b0 + 32 * r + lane;
+        int e = ev[r];
+        if (e >= E) e = -1;  // already reported by the histogram
+        const unsigned peers = __match_any_sync(0xffffffffu, e);
+        const int start = (e >= 0) ? run[e] : 0;
+        __syncwarp();
+        const int p = start + __popc(peers & lt);
+        if (e >= 0 && lane == __ffs(peers) - 1) run[e] = start + __popc(peers);
+        __syncwarp();
+        if (a < n) {
+          pos[a] = (e >= 0) ? p : -1;
+          if (e >= 0) {
+            perm_token[p] = t0 + a / k;
+            perm_w[p] = wv[r];
+            inv_row[a0 + a] = p;
+          } else {
+            inv_row[a0 + a] = -1;
+          }
         }
       }
     }
