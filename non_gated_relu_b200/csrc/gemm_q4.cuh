@@ -1,5 +1,6 @@
 // gemm_q4.cuh -- expert GEMM with NVFP4 weights (W4A16, group size 16) on the
-// sm_100a tensor cores, decode orientation.
+// sm_100a tensor cores, weights on the MMA M side; used for tile entries of 64
+// tokens (tiles of at most 32 tokens go to the register GEMV of gemv_q4.cuh).
 //
 // Weight storage (vllm.cpp PR #518 names it for the checkpoint's routed and
 // shared experts): every weight is an E2M1 code times an E4M3 scale shared by

@@ -289,10 +289,6 @@ static nh_status set_attrs(int dev) {
                                cudaFuncAttributeMaxDynamicSharedMemorySize, TcSwap64::SMEM));
   NH_CUDA(cudaFuncSetAttribute(tc2::tc2_grouped_gemm, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                tc2::SMEM));
-  NH_CUDA(cudaFuncSetAttribute(q4::tc_q4_gemm<16, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               q4::Shape<16, 8>::SMEM));
-  NH_CUDA(cudaFuncSetAttribute(q4::tc_q4_gemm<32, 6>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                               q4::Shape<32, 6>::SMEM));
   NH_CUDA(cudaFuncSetAttribute(q4::tc_q4_gemm<64, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                q4::Shape<64, 4>::SMEM));
   NH_CUDA(cudaFuncSetAttribute(route_permute_small<__nv_bfloat16>,
