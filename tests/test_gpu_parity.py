@@ -51,6 +51,16 @@ SMALL = {
     "small_nvfp4_t64": small("small_nvfp4_t64", T=64, seed=43, weight_format="nvfp4",
                              moe_intermediate_size=192),
     "small_nvfp4_t150": small("small_nvfp4_t150", T=150, seed=44, weight_format="nvfp4"),
+    # selection paths: 128 candidate experts (the ranking pass at its limit)
+    # and 256 (the sequential top-k rounds)
+    "small_cand128": small("small_cand128", T=45, hidden_size=128, n_routed_experts=256,
+                           n_group=2, topk_group=1, num_experts_per_tok=8,
+                           moe_intermediate_size=64, moe_shared_expert_intermediate_size=64,
+                           seed=15),
+    "small_cand256": small("small_cand256", T=20, hidden_size=128, n_routed_experts=512,
+                           n_group=2, topk_group=1, num_experts_per_tok=8,
+                           moe_intermediate_size=64, moe_shared_expert_intermediate_size=64,
+                           seed=16),
     # single expert (routing is trivial)
     "small_one_expert": small("small_one_expert", T=40, n_routed_experts=1, n_group=1,
                               topk_group=1, num_experts_per_tok=1, seed=14),
