@@ -128,6 +128,10 @@ def test_host_api_graph_matches_eager():
     np.testing.assert_array_equal(y_host, y_eager)
     y2 = blk(inp.x).float().numpy()          # second replay
     np.testing.assert_array_equal(y2, y_eager)
+    # another input through the same graph (the staging buffer is refilled)
+    x2 = np.ascontiguousarray(inp.x[::-1])
+    y3 = blk(x2).float().numpy()
+    np.testing.assert_array_equal(y3, blk.forward(to_dev(x2)).float().cpu().numpy())
 
 
 # ----------------------------------------------------------------------------- full size
