@@ -49,6 +49,12 @@
  * and each matrix has one float32 global scale.  The weight is
  *   w = e2m1(code) * e4m3(scale) * global.
  *
+ * nho_forward_latent adds latent projections around the routed experts
+ * (ModelOpt descriptor NemotronHMoELayerDescriptor names fc1_latent_proj and
+ * fc2_latent_proj and gives no formula): PARITY UNPINNED as a reading of the
+ * sources; its tests pin it to the plain block at identity and permutation
+ * projections.
+ *
  * Single-threaded, plain loops, built -O2 without fast-math.
  */
 #include <math.h>
