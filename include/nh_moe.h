@@ -235,10 +235,11 @@ nh_status nh_moe_forward(const nh_moe_config *cfg, int64_t T, const void *x, con
 /*
  * nh_moe_forward with NVFP4 routed-expert weights (cfg->weight_format ==
  * NH_WEIGHTS_NVFP4): w_up [E][I][H], w_down [E][H][I] as nh_nvfp4_weight.
- * The weights are dequantized stage by stage in shared memory (code x block
- * scale, exact in bf16), multiplied on the tensor cores, and the float32
- * matrix scale is applied in the epilogue.  Same results layout as
- * nh_moe_forward.
+ * Each weight is dequantized in registers (code x block scale, exact in
+ * bf16): for tiles of up to 32 tokens per expert straight into warp-level MMA
+ * fragments, for 64-token tiles into tensor memory as the A operand of
+ * tcgen05.mma.  The float32 matrix scale is applied in the epilogue.  Same
+ * results layout as nh_moe_forward.
  */
 nh_status nh_moe_forward_nvfp4(const nh_moe_config *cfg, int64_t T, const void *x,
                                const nh_nvfp4_weight *w_up, const nh_nvfp4_weight *w_down,

@@ -135,3 +135,66 @@ def test_zero_tokens_is_a_no_op_plan():
     cfg = synth.CONFIGS["decode_bf16_t8"]
     L = nh.workspace_layout(cfg, 0)
     assert L.total_bytes > 0 and L.n_chunks == 0
+
+
+def test_latent_config_is_the_expert_width_block():
+    cfg = synth.CONFIGS["decode_latent_bf16_t8"]
+    e = nh.latent_config(cfg)
+    c = nh.config_from(cfg)
+    assert (e.hidden_size, e.latent_size, e.n_shared_experts) == (cfg.latent_size, 0, 0)
+    for f in ("n_routed_experts", "n_group", "topk_group", "num_experts_per_tok",
+              "moe_intermediate_size", "norm_topk_prob", "routed_scaling_factor", "dtype",
+              "group_score", "weight_format"):
+        assert getattr(e, f) == getattr(c, f), f
+    assert nh.latent_workspace_size(cfg, cfg.T) >= 16 * 4
+    # a plain block has no expert-width config and no latent workspace
+    plain = synth.CONFIGS["decode_bf16_t8"]
+    for fn in (lambda: nh.latent_config(plain), lambda: nh.latent_workspace_size(plain, 8)):
+        with pytest.raises(nh.NHMoEError) as e:
+            fn()
+        assert e.value.status == nh.NH_ERR_INVALID_ARG
+    # bf16 tiles need a latent width that is a multiple of 64
+    with pytest.raises(nh.NHMoEError) as e:
+        nh.validate(cfg.replace(latent_size=100))
+    assert e.value.status in (nh.NH_ERR_INVALID_ARG, nh.NH_ERR_UNSUPPORTED)
+    nh.validate(cfg.replace(dtype="f32", latent_size=100))
+
+
+def test_next_row_argument_checks_before_any_device_work():
+    lib = nh.load()
+    P = ctypes.c_void_p
+    lat = nh.config_from(synth.CONFIGS["decode_latent_bf16_t8"])
+    need = nh.workspace_size(synth.CONFIGS["decode_bf16_t8"], 8)
+    # routed-expert calls refuse the full latent config
+    for rc in (lib.nh_moe_permute(ctypes.byref(lat), 8, P(256), P(256), P(256), P(256), need, None),
+               lib.nh_moe_forward(ctypes.byref(lat), 8, P(256), P(256), P(256), P(256), need, None),
+               lib.nh_moe_finalize(ctypes.byref(lat), 8, P(256), need, P(256), P(256), None)):
+        assert rc == nh.NH_ERR_INVALID_ARG and b"latent_size" in lib.nh_last_error()
+    # latent projections: workspace and pointer checks
+    rc = lib.nh_moe_latent_in(ctypes.byref(lat), 8, P(256), P(256), P(256), None, 256, None)
+    assert rc == nh.NH_ERR_INVALID_ARG and b"ws_latent" in lib.nh_last_error()
+    rc = lib.nh_moe_latent_in(ctypes.byref(lat), 8, P(256), P(256), P(256), P(256), 8, None)
+    assert rc == nh.NH_ERR_INVALID_ARG and b"needed" in lib.nh_last_error()
+    rc = lib.nh_moe_latent_out(ctypes.byref(lat), 8, P(256), P(258), P(256), P(256), 256, None)
+    assert rc == nh.NH_ERR_INVALID_ARG and b"aligned" in lib.nh_last_error()
+    # NVFP4 entry points: NULL weight descriptors, and the format must match the call
+    q4 = nh.config_from(synth.CONFIGS["decode_nvfp4_t8"])
+    rc = lib.nh_moe_forward_nvfp4(ctypes.byref(q4), 8, P(256), None, None, P(256), need, None)
+    assert rc == nh.NH_ERR_INVALID_ARG and b"NULL" in lib.nh_last_error()
+    rc = lib.nh_moe_forward(ctypes.byref(q4), 8, P(256), P(256), P(256), P(256),
+                            nh.workspace_size(synth.CONFIGS["decode_nvfp4_t8"], 8), None)
+    assert rc == nh.NH_ERR_INVALID_ARG and b"NVFP4" in lib.nh_last_error()
+    w = nh.NvFp4Weight(256, 256, 256)
+    bf = nh.config_from(synth.CONFIGS["decode_bf16_t8"])
+    rc = lib.nh_moe_forward_nvfp4(ctypes.byref(bf), 8, P(256), ctypes.byref(w), ctypes.byref(w),
+                                  P(256), need, None)
+    assert rc == nh.NH_ERR_INVALID_ARG and b"native" in lib.nh_last_error()
+    # tensor-parallel partial finalize and the one rounding
+    rc = lib.nh_moe_finalize_partial(ctypes.byref(bf), 8, P(256), need, P(256), P(250), None)
+    assert rc == nh.NH_ERR_INVALID_ARG and b"y_f32" in lib.nh_last_error()
+    rc = lib.nh_moe_cast_output(ctypes.byref(bf), -1, P(256), P(256), None)
+    assert rc == nh.NH_ERR_INVALID_ARG
+    rc = lib.nh_moe_cast_output(ctypes.byref(bf), 8, P(256), P(264), None)
+    assert rc == nh.NH_ERR_INVALID_ARG and b"aligned" in lib.nh_last_error()
+    # zero tokens: nothing to do, no device needed
+    assert lib.nh_moe_cast_output(ctypes.byref(bf), 0, None, None, None) == nh.NH_OK
