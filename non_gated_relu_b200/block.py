@@ -287,7 +287,12 @@ class NemotronHMoE:
         """y = block(x).  A device tensor is computed in place on the current
         stream; a host tensor (or numpy array) goes through pinned staging
         buffers: host->device copy, the block (as a CUDA graph when
-        ``use_graph``), device->host copy; returns a host tensor."""
+        ``use_graph``), device->host copy.
+
+        Both forms return a buffer the block owns, like a CUDA graph's static
+        output: the device y of ``forward`` for T tokens, or the pinned host
+        output buffer for T tokens.  The next call with the same T overwrites
+        it; clone the result to keep it."""
         if isinstance(x, torch.Tensor) and x.is_cuda:
             return self.forward(x)
         xh = _to_device(x, self.dtype, "cpu") if isinstance(x, np.ndarray) else x
