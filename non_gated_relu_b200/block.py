@@ -75,6 +75,10 @@ class NemotronHMoE:
     ``w_shared_down [H, S]`` in the block dtype (bf16 or float32), and an
     optional router correction bias ``[E]`` float32.  numpy uint16 arrays are
     taken as bf16 bit patterns.
+
+    libnhmoe launches on the current CUDA device, so call the block with its
+    own device current (``torch.cuda.set_device`` or a ``torch.cuda.device``
+    context), as one process per GPU does.
     """
 
     def __init__(self, cfg, w_router, w_up=None, w_down=None, w_shared_up=None,
