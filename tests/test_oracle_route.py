@@ -209,3 +209,60 @@ def test_bad_configs_rejected():
     assert oracle.check_config(tiny_cfg(8, 4, 5, 2)) != 0     # tg > G
     assert oracle.check_config(tiny_cfg(8, 4, 1, 3)) != 0     # k > tg * g
     assert oracle.check_config(tiny_cfg(8, 4, 1, 2)) == 0
+
+
+def brute_force_variant(l, b, E, G, tg, k, top2, alpha=2.5):
+    """Enumeration for the router variants: selection scores s + b (b the
+    correction bias), group score the max or the sum of the two largest
+    selection scores of the group; the weights use the unbiased s."""
+    s = 1.0 / (1.0 + np.exp(-l))
+    sel = s + b
+    g = E // G
+
+    def gscore(q):
+        v = sorted(sel[q * g:(q + 1) * g], reverse=True)
+        return v[0] + v[1] if top2 else v[0]
+
+    def better(va, ta, vb, tb):
+        return va > vb or (va == vb and ta < tb)
+
+    bestQ = bestv = None
+    for Q in itertools.combinations(range(G), tg):
+        v = sorted((gscore(q) for q in Q), reverse=True)
+        if bestQ is None or better(v, Q, bestv, bestQ):
+            bestQ, bestv = Q, v
+    cand = [q * g + i for q in bestQ for i in range(g)]
+    bestK = bestv = None
+    for K in itertools.combinations(sorted(cand), k):
+        v = sorted((sel[e] for e in K), reverse=True)
+        if bestK is None or better(v, K, bestv, bestK):
+            bestK, bestv = K, v
+    picks = sorted(bestK, key=lambda e: (-sel[e], e))
+    ssum = sum(s[e] for e in picks)
+    return picks, [alpha * s[e] / ssum for e in picks]
+
+
+@pytest.mark.parametrize("top2", [0, 1])
+@pytest.mark.parametrize("seed", range(3))
+def test_brute_force_router_variants(seed, top2):
+    """Correction bias (selection only) and the top-2-sum group score against
+    enumeration, with exact ties in the logits and in the bias."""
+    vals = np.array([-2.0, -1.0, -0.5, 0.0, 0.5, 1.0, 2.0], np.float32)
+    bvals = np.array([0.0, 0.25, 0.5], np.float32)
+    n = 0
+    for E, G, tg, k in _tiny_cases(60, 100 + seed):
+        if top2 and E // G < 2:
+            continue
+        cfg = tiny_cfg(E, G, tg, k)
+        rng = np.random.default_rng([seed, top2, E, G, tg, k])
+        x = vals[rng.integers(0, 3 + seed % 4, size=(16, E))]
+        b = bvals[rng.integers(0, 3, size=E)]
+        idx, w, _, _ = oracle.route(cfg, x, np.eye(E, dtype=np.float32), bias=b,
+                                    group_score=top2)
+        for t in range(x.shape[0]):
+            want, wt = brute_force_variant(x[t].astype(np.float64), b.astype(np.float64),
+                                           E, G, tg, k, top2)
+            assert idx[t].tolist() == want, (E, G, tg, k, x[t], b)
+            np.testing.assert_allclose(w[t], wt, rtol=1e-12)
+        n += 1
+    assert n >= 20
