@@ -167,3 +167,6 @@ def test_permute_invariants():
     assert np.all(p["inv_row"][p["perm_token"], p["perm_slot"]] == rows)  # inverse
     assert np.all(np.diff(p["perm_token"])[np.diff(seg) == 0] > 0)        # stable (t increasing)
     np.testing.assert_array_equal(p["counts"], np.bincount(idx.reshape(-1), minlength=E))
+    # the whole order is numpy's stable sort of the (token, slot) assignments by expert
+    np.testing.assert_array_equal(p["perm_token"] * k + p["perm_slot"],
+                                  np.argsort(idx.reshape(-1), kind="stable"))
