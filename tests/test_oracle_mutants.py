@@ -38,6 +38,12 @@ MUTANTS = {
     "norm_over_k_minus_1": ("for (int64_t j = 0; j < c->k; ++j) sum += s[cand[j]];",
                             "for (int64_t j = 0; j + 1 < c->k; ++j) sum += s[cand[j]];"),
     "bf16_widen_wrong_shift": ("<< 16;", "<< 15;"),
+    "top2_sum_takes_group_min": ("gs[q] = sel[tmp[0]] + sel[tmp[1]];",
+                                 "gs[q] = sel[tmp[0]] + sel[tmp[g - 1]];"),
+    "bias_ignored_in_selection": ("sel[e] = s[e] + (bias ? (double)bias[e] : 0.0);",
+                                  "sel[e] = s[e];"),
+    "bias_subtracted": ("sel[e] = s[e] + (bias ? (double)bias[e] : 0.0);",
+                        "sel[e] = s[e] - (bias ? (double)bias[e] : 0.0);"),
 }
 
 PINS = ["tests/test_oracle_route.py", "tests/test_oracle_forward.py",
