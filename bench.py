@@ -115,6 +115,17 @@ def max_over_ranks(elapsed_ms, dist, device):
     return float(t.item())
 
 
+def agree_steps(steps, dist, device):
+    """Rank 0's step count on every rank, so that all ranks time the same work
+    and take the same collective steps."""
+    if dist is None:
+        return int(steps)
+    import torch
+    t = torch.tensor([int(steps)], dtype=torch.int64, device=device)
+    dist.broadcast(t, 0)
+    return int(t.item())
+
+
 def job_throughput(tokens_per_rank_step, world, steps, elapsed_ms):
     """Whole-job tokens/s: the tokens all ranks processed over the max-over-ranks time."""
     return tokens_per_rank_step * world * steps / (elapsed_ms / 1e3)
@@ -256,6 +267,7 @@ def run_ours(args, rank, world, local_rank):
     dist = None
     if world > 1:
         import torch.distributed as dist
+    steps = agree_steps(steps, dist, dev)
     clocks = ClockSampler(local_rank)
     if rank == 0:
         clocks.start()
@@ -544,9 +556,7 @@ def run_tp(args, rank, world, local_rank):
         import torch.distributed as dist
         dist_mod = dist
         # every rank runs the same number of steps (and so the same collectives)
-        st = torch.tensor([steps], device=dev)
-        dist.broadcast(st, 0)
-        steps = int(st.item())
+        steps = agree_steps(steps, dist, dev)
     else:
         dist_mod = None
     clocks = ClockSampler(local_rank)

@@ -1,8 +1,9 @@
 """The benchmark's multi-rank path on CPU: two gloo ranks.
 
 Token data parallelism has no data-path collective; what the ranks share is
-the bookkeeping: disjoint input batches per rank, the max-over-ranks time of
-the timed region, and the whole-job throughput computed from it.  The
+the bookkeeping: disjoint input batches per rank, one step count for all
+ranks, the max-over-ranks time of the timed region, and the whole-job
+throughput computed from it.  The
 reference arm runs on rank 0 only.
 """
 import os
@@ -32,9 +33,10 @@ def _rank_main(rank, world, port, q):
         elapsed = 100.0 + 25.0 * rank            # rank 1 is the slow one
         mx = bench.max_over_ranks(elapsed, dist, torch.device("cpu"))
         ids = bench.rank_batch_ids(4, rank)
+        steps = bench.agree_steps(100 + 7 * rank, dist, torch.device("cpu"))
         gathered = [None] * world
         dist.all_gather_object(gathered, ids)
-        q.put((rank, mx, gathered))
+        q.put((rank, mx, gathered, steps))
     finally:
         dist.destroy_process_group()
 
@@ -51,8 +53,9 @@ def test_two_gloo_ranks_bookkeeping():
     for p in procs:
         p.join(timeout=60)
         assert p.exitcode == 0
-    for rank, mx, gathered in out:
+    for rank, mx, gathered, steps in out:
         assert mx == 125.0                        # every rank sees the slowest rank's time
+        assert steps == 100                       # every rank times rank 0's step count
         flat = [i for ids in gathered for i in ids]
         assert len(flat) == len(set(flat)) == 8   # batches are disjoint across ranks
     # whole-job throughput: all ranks' tokens over the max time
