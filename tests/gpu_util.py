@@ -16,7 +16,6 @@ import os
 import numpy as np
 
 import oracle
-import synth
 
 EXCUSE_GAP = 1e-5
 TOL = {"bf16": 2e-2, "f32": 1e-4}
