@@ -124,10 +124,12 @@ typedef struct {
     size_t perm_token;    /* int32 [T * k] token of each permuted row           */
     size_t perm_w;        /* float [T * k] routing weight of each permuted row  */
     size_t inv_row;       /* int32 [T, k] permuted row of assignment (t, j)     */
-    size_t tiles;         /* int32 [max_tiles, 4] (expert, first row, rows, 0)  */
+    size_t tiles;         /* int32 [max_tiles, 4] (expert, first row, rows,
+                             kind: 1 = an expert's partial last tile of the
+                             CTA-pair GEMM, computed with weights on M)        */
     size_t num_tiles;     /* int32 [1] number of valid tile entries             */
     size_t x_perm;        /* dtype [rows_alloc, H] x gathered in permuted order
-                             (empty when swap_ab: decode reads x directly)    */
+                             (empty when x_direct: the GEMM reads x itself)   */
     size_t h;             /* dtype [rows_alloc, I] relu^2(up) in permuted order */
     size_t y_part;        /* dtype [rows_alloc, H] weighted routed partial rows */
     int64_t rows_alloc;   /* T * k rounded up to the tile height                */
