@@ -353,7 +353,8 @@ nh_status nh_moe_reset_status(void *ws, void *stream);
 /*
  * Synchronises `stream`, reads the workspace status word and returns it
  * (NH_OK, NH_ERR_TIMEOUT or NH_ERR_DEVICE_CHECK); a pending CUDA error is
- * returned as NH_ERR_CUDA.  `ws` is a routed-path workspace.
+ * returned as NH_ERR_CUDA.  `ws` is any of the library's workspaces
+ * (routed, shared or latent): each starts with its own status word.
  */
 nh_status nh_moe_check_device(void *ws, void *stream);
 
