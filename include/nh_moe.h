@@ -186,11 +186,12 @@ nh_status nh_moe_route_permute(const nh_moe_config *cfg, int64_t T, const void *
 
 /*
  * nh_moe_route_noalloc: the router of nh_moe_route for decode-sized batches,
- * for callers that cannot allocate device memory or pass a workspace (for
- * example code running under a CUDA graph capture where allocation is not
- * allowed, serving stacks whose memory pool has already claimed the device,
- * or plugin hosts that give an op no scratch buffer).  None of the cited
- * sources has such a call: it is a packaging choice of this library.
+ * for callers that cannot allocate device memory or pass a workspace: serving
+ * stacks whose memory pool has already claimed the device's free memory, and
+ * plugin hosts that hand an op its inputs and outputs but no scratch buffer
+ * and whose op code may not call cudaMalloc (it is not stream-ordered and can
+ * synchronise the device).  None of the cited sources has such a call: it is
+ * a packaging choice of this library.
  *   Same arguments and results as nh_moe_route, without ws / ws_bytes.
  *   Limits: T <= 32 and T * n_routed_experts <= 16384; larger sizes return
  *   NH_ERR_INVALID_ARG with a message naming the limit (use nh_moe_route).

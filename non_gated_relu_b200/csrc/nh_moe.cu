@@ -813,10 +813,10 @@ __global__ void selftest_timeout_kernel(int* status, uint64_t timeout_ns) {
 // ----------------------------------------------------------------------------
 // Router without caller-provided scratch (nh_moe_route_noalloc).
 //
-// Some callers cannot hand the library a workspace: code that runs while a
-// CUDA graph is being captured with allocations forbidden, serving stacks
-// whose memory pool reserves all of device memory up front, or plugin hosts
-// that give an op no scratch buffer.  For decode-sized batches the router's
+// Some callers cannot hand the library a workspace: serving stacks whose
+// memory pool reserves all of device memory up front, or plugin hosts that
+// give an op no scratch buffer and may not call cudaMalloc (not
+// stream-ordered; it can synchronise the device).  For decode-sized batches the router's
 // only scratch is the logits block, a status word and a completion counter,
 // which fit in a fixed array compiled into the library.  Every device that
 // loads the library holds this array until the process exits.
@@ -990,6 +990,8 @@ nh_status nh_moe_route_noalloc(const nh_moe_config* cfg, int64_t T, const void* 
     return fail(NH_ERR_INVALID_ARG,
                 "nh_moe_route_noalloc takes at most %lld tokens (got %lld); use nh_moe_route",
                 (long long)NOALLOC_MAX_T, (long long)T);
+  // T <= 32 and n_routed_experts <= MAX_E (512) already keep T * E within the
+  // scratch today; this check guards the logits block if MAX_E ever grows
   if (T * cfg->n_routed_experts > NOALLOC_MAX_LOGITS)
     return fail(NH_ERR_INVALID_ARG,
                 "nh_moe_route_noalloc: T * n_routed_experts = %lld exceeds its fixed scratch of "

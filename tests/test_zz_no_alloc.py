@@ -1,8 +1,8 @@
 """nh_moe_route_noalloc: the router for callers that cannot allocate.
 
-Some callers cannot give the library a workspace (graph capture with
-allocation forbidden, a memory pool that owns the whole device, a plugin
-host without scratch).  For them the library keeps the router's scratch in a
+Some callers cannot give the library a workspace (a serving memory pool that
+owns the whole device, a plugin host that passes no scratch buffer and may
+not call cudaMalloc).  For them the library keeps the router's scratch in a
 fixed array of its own.  This test calls that entry point through the C ABI
 twice in a row and checks both results against nh_moe_route, the entry point
 with a caller workspace, within the routing tolerance of the other GPU tests
