@@ -371,7 +371,7 @@ def kernel_times(blk, xs, b, nb, steps):
     import non_gated_relu_b200 as nh
     main = torch.cuda.current_stream(blk.device)
     T = xs[0].shape[0]
-    names = ["route", "permute", "experts_up", "experts_down", "shared", "finalize"]
+    names = ["zero_acc", "route", "permute", "experts_up", "experts_down", "shared", "finalize"]
     acc = {n: 0.0 for n in names}
     ev = {n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for n in names}
@@ -381,13 +381,18 @@ def kernel_times(blk, xs, b, nb, steps):
             ev[n][0].record(stream)
             fn()
             ev[n][1].record(stream)
+        if blk.latent:
+            timed("zero_acc", lambda: (nh.zero_acc(blk.c, T, b.y_acc, stream=main),
+                                       nh.zero_acc(blk.c_exp, T, b.y_lat_acc, stream=main)))
+        else:
+            timed("zero_acc", lambda: nh.zero_acc(blk.c, T, b.y_acc, stream=main))
         if blk.has_shared and blk.nvfp4:
             timed("shared", lambda: nh.shared_nvfp4(blk.c, x, blk.q4["shared_up"],
-                                                     blk.q4["shared_down"], b.y_shared,
+                                                     blk.q4["shared_down"], b.y_acc,
                                                      b.ws_shared, stream=main))
         elif blk.has_shared:
             timed("shared", lambda: nh.shared(blk.c, x, blk.w_shared_up, blk.w_shared_down,
-                                               b.y_shared, b.ws_shared, stream=main))
+                                               b.y_acc, b.ws_shared, stream=main))
         if blk.latent:
             # routing on x, fc1 (counted with the permute), experts in width L
             ce = blk.c_exp
@@ -398,29 +403,29 @@ def kernel_times(blk, xs, b, nb, steps):
                                       nh.reset_status(b.ws, stream=main),
                                       nh.permute(ce, b.x_lat, b.topk_idx, b.topk_w, b.ws,
                                                  stream=main)))
-            xe = b.x_lat
+            xe, yacc = b.x_lat, b.y_lat_acc
         else:
             ce = blk.c
             timed("route", lambda: nh.route(blk.c, x, blk.w_router, blk.bias, b.topk_idx,
                                              b.topk_w, b.ws, stream=main))
             timed("permute", lambda: nh.permute(blk.c, x, b.topk_idx, b.topk_w, b.ws, stream=main))
-            xe = x
+            xe, yacc = x, b.y_acc
         if blk.nvfp4 and not blk.latent:
             # up and down run back to back in one call; each is timed as half
             timed("experts_up", lambda: nh.forward_nvfp4(blk.c, x, blk.q4["up"], blk.q4["down"],
-                                                          b.ws, stream=main))
+                                                          b.ws, yacc, stream=main))
         else:
             timed("experts_up", lambda: nh.experts_up(ce, xe, blk.w_up, b.ws, stream=main))
-            timed("experts_down", lambda: nh.experts_down(ce, T, blk.w_down, b.ws,
+            timed("experts_down", lambda: nh.experts_down(ce, T, blk.w_down, b.ws, yacc,
                                                            stream=main))
         if blk.latent:
-            # finalize in width L, fc2 onto the shared output, the one rounding
-            timed("finalize", lambda: (nh.finalize(ce, T, b.ws, None, b.y_lat, stream=main),
+            # routed sum rounded in width L, fc2 onto y_acc, the one rounding
+            timed("finalize", lambda: (nh.finalize(ce, T, b.y_lat_acc, b.y_lat, stream=main),
                                        nh.latent_out(blk.c, T, b.y_lat, blk.w_latent_fc2,
                                                      b.y_acc, b.ws_lat, stream=main),
-                                       nh.cast_output(blk.c, T, b.y_acc, b.y, stream=main)))
+                                       nh.finalize(blk.c, T, b.y_acc, b.y, stream=main)))
         else:
-            timed("finalize", lambda: nh.finalize(blk.c, T, b.ws, b.y_shared, b.y, stream=main))
+            timed("finalize", lambda: nh.finalize(blk.c, T, b.y_acc, b.y, stream=main))
         torch.cuda.synchronize(blk.device)
         for n in names:
             if (n == "shared" and not blk.has_shared) or (n == "experts_down" and blk.nvfp4):
@@ -582,8 +587,8 @@ def run_tp(args, rank, world, local_rank):
 
     def step(i):
         graphs[i % nb].replay()
-        tp.all_reduce_sum(b.y_f32)
-        return blk.output(b.y_f32)
+        tp.all_reduce_sum(b.y_acc)
+        return blk.output(b.y_acc)
 
     main = torch.cuda.current_stream(dev)
     for i in range(max(3, args.warmup)):
@@ -633,8 +638,8 @@ def run_tp(args, rank, world, local_rank):
     def e2e_step(i):
         xd.copy_(xh[i % nb], non_blocking=True)
         blk.partial(xd)
-        tp.all_reduce_sum(b.y_f32)
-        yh.copy_(blk.output(b.y_f32), non_blocking=True)
+        tp.all_reduce_sum(b.y_acc)
+        yh.copy_(blk.output(b.y_acc), non_blocking=True)
         main.synchronize()
     for i in range(3):
         e2e_step(i)

@@ -11,8 +11,14 @@
  * issue #46, "Architecture (config.json)"; expert shapes in the auto-round PR
  * #1712 log).  One block call is, in stream order:
  *
- *   stream A:  nh_moe_route -> nh_moe_permute -> nh_moe_forward ---+
- *   stream B:  nh_moe_shared ---------------------------------------+-> nh_moe_finalize
+ *   stream B:  nh_moe_zero_acc -> nh_moe_shared --------------------------+
+ *   stream A:  nh_moe_route -> nh_moe_permute -> nh_moe_forward ----------+-> nh_moe_finalize
+ *              (nh_moe_forward's down projection after nh_moe_zero_acc)
+ *
+ * The routed experts' down projection adds each token's k weighted expert
+ * outputs straight into a float32 accumulator y_acc [T, H] (float32 atomic
+ * adds in the GEMM epilogue), the shared expert adds its output into the
+ * same y_acc, and nh_moe_finalize rounds y_acc once to the dtype of x.
  *
  * Conventions (every entry point):
  *   - All pointers named x, w_*, topk_*, y*, ws* are DEVICE pointers of the
@@ -129,15 +135,17 @@ typedef struct {
                              CTA-pair GEMM, computed with weights on M)        */
     size_t num_tiles;     /* int32 [1] number of valid tile entries             */
     size_t x_perm;        /* dtype [rows_alloc, H] x gathered in permuted order
-                             (empty when x_direct: the GEMM reads x itself)   */
+                             (empty when x_direct or x_gather: the GEMM reads
+                             x itself)                                        */
     size_t h;             /* dtype [rows_alloc, I] relu^2(up) in permuted order */
-    size_t y_part;        /* dtype [rows_alloc, H] weighted routed partial rows */
     int64_t rows_alloc;   /* T * k rounded up to the tile height                */
     int32_t tile_rows;    /* rows per tile entry of this (cfg, T)               */
     int32_t max_tiles;
     int32_t n_chunks;     /* token chunks of the permute histogram              */
     int32_t swap_ab;      /* 1: weights on the MMA M side (small T, or NVFP4)   */
     int32_t x_direct;     /* 1: the up projection reads x itself (no x_perm)    */
+    int32_t x_gather;     /* 1: the up projection gathers the rows x[perm_token]
+                             by TMA (CTA-pair tiles; no x_perm)               */
 } nh_moe_ws_layout;
 
 /* Validate a configuration (no device work). */
@@ -213,7 +221,8 @@ nh_status nh_moe_route_noalloc(const nh_moe_config *cfg, int64_t T, const void *
 /*
  * Token permute: per-expert histogram, exclusive scan, stable scatter of the
  * (t, j) assignments in (t, j) order, the tile table of the expert GEMMs and
- * the gather x_perm[row] = x[perm_token[row]].  The routed experts are
+ * (unless the layout's x_direct or x_gather is set) the gather
+ * x_perm[row] = x[perm_token[row]].  The routed experts are
  * applied per expert id (MLX SwitchMLP fc1/fc2 indexed by the router's
  * expert ids, exo commit "Add support for Nemotron sharding").
  *   topk_idx / topk_w as produced by nh_moe_route (any valid ids in [0, E)
@@ -224,16 +233,27 @@ nh_status nh_moe_permute(const nh_moe_config *cfg, int64_t T, const void *x,
                          void *stream);
 
 /*
- * Routed experts: h[r] = relu(x[perm_token[r]] W_up[e]^T)^2 (float32
- * accumulate, h stored in dtype), then the weighted partial rows
- *   y_part[r] = perm_w[r] * (h[r] W_down[e]^T)     (dtype, permuted row order)
- * which nh_moe_finalize sums per token.  Both live in the workspace.
+ * Routed experts with the weighted combine (exo commit "Add support for
+ * Nemotron sharding": switch_layers.pyi SwitchMLP fc1 / fc2 per expert id,
+ * and nemotron_h.pyi NemotronHMoE.__call__, which sums the k experts of a
+ * token weighted by the router):
+ *   h[r] = relu(x[perm_token[r]] W_up[e]^T)^2      (float32 accumulate, h in
+ *                                                   dtype, in the workspace)
+ *   y_acc[perm_token[r]] += perm_w[r] * (h[r] W_down[e]^T)      (float32)
+ * for every permuted row r of expert e.  The adds are float32 atomic adds
+ * issued by the down projection's epilogue, so the order in which a token's
+ * k contributions (and the shared expert's) are summed is not fixed: results
+ * can differ between runs in the last float32 bits.
  *   x [T, H] dtype (the same x that nh_moe_permute saw); w_up [E, I, H] dtype;
- *   w_down [E, H, I] dtype.
+ *   w_down [E, H, I] dtype; y_acc [T, H] float32, read and added to: it must
+ *   hold its starting value (zeros from nh_moe_zero_acc, optionally plus the
+ *   shared expert) before the down projection runs, and no other stream may
+ *   write it meanwhile except nh_moe_shared's adds.
  * Needs nh_moe_permute's workspace contents.
  */
 nh_status nh_moe_forward(const nh_moe_config *cfg, int64_t T, const void *x, const void *w_up,
-                         const void *w_down, void *ws, size_t ws_bytes, void *stream);
+                         const void *w_down, void *ws, size_t ws_bytes, float *y_acc,
+                         void *stream);
 
 /*
  * nh_moe_forward with NVFP4 routed-expert weights (cfg->weight_format ==
@@ -241,73 +261,70 @@ nh_status nh_moe_forward(const nh_moe_config *cfg, int64_t T, const void *x, con
  * Each weight is dequantized in registers (code x block scale, exact in
  * bf16): for tiles of up to 32 tokens per expert straight into warp-level MMA
  * fragments, for 64-token tiles into tensor memory as the A operand of
- * tcgen05.mma.  The float32 matrix scale is applied in the epilogue.  Same
- * results layout as nh_moe_forward.
+ * tcgen05.mma.  The float32 matrix scale is applied in the epilogue.  Adds
+ * into y_acc exactly like nh_moe_forward.
  */
 nh_status nh_moe_forward_nvfp4(const nh_moe_config *cfg, int64_t T, const void *x,
                                const nh_nvfp4_weight *w_up, const nh_nvfp4_weight *w_down,
-                               void *ws, size_t ws_bytes, void *stream);
+                               void *ws, size_t ws_bytes, float *y_acc, void *stream);
 
 /*
  * The two phases of nh_moe_forward, for callers that schedule or time them
  * separately (same arguments and requirements):
  *   nh_moe_experts_up:   h = relu(x[perm_token] W_up[e]^T)^2 into the workspace;
- *   nh_moe_experts_down: y_part[r] = perm_w[r] * (h[r] W_down[e]^T).
+ *   nh_moe_experts_down: y_acc[perm_token[r]] += perm_w[r] * (h[r] W_down[e]^T).
  */
 nh_status nh_moe_experts_up(const nh_moe_config *cfg, int64_t T, const void *x, const void *w_up,
                             void *ws, size_t ws_bytes, void *stream);
 nh_status nh_moe_experts_down(const nh_moe_config *cfg, int64_t T, const void *w_down, void *ws,
-                              size_t ws_bytes, void *stream);
+                              size_t ws_bytes, float *y_acc, void *stream);
 
 /*
- * Shared expert (NemotronHMLP up_proj / down_proj, always on, unscaled):
- * y_shared = relu(x W_su^T)^2 W_sd^T, written (not accumulated).
- *   w_shared_up [S, H]; w_shared_down [H, S] (dtype); y_shared [T, H] float32;
- *   ws_shared: nh_moe_shared_workspace_size bytes.
- * Independent of the routed path: may run on a second stream.
+ * Shared expert (NemotronHMLP up_proj / down_proj, always on, unscaled; exo
+ * commit "Add support for Nemotron sharding", nemotron_h.pyi):
+ *   y_acc += relu(x W_su^T)^2 W_sd^T      (float32 atomic adds)
+ *   w_shared_up [S, H]; w_shared_down [H, S] (dtype); y_acc [T, H] float32,
+ *   the accumulator nh_moe_forward adds into; ws_shared:
+ *   nh_moe_shared_workspace_size bytes.
+ * Independent of the routed path: may run on a second stream, concurrently
+ * with nh_moe_forward, once y_acc holds its starting value.
  */
 nh_status nh_moe_shared(const nh_moe_config *cfg, int64_t T, const void *x, const void *w_shared_up,
-                        const void *w_shared_down, float *y_shared, void *ws_shared,
+                        const void *w_shared_down, float *y_acc, void *ws_shared,
                         size_t ws_shared_bytes, void *stream);
 
 /* nh_moe_shared with NVFP4 shared-expert weights: w_shared_up [1][S][H],
  * w_shared_down [1][H][S]. */
 nh_status nh_moe_shared_nvfp4(const nh_moe_config *cfg, int64_t T, const void *x,
                               const nh_nvfp4_weight *w_shared_up,
-                              const nh_nvfp4_weight *w_shared_down, float *y_shared,
+                              const nh_nvfp4_weight *w_shared_down, float *y_acc,
                               void *ws_shared, size_t ws_shared_bytes, void *stream);
 
 /*
- * y[t] = dtype( y_shared[t] + sum_j y_part[inv_row[t, j]] ), summed in float32
- * in that order (deterministic; no atomics anywhere on the path).
- *   ws: the routed workspace after nh_moe_forward; y_shared [T, H] float32
- *   (NULL when the config has no shared expert); y [T, H] dtype (out).
+ * y_acc = 0: the starting value of the float32 accumulator [T, H] (H =
+ * cfg->hidden_size) that nh_moe_shared and nh_moe_forward add into.  An
+ * asynchronous memset on `stream`; no kernel.
  */
-nh_status nh_moe_finalize(const nh_moe_config *cfg, int64_t T, const void *ws, size_t ws_bytes,
-                          const float *y_shared, void *y, void *stream);
+nh_status nh_moe_zero_acc(const nh_moe_config *cfg, int64_t T, float *y_acc, void *stream);
 
 /*
+ * y = dtype(y_acc): the block output, rounded once (float32 dtype: a copy).
+ *   y_acc [T, H] float32 after nh_moe_forward and nh_moe_shared; y [T, H]
+ *   dtype (out).  H = cfg->hidden_size.
+ *
  * Tensor-parallel shards (exo commit "Add support for Nemotron sharding",
  * the NemotronHMoE branch of the sharding strategy: the routed fc1 and the
  * shared up_proj are split over their output features, the routed fc2 and the
  * shared down_proj over their input features, the router is replicated, and
- * one all-reduce sums the block output).
- * A rank runs the whole path with the config of its shard
- * (moe_intermediate_size and moe_shared_expert_intermediate_size set to its
- * share of I and S, each a multiple of 64) and its slices of the weights,
- * then calls nh_moe_finalize_partial instead of nh_moe_finalize:
- *   y_f32[t] = y_shared[t] + sum_j y_part[inv_row[t, j]]     (float32, no rounding)
- * The caller sums y_f32 over the ranks (an all-reduce) and rounds the sum once
- * with nh_moe_cast_output:
- *   y[t] = dtype(y_f32[t])
- * y_f32 [T, H] float32 and y [T, H] dtype are device buffers, 16-byte aligned.
- * Errors as nh_moe_finalize.
+ * one all-reduce sums the block output): a rank runs the whole path with the
+ * config of its shard (moe_intermediate_size and
+ * moe_shared_expert_intermediate_size set to its share of I and S, each a
+ * multiple of 64) and its slices of the weights.  Its y_acc is then its
+ * float32 contribution; the caller sums y_acc over the ranks (an all-reduce)
+ * and calls nh_moe_finalize on the sum, so the output is rounded once.
  */
-nh_status nh_moe_finalize_partial(const nh_moe_config *cfg, int64_t T, const void *ws,
-                                  size_t ws_bytes, const float *y_shared, float *y_f32,
-                                  void *stream);
-nh_status nh_moe_cast_output(const nh_moe_config *cfg, int64_t T, const float *y_f32, void *y,
-                             void *stream);
+nh_status nh_moe_finalize(const nh_moe_config *cfg, int64_t T, const float *y_acc, void *y,
+                          void *stream);
 
 /*
  * Latent MoE projections (ModelOpt descriptor NemotronHMoELayerDescriptor:
@@ -316,21 +333,22 @@ nh_status nh_moe_cast_output(const nh_moe_config *cfg, int64_t T, const float *y
  * L = cfg->latent_size > 0:
  *   x_lat = dtype(x W_fc1^T)                     W_fc1 [L, H]   (nh_moe_latent_in)
  *   routed experts on x_lat, in width L: W_up [E, I, L], W_down [E, L, I],
- *     routing on x (nh_moe_route with cfg), combined as usual into
- *     y_lat [T, L] (nh_moe_finalize, rounded to dtype)
+ *     routing on x (nh_moe_route with cfg), combined as usual into a zeroed
+ *     float32 y_lat_acc [T, L] and rounded to y_lat [T, L] (nh_moe_zero_acc,
+ *     nh_moe_forward, nh_moe_finalize with the expert-width config)
  *   y_acc += y_lat W_fc2^T                       W_fc2 [H, L]   (nh_moe_latent_out)
- *     where y_acc holds the shared expert's y_shared; without a shared
- *     expert nh_moe_latent_out writes y_acc = y_lat W_fc2^T instead
- *   y = dtype(y_acc)                                            (nh_moe_cast_output)
+ *     where y_acc holds zeros plus the shared expert (nh_moe_zero_acc and
+ *     nh_moe_shared with cfg), complete before this call
+ *   y = dtype(y_acc)                                            (nh_moe_finalize)
  * The routed-expert calls (nh_moe_permute, nh_moe_forward[_nvfp4],
- * nh_moe_experts_*, nh_moe_finalize[_partial]) take the expert-width config
+ * nh_moe_experts_*) take the expert-width config
  * that nh_moe_latent_config writes (hidden_size = L, latent_size = 0,
  * n_shared_experts = 0) and return NH_ERR_INVALID_ARG for a config with
  * latent_size > 0; nh_moe_route and nh_moe_shared take cfg itself.
  * nh_moe_route needs only the first `counts` bytes of its workspace layout.
  *   x [T, H], x_lat [T, L], y_lat [T, L]: dtype; W_fc1, W_fc2: dtype (also
  *   with NVFP4 expert weights); y_acc [T, H] float32 (read and written; each
- *   element by one thread, deterministic); ws_latent:
+ *   element by one thread); ws_latent:
  *   nh_moe_latent_workspace_size bytes.  Device pointers, 16-byte aligned.
  */
 nh_status nh_moe_latent_config(const nh_moe_config *cfg, nh_moe_config *expert_cfg);

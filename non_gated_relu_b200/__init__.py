@@ -6,7 +6,7 @@ memory and streams.  There is no CPU fallback: when the library cannot be
 built or loaded, or no sm_100 device is present, the calls raise.
 
 Low level (same names as the C ABI, minus the ``nh_moe_`` prefix):
-``route``, ``permute``, ``forward``, ``shared``, ``finalize``,
+``route``, ``permute``, ``forward``, ``shared``, ``zero_acc``, ``finalize``,
 ``check_device``, ``workspace_size``, ``workspace_layout``,
 ``shared_workspace_size``, ``validate``, ``selftest_timeout``.
 
@@ -23,7 +23,7 @@ from . import build as _build
 
 __all__ = ["NHMoEError", "Config", "Layout", "config_from", "load", "validate", "workspace_size",
            "workspace_layout", "shared_workspace_size", "route", "route_noalloc", "route_permute", "permute", "forward", "experts_up", "experts_down", "shared", "forward_nvfp4", "shared_nvfp4", "nvfp4_weight",
-           "finalize", "finalize_partial", "cast_output", "latent_config", "latent_workspace_size",
+           "zero_acc", "finalize", "latent_config", "latent_workspace_size",
            "latent_in", "latent_out", "reset_status", "check_device", "selftest_timeout", "library_path", "NemotronHMoE"]
 
 NH_OK, NH_ERR_INVALID_ARG, NH_ERR_UNSUPPORTED, NH_ERR_CUDA, NH_ERR_TIMEOUT, NH_ERR_DEVICE_CHECK = range(6)
@@ -63,10 +63,10 @@ class Layout(ctypes.Structure):
     """nh_moe_ws_layout: byte offsets of the routed-path workspace regions."""
     _fields_ = [(n, ctypes.c_size_t) for n in (
         "total_bytes", "status", "logits", "router_w", "counts", "offsets", "chunk_counts", "perm_token",
-        "perm_w", "inv_row", "tiles", "num_tiles", "x_perm", "h", "y_part")] + [
+        "perm_w", "inv_row", "tiles", "num_tiles", "x_perm", "h")] + [
         ("rows_alloc", ctypes.c_int64), ("tile_rows", ctypes.c_int32),
         ("max_tiles", ctypes.c_int32), ("n_chunks", ctypes.c_int32), ("swap_ab", ctypes.c_int32),
-        ("x_direct", ctypes.c_int32)]
+        ("x_direct", ctypes.c_int32), ("x_gather", ctypes.c_int32)]
 
 
 def config_from(c, group_score: int = 0) -> Config:
@@ -91,7 +91,8 @@ _lib = None
 _EXPORTS = ["nh_moe_validate", "nh_moe_workspace_size", "nh_moe_workspace_layout",
             "nh_moe_shared_workspace_size", "nh_moe_route", "nh_moe_route_noalloc", "nh_moe_route_permute",
             "nh_moe_permute", "nh_moe_forward", "nh_moe_experts_up", "nh_moe_experts_down",
-            "nh_moe_shared", "nh_moe_finalize", "nh_moe_finalize_partial", "nh_moe_cast_output",
+            "nh_moe_forward_nvfp4", "nh_moe_shared", "nh_moe_shared_nvfp4", "nh_moe_zero_acc",
+            "nh_moe_finalize",
             "nh_moe_latent_config", "nh_moe_latent_workspace_size", "nh_moe_latent_in",
             "nh_moe_latent_out", "nh_moe_reset_status", "nh_moe_check_device",
             "nh_moe_selftest_timeout",
@@ -121,17 +122,16 @@ def load():
             "nh_moe_route_noalloc": [C, I64, P, P, P, P, P, P],
             "nh_moe_route_permute": [C, I64, P, P, P, P, P, P, S, P],
             "nh_moe_permute": [C, I64, P, P, P, P, S, P],
-            "nh_moe_forward": [C, I64, P, P, P, P, S, P],
+            "nh_moe_forward": [C, I64, P, P, P, P, S, P, P],
             "nh_moe_experts_up": [C, I64, P, P, P, S, P],
-            "nh_moe_experts_down": [C, I64, P, P, S, P],
+            "nh_moe_experts_down": [C, I64, P, P, S, P, P],
             "nh_moe_shared": [C, I64, P, P, P, P, P, S, P],
             "nh_moe_forward_nvfp4": [C, I64, P, ctypes.POINTER(NvFp4Weight),
-                                     ctypes.POINTER(NvFp4Weight), P, S, P],
+                                     ctypes.POINTER(NvFp4Weight), P, S, P, P],
             "nh_moe_shared_nvfp4": [C, I64, P, ctypes.POINTER(NvFp4Weight),
                                     ctypes.POINTER(NvFp4Weight), P, P, S, P],
-            "nh_moe_finalize": [C, I64, P, S, P, P, P],
-            "nh_moe_finalize_partial": [C, I64, P, S, P, P, P],
-            "nh_moe_cast_output": [C, I64, P, P, P],
+            "nh_moe_zero_acc": [C, I64, P, P],
+            "nh_moe_finalize": [C, I64, P, P, P],
             "nh_moe_latent_config": [C, C],
             "nh_moe_latent_workspace_size": [C, I64, ctypes.POINTER(S)],
             "nh_moe_latent_in": [C, I64, P, P, P, P, S, P],
@@ -230,10 +230,11 @@ def permute(cfg, x, topk_idx, topk_w, ws, stream=None):
                                  _p(ws), _nbytes(ws), _stream(stream)))
 
 
-def forward(cfg, x, w_up, w_down, ws, stream=None):
+def forward(cfg, x, w_up, w_down, ws, y_acc, stream=None):
+    """Routed experts: y_acc[token] += the token's weighted expert outputs (float32)."""
     c = config_from(cfg)
     _check(load().nh_moe_forward(ctypes.byref(c), x.shape[0], _p(x), _p(w_up), _p(w_down), _p(ws),
-                                 _nbytes(ws), _stream(stream)))
+                                 _nbytes(ws), _p(y_acc), _stream(stream)))
 
 
 def experts_up(cfg, x, w_up, ws, stream=None):
@@ -242,16 +243,17 @@ def experts_up(cfg, x, w_up, ws, stream=None):
                                     _nbytes(ws), _stream(stream)))
 
 
-def experts_down(cfg, T: int, w_down, ws, stream=None):
+def experts_down(cfg, T: int, w_down, ws, y_acc, stream=None):
     c = config_from(cfg)
     _check(load().nh_moe_experts_down(ctypes.byref(c), T, _p(w_down), _p(ws), _nbytes(ws),
-                                      _stream(stream)))
+                                      _p(y_acc), _stream(stream)))
 
 
-def shared(cfg, x, w_shared_up, w_shared_down, y_shared, ws_shared, stream=None):
+def shared(cfg, x, w_shared_up, w_shared_down, y_acc, ws_shared, stream=None):
+    """Shared expert: y_acc += relu(x W_su^T)^2 W_sd^T (float32)."""
     c = config_from(cfg)
     _check(load().nh_moe_shared(ctypes.byref(c), x.shape[0], _p(x), _p(w_shared_up),
-                                _p(w_shared_down), _p(y_shared), _p(ws_shared),
+                                _p(w_shared_down), _p(y_acc), _p(ws_shared),
                                 _nbytes(ws_shared), _stream(stream)))
 
 
@@ -260,38 +262,31 @@ def nvfp4_weight(codes, scales, global_scale) -> NvFp4Weight:
     return NvFp4Weight(codes.data_ptr(), scales.data_ptr(), global_scale.data_ptr())
 
 
-def forward_nvfp4(cfg, x, w_up, w_down, ws, stream=None):
+def forward_nvfp4(cfg, x, w_up, w_down, ws, y_acc, stream=None):
     """nh_moe_forward with NVFP4 weights; w_up / w_down are NvFp4Weight structs."""
     c = config_from(cfg)
     _check(load().nh_moe_forward_nvfp4(ctypes.byref(c), x.shape[0], _p(x), ctypes.byref(w_up),
-                                       ctypes.byref(w_down), _p(ws), _nbytes(ws), _stream(stream)))
+                                       ctypes.byref(w_down), _p(ws), _nbytes(ws), _p(y_acc),
+                                       _stream(stream)))
 
 
-def shared_nvfp4(cfg, x, w_shared_up, w_shared_down, y_shared, ws_shared, stream=None):
+def shared_nvfp4(cfg, x, w_shared_up, w_shared_down, y_acc, ws_shared, stream=None):
     c = config_from(cfg)
     _check(load().nh_moe_shared_nvfp4(ctypes.byref(c), x.shape[0], _p(x), ctypes.byref(w_shared_up),
-                                      ctypes.byref(w_shared_down), _p(y_shared), _p(ws_shared),
+                                      ctypes.byref(w_shared_down), _p(y_acc), _p(ws_shared),
                                       _nbytes(ws_shared), _stream(stream)))
 
 
-def finalize(cfg, T: int, ws, y_shared, y, stream=None):
+def zero_acc(cfg, T: int, y_acc, stream=None):
+    """y_acc = 0 ([T, hidden_size] float32), asynchronously on `stream`."""
     c = config_from(cfg)
-    _check(load().nh_moe_finalize(ctypes.byref(c), T, _p(ws), _nbytes(ws), _p(y_shared), _p(y),
-                                  _stream(stream)))
+    _check(load().nh_moe_zero_acc(ctypes.byref(c), T, _p(y_acc), _stream(stream)))
 
 
-def finalize_partial(cfg, T: int, ws, y_shared, y_f32, stream=None):
-    """Tensor-parallel rank: y_f32 = the float32 sum of this rank's partial
-    rows and shared output, without the final rounding."""
+def finalize(cfg, T: int, y_acc, y, stream=None):
+    """y = dtype(y_acc): the one rounding of the block output."""
     c = config_from(cfg)
-    _check(load().nh_moe_finalize_partial(ctypes.byref(c), T, _p(ws), _nbytes(ws), _p(y_shared),
-                                          _p(y_f32), _stream(stream)))
-
-
-def cast_output(cfg, T: int, y_f32, y, stream=None):
-    """y = dtype(y_f32), the one rounding of an all-reduced block output."""
-    c = config_from(cfg)
-    _check(load().nh_moe_cast_output(ctypes.byref(c), T, _p(y_f32), _p(y), _stream(stream)))
+    _check(load().nh_moe_finalize(ctypes.byref(c), T, _p(y_acc), _p(y), _stream(stream)))
 
 
 def latent_config(cfg) -> Config:

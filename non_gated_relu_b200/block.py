@@ -5,16 +5,17 @@ The Nemotron-H MoE block (``NemotronHMoE.__call__(x) -> y`` with a
 commit "Add support for Nemotron sharding", nemotron_h.pyi) on one GPU.  One
 call runs, on the caller's stream and a side stream:
 
-    main: route + permute -> forward (routed experts) --+
-    side: shared expert ----------------------------------+-> finalize
+    side: y_acc = 0 --+-> shared expert: y_acc += shared(x) ----------+
+    main: route + permute -> forward: y_acc += routed experts (x) ---+-> finalize: y = dtype(y_acc)
+                      (forward's down projection waits for y_acc = 0)
 
 With latent projections (config ``latent_size`` L > 0; the modules
 fc1_latent_proj / fc2_latent_proj of the ModelOpt descriptor
 NemotronHMoELayerDescriptor) the routed experts run in width L:
 
-    main: route(x) -> fc1: x_lat -> permute + forward + finalize in width L
-          -> y_lat --+-> fc2: y_shared += y_lat W_fc2^T -> cast -> y
-    side: shared expert(x) -> y_shared
+    side: y_acc = 0, y_lat_acc = 0 -> shared expert(x) into y_acc ------+
+    main: route(x) -> fc1: x_lat -> permute + forward into y_lat_acc      |
+          -> y_lat = dtype(y_lat_acc) --+-> fc2: y_acc += y_lat W_fc2^T -> y = dtype(y_acc)
 
 All arithmetic happens in libnhmoe's kernels; this class only owns buffers,
 streams, events and (optionally) a CUDA graph of the call sequence.
@@ -27,11 +28,10 @@ from typing import Dict, Optional
 import numpy as np
 import torch
 
-from . import (cast_output, check_device, config_from, finalize, finalize_partial, forward,
-               forward_nvfp4, latent_config, latent_in, latent_out, latent_workspace_size,
-               nvfp4_weight, permute, reset_status, route, route_permute, shared, shared_nvfp4,
-               shared_workspace_size, validate, workspace_layout, workspace_size, NH_BF16,
-               NH_WEIGHTS_NVFP4)
+from . import (check_device, config_from, finalize, forward, forward_nvfp4, latent_config,
+               latent_in, latent_out, latent_workspace_size, nvfp4_weight, permute, reset_status,
+               route, route_permute, shared, shared_nvfp4, shared_workspace_size, validate,
+               workspace_layout, workspace_size, zero_acc, NH_BF16, NH_WEIGHTS_NVFP4)
 
 
 def _to_device(a, dtype: torch.dtype, device) -> torch.Tensor:
@@ -55,16 +55,15 @@ class Buffers:
     ws_shared: Optional[torch.Tensor]
     topk_idx: torch.Tensor
     topk_w: torch.Tensor
-    y_shared: Optional[torch.Tensor]
+    y_acc: torch.Tensor                      # float32 [T, H]: shared + weighted routed experts
     y: torch.Tensor
-    y_f32: Optional[torch.Tensor] = None     # tensor-parallel partial sum (float32)
     # latent blocks: routing workspace (full width), projection workspace,
-    # x_lat / y_lat [T, L], float32 accumulator [T, H] (y_shared when present)
+    # x_lat / y_lat [T, L] and the float32 accumulator of the routed experts [T, L]
     ws_route: Optional[torch.Tensor] = None
     ws_lat: Optional[torch.Tensor] = None
     x_lat: Optional[torch.Tensor] = None
     y_lat: Optional[torch.Tensor] = None
-    y_acc: Optional[torch.Tensor] = None
+    y_lat_acc: Optional[torch.Tensor] = None
 
 
 class NemotronHMoE:
@@ -145,13 +144,13 @@ class NemotronHMoE:
         if b is None:
             dev = self.device
             ws = torch.empty(workspace_size(self.c_exp, T), dtype=torch.uint8, device=dev)
-            wss = ys = None
+            wss = None
             if self.has_shared:
                 wss = torch.empty(shared_workspace_size(self.c, T), dtype=torch.uint8, device=dev)
-                ys = torch.empty((T, self.H), dtype=torch.float32, device=dev)
             b = Buffers(T, ws, wss,
                         torch.empty((T, self.k), dtype=torch.int32, device=dev),
-                        torch.empty((T, self.k), dtype=torch.float32, device=dev), ys,
+                        torch.empty((T, self.k), dtype=torch.float32, device=dev),
+                        torch.empty((T, self.H), dtype=torch.float32, device=dev),
                         torch.empty((T, self.H), dtype=self.dtype, device=dev))
             if self.latent:
                 b.ws_route = torch.empty(max(256, workspace_layout(self.c, T).counts),
@@ -160,8 +159,7 @@ class NemotronHMoE:
                                        device=dev)
                 b.x_lat = torch.empty((T, self.L), dtype=self.dtype, device=dev)
                 b.y_lat = torch.empty((T, self.L), dtype=self.dtype, device=dev)
-                b.y_acc = (b.y_shared if self.has_shared else
-                           torch.empty((T, self.H), dtype=torch.float32, device=dev))
+                b.y_lat_acc = torch.empty((T, self.L), dtype=torch.float32, device=dev)
             self._bufs[T] = b
         return b
 
@@ -171,11 +169,10 @@ class NemotronHMoE:
         """y for a device tensor x [T, H]; returns the buffer-owned y [T, H].
         ``nvtx`` wraps each call in an NVTX range of its name (for profilers).
         ``partial`` (a tensor-parallel shard) returns instead the float32
-        sum of this shard's contributions, unrounded, for an all-reduce."""
+        accumulator y_acc of this shard's contributions, unrounded, for an
+        all-reduce."""
         T = x.shape[0]
         b = bufs or self.buffers(T)
-        if partial and b.y_f32 is None:
-            b.y_f32 = torch.empty((T, self.H), dtype=torch.float32, device=self.device)
         caller = torch.cuda.current_stream(self.device)
         main = self.hi
         push = torch.cuda.nvtx.range_push if nvtx else (lambda name: None)
@@ -183,42 +180,48 @@ class NemotronHMoE:
         fork = torch.cuda.Event()
         fork.record(caller)
         main.wait_event(fork)
+        self.side.wait_event(fork)
+        # side stream: the accumulators start at zero, then the shared expert
+        # adds into y_acc (beside the routed path)
+        push("zero_acc")
+        zero_acc(self.c, T, b.y_acc, stream=self.side)
+        if self.latent:
+            zero_acc(self.c_exp, T, b.y_lat_acc, stream=self.side)
+        pop()
+        zero = torch.cuda.Event()
+        zero.record(self.side)
         if self.has_shared:
-            self.side.wait_event(fork)
             push("shared")
             if self.nvfp4:
-                shared_nvfp4(self.c, x, self.q4["shared_up"], self.q4["shared_down"], b.y_shared,
+                shared_nvfp4(self.c, x, self.q4["shared_up"], self.q4["shared_down"], b.y_acc,
                              b.ws_shared, stream=self.side)
             else:
-                shared(self.c, x, self.w_shared_up, self.w_shared_down, b.y_shared, b.ws_shared,
+                shared(self.c, x, self.w_shared_up, self.w_shared_down, b.y_acc, b.ws_shared,
                        stream=self.side)
             pop()
-            join = torch.cuda.Event()
-            join.record(self.side)
+        join = torch.cuda.Event()
+        join.record(self.side)
         if self.latent:
-            out = self._forward_latent(x, b, main, join if self.has_shared else None, partial,
-                                       push, pop)
+            out = self._forward_latent(x, b, main, zero, join, partial, push, pop)
             self._join(caller, main)
             return out
         push("route_permute")
         route_permute(self.c, x, self.w_router, self.bias, b.topk_idx, b.topk_w, b.ws, stream=main)
         pop()
+        main.wait_event(zero)
         push("forward")
         if self.nvfp4:
-            forward_nvfp4(self.c, x, self.q4["up"], self.q4["down"], b.ws, stream=main)
+            forward_nvfp4(self.c, x, self.q4["up"], self.q4["down"], b.ws, b.y_acc, stream=main)
         else:
-            forward(self.c, x, self.w_up, self.w_down, b.ws, stream=main)
+            forward(self.c, x, self.w_up, self.w_down, b.ws, b.y_acc, stream=main)
         pop()
-        if self.has_shared:
-            main.wait_event(join)
-        push("finalize")
-        if partial:
-            finalize_partial(self.c, T, b.ws, b.y_shared, b.y_f32, stream=main)
-        else:
-            finalize(self.c, T, b.ws, b.y_shared, b.y, stream=main)
-        pop()
+        main.wait_event(join)
+        if not partial:
+            push("finalize")
+            finalize(self.c, T, b.y_acc, b.y, stream=main)
+            pop()
         self._join(caller, main)
-        return b.y_f32 if partial else b.y
+        return b.y_acc if partial else b.y
 
     @staticmethod
     def _join(caller, main):
@@ -226,7 +229,7 @@ class NemotronHMoE:
         done.record(main)
         caller.wait_event(done)
 
-    def _forward_latent(self, x, b, main, join, partial, push, pop):
+    def _forward_latent(self, x, b, main, zero, join, partial, push, pop):
         T = x.shape[0]
         push("route")
         route(self.c, x, self.w_router, self.bias, b.topk_idx, b.topk_w, b.ws_route, stream=main)
@@ -238,21 +241,22 @@ class NemotronHMoE:
         ce = self.c_exp
         reset_status(b.ws, stream=main)
         permute(ce, b.x_lat, b.topk_idx, b.topk_w, b.ws, stream=main)
+        main.wait_event(zero)
         if self.nvfp4:
-            forward_nvfp4(ce, b.x_lat, self.q4["up"], self.q4["down"], b.ws, stream=main)
+            forward_nvfp4(ce, b.x_lat, self.q4["up"], self.q4["down"], b.ws, b.y_lat_acc,
+                          stream=main)
         else:
-            forward(ce, b.x_lat, self.w_up, self.w_down, b.ws, stream=main)
-        finalize(ce, T, b.ws, None, b.y_lat, stream=main)
+            forward(ce, b.x_lat, self.w_up, self.w_down, b.ws, b.y_lat_acc, stream=main)
+        finalize(ce, T, b.y_lat_acc, b.y_lat, stream=main)
         pop()
-        if join is not None:
-            main.wait_event(join)
+        main.wait_event(join)
         push("latent_out")
         latent_out(self.c, T, b.y_lat, self.w_latent_fc2, b.y_acc, b.ws_lat, stream=main)
         pop()
         if partial:
             return b.y_acc
-        push("cast")
-        cast_output(self.c, T, b.y_acc, b.y, stream=main)
+        push("finalize")
+        finalize(self.c, T, b.y_acc, b.y, stream=main)
         pop()
         return b.y
 

@@ -11,11 +11,15 @@ namespace nh {
 
 enum Epilogue : int {
   EPI_UP_RELU2 = 0,      // out (dtype) [rows, N] = relu(acc)^2
-  EPI_DOWN_WEIGHTED = 1, // out (dtype) [rows, N] = perm_w[r] * acc   (routed partial rows)
+  EPI_DOWN_COMBINE = 1,  // out (float32) [T, N]: out[dst_row[r]] += perm_w[r] * acc
+                         //   (routed down projection: the weighted combine of a
+                         //   token's k experts, float32 atomic adds)
   EPI_STORE_F32 = 2,     // out (float32) [rows, N] = acc
   EPI_STORE = 3,         // out (dtype) [rows, N] = acc             (latent fc1 projection)
   EPI_ADD_F32 = 4,       // out (float32) [rows, N] += acc          (latent fc2 projection;
                          //   each element has one owner tile: no atomics)
+  EPI_ACC_F32 = 5,       // out (float32) [rows, N] += acc, atomic adds (shared expert,
+                         //   which may run beside the routed combine)
 };
 
 struct GemmArgs {
@@ -30,6 +34,7 @@ struct GemmArgs {
   void* out;
   int64_t ldo;            // row stride of out, elements
   const float* perm_w;
+  const int32_t* dst_row; // EPI_DOWN_COMBINE: output row (token) of each permuted row
 };
 
 __device__ __forceinline__ bool tile_entry(const GemmArgs& g, int m, int4& ent) {
@@ -98,12 +103,15 @@ __global__ void __launch_bounds__(256) simt_grouped_gemm(GemmArgs g) {
       const float v = acc[i][j];
       if (g.epi == EPI_UP_RELU2) {
         static_cast<Tin*>(g.out)[(size_t)r * g.ldo + n] = from_f32<Tin>(relu2(v));
-      } else if (g.epi == EPI_DOWN_WEIGHTED) {
-        static_cast<Tin*>(g.out)[(size_t)r * g.ldo + n] = from_f32<Tin>(g.perm_w[r] * v);
+      } else if (g.epi == EPI_DOWN_COMBINE) {
+        red_add_f32(static_cast<float*>(g.out) + (size_t)g.dst_row[r] * g.ldo + n,
+                    g.perm_w[r] * v);
       } else if (g.epi == EPI_STORE) {
         static_cast<Tin*>(g.out)[(size_t)r * g.ldo + n] = from_f32<Tin>(v);
       } else if (g.epi == EPI_ADD_F32) {
         static_cast<float*>(g.out)[(size_t)r * g.ldo + n] += v;
+      } else if (g.epi == EPI_ACC_F32) {
+        red_add_f32(static_cast<float*>(g.out) + (size_t)r * g.ldo + n, v);
       } else {
         static_cast<float*>(g.out)[(size_t)r * g.ldo + n] = v;
       }

@@ -8,9 +8,9 @@
 //   up_proj:   h = relu(D)^2 stored in bf16              (non-gated expert:
 //              no gate projection, squared relu between the two
 //              projections; vllm.cpp PR #518)
-//   down_proj: y_part[row] = routing weight * D in bf16     (per-(token, expert)
-//              partial rows, summed per token by the finalize kernel)
-//   shared:    y_shared = D                                 (always-on expert)
+//   down_proj: y_acc[token of row] += routing weight * D    (the weighted
+//              combine of a token's k experts, float32 atomic adds)
+//   shared:    y_acc += D                                   (always-on expert)
 //
 // Two orientations:
 //   prefill (SWAP = false): MMA M = 128 activation rows, N = NT weight rows;
@@ -50,9 +50,12 @@ struct TcArgs {
   void* out;
   int64_t ldo;                // row stride of out, elements
   const float* perm_w;
+  const int32_t* dst_row;     // EPI_DOWN_COMBINE: output row (token) of each permuted row
   const int32_t* row_token;   // decode up projection: activations are x itself (rows
                               // 0..NT-1) and permuted row r takes accumulator column
                               // row_token[r]; null otherwise
+  const int32_t* gather_rows; // prefill up projection (pair kernel): activation row r is
+                              // x[gather_rows[r]], gathered by TMA; null otherwise
   int* status;
   uint64_t timeout_ns;
   unsigned int* sched;        // [2]: next tile, CTAs finished; zero on entry, reset on exit
@@ -94,6 +97,18 @@ __device__ __forceinline__ void mbar_drain(uint32_t bar, uint32_t parity, uint64
 
 // epilogue of 32 consecutive output features of one row (prefill orientation)
 __device__ __forceinline__ void epi_row32(const TcArgs& g, int r, int n, const float* v) {
+  if (g.epi == EPI_DOWN_COMBINE || g.epi == EPI_ACC_F32) {
+    // float32 adds into the accumulator row of the token: 16 bytes per add
+    const bool down = g.epi == EPI_DOWN_COMBINE;
+    const float w = down ? g.perm_w[r] : 1.f;
+    const int64_t row = down ? g.dst_row[r] : r;
+    float* dst = static_cast<float*>(g.out) + (size_t)row * g.ldo + n;
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      red_add_f32x4(dst + 4 * i, w * v[4 * i], w * v[4 * i + 1], w * v[4 * i + 2],
+                    w * v[4 * i + 3]);
+    return;
+  }
   if (g.epi == EPI_STORE_F32 || g.epi == EPI_ADD_F32) {
     float4* dst = reinterpret_cast<float4*>(static_cast<float*>(g.out) + (size_t)r * g.ldo + n);
     const bool add = g.epi == EPI_ADD_F32;
@@ -109,10 +124,9 @@ __device__ __forceinline__ void epi_row32(const TcArgs& g, int r, int n, const f
     return;
   }
   const bool up = g.epi == EPI_UP_RELU2;
-  const float w = (up || g.epi == EPI_STORE) ? 1.f : g.perm_w[r];
   float o[32];
 #pragma unroll
-  for (int i = 0; i < 32; ++i) o[i] = up ? relu2(v[i]) : w * v[i];
+  for (int i = 0; i < 32; ++i) o[i] = up ? relu2(v[i]) : v[i];
   uint4* dst = reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(g.out) + (size_t)r * g.ldo + n);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
@@ -129,12 +143,14 @@ __device__ __forceinline__ void epi_row32(const TcArgs& g, int r, int n, const f
 __device__ __forceinline__ void epi_elem(const TcArgs& g, int r, int f, float v) {
   if (g.epi == EPI_UP_RELU2) {
     static_cast<__nv_bfloat16*>(g.out)[(size_t)r * g.ldo + f] = __float2bfloat16_rn(relu2(v));
-  } else if (g.epi == EPI_DOWN_WEIGHTED) {
-    static_cast<__nv_bfloat16*>(g.out)[(size_t)r * g.ldo + f] = __float2bfloat16_rn(g.perm_w[r] * v);
+  } else if (g.epi == EPI_DOWN_COMBINE) {
+    red_add_f32(static_cast<float*>(g.out) + (size_t)g.dst_row[r] * g.ldo + f, g.perm_w[r] * v);
   } else if (g.epi == EPI_STORE) {
     static_cast<__nv_bfloat16*>(g.out)[(size_t)r * g.ldo + f] = __float2bfloat16_rn(v);
   } else if (g.epi == EPI_ADD_F32) {
     static_cast<float*>(g.out)[(size_t)r * g.ldo + f] += v;
+  } else if (g.epi == EPI_ACC_F32) {
+    red_add_f32(static_cast<float*>(g.out) + (size_t)r * g.ldo + f, v);
   } else {
     static_cast<float*>(g.out)[(size_t)r * g.ldo + f] = v;
   }

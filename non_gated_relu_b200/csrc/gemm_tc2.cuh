@@ -12,12 +12,23 @@
 // An expert's last, partial tile (fewer than 256 rows) is computed swapped:
 // 256 weight rows (128 per CTA) on the MMA M side and the remaining token rows
 // (rounded up to 16) on N, so the tensor cores do not multiply padding rows.
-// Both tile kinds use the same tensor maps and the same accumulator layout;
-// only the operand roles, the MMA shape and the epilogue's indexing change.
+// A partial tile of at most 64 rows rides on the expert's last full tile
+// instead (kind 2): each K step also stages those rows (32 per CTA) and
+// issues a second, swapped MMA whose A operand is the weight tile already in
+// shared memory, into the other tensor-memory accumulator.  The expert's
+// weights then cross from L2 once per feature block for both parts; a
+// separate small tile would stream them again for a few rows of work.
+// All tile kinds use the same tensor maps and accumulator layout; only the
+// operand roles, the MMA shapes and the epilogue's indexing change.
+//
+// With g.gather_rows set (the up projection), the activation rows are
+// gathered from x itself by TMA (tile::gather4, four rows per copy, no
+// multicast) instead of being read from a permuted copy of x.
 //
 // Roles per CTA (192 threads), as in the one-CTA kernel:
-//   warp 0 lane 0  TMA producer (both CTAs; the leader also runs the tile
-//                  scheduler and forwards each tile id to the peer);
+//   warp 0         TMA producer (both CTAs; lane 0 waits on the barriers, and
+//                  on the leader runs the tile scheduler and forwards each
+//                  tile id to the peer; all lanes issue row gathers);
 //   warp 1         tensor memory owner; lane 0 of the leader issues the MMAs;
 //   warps 2..5     epilogue of the CTA's 128 accumulator rows.
 // Both CTAs' TMA loads complete on the leader's stage barrier; the leader's
@@ -28,6 +39,7 @@
 #pragma once
 
 #include "gemm_tc.cuh"
+#include "permute.cuh"  // PAIR_ATTACH_ROWS
 
 namespace nh {
 namespace tc2 {
@@ -37,11 +49,14 @@ constexpr int UMMA_K = 16;
 constexpr int MP = 256;       // tile rows (MMA M across the pair)
 constexpr int NT = 256;       // tile features (MMA N)
 constexpr int HALF = 128;     // rows of A and of B staged per CTA
-constexpr int STAGES = 7;
+constexpr int C_ROWS = PAIR_ATTACH_ROWS / 2;   // attached remainder rows staged per CTA
+constexpr int STAGES = 6;
 constexpr int THREADS = 192;
 constexpr int A_BYTES = HALF * BK * 2;
 constexpr int B_BYTES = HALF * BK * 2;
-constexpr int STAGE_BYTES = A_BYTES + B_BYTES;
+constexpr int C_BYTES = C_ROWS * BK * 2;
+constexpr int AB_BYTES = A_BYTES + B_BYTES;
+constexpr int STAGE_BYTES = A_BYTES + B_BYTES + C_BYTES;
 constexpr int TMEM_COLS = 2 * NT;
 constexpr int TQ = 4;
 constexpr int NBAR = 2 * STAGES + 5 + 2 * TQ;
@@ -51,7 +66,8 @@ static_assert(STAGE_BYTES % 1024 == 0, "stage alignment");
 // MMA N of a swapped remainder tile of `rows` token rows
 __device__ __forceinline__ int swap_n(int rows) { return (rows + 15) & ~15; }
 
-// tile entry (expert, first row, rows, kind); kind 1 = swapped remainder tile
+// tile entry (expert, first row, rows, kind); kind 1 = swapped remainder tile,
+// kind 2 = a full tile plus rows - MP attached remainder rows
 __device__ __forceinline__ int4 pair_entry(const tc::TcArgs& g, int m) {
   if (g.tiles) return g.tiles[m];
   const int r0 = m * g.tile_rows;
@@ -61,7 +77,8 @@ __device__ __forceinline__ int4 pair_entry(const tc::TcArgs& g, int m) {
 
 __global__ void __launch_bounds__(THREADS, 1)
     tc2_grouped_gemm(const __grid_constant__ CUtensorMap map_act,
-                     const __grid_constant__ CUtensorMap map_w, const tc::TcArgs g) {
+                     const __grid_constant__ CUtensorMap map_w,
+                     const __grid_constant__ CUtensorMap map_rem, const tc::TcArgs g) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t base = (raw + 1023u) & ~1023u;
@@ -99,6 +116,7 @@ __global__ void __launch_bounds__(THREADS, 1)
     fence_barrier_init();
     tma_prefetch_map(&map_act);
     tma_prefetch_map(&map_w);
+    tma_prefetch_map(&map_rem);
   }
   if (warp == 1) {
     tmem_alloc_pair(smem_u32(tmem_slot), TMEM_COLS);
@@ -119,8 +137,12 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int total = num_m * n_blocks;
   const int nk = g.K / BK;
 
-  if (warp == 0 && lane == 0) {
+  if (warp == 0) {
     // ---------------- producer (+ scheduler on the leader) ----------------
+    // Lane 0 takes the tiles and waits on the barriers.  Activation rows
+    // gathered from x (g.gather_rows) are fetched by the whole warp: lane l
+    // issues the 4-row TMA gather of rows 4l .. 4l+3 of the CTA's operand.
+    const bool gather = g.gather_rows != nullptr;
     int stage = 0;
     uint32_t phase = 0;
     long issued = 0;
@@ -128,54 +150,106 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int i = 0; ok; ++i) {
       const int q = i % TQ;
       const uint32_t ph = (uint32_t)((i / TQ) & 1);
-      int tile;
-      if (leader) {
-        if (!mbar_wait_cluster(tq_empty_bar(q), ph ^ 1u, wc, SITE_TC_PRODUCER)) {
-          ok = false;
-          break;
+      int tile = -1, lok = 1;
+      if (lane == 0) {
+        if (leader) {
+          if (!mbar_wait_cluster(tq_empty_bar(q), ph ^ 1u, wc, SITE_TC_PRODUCER)) {
+            lok = 0;
+          } else {
+            tile = (int)atomicAdd(g.sched, 1u);
+            if (tile >= total) tile = -1;
+            tile_q[q] = tile;
+            st_cluster_u32(map_to_rank(smem_u32((const void*)&tile_q[q]), 1), (uint32_t)tile);
+            mbar_arrive(tq_full_bar(q));
+            mbar_arrive_cluster(map_to_rank(tq_full_bar(q), 1));
+          }
+        } else {
+          if (!mbar_wait_cluster(tq_full_bar(q), ph, wc, SITE_TC_PRODUCER)) {
+            lok = 0;
+          } else {
+            tile = tile_q[q];
+            mbar_arrive_cluster(map_to_rank(tq_empty_bar(q), 0));
+          }
         }
-        tile = (int)atomicAdd(g.sched, 1u);
-        if (tile >= total) tile = -1;
-        tile_q[q] = tile;
-        st_cluster_u32(map_to_rank(smem_u32((const void*)&tile_q[q]), 1), (uint32_t)tile);
-        mbar_arrive(tq_full_bar(q));
-        mbar_arrive_cluster(map_to_rank(tq_full_bar(q), 1));
-      } else {
-        if (!mbar_wait_cluster(tq_full_bar(q), ph, wc, SITE_TC_PRODUCER)) {
-          ok = false;
-          break;
-        }
-        tile = tile_q[q];
-        mbar_arrive_cluster(map_to_rank(tq_empty_bar(q), 0));
       }
-      if (tile < 0) break;
+      ok = __shfl_sync(0xffffffffu, lok, 0) != 0;
+      tile = __shfl_sync(0xffffffffu, tile, 0);
+      if (!ok || tile < 0) break;
       const int m = tile / n_blocks, nb = tile - m * n_blocks;
       const int4 ent = pair_entry(g, m);
       const int n0 = nb * NT;
-      // operand rows staged by this CTA: slot A (M side) and slot B (N side)
+      // operand rows staged by this CTA: slot A (M side), slot B (N side) and,
+      // for kind 2, slot C (the attached remainder rows)
+      const bool swapped = ent.w == 1, attached = ent.w == 2;
       int a_row, b_row;
-      if (ent.w == 0) {                                     // activations x weights
+      if (!swapped) {                                       // activations x weights
         a_row = ent.y + (int)rank * HALF;
         b_row = n0 + (int)rank * (min(NT, g.N - n0) / 2);
       } else {                                              // weights x remainder rows
         a_row = n0 + (int)rank * HALF;
         b_row = ent.y + (int)rank * (swap_n(ent.z) / 2);
       }
+      const int c_row = ent.y + MP + (int)rank * (attached ? swap_n(ent.z - MP) / 2 : 0);
+      // gathered activation rows of this CTA: HALF (full tile) or half of the
+      // remainder's MMA N, and C_ROWS attached rows; padding rows past the
+      // expert repeat its last token
+      const int last = ent.y + ent.z - 1;
+      const int g_rows = !swapped ? HALF : swap_n(ent.z) / 2;
+      const int g_first = !swapped ? a_row : b_row;
+      const bool g_lane = gather && 4 * lane < g_rows;
+      const bool c_lane = gather && attached && 4 * lane < C_ROWS;
+      int tok[4] = {0, 0, 0, 0}, tokc[4] = {0, 0, 0, 0};
+      if (g_lane) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) tok[u] = g.gather_rows[min(g_first + 4 * lane + u, last)];
+      }
+      if (c_lane) {
+#pragma unroll
+        for (int u = 0; u < 4; ++u) tokc[u] = g.gather_rows[min(c_row + 4 * lane + u, last)];
+      }
+      const uint32_t tx_bytes = attached ? 2u * STAGE_BYTES
+                                : (!gather || !swapped)
+                                    ? 2u * AB_BYTES
+                                    : 2u * (uint32_t)(A_BYTES + g_rows * BK * 2);
       for (int kb = 0; kb < nk; ++kb) {
-        if (!mbar_wait_cluster(empty_bar(stage), phase ^ 1u, wc, SITE_TC_PRODUCER)) {
+        lok = 1;
+        if (lane == 0)
+          lok = mbar_wait_cluster(empty_bar(stage), phase ^ 1u, wc, SITE_TC_PRODUCER) ? 1 : 0;
+        if (!__shfl_sync(0xffffffffu, lok, 0)) {
           ok = false;
           break;
         }
-        const uint32_t sa = base + stage * STAGE_BYTES, sb = sa + A_BYTES;
+        const uint32_t sa = base + stage * STAGE_BYTES, sb = sa + A_BYTES, sc = sb + B_BYTES;
         const uint32_t fb = map_to_rank(full_bar(stage), 0);
         const int ka = g.a_kwrap ? (kb * BK) % g.a_kwrap : kb * BK;
-        if (leader) mbar_arrive_expect_tx(full_bar(stage), 2 * STAGE_BYTES);
-        if (ent.w == 0) {
-          tma_load_2d_pair(sa, &map_act, fb, ka, a_row);
-          tma_load_3d_pair(sb, &map_w, fb, kb * BK, b_row, ent.x);
+        if (lane == 0 && leader) mbar_arrive_expect_tx(full_bar(stage), tx_bytes);
+        if (attached) {
+          if (gather) {
+            if (c_lane)
+              tma_gather4_pair(sc + (uint32_t)(4 * lane * BK * 2), &map_act, fb, ka, tokc[0],
+                               tokc[1], tokc[2], tokc[3]);
+          } else if (lane == 0) {
+            tma_load_2d_pair(sc, &map_rem, fb, ka, c_row);
+          }
+        }
+        if (!swapped) {
+          if (gather) {
+            if (g_lane)
+              tma_gather4_pair(sa + (uint32_t)(4 * lane * BK * 2), &map_act, fb, ka, tok[0],
+                               tok[1], tok[2], tok[3]);
+          } else if (lane == 0) {
+            tma_load_2d_pair(sa, &map_act, fb, ka, a_row);
+          }
+          if (lane == 0) tma_load_3d_pair(sb, &map_w, fb, kb * BK, b_row, ent.x);
         } else {
-          tma_load_3d_pair(sa, &map_w, fb, kb * BK, a_row, ent.x);
-          tma_load_2d_pair(sb, &map_act, fb, ka, b_row);
+          if (lane == 0) tma_load_3d_pair(sa, &map_w, fb, kb * BK, a_row, ent.x);
+          if (gather) {
+            if (g_lane)
+              tma_gather4_pair(sb + (uint32_t)(4 * lane * BK * 2), &map_act, fb, ka, tok[0],
+                               tok[1], tok[2], tok[3]);
+          } else if (lane == 0) {
+            tma_load_2d_pair(sb, &map_act, fb, ka, b_row);
+          }
         }
         ++issued;
         if (++stage == STAGES) {
@@ -184,7 +258,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
     }
-    if (!ok && leader) {
+    if (!ok && leader && lane == 0) {
       // the leader's stage barriers count both CTAs' copies: wait for those in flight
       const long first = issued > STAGES ? issued - STAGES : 0;
       for (long i = first; i < issued; ++i)
@@ -208,27 +282,37 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (tile < 0) break;
       const int nb = tile % n_blocks;
       const int4 ent = pair_entry(g, tile / n_blocks);
-      const int acc = it & 1;
-      const uint32_t aph = (uint32_t)((it >> 1) & 1);
-      if (!mbar_wait_cluster(tempty_bar(acc), aph ^ 1u, wc, SITE_TC_MMA)) {
+      const bool attached = ent.w == 2;
+      // a kind-2 tile takes both accumulators: the full tile, then the remainder
+      const int acc = it & 1, acc2 = (it + 1) & 1;
+      if (!mbar_wait_cluster(tempty_bar(acc), (uint32_t)((it >> 1) & 1) ^ 1u, wc, SITE_TC_MMA) ||
+          (attached && !mbar_wait_cluster(tempty_bar(acc2), (uint32_t)(((it + 1) >> 1) & 1) ^ 1u,
+                                          wc, SITE_TC_MMA))) {
         ok = false;
         break;
       }
       tc_fence_after();
-      const int n_mma = ent.w == 0 ? min(NT, g.N - nb * NT) : swap_n(ent.z);
+      const int n_mma = ent.w == 1 ? swap_n(ent.z) : min(NT, g.N - nb * NT);
       const uint32_t idesc = make_idesc_bf16(MP, n_mma);
+      const uint32_t idesc2 = make_idesc_bf16(MP, attached ? swap_n(ent.z - MP) : 16);
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * NT);
+      const uint32_t d2_tmem = tmem_base + (uint32_t)(acc2 * NT);
       for (int kb = 0; kb < nk; ++kb) {
         if (!mbar_wait_cluster(full_bar(stage), phase, wc, SITE_TC_MMA)) {
           ok = false;
           break;
         }
         tc_fence_after();
-        const uint32_t sa = base + stage * STAGE_BYTES, sb = sa + A_BYTES;
+        const uint32_t sa = base + stage * STAGE_BYTES, sb = sa + A_BYTES, sc = sb + B_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < BK / UMMA_K; ++kk)
+        for (int kk = 0; kk < BK / UMMA_K; ++kk) {
           umma_bf16_pair(d_tmem, make_sdesc_sw128(sa + kk * UMMA_K * 2),
                          make_sdesc_sw128(sb + kk * UMMA_K * 2), idesc, (kb | kk) != 0);
+          // attached remainder: the staged weight rows on M, the remainder rows on N
+          if (attached)
+            umma_bf16_pair(d2_tmem, make_sdesc_sw128(sb + kk * UMMA_K * 2),
+                           make_sdesc_sw128(sc + kk * UMMA_K * 2), idesc2, (kb | kk) != 0);
+        }
         any = true;
         umma_commit_pair(empty_bar(stage));
         umma_commit_pair(map_to_rank(empty_bar(stage), 1));
@@ -240,7 +324,11 @@ __global__ void __launch_bounds__(THREADS, 1)
       if (!ok) break;
       umma_commit_pair(tfull_bar(acc));
       umma_commit_pair(map_to_rank(tfull_bar(acc), 1));
-      ++it;
+      if (attached) {
+        umma_commit_pair(tfull_bar(acc2));
+        umma_commit_pair(map_to_rank(tfull_bar(acc2), 1));
+      }
+      it += attached ? 2 : 1;
     }
     if (!ok && any) {
       umma_commit_pair(drain_bar);
@@ -269,47 +357,73 @@ __global__ void __launch_bounds__(THREADS, 1)
       tile = __shfl_sync(0xffffffffu, tile, 0);
       if (!ok || tile < 0) break;
       const int m = tile / n_blocks, nb = tile - m * n_blocks;
-      const int acc = it & 1;
-      const uint32_t aph = (uint32_t)((it >> 1) & 1);
-      if (lane == 0) ok = mbar_wait_cluster(tfull_bar(acc), aph, wc, SITE_TC_EPILOGUE) ? 1 : 0;
-      ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
-      tc_fence_after();
       const int4 ent = pair_entry(g, m);
       const int n0 = nb * NT;
-      const uint32_t tq = tmem_base + ((uint32_t)(qw * 32) << 16) + (uint32_t)(acc * NT);
-      if (ent.w == 0) {
+      const int n_eff = min(NT, g.N - n0);
+      // wait for accumulator use `u` (slot u & 1), or give up with the CTA
+      auto acquire = [&](int u) {
+        int r = 1;
+        if (lane == 0)
+          r = mbar_wait_cluster(tfull_bar(u & 1), (uint32_t)((u >> 1) & 1), wc, SITE_TC_EPILOGUE)
+                  ? 1 : 0;
+        r = __shfl_sync(0xffffffffu, r, 0);
+        if (r) tc_fence_after();
+        return r != 0;
+      };
+      auto release = [&](int u) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) {
+          if (leader)
+            mbar_arrive(tempty_bar(u & 1));
+          else
+            mbar_arrive_cluster(map_to_rank(tempty_bar(u & 1), 0));
+        }
+      };
+      // accumulator lane = output feature, column = token row: the rows
+      // [r0, r0 + rows) of a swapped MMA; this CTA's lanes hold features
+      // f0 + lane index, valid below f_end
+      auto swapped_rows = [&](uint32_t tq, int r0, int rows, int f0, int f_end) {
+        const int f = f0 + qw * 32 + lane;
+        const bool valid = f < f_end;
+        const int n_mma = swap_n(rows);
+        for (int c = 0; c < n_mma; c += 16) {
+          float v[16];
+          tmem_ld_x16(tq + (uint32_t)c, v);
+#pragma unroll
+          for (int j = 0; j < 16; ++j)
+            if (valid && c + j < rows) tc::epi_elem(g, r0 + c + j, f, v[j]);
+        }
+      };
+      if (!acquire(it)) break;
+      const uint32_t tq = tmem_base + ((uint32_t)(qw * 32) << 16) + (uint32_t)((it & 1) * NT);
+      if (ent.w != 1) {
         // accumulator lane = token row, column = output feature
         const int row = (int)rank * HALF + qw * 32 + lane;
-        const bool valid = row < ent.z;
-        const int n_eff = min(NT, g.N - n0);
+        const bool valid = row < min(ent.z, MP);
         for (int c = 0; c < n_eff; c += 32) {
           float v[32];
           tmem_ld_x32(tq + (uint32_t)c, v);
           if (valid) tc::epi_row32(g, ent.y + row, n0 + c, v);
         }
       } else {
-        // accumulator lane = output feature, column = token row of the remainder
-        const int f = n0 + (int)rank * HALF + qw * 32 + lane;
-        const bool valid = f < g.N;
-        const int n_mma = swap_n(ent.z);
-        for (int c = 0; c < n_mma; c += 16) {
-          float v[16];
-          tmem_ld_x16(tq + (uint32_t)c, v);
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (valid && c + j < ent.z) tc::epi_elem(g, ent.y + c + j, f, v[j]);
-        }
+        // weights on M: this CTA's 128 weight rows start at n0 + rank * 128
+        swapped_rows(tq, ent.y, ent.z, n0 + (int)rank * HALF, g.N);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) {
-        if (leader)
-          mbar_arrive(tempty_bar(acc));
-        else
-          mbar_arrive_cluster(map_to_rank(tempty_bar(acc), 0));
+      release(it);
+      if (ent.w == 2) {
+        // attached remainder: the weight rows of the B slot on M (this CTA's
+        // n_eff / 2 rows start at n0 + rank * n_eff / 2), remainder rows on N
+        if (!acquire(it + 1)) break;
+        const uint32_t tq2 =
+            tmem_base + ((uint32_t)(qw * 32) << 16) + (uint32_t)(((it + 1) & 1) * NT);
+        const int f0 = n0 + (int)rank * (n_eff / 2);
+        swapped_rows(tq2, ent.y + MP, ent.z - MP, f0, min(g.N, f0 + n_eff / 2));
+        release(it + 1);
+        it += 2;
+      } else {
+        ++it;
       }
-      ++it;
     }
   }
   tc_fence_before();

@@ -183,6 +183,9 @@ static nh_status make_plan(const nh_moe_config* c, int64_t T, Plan* p) {
   L.tile_rows = tr;
   L.swap_ab = sw;
   L.x_direct = (sw && T <= 64) ? 1 : 0;   // every token fits one activation tile
+  // CTA-pair tiles (bf16, native weights, T > 64): the up projection gathers
+  // its activation rows from x by TMA, so no permuted copy of x is made
+  L.x_gather = (p->bf16 && !sw && c->weight_format == NH_WEIGHTS_NATIVE) ? 1 : 0;
   L.max_tiles = (int)((rows + tr - 1) / tr + p->E);
   L.n_chunks = (int)((T + PERM_CHUNK - 1) / PERM_CHUNK);
   L.rows_alloc = rows;
@@ -203,9 +206,8 @@ static nh_status make_plan(const nh_moe_config* c, int64_t T, Plan* p) {
   L.inv_row = take((size_t)rows * 4);
   L.tiles = take((size_t)L.max_tiles * 16);
   L.num_tiles = take(4);
-  L.x_perm = take(L.x_direct ? 0 : (size_t)rows * p->H * p->elem);
+  L.x_perm = take((L.x_direct || L.x_gather) ? 0 : (size_t)rows * p->H * p->elem);
   L.h = take((size_t)rows * p->I * p->elem);
-  L.y_part = take((size_t)rows * p->H * p->elem);
   L.total_bytes = o;
   return NH_OK;
 }
@@ -254,7 +256,7 @@ static PermuteOut permute_out(void* ws, const nh_moe_ws_layout& L, int* status) 
   o.x_perm = at<void>(ws, L.x_perm);
   o.status = status;
   o.sched_zero = reinterpret_cast<unsigned int*>(status + SCHED_UP);
-  o.gather = L.x_direct ? 0 : 1;
+  o.gather = (L.x_direct || L.x_gather) ? 0 : 1;
   return o;
 }
 
@@ -437,7 +439,9 @@ struct GemmCall {
   void* out;
   int64_t ldo;
   const float* perm_w;
+  const int32_t* dst_row;    // routed down projection: token of each permuted row
   const int32_t* row_token;  // decode up projection reads x directly
+  const int32_t* gather_rows;  // prefill up projection gathers x rows by TMA (pair kernel)
   int* status;
   unsigned int* sched;  // tile scheduler counters (tensor-core path)
 };
@@ -460,7 +464,9 @@ static nh_status launch_tc(const GemmCall& c, int dev, cudaStream_t st) {
   g.out = c.out;
   g.ldo = c.ldo;
   g.perm_w = c.perm_w;
+  g.dst_row = c.dst_row;
   g.row_token = c.row_token;
+  g.gather_rows = nullptr;
   g.status = c.status;
   g.timeout_ns = timeout_ns();
   g.sched = c.sched;
@@ -477,9 +483,15 @@ static nh_status launch_tc(const GemmCall& c, int dev, cudaStream_t st) {
 // prefill orientation on CTA pairs: 256-row tiles, each CTA stages 128 rows of
 // the activations and half of the weight rows
 static nh_status launch_tc2(const GemmCall& c, int dev, cudaStream_t st) {
-  CUtensorMap ma, mw;
-  NH_TRY(map_2d(&ma, c.A, c.a_kwrap ? c.a_kwrap : c.K, c.rows, tc2::HALF));
+  CUtensorMap ma, mw, mr;
+  // gathered activations: a box one row high, four rows per TMA gather
+  NH_TRY(map_2d(&ma, c.A, c.a_kwrap ? c.a_kwrap : c.K, c.rows, c.gather_rows ? 1 : tc2::HALF));
   NH_TRY(map_3d(&mw, c.W, c.K, c.N, c.n_exp, tc2::HALF));
+  // attached remainder rows (kind-2 tiles) when they are not gathered
+  if (c.gather_rows)
+    mr = ma;
+  else
+    NH_TRY(map_2d(&mr, c.A, c.a_kwrap ? c.a_kwrap : c.K, c.rows, tc2::C_ROWS));
   tc::TcArgs g;
   g.tiles = c.tiles;
   g.num_tiles = c.num_tiles;
@@ -492,12 +504,15 @@ static nh_status launch_tc2(const GemmCall& c, int dev, cudaStream_t st) {
   g.out = c.out;
   g.ldo = c.ldo;
   g.perm_w = c.perm_w;
+  g.dst_row = c.dst_row;
   g.row_token = nullptr;
+  g.gather_rows = c.gather_rows;
   g.status = c.status;
   g.timeout_ns = timeout_ns();
   g.sched = c.sched;
   if (!g.sched) return fail(NH_ERR_INVALID_ARG, "internal: no tile scheduler counters");
   if (c.tile_rows != tc2::MP) return fail(NH_ERR_INVALID_ARG, "internal: pair tiles are 256 rows");
+  if (c.gather_rows && c.a_kwrap) return fail(NH_ERR_INVALID_ARG, "internal: gather with K wrap");
   const int n_blocks = (c.N + tc2::NT - 1) / tc2::NT;
   const int64_t m_max = c.tiles ? c.max_tiles : (c.rows + c.tile_rows - 1) / c.tile_rows;
   const int64_t pairs = std::min<int64_t>(m_max * n_blocks, g_pair_clusters[dev]);
@@ -518,7 +533,7 @@ static nh_status launch_tc2(const GemmCall& c, int dev, cudaStream_t st) {
   at[2].val.priority = stream_priority(st);
   lc.attrs = at;
   lc.numAttrs = 3;
-  NH_CUDA(cudaLaunchKernelEx(&lc, tc2::tc2_grouped_gemm, ma, mw, g));
+  NH_CUDA(cudaLaunchKernelEx(&lc, tc2::tc2_grouped_gemm, ma, mw, mr, g));
   return launch_check("tc2_grouped_gemm");
 }
 
@@ -562,7 +577,9 @@ static nh_status launch_q4(const GemmCall& c, const nh_nvfp4_weight& w, int dev,
   g.out = c.out;
   g.ldo = c.ldo;
   g.perm_w = c.perm_w;
+  g.dst_row = c.dst_row;
   g.row_token = c.row_token;
+  g.gather_rows = nullptr;
   g.status = c.status;
   g.timeout_ns = timeout_ns();
   g.sched = c.sched;
@@ -592,7 +609,9 @@ static nh_status launch_q4v(const GemmCall& c, const nh_nvfp4_weight& w, int dev
   g.out = c.out;
   g.ldo = c.ldo;
   g.perm_w = c.perm_w;
+  g.dst_row = c.dst_row;
   g.row_token = c.row_token;
+  g.gather_rows = nullptr;
   g.status = c.status;
   g.timeout_ns = timeout_ns();
   g.sched = c.sched;
@@ -651,7 +670,9 @@ static nh_status launch_dgv(const GemmCall& c, int dev, cudaStream_t st) {
   g.out = c.out;
   g.ldo = c.ldo;
   g.perm_w = c.perm_w;
+  g.dst_row = c.dst_row;
   g.row_token = nullptr;
+  g.gather_rows = nullptr;
   g.status = c.status;
   g.timeout_ns = timeout_ns();
   g.sched = c.sched;
@@ -684,6 +705,7 @@ static nh_status run_gemm(const Plan& p, const GemmCall& c, int dev, cudaStream_
     g.out = c.out;
     g.ldo = c.ldo;
     g.perm_w = c.perm_w;
+    g.dst_row = c.dst_row;
     const int64_t m_max = c.tiles ? c.max_tiles : (c.rows + c.tile_rows - 1) / c.tile_rows;
     if (m_max > 65535) return fail(NH_ERR_UNSUPPORTED, "float32 path: too many row tiles");
     dim3 grid((c.N + SG_BN - 1) / SG_BN, (unsigned)m_max);
@@ -702,95 +724,27 @@ static nh_status run_gemm(const Plan& p, const GemmCall& c, int dev, cudaStream_
 // ----------------------------------------------------------------------------
 // small kernels
 // ----------------------------------------------------------------------------
-// y[t] = y_shared[t] + sum_j y_part[inv_row[t, j]], summed in fp32 in that
-// order (deterministic), rounded once to the output type (float32 output:
-// no rounding, for the tensor-parallel partial sums).
-template <typename Tin, typename Tout>
-__global__ void finalize_gather(const Tin* __restrict__ y_part, const int32_t* __restrict__ inv_row,
-                                const float* __restrict__ y_sh, Tout* __restrict__ y, int64_t T,
-                                int k, int H) {
-  pdl_wait();
-  pdl_trigger();
-  const int64_t n = T * H;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t t = i / H;
-    const int h = (int)(i - t * H);
-    float v = y_sh ? y_sh[i] : 0.f;
-    for (int j = 0; j < k; ++j) {
-      const int r = inv_row[t * k + j];
-      if (r >= 0) v += to_f32(y_part[(size_t)r * H + h]);
-    }
-    y[i] = from_f32<Tout>(v);
-  }
-}
-
-// bf16, eight consecutive features per thread (16-byte loads and stores);
-// output bf16 (uint4 per thread) or, with OUT_F32, float32 (two float4)
-template <bool OUT_F32>
-__global__ void finalize_gather_bf16x8(const uint4* __restrict__ y_part,
-                                       const int32_t* __restrict__ inv_row,
-                                       const float4* __restrict__ y_sh, void* __restrict__ y,
-                                       int64_t T, int k, int H8) {
-  pdl_wait();
-  pdl_trigger();
-  const int64_t n = T * H8;
-  for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
-       i += (int64_t)gridDim.x * blockDim.x) {
-    const int64_t t = i / H8;
-    const int c = (int)(i - t * H8);
-    float a[8];
-    if (y_sh) {
-      const float4 s0 = y_sh[2 * i], s1 = y_sh[2 * i + 1];
-      a[0] = s0.x; a[1] = s0.y; a[2] = s0.z; a[3] = s0.w;
-      a[4] = s1.x; a[5] = s1.y; a[6] = s1.z; a[7] = s1.w;
-    } else {
-#pragma unroll
-      for (int q = 0; q < 8; ++q) a[q] = 0.f;
-    }
-    for (int j = 0; j < k; ++j) {
-      const int r = inv_row[t * k + j];
-      if (r < 0) continue;
-      const uint4 u = y_part[(size_t)r * H8 + c];
-      const uint32_t w[4] = {u.x, u.y, u.z, u.w};
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        a[2 * q] += __uint_as_float(w[q] << 16);
-        a[2 * q + 1] += __uint_as_float(w[q] & 0xffff0000u);
-      }
-    }
-    if (OUT_F32) {
-      float4* yf = static_cast<float4*>(y);
-      yf[2 * i] = make_float4(a[0], a[1], a[2], a[3]);
-      yf[2 * i + 1] = make_float4(a[4], a[5], a[6], a[7]);
-    } else {
-      static_cast<uint4*>(y)[i] =
-          make_uint4(pack_bf16x2(a[0], a[1]), pack_bf16x2(a[2], a[3]), pack_bf16x2(a[4], a[5]),
-                     pack_bf16x2(a[6], a[7]));
-    }
-  }
-}
-
-// y = dtype(y_f32): the one rounding of a tensor-parallel block output
-__global__ void cast_output_bf16x8(const float4* __restrict__ y_f32, uint4* __restrict__ y,
+// y = dtype(y_acc): the one rounding of the block output, after the routed
+// experts' weighted combine and the shared expert were added into y_acc
+__global__ void cast_output_bf16x8(const float4* __restrict__ y_acc, uint4* __restrict__ y,
                                    int64_t n8) {
   pdl_wait();
   pdl_trigger();
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n8;
        i += (int64_t)gridDim.x * blockDim.x) {
-    const float4 a = y_f32[2 * i], b = y_f32[2 * i + 1];
+    const float4 a = y_acc[2 * i], b = y_acc[2 * i + 1];
     y[i] = make_uint4(pack_bf16x2(a.x, a.y), pack_bf16x2(a.z, a.w), pack_bf16x2(b.x, b.y),
                       pack_bf16x2(b.z, b.w));
   }
 }
 
 template <typename Tout>
-__global__ void cast_output(const float* __restrict__ y_f32, Tout* __restrict__ y, int64_t n) {
+__global__ void cast_output(const float* __restrict__ y_acc, Tout* __restrict__ y, int64_t n) {
   pdl_wait();
   pdl_trigger();
   for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
        i += (int64_t)gridDim.x * blockDim.x)
-    y[i] = from_f32<Tout>(y_f32[i]);
+    y[i] = from_f32<Tout>(y_acc[i]);
 }
 
 __global__ void selftest_timeout_kernel(int* status, uint64_t timeout_ns) {
@@ -1089,6 +1043,7 @@ nh_status nh_moe_permute(const nh_moe_config* cfg, int64_t T, const void* x,
         at<int32_t>(ws, L.perm_token), at<float>(ws, L.perm_w), at<int32_t>(ws, L.inv_row),
         at<__nv_bfloat16>(ws, L.x_perm), status, 0)));
     NH_TRY(launch_check("permute_scatter"));
+    if (L.x_gather) return NH_OK;   // the up projection gathers x rows itself
     NH_TRY((launch_k("permute_gather", permute_gather<__nv_bfloat16>, dim3(gather_blocks), dim3(256), 0, st, 
         static_cast<const __nv_bfloat16*>(x), at<int32_t>(ws, L.perm_token),
         at<int32_t>(ws, L.offsets), p.E, p.H, at<__nv_bfloat16>(ws, L.x_perm))));
@@ -1154,8 +1109,8 @@ nh_status nh_moe_route_permute(const nh_moe_config* cfg, int64_t T, const void* 
 }
 
 static nh_status experts_phase(const nh_moe_config* cfg, int64_t T, const void* x, const void* w,
-                               void* ws, size_t ws_bytes, void* stream, bool up_phase,
-                               const nh_nvfp4_weight* wq = nullptr) {
+                               void* ws, size_t ws_bytes, float* y_acc, void* stream,
+                               bool up_phase, const nh_nvfp4_weight* wq = nullptr) {
   NH_TRY(no_latent(cfg, "routed experts"));
   Plan p;
   NH_TRY(make_plan(cfg, T, &p));
@@ -1167,6 +1122,7 @@ static nh_status experts_phase(const nh_moe_config* cfg, int64_t T, const void* 
   if (T == 0) return NH_OK;
   if (!nvfp4) NH_TRY(check_ptr(w, up_phase ? "w_up" : "w_down"));
   if (up_phase) NH_TRY(check_ptr(x, "x"));
+  else NH_TRY(check_ptr(y_acc, "y_acc"));
   int dev;
   NH_TRY(device_setup(&dev));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -1188,6 +1144,11 @@ static nh_status experts_phase(const nh_moe_config* cfg, int64_t T, const void* 
       c.A = x;
       c.rows = T;
       c.row_token = at<int32_t>(ws, L.perm_token);
+    } else if (L.x_gather && !nvfp4) {
+      // prefill: permuted row r is x[perm_token[r]], gathered by the GEMM's TMA
+      c.A = x;
+      c.rows = T;
+      c.gather_rows = at<int32_t>(ws, L.perm_token);
     } else {
       c.A = at<void>(ws, L.x_perm);
     }
@@ -1197,13 +1158,15 @@ static nh_status experts_phase(const nh_moe_config* cfg, int64_t T, const void* 
     c.out = at<void>(ws, L.h);
     c.ldo = p.I;
   } else {
+    // the weighted combine: y_acc[perm_token[r]] += perm_w[r] * (h[r] W_down[e]^T)
     c.A = at<void>(ws, L.h);
     c.N = p.H;
     c.K = p.I;
-    c.epi = EPI_DOWN_WEIGHTED;
-    c.out = at<void>(ws, L.y_part);
+    c.epi = EPI_DOWN_COMBINE;
+    c.out = y_acc;
     c.ldo = p.H;
     c.perm_w = at<float>(ws, L.perm_w);
+    c.dst_row = at<int32_t>(ws, L.perm_token);
   }
   if (nvfp4) return run_gemm_q4(c, wq, dev, st);
   return run_gemm(p, c, dev, st);
@@ -1211,16 +1174,17 @@ static nh_status experts_phase(const nh_moe_config* cfg, int64_t T, const void* 
 
 nh_status nh_moe_experts_up(const nh_moe_config* cfg, int64_t T, const void* x, const void* w_up,
                             void* ws, size_t ws_bytes, void* stream) {
-  return experts_phase(cfg, T, x, w_up, ws, ws_bytes, stream, true);
+  return experts_phase(cfg, T, x, w_up, ws, ws_bytes, nullptr, stream, true);
 }
 
 nh_status nh_moe_experts_down(const nh_moe_config* cfg, int64_t T, const void* w_down, void* ws,
-                              size_t ws_bytes, void* stream) {
-  return experts_phase(cfg, T, nullptr, w_down, ws, ws_bytes, stream, false);
+                              size_t ws_bytes, float* y_acc, void* stream) {
+  return experts_phase(cfg, T, nullptr, w_down, ws, ws_bytes, y_acc, stream, false);
 }
 
 nh_status nh_moe_forward(const nh_moe_config* cfg, int64_t T, const void* x, const void* w_up,
-                         const void* w_down, void* ws, size_t ws_bytes, void* stream) {
+                         const void* w_down, void* ws, size_t ws_bytes, float* y_acc,
+                         void* stream) {
   Plan p;
   NH_TRY(make_plan(cfg, T, &p));
   NH_TRY(check_ws(p, ws, ws_bytes));
@@ -1228,42 +1192,44 @@ nh_status nh_moe_forward(const nh_moe_config* cfg, int64_t T, const void* x, con
   NH_TRY(check_ptr(x, "x"));
   NH_TRY(check_ptr(w_up, "w_up"));
   NH_TRY(check_ptr(w_down, "w_down"));
+  NH_TRY(check_ptr(y_acc, "y_acc"));
   NH_TRY(nh_moe_experts_up(cfg, T, x, w_up, ws, ws_bytes, stream));
-  return nh_moe_experts_down(cfg, T, w_down, ws, ws_bytes, stream);
+  return nh_moe_experts_down(cfg, T, w_down, ws, ws_bytes, y_acc, stream);
 }
 
 nh_status nh_moe_forward_nvfp4(const nh_moe_config* cfg, int64_t T, const void* x,
                                const nh_nvfp4_weight* w_up, const nh_nvfp4_weight* w_down,
-                               void* ws, size_t ws_bytes, void* stream) {
+                               void* ws, size_t ws_bytes, float* y_acc, void* stream) {
   if (!w_up || !w_down) return fail(NH_ERR_INVALID_ARG, "w_up / w_down is NULL");
-  NH_TRY(experts_phase(cfg, T, x, nullptr, ws, ws_bytes, stream, true, w_up));
-  return experts_phase(cfg, T, x, nullptr, ws, ws_bytes, stream, false, w_down);
+  if (T > 0) NH_TRY(check_ptr(y_acc, "y_acc"));
+  NH_TRY(experts_phase(cfg, T, x, nullptr, ws, ws_bytes, nullptr, stream, true, w_up));
+  return experts_phase(cfg, T, x, nullptr, ws, ws_bytes, y_acc, stream, false, w_down);
 }
 
 static nh_status shared_impl(const nh_moe_config* cfg, int64_t T, const void* x, const void* w_su,
                              const void* w_sd, const nh_nvfp4_weight* q_su,
-                             const nh_nvfp4_weight* q_sd, float* y_shared, void* ws_shared,
+                             const nh_nvfp4_weight* q_sd, float* y_acc, void* ws_shared,
                              size_t ws_shared_bytes, void* stream);
 
 nh_status nh_moe_shared_nvfp4(const nh_moe_config* cfg, int64_t T, const void* x,
                               const nh_nvfp4_weight* w_su, const nh_nvfp4_weight* w_sd,
-                              float* y_shared, void* ws_shared, size_t ws_shared_bytes,
+                              float* y_acc, void* ws_shared, size_t ws_shared_bytes,
                               void* stream) {
   if (!w_su || !w_sd) return fail(NH_ERR_INVALID_ARG, "w_shared_up / w_shared_down is NULL");
-  return shared_impl(cfg, T, x, nullptr, nullptr, w_su, w_sd, y_shared, ws_shared,
+  return shared_impl(cfg, T, x, nullptr, nullptr, w_su, w_sd, y_acc, ws_shared,
                      ws_shared_bytes, stream);
 }
 
 nh_status nh_moe_shared(const nh_moe_config* cfg, int64_t T, const void* x, const void* w_su,
-                        const void* w_sd, float* y_shared, void* ws_shared, size_t ws_shared_bytes,
+                        const void* w_sd, float* y_acc, void* ws_shared, size_t ws_shared_bytes,
                         void* stream) {
-  return shared_impl(cfg, T, x, w_su, w_sd, nullptr, nullptr, y_shared, ws_shared,
+  return shared_impl(cfg, T, x, w_su, w_sd, nullptr, nullptr, y_acc, ws_shared,
                      ws_shared_bytes, stream);
 }
 
 static nh_status shared_impl(const nh_moe_config* cfg, int64_t T, const void* x, const void* w_su,
                              const void* w_sd, const nh_nvfp4_weight* q_su,
-                             const nh_nvfp4_weight* q_sd, float* y_shared, void* ws_shared,
+                             const nh_nvfp4_weight* q_sd, float* y_acc, void* ws_shared,
                              size_t ws_shared_bytes, void* stream) {
   Plan p;
   NH_TRY(make_plan(cfg, T, &p));
@@ -1282,7 +1248,7 @@ static nh_status shared_impl(const nh_moe_config* cfg, int64_t T, const void* x,
     NH_TRY(check_ptr(w_su, "w_shared_up"));
     NH_TRY(check_ptr(w_sd, "w_shared_down"));
   }
-  NH_TRY(check_ptr(y_shared, "y_shared"));
+  NH_TRY(check_ptr(y_acc, "y_acc"));
   int dev;
   NH_TRY(device_setup(&dev));
   cudaStream_t st = static_cast<cudaStream_t>(stream);
@@ -1311,80 +1277,31 @@ static nh_status shared_impl(const nh_moe_config* cfg, int64_t T, const void* x,
   dn.W = w_sd;
   dn.N = p.H;
   dn.K = p.S;
-  dn.epi = EPI_STORE_F32;
-  dn.out = y_shared;
+  dn.epi = EPI_ACC_F32;   // y_acc += shared expert, beside the routed combine
+  dn.out = y_acc;
   dn.ldo = p.H;
   dn.sched = reinterpret_cast<unsigned int*>(status + 6);
   if (nvfp4) return run_gemm_q4(dn, q_sd, dev, st);
   return run_gemm(p, dn, dev, st);
 }
 
-// y (dtype, rounded once) or, with out_f32, the float32 sum without rounding
-static nh_status finalize_impl(const nh_moe_config* cfg, int64_t T, const void* ws,
-                               size_t ws_bytes, const float* y_shared, void* y, bool out_f32,
-                               void* stream) {
-  NH_TRY(no_latent(cfg, "finalize"));
-  Plan p;
-  NH_TRY(make_plan(cfg, T, &p));
-  NH_TRY(check_ws(p, const_cast<void*>(ws), ws_bytes));
-  if (T == 0) return NH_OK;
-  NH_TRY(check_ptr(y, out_f32 ? "y_f32" : "y"));
-  if (y_shared) NH_TRY(check_ptr(y_shared, "y_shared"));
-  if (cfg->n_shared_experts && !y_shared)
-    return fail(NH_ERR_INVALID_ARG, "y_shared is NULL but the config has a shared expert");
-  int dev;
-  NH_TRY(device_setup(&dev));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
-  const nh_moe_ws_layout& L = p.lay;
-  void* ws_nc = const_cast<void*>(ws);
-  const int32_t* inv = at<int32_t>(ws_nc, L.inv_row);
-  const dim3 blk(256);
-  if (p.bf16 && p.H % 8 == 0) {
-    const int H8 = p.H / 8;
-    const dim3 grid(grid_for(T * H8, 256, dev));
-    const uint4* yp = at<uint4>(ws_nc, L.y_part);
-    const float4* ys = reinterpret_cast<const float4*>(y_shared);
-    if (out_f32)
-      NH_TRY((launch_k("finalize_gather_bf16x8", finalize_gather_bf16x8<true>, grid, blk, 0, st,
-                       yp, inv, ys, y, T, p.k, H8)));
-    else
-      NH_TRY((launch_k("finalize_gather_bf16x8", finalize_gather_bf16x8<false>, grid, blk, 0, st,
-                       yp, inv, ys, y, T, p.k, H8)));
-  } else if (p.bf16) {
-    const dim3 grid(grid_for(T * p.H, 256, dev));
-    const __nv_bfloat16* yp = at<__nv_bfloat16>(ws_nc, L.y_part);
-    if (out_f32)
-      NH_TRY((launch_k("finalize_gather", finalize_gather<__nv_bfloat16, float>, grid, blk, 0, st,
-                       yp, inv, y_shared, static_cast<float*>(y), T, p.k, p.H)));
-    else
-      NH_TRY((launch_k("finalize_gather", finalize_gather<__nv_bfloat16, __nv_bfloat16>, grid,
-                       blk, 0, st, yp, inv, y_shared, static_cast<__nv_bfloat16*>(y), T, p.k,
-                       p.H)));
-  } else {
-    NH_TRY((launch_k("finalize_gather", finalize_gather<float, float>,
-                     dim3(grid_for(T * p.H, 256, dev)), blk, 0, st, at<float>(ws_nc, L.y_part),
-                     inv, y_shared, static_cast<float*>(y), T, p.k, p.H)));
-  }
-  return launch_check("finalize");
-}
-
-nh_status nh_moe_finalize(const nh_moe_config* cfg, int64_t T, const void* ws, size_t ws_bytes,
-                          const float* y_shared, void* y, void* stream) {
-  return finalize_impl(cfg, T, ws, ws_bytes, y_shared, y, false, stream);
-}
-
-nh_status nh_moe_finalize_partial(const nh_moe_config* cfg, int64_t T, const void* ws,
-                                  size_t ws_bytes, const float* y_shared, float* y_f32,
-                                  void* stream) {
-  return finalize_impl(cfg, T, ws, ws_bytes, y_shared, y_f32, true, stream);
-}
-
-nh_status nh_moe_cast_output(const nh_moe_config* cfg, int64_t T, const float* y_f32, void* y,
-                             void* stream) {
-  NH_TRY(nh_moe_validate(cfg));
+nh_status nh_moe_zero_acc(const nh_moe_config* cfg, int64_t T, float* y_acc, void* stream) {
+  NH_TRY(validate(cfg));
   if (T < 0) return fail(NH_ERR_INVALID_ARG, "T must be >= 0");
   if (T == 0) return NH_OK;
-  NH_TRY(check_ptr(y_f32, "y_f32"));
+  NH_TRY(check_ptr(y_acc, "y_acc"));
+  NH_CUDA(cudaMemsetAsync(y_acc, 0, (size_t)T * cfg->hidden_size * sizeof(float),
+                          static_cast<cudaStream_t>(stream)));
+  return NH_OK;
+}
+
+// y = dtype(y_acc): the one rounding of the block output
+nh_status nh_moe_finalize(const nh_moe_config* cfg, int64_t T, const float* y_acc, void* y,
+                          void* stream) {
+  NH_TRY(validate(cfg));
+  if (T < 0) return fail(NH_ERR_INVALID_ARG, "T must be >= 0");
+  if (T == 0) return NH_OK;
+  NH_TRY(check_ptr(y_acc, "y_acc"));
   NH_TRY(check_ptr(y, "y"));
   int dev;
   NH_TRY(device_setup(&dev));
@@ -1392,14 +1309,14 @@ nh_status nh_moe_cast_output(const nh_moe_config* cfg, int64_t T, const float* y
   const int64_t n = T * (int64_t)cfg->hidden_size;
   if (cfg->dtype == NH_BF16 && n % 8 == 0) {
     NH_TRY((launch_k("cast_output_bf16x8", cast_output_bf16x8, dim3(grid_for(n / 8, 256, dev)),
-                     dim3(256), 0, st, reinterpret_cast<const float4*>(y_f32),
+                     dim3(256), 0, st, reinterpret_cast<const float4*>(y_acc),
                      static_cast<uint4*>(y), n / 8)));
   } else if (cfg->dtype == NH_BF16) {
     NH_TRY((launch_k("cast_output", cast_output<__nv_bfloat16>, dim3(grid_for(n, 256, dev)),
-                     dim3(256), 0, st, y_f32, static_cast<__nv_bfloat16*>(y), n)));
+                     dim3(256), 0, st, y_acc, static_cast<__nv_bfloat16*>(y), n)));
   } else {
     NH_TRY((launch_k("cast_output", cast_output<float>, dim3(grid_for(n, 256, dev)), dim3(256), 0,
-                     st, y_f32, static_cast<float*>(y), n)));
+                     st, y_acc, static_cast<float*>(y), n)));
   }
   return launch_check("cast_output");
 }
@@ -1462,8 +1379,9 @@ static nh_status latent_gemm(const nh_moe_config* cfg, int64_t T, const void* a,
   g.tiles = nullptr;
   g.tile_rows = tr;
   g.swap = sw;
-  // fc2 adds onto the shared expert's output; without a shared expert it writes
-  g.epi = fc1 ? EPI_STORE : (cfg->n_shared_experts ? EPI_ADD_F32 : EPI_STORE_F32);
+  // fc2 adds onto y_acc (the shared expert's output, or zeros): one owner per
+  // element, ordered after the shared expert by the caller
+  g.epi = fc1 ? EPI_STORE : EPI_ADD_F32;
   g.out = out;
   g.ldo = g.N;
   g.status = status;

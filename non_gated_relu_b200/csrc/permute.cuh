@@ -15,11 +15,33 @@ namespace nh {
 
 constexpr int PERM_CHUNK = 256;  // tokens per histogram chunk
 constexpr int PAIR_TILE_ROWS = 256;
+constexpr int PAIR_ATTACH_ROWS = 64;  // largest remainder that rides on a full pair tile
 
-// kind of a tile entry: 1 marks the partial last tile of an expert in the
-// CTA-pair GEMM (256-row tiles), which that GEMM computes swapped
-__device__ __forceinline__ int tile_kind(int rows, int tile_rows) {
-  return (tile_rows == PAIR_TILE_ROWS && rows < tile_rows) ? 1 : 0;
+// Tiles of an expert with `total` rows.  Tiles never cross an expert
+// boundary.  For the CTA-pair GEMM (256-row tiles) an expert's rows past its
+// full tiles form its partial last tile; a partial tile of at most
+// PAIR_ATTACH_ROWS rows is attached to the expert's last full tile instead,
+// so the expert's weights are streamed once per feature block for both.
+__device__ __forceinline__ int expert_tile_count(int total, int tile_rows) {
+  int nt = (total + tile_rows - 1) / tile_rows;
+  if (tile_rows == PAIR_TILE_ROWS) {
+    const int r = total % tile_rows;
+    if (r > 0 && r <= PAIR_ATTACH_ROWS && total > tile_rows) --nt;
+  }
+  return nt;
+}
+
+// Tile i of nt of an expert: (expert, first row, rows, kind).  Kinds of the
+// CTA-pair GEMM: 0 a full tile, 1 a partial tile (computed swapped), 2 a full
+// tile plus an attached partial tile of rows - 256 rows.  Other tile heights
+// use kind 0 only.
+__device__ __forceinline__ int4 expert_tile(int e, int off, int total, int tile_rows, int i,
+                                            int nt) {
+  const int r0 = i * tile_rows;
+  const int rows = (i == nt - 1) ? total - r0 : tile_rows;
+  int kind = 0;
+  if (tile_rows == PAIR_TILE_ROWS) kind = rows < tile_rows ? 1 : (rows > tile_rows ? 2 : 0);
+  return make_int4(e, off + r0, rows, kind);
 }
 
 // per-chunk expert histogram: chunk_counts[c][e]
@@ -79,8 +101,8 @@ __device__ __forceinline__ int block_exclusive_scan(int v, int* smem_warp, int* 
 
 // One block, blockDim.x >= E (rounded to a warp multiple).  Turns the chunk
 // histograms into absolute chunk bases (in place), writes counts, offsets,
-// the tile table (expert, first row, rows, 0) with tiles of `tile_rows` rows
-// that never cross an expert boundary, and the number of tiles.
+// the tile table (expert, first row, rows, kind) of expert_tile, and the
+// number of tiles.
 __global__ void permute_scan(int32_t* __restrict__ chunk_counts, int n_chunks, int E,
                              int tile_rows, int32_t* __restrict__ counts,
                              int32_t* __restrict__ offsets, int4* __restrict__ tiles,
@@ -96,7 +118,7 @@ __global__ void permute_scan(int32_t* __restrict__ chunk_counts, int n_chunks, i
     for (int c = 0; c < n_chunks; ++c) total += chunk_counts[(size_t)c * E + e];
   int all_rows;
   const int off = block_exclusive_scan(e < E ? total : 0, warp_sums, &all_rows);
-  const int nt = (e < E) ? (total + tile_rows - 1) / tile_rows : 0;
+  const int nt = (e < E) ? expert_tile_count(total, tile_rows) : 0;
   int all_tiles;
   const int toff = block_exclusive_scan(nt, warp_sums, &all_tiles);
   if (e < E) {
@@ -108,11 +130,8 @@ __global__ void permute_scan(int32_t* __restrict__ chunk_counts, int n_chunks, i
       chunk_counts[(size_t)c * E + e] = run;
       run += v;
     }
-    for (int i = 0; i < nt && toff + i < max_tiles; ++i) {
-      const int r0 = i * tile_rows;
-      const int rows = min(tile_rows, total - r0);
-      tiles[toff + i] = make_int4(e, off + r0, rows, tile_kind(rows, tile_rows));
-    }
+    for (int i = 0; i < nt && toff + i < max_tiles; ++i)
+      tiles[toff + i] = expert_tile(e, off, total, tile_rows, i, nt);
   }
   if (e == 0) {
     offsets[E] = all_rows;
@@ -264,15 +283,13 @@ __device__ __forceinline__ void permute_block(
   const int total = e < E ? cnt[e] : 0;
   int all_rows, all_tiles;
   const int off = block_exclusive_scan(total, warp_sums, &all_rows);
-  const int nt = (total + tile_rows - 1) / tile_rows;
+  const int nt = expert_tile_count(total, tile_rows);
   const int toff = block_exclusive_scan(nt, warp_sums, &all_tiles);
   if (e < E) {
     counts[e] = total;
     offsets[e] = off;
-    for (int i = 0; i < nt && toff + i < max_tiles; ++i) {
-      const int rows = min(tile_rows, total - i * tile_rows);
-      tiles[toff + i] = make_int4(e, off + i * tile_rows, rows, tile_kind(rows, tile_rows));
-    }
+    for (int i = 0; i < nt && toff + i < max_tiles; ++i)
+      tiles[toff + i] = expert_tile(e, off, total, tile_rows, i, nt);
     cnt[e] = off;  // running position for the ranking
   }
   if (e == 0) {

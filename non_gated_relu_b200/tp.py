@@ -18,9 +18,9 @@ Layout choice of this library: I and S are split in blocks of 64 features
 (the K tile of the expert GEMMs), rank r taking blocks
 [r * nb // world, (r + 1) * nb // world).  Shares differ by at most one
 block when 64 * world does not divide I (Nemotron-H's I = 1856 is 29
-blocks).  Each rank sums its own contributions in float32 without rounding
-(nh_moe_finalize_partial); the all-reduce sums those in float32 and
-nh_moe_cast_output rounds once, as the unsharded block does.
+blocks).  Each rank adds its own contributions into its float32
+accumulator y_acc without rounding; the all-reduce sums those in float32 and
+nh_moe_finalize rounds the sum once, as the unsharded block does.
 """
 from __future__ import annotations
 
@@ -30,7 +30,7 @@ from typing import Optional, Tuple
 import numpy as np
 import torch
 
-from . import NH_WEIGHTS_NVFP4, cast_output, config_from
+from . import NH_WEIGHTS_NVFP4, config_from, finalize
 from .block import NemotronHMoE
 
 BLOCK = 64
@@ -164,14 +164,13 @@ class TPNemotronHMoE:
         return self.block.forward(x, partial=True)
 
     def output(self, y_f32: torch.Tensor) -> torch.Tensor:
-        """y = dtype(y_f32) into this rank's output buffer."""
+        """y = dtype(y_f32) into this rank's output buffer (the one rounding)."""
         T = y_f32.shape[0]
         y = self._y.get(T)
         if y is None:
             y = torch.empty((T, self.block.H), dtype=self.block.dtype, device=self.block.device)
             self._y[T] = y
-        cast_output(self.c_full, T, y_f32, y,
-                    stream=torch.cuda.current_stream(self.block.device))
+        finalize(self.c_full, T, y_f32, y, stream=torch.cuda.current_stream(self.block.device))
         return y
 
     def forward(self, x: torch.Tensor) -> torch.Tensor:

@@ -107,6 +107,52 @@ def check_output(inp, y_gpu, idx_gpu, w_gpu, tokens, excused):
     return err / scale
 
 
+def assert_same_up_to_sum_order(a, b, dtype):
+    """Two runs of the block on the same input: equal up to the order of the
+    float32 atomic adds of the combine.  The float32 sums differ by a few
+    float32 roundings of the largest term; after the output rounding that is
+    at most one ulp of the output type per element (2^-7 relative for bf16),
+    plus an absolute float32-level term for sums that cancel to near zero."""
+    a = np.asarray(a, np.float64)
+    b = np.asarray(b, np.float64)
+    scale = np.abs(b).max()
+    rel = 2.0 ** -7 if dtype == "bf16" else 2.0 ** -20
+    bound = rel * np.maximum(np.abs(a), np.abs(b)) + 1e-5 * scale
+    bad = np.abs(a - b) > bound
+    assert not bad.any(), (f"{int(bad.sum())} elements differ beyond the summation-order bound, "
+                           f"max |diff| {np.abs(a - b).max():.3g}")
+
+
+def tile_tokens(blk, T):
+    """Tokens that put every tile of the GPU's tile table under test.
+
+    Reads the tile table (expert, first row, rows, kind) and perm_token from
+    the block's workspace after a call.  A full 256-row tile (kind 0) is
+    computed by a CTA pair, each CTA owning 128 rows: one token from each
+    half.  An expert's partial last tile (kind 1, computed swapped), and a
+    partial tile attached to a full one (kind 2), give their first and last
+    rows.  Returns (tokens, number of tiles, number of kind-1 and kind-2
+    tiles)."""
+    import non_gated_relu_b200 as nh
+    b = blk.buffers(T)
+    lay = nh.workspace_layout(blk.c_exp, T)
+    ws = b.ws.cpu().numpy()
+    n_tiles = int(ws[lay.num_tiles:lay.num_tiles + 4].view(np.int32)[0])
+    tiles = ws[lay.tiles:lay.tiles + 16 * n_tiles].view(np.int32).reshape(n_tiles, 4)
+    rows = T * blk.k
+    perm_token = ws[lay.perm_token:lay.perm_token + 4 * rows].view(np.int32)
+    picks = []
+    for e, r0, nr, kind in tiles:
+        if kind in (0, 2):
+            picks += [r0 + 64, r0 + 128 + 63]
+            if kind == 2:            # the attached partial tile's first and last rows
+                picks += [r0 + 256, r0 + nr - 1]
+        else:
+            picks += [r0, r0 + nr - 1]
+    return (np.unique(perm_token[np.asarray(picks, np.int64)]).astype(np.int64), n_tiles,
+            int((tiles[:, 3] >= 1).sum()))
+
+
 def sample_tokens(T, n, seed, extra=()):
     rng = np.random.default_rng(seed)
     base = rng.choice(T, size=min(n, T), replace=False)

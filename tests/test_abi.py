@@ -83,8 +83,8 @@ def test_workspace_layout(name):
                ("counts", cfg.E * 4),
                ("offsets", (cfg.E + 1) * 4), ("chunk_counts", L.n_chunks * cfg.E * 4),
                ("perm_token", rows * 4), ("perm_w", rows * 4), ("inv_row", rows * 4),
-               ("tiles", L.max_tiles * 16), ("num_tiles", 4), ("x_perm", 0 if L.x_direct else rows * cfg.H * elem),
-               ("h", rows * cfg.I * elem), ("y_part", rows * cfg.H * elem)]
+               ("tiles", L.max_tiles * 16), ("num_tiles", 4), ("x_perm", 0 if (L.x_direct or L.x_gather) else rows * cfg.H * elem),
+               ("h", rows * cfg.I * elem)]
     spans = sorted((getattr(L, n), getattr(L, n) + sz, n) for n, sz in regions)
     for (a0, a1, an), (b0, b1, bn) in zip(spans, spans[1:]):
         assert a1 <= b0, (an, bn)
@@ -99,6 +99,7 @@ def test_workspace_layout(name):
         assert L.swap_ab == 1 and L.tile_rows >= T and L.tile_rows % 16 == 0
     else:
         assert L.swap_ab == 0 and L.tile_rows == 256     # CTA-pair tiles
+        assert L.x_gather == 1 and L.x_direct == 0       # rows gathered from x by TMA
     assert L.max_tiles >= -(-rows // L.tile_rows) + cfg.E - 1
 
 
@@ -114,8 +115,13 @@ def test_argument_checks_before_any_device_work():
     assert rc == nh.NH_ERR_INVALID_ARG and b"needed" in lib.nh_last_error()
     # misaligned pointer
     need = nh.workspace_size(c, 8)
-    rc = lib.nh_moe_forward(ctypes.byref(c), 8, P(16), P(18), P(16), P(256), need, None)
+    rc = lib.nh_moe_forward(ctypes.byref(c), 8, P(16), P(18), P(16), P(256), need, P(256), None)
     assert rc == nh.NH_ERR_INVALID_ARG and b"aligned" in lib.nh_last_error()
+    # the routed combine needs its float32 accumulator
+    rc = lib.nh_moe_forward(ctypes.byref(c), 8, P(16), P(16), P(16), P(256), need, None, None)
+    assert rc == nh.NH_ERR_INVALID_ARG and b"y_acc" in lib.nh_last_error()
+    rc = lib.nh_moe_experts_down(ctypes.byref(c), 8, P(16), P(256), need, P(260), None)
+    assert rc == nh.NH_ERR_INVALID_ARG and b"y_acc" in lib.nh_last_error()
     # negative T
     rc = lib.nh_moe_workspace_size(ctypes.byref(c), -1, ctypes.byref(ctypes.c_size_t()))
     assert rc == nh.NH_ERR_INVALID_ARG
@@ -123,9 +129,18 @@ def test_argument_checks_before_any_device_work():
     c0 = nh.config_from(synth.CONFIGS["decode_bf16_t8"].replace(n_shared_experts=0))
     rc = lib.nh_moe_shared_workspace_size(ctypes.byref(c0), 8, ctypes.byref(ctypes.c_size_t()))
     assert rc == nh.NH_ERR_INVALID_ARG
-    # finalize requires y_shared when the config has a shared expert
-    rc = lib.nh_moe_finalize(ctypes.byref(c), 8, P(256), need, None, P(16), None)
-    assert rc == nh.NH_ERR_INVALID_ARG and b"y_shared" in lib.nh_last_error()
+    # finalize reads the accumulator and writes y
+    rc = lib.nh_moe_finalize(ctypes.byref(c), 8, None, P(16), None)
+    assert rc == nh.NH_ERR_INVALID_ARG and b"y_acc" in lib.nh_last_error()
+    rc = lib.nh_moe_finalize(ctypes.byref(c), 8, P(256), P(264), None)
+    assert rc == nh.NH_ERR_INVALID_ARG and b"aligned" in lib.nh_last_error()
+    rc = lib.nh_moe_finalize(ctypes.byref(c), -1, P(256), P(256), None)
+    assert rc == nh.NH_ERR_INVALID_ARG
+    rc = lib.nh_moe_zero_acc(ctypes.byref(c), 8, P(250), None)
+    assert rc == nh.NH_ERR_INVALID_ARG and b"aligned" in lib.nh_last_error()
+    # zero tokens: nothing to do, no device needed
+    assert lib.nh_moe_finalize(ctypes.byref(c), 0, None, None, None) == nh.NH_OK
+    assert lib.nh_moe_zero_acc(ctypes.byref(c), 0, None, None) == nh.NH_OK
     # selftest timeout bound
     rc = lib.nh_moe_selftest_timeout(P(256), 0, None)
     assert rc == nh.NH_ERR_INVALID_ARG
@@ -167,8 +182,8 @@ def test_next_row_argument_checks_before_any_device_work():
     need = nh.workspace_size(synth.CONFIGS["decode_bf16_t8"], 8)
     # routed-expert calls refuse the full latent config
     for rc in (lib.nh_moe_permute(ctypes.byref(lat), 8, P(256), P(256), P(256), P(256), need, None),
-               lib.nh_moe_forward(ctypes.byref(lat), 8, P(256), P(256), P(256), P(256), need, None),
-               lib.nh_moe_finalize(ctypes.byref(lat), 8, P(256), need, P(256), P(256), None)):
+               lib.nh_moe_forward(ctypes.byref(lat), 8, P(256), P(256), P(256), P(256), need,
+                                  P(256), None)):
         assert rc == nh.NH_ERR_INVALID_ARG and b"latent_size" in lib.nh_last_error()
     # latent projections: workspace and pointer checks
     rc = lib.nh_moe_latent_in(ctypes.byref(lat), 8, P(256), P(256), P(256), None, 256, None)
@@ -179,22 +194,17 @@ def test_next_row_argument_checks_before_any_device_work():
     assert rc == nh.NH_ERR_INVALID_ARG and b"aligned" in lib.nh_last_error()
     # NVFP4 entry points: NULL weight descriptors, and the format must match the call
     q4 = nh.config_from(synth.CONFIGS["decode_nvfp4_t8"])
-    rc = lib.nh_moe_forward_nvfp4(ctypes.byref(q4), 8, P(256), None, None, P(256), need, None)
+    rc = lib.nh_moe_forward_nvfp4(ctypes.byref(q4), 8, P(256), None, None, P(256), need, P(256),
+                                  None)
     assert rc == nh.NH_ERR_INVALID_ARG and b"NULL" in lib.nh_last_error()
     rc = lib.nh_moe_forward(ctypes.byref(q4), 8, P(256), P(256), P(256), P(256),
-                            nh.workspace_size(synth.CONFIGS["decode_nvfp4_t8"], 8), None)
+                            nh.workspace_size(synth.CONFIGS["decode_nvfp4_t8"], 8), P(256), None)
     assert rc == nh.NH_ERR_INVALID_ARG and b"NVFP4" in lib.nh_last_error()
     w = nh.NvFp4Weight(256, 256, 256)
     bf = nh.config_from(synth.CONFIGS["decode_bf16_t8"])
     rc = lib.nh_moe_forward_nvfp4(ctypes.byref(bf), 8, P(256), ctypes.byref(w), ctypes.byref(w),
-                                  P(256), need, None)
+                                  P(256), need, P(256), None)
     assert rc == nh.NH_ERR_INVALID_ARG and b"native" in lib.nh_last_error()
-    # tensor-parallel partial finalize and the one rounding
-    rc = lib.nh_moe_finalize_partial(ctypes.byref(bf), 8, P(256), need, P(256), P(250), None)
-    assert rc == nh.NH_ERR_INVALID_ARG and b"y_f32" in lib.nh_last_error()
-    rc = lib.nh_moe_cast_output(ctypes.byref(bf), -1, P(256), P(256), None)
-    assert rc == nh.NH_ERR_INVALID_ARG
-    rc = lib.nh_moe_cast_output(ctypes.byref(bf), 8, P(256), P(264), None)
-    assert rc == nh.NH_ERR_INVALID_ARG and b"aligned" in lib.nh_last_error()
-    # zero tokens: nothing to do, no device needed
-    assert lib.nh_moe_cast_output(ctypes.byref(bf), 0, None, None, None) == nh.NH_OK
+    rc = lib.nh_moe_forward_nvfp4(ctypes.byref(q4), 8, P(256), ctypes.byref(w), ctypes.byref(w),
+                                  P(256), need, None, None)
+    assert rc == nh.NH_ERR_INVALID_ARG and b"y_acc" in lib.nh_last_error()

@@ -61,6 +61,6 @@ def test_argument_errors_enqueue_nothing():
         nh.route(blk.c, x, blk.w_router, None, b.topk_idx, b.topk_w, b.ws[:100])
     assert e.value.status == nh.NH_ERR_INVALID_ARG
     with pytest.raises(nh.NHMoEError) as e:
-        nh.forward(blk.c, x, blk.w_up, None, b.ws)
+        nh.forward(blk.c, x, blk.w_up, None, b.ws, b.y_acc)
     assert e.value.status == nh.NH_ERR_INVALID_ARG
     torch.cuda.synchronize()

@@ -4,8 +4,8 @@ The routed experts run in width L between fc1_latent_proj and
 fc2_latent_proj (nh_moe_latent_in / nh_moe_latent_out around the unchanged
 routed path in its expert-width config); routing and the shared expert see
 the full-width x.  The GPU rounds x_lat and the combined y_lat to the
-activation dtype (the oracle rounds nothing), so the bf16 tolerance covers
-two more roundings than the plain block's.
+activation dtype (they are Linear inputs; the oracle rounds nothing), which
+the bf16 tolerance covers.
 """
 import numpy as np
 import pytest

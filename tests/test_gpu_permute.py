@@ -2,10 +2,12 @@
 
 Checks, for the single-block path (T <= 256), the multi-kernel path and the
 fused decode router+permute: counts, offsets, perm_token, perm_w, inv_row
-equal oracle.permute of the GPU's own routing; x_perm rows equal x rows; the
+equal oracle.permute of the GPU's own routing; x_perm rows (where the plan
+makes them) equal x rows; the
 tile table covers every expert's rows exactly once in order, with tiles no
 taller than the plan's tile height and the partial-tile kind flag set as
-documented.
+documented (kind 1: an expert's partial last tile; kind 2: a full tile with
+an attached partial tile of at most 64 rows).
 """
 import numpy as np
 import pytest
@@ -37,16 +39,26 @@ def check_permute(cfg, x_np, idx, w, ws, lay, x_dev):
     np.testing.assert_array_equal(region(ws, lay.inv_row, rows, np.int32).reshape(T, k),
                                   ref["inv_row"])
     elem = np.uint16 if cfg.dtype == "bf16" else np.float32
-    if not lay.x_direct:   # the decode orientation reads x directly (no x_perm)
+    if not (lay.x_direct or lay.x_gather):   # else the up projection reads x itself
         xp = region(ws, lay.x_perm, rows * cfg.H, elem).reshape(rows, cfg.H)
         np.testing.assert_array_equal(xp, x_np[ref["perm_token"]])
     nt = int(region(ws, lay.num_tiles, 1, np.int32)[0])
     tiles = region(ws, lay.tiles, nt * 4, np.int32).reshape(nt, 4)
     covered = np.zeros(rows, np.int32)
+    pair = lay.tile_rows == 256
     for e_, r0, n, kind in tiles:
-        assert 1 <= n <= lay.tile_rows
+        # CTA-pair tiles: a partial tile of at most 64 rows rides on the
+        # expert's last full tile (kind 2); a larger one is its own (kind 1)
+        assert 1 <= n <= lay.tile_rows + (64 if pair else 0)
         assert ref["offsets"][e_] <= r0 and r0 + n <= ref["offsets"][e_ + 1]
-        assert kind == (1 if (lay.tile_rows == 256 and n < 256) else 0)
+        want = 0
+        if pair:
+            want = 1 if n < 256 else (2 if n > 256 else 0)
+        assert kind == want
+        if kind == 1:           # a small partial tile stands alone only without a full one
+            assert n > 64 or ref["counts"][e_] < 256
+        if kind == 2:   # the expert's last tile
+            assert r0 + n == ref["offsets"][e_ + 1]
         covered[r0:r0 + n] += 1
     assert np.all(covered == 1)
     assert np.all(np.diff(tiles[:, 1]) > 0)
@@ -59,6 +71,11 @@ CASES = {
     "t1500_multi_chunk": dict(T=1500, seed=33, n_routed_experts=64),
     "t700_top8_e256": dict(T=700, seed=34, n_routed_experts=256, n_group=8, topk_group=2,
                            num_experts_per_tok=8),
+    # few experts: several pair tiles per expert, partial tiles attached or not
+    "t1100_e8": dict(T=1100, seed=35, n_routed_experts=8, n_group=2, topk_group=1,
+                     num_experts_per_tok=2),
+    "t1300_e8": dict(T=1300, seed=36, n_routed_experts=8, n_group=2, topk_group=1,
+                     num_experts_per_tok=2),
 }
 
 

@@ -1,10 +1,10 @@
 """Tensor-parallel shards on one GPU, through the C ABI, against the oracle.
 
 Each rank of a world of 2 or 3 runs the whole path on its 64-feature blocks
-of I and S (nh_moe_finalize_partial gives its float32 contribution).  The
+of I and S (its float32 accumulator y_acc is its contribution).  The
 ranks do not wait on one another, so they run one after the other on the
 same GPU; the test adds their float32 partials (what the all-reduce does)
-and nh_moe_cast_output rounds the sum once.  The result must match the
+and nh_moe_finalize rounds the sum once.  The result must match the
 oracle like the unsharded block, and the unsharded GPU block closely.
 """
 import numpy as np
