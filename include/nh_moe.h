@@ -135,8 +135,7 @@ typedef struct {
                              CTA-pair GEMM, computed with weights on M)        */
     size_t num_tiles;     /* int32 [1] number of valid tile entries             */
     size_t x_perm;        /* dtype [rows_alloc, H] x gathered in permuted order
-                             (empty when x_direct or x_gather: the GEMM reads
-                             x itself)                                        */
+                             (empty when x_direct: the GEMM reads x itself)   */
     size_t h;             /* dtype [rows_alloc, I] relu^2(up) in permuted order */
     int64_t rows_alloc;   /* T * k rounded up to the tile height                */
     int32_t tile_rows;    /* rows per tile entry of this (cfg, T)               */
@@ -144,8 +143,6 @@ typedef struct {
     int32_t n_chunks;     /* token chunks of the permute histogram              */
     int32_t swap_ab;      /* 1: weights on the MMA M side (small T, or NVFP4)   */
     int32_t x_direct;     /* 1: the up projection reads x itself (no x_perm)    */
-    int32_t x_gather;     /* 1: the up projection gathers the rows x[perm_token]
-                             by TMA (CTA-pair tiles; no x_perm)               */
 } nh_moe_ws_layout;
 
 /* Validate a configuration (no device work). */
@@ -221,7 +218,7 @@ nh_status nh_moe_route_noalloc(const nh_moe_config *cfg, int64_t T, const void *
 /*
  * Token permute: per-expert histogram, exclusive scan, stable scatter of the
  * (t, j) assignments in (t, j) order, the tile table of the expert GEMMs and
- * (unless the layout's x_direct or x_gather is set) the gather
+ * (unless the layout's x_direct is set) the gather
  * x_perm[row] = x[perm_token[row]].  The routed experts are
  * applied per expert id (MLX SwitchMLP fc1/fc2 indexed by the router's
  * expert ids, exo commit "Add support for Nemotron sharding").

@@ -66,7 +66,7 @@ class Layout(ctypes.Structure):
         "perm_w", "inv_row", "tiles", "num_tiles", "x_perm", "h")] + [
         ("rows_alloc", ctypes.c_int64), ("tile_rows", ctypes.c_int32),
         ("max_tiles", ctypes.c_int32), ("n_chunks", ctypes.c_int32), ("swap_ab", ctypes.c_int32),
-        ("x_direct", ctypes.c_int32), ("x_gather", ctypes.c_int32)]
+        ("x_direct", ctypes.c_int32)]
 
 
 def config_from(c, group_score: int = 0) -> Config:

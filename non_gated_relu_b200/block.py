@@ -9,6 +9,14 @@ call runs, on the caller's stream and a side stream:
     main: route + permute -> forward: y_acc += routed experts (x) ---+-> finalize: y = dtype(y_acc)
                       (forward's down projection waits for y_acc = 0)
 
+That is the schedule while the routed experts stream their weights, with fewer
+than 256 rows (one CTA-pair tile) per expert on average: the shared expert
+then fills what the routed path leaves idle.  With more rows per expert every
+GEMM is bound by the tensor cores, and running the shared expert's GEMMs beside
+the routed ones only makes them contend (their float32 adds into the same y_acc
+included); there every step runs on the caller's stream in turn: y_acc = 0,
+shared expert, route + permute, forward, finalize.
+
 With latent projections (config ``latent_size`` L > 0; the modules
 fc1_latent_proj / fc2_latent_proj of the ModelOpt descriptor
 NemotronHMoELayerDescriptor) the routed experts run in width L:
@@ -79,6 +87,10 @@ class NemotronHMoE:
     own device current (``torch.cuda.set_device`` or a ``torch.cuda.device``
     context), as one process per GPU does.
     """
+
+    #: the shared expert runs on a side stream, beside the routed path, while
+    #: T * k < concurrent_rows_per_expert * E (mean rows per routed expert)
+    concurrent_rows_per_expert = 256
 
     def __init__(self, cfg, w_router, w_up=None, w_down=None, w_shared_up=None,
                  w_shared_down=None, bias=None, device=None, nvfp4=None, w_latent_fc1=None,
@@ -180,27 +192,30 @@ class NemotronHMoE:
         fork = torch.cuda.Event()
         fork.record(caller)
         main.wait_event(fork)
-        self.side.wait_event(fork)
-        # side stream: the accumulators start at zero, then the shared expert
-        # adds into y_acc (beside the routed path)
+        # weight-streaming calls run the shared expert beside the routed path
+        E = self.c.n_routed_experts
+        side = self.side if T * self.k < self.concurrent_rows_per_expert * E else main
+        if side is not main:
+            side.wait_event(fork)
+        # the accumulators start at zero, then the shared expert adds into y_acc
         push("zero_acc")
-        zero_acc(self.c, T, b.y_acc, stream=self.side)
+        zero_acc(self.c, T, b.y_acc, stream=side)
         if self.latent:
-            zero_acc(self.c_exp, T, b.y_lat_acc, stream=self.side)
+            zero_acc(self.c_exp, T, b.y_lat_acc, stream=side)
         pop()
         zero = torch.cuda.Event()
-        zero.record(self.side)
+        zero.record(side)
         if self.has_shared:
             push("shared")
             if self.nvfp4:
                 shared_nvfp4(self.c, x, self.q4["shared_up"], self.q4["shared_down"], b.y_acc,
-                             b.ws_shared, stream=self.side)
+                             b.ws_shared, stream=side)
             else:
                 shared(self.c, x, self.w_shared_up, self.w_shared_down, b.y_acc, b.ws_shared,
-                       stream=self.side)
+                       stream=side)
             pop()
         join = torch.cuda.Event()
-        join.record(self.side)
+        join.record(side)
         if self.latent:
             out = self._forward_latent(x, b, main, zero, join, partial, push, pop)
             self._join(caller, main)

@@ -54,8 +54,6 @@ struct TcArgs {
   const int32_t* row_token;   // decode up projection: activations are x itself (rows
                               // 0..NT-1) and permuted row r takes accumulator column
                               // row_token[r]; null otherwise
-  const int32_t* gather_rows; // prefill up projection (pair kernel): activation row r is
-                              // x[gather_rows[r]], gathered by TMA; null otherwise
   int* status;
   uint64_t timeout_ns;
   unsigned int* sched;        // [2]: next tile, CTAs finished; zero on entry, reset on exit

@@ -21,14 +21,9 @@
 // All tile kinds use the same tensor maps and accumulator layout; only the
 // operand roles, the MMA shapes and the epilogue's indexing change.
 //
-// With g.gather_rows set (the up projection), the activation rows are
-// gathered from x itself by TMA (tile::gather4, four rows per copy, no
-// multicast) instead of being read from a permuted copy of x.
-//
 // Roles per CTA (192 threads), as in the one-CTA kernel:
-//   warp 0         TMA producer (both CTAs; lane 0 waits on the barriers, and
-//                  on the leader runs the tile scheduler and forwards each
-//                  tile id to the peer; all lanes issue row gathers);
+//   warp 0 lane 0  TMA producer (both CTAs; the leader also runs the tile
+//                  scheduler and forwards each tile id to the peer);
 //   warp 1         tensor memory owner; lane 0 of the leader issues the MMAs;
 //   warps 2..5     epilogue of the CTA's 128 accumulator rows.
 // Both CTAs' TMA loads complete on the leader's stage barrier; the leader's
@@ -137,12 +132,8 @@ __global__ void __launch_bounds__(THREADS, 1)
   const int total = num_m * n_blocks;
   const int nk = g.K / BK;
 
-  if (warp == 0) {
+  if (warp == 0 && lane == 0) {
     // ---------------- producer (+ scheduler on the leader) ----------------
-    // Lane 0 takes the tiles and waits on the barriers.  Activation rows
-    // gathered from x (g.gather_rows) are fetched by the whole warp: lane l
-    // issues the 4-row TMA gather of rows 4l .. 4l+3 of the CTA's operand.
-    const bool gather = g.gather_rows != nullptr;
     int stage = 0;
     uint32_t phase = 0;
     long issued = 0;
@@ -150,31 +141,27 @@ __global__ void __launch_bounds__(THREADS, 1)
     for (int i = 0; ok; ++i) {
       const int q = i % TQ;
       const uint32_t ph = (uint32_t)((i / TQ) & 1);
-      int tile = -1, lok = 1;
-      if (lane == 0) {
-        if (leader) {
-          if (!mbar_wait_cluster(tq_empty_bar(q), ph ^ 1u, wc, SITE_TC_PRODUCER)) {
-            lok = 0;
-          } else {
-            tile = (int)atomicAdd(g.sched, 1u);
-            if (tile >= total) tile = -1;
-            tile_q[q] = tile;
-            st_cluster_u32(map_to_rank(smem_u32((const void*)&tile_q[q]), 1), (uint32_t)tile);
-            mbar_arrive(tq_full_bar(q));
-            mbar_arrive_cluster(map_to_rank(tq_full_bar(q), 1));
-          }
-        } else {
-          if (!mbar_wait_cluster(tq_full_bar(q), ph, wc, SITE_TC_PRODUCER)) {
-            lok = 0;
-          } else {
-            tile = tile_q[q];
-            mbar_arrive_cluster(map_to_rank(tq_empty_bar(q), 0));
-          }
+      int tile;
+      if (leader) {
+        if (!mbar_wait_cluster(tq_empty_bar(q), ph ^ 1u, wc, SITE_TC_PRODUCER)) {
+          ok = false;
+          break;
         }
+        tile = (int)atomicAdd(g.sched, 1u);
+        if (tile >= total) tile = -1;
+        tile_q[q] = tile;
+        st_cluster_u32(map_to_rank(smem_u32((const void*)&tile_q[q]), 1), (uint32_t)tile);
+        mbar_arrive(tq_full_bar(q));
+        mbar_arrive_cluster(map_to_rank(tq_full_bar(q), 1));
+      } else {
+        if (!mbar_wait_cluster(tq_full_bar(q), ph, wc, SITE_TC_PRODUCER)) {
+          ok = false;
+          break;
+        }
+        tile = tile_q[q];
+        mbar_arrive_cluster(map_to_rank(tq_empty_bar(q), 0));
       }
-      ok = __shfl_sync(0xffffffffu, lok, 0) != 0;
-      tile = __shfl_sync(0xffffffffu, tile, 0);
-      if (!ok || tile < 0) break;
+      if (tile < 0) break;
       const int m = tile / n_blocks, nb = tile - m * n_blocks;
       const int4 ent = pair_entry(g, m);
       const int n0 = nb * NT;
@@ -190,66 +177,23 @@ __global__ void __launch_bounds__(THREADS, 1)
         b_row = ent.y + (int)rank * (swap_n(ent.z) / 2);
       }
       const int c_row = ent.y + MP + (int)rank * (attached ? swap_n(ent.z - MP) / 2 : 0);
-      // gathered activation rows of this CTA: HALF (full tile) or half of the
-      // remainder's MMA N, and C_ROWS attached rows; padding rows past the
-      // expert repeat its last token
-      const int last = ent.y + ent.z - 1;
-      const int g_rows = !swapped ? HALF : swap_n(ent.z) / 2;
-      const int g_first = !swapped ? a_row : b_row;
-      const bool g_lane = gather && 4 * lane < g_rows;
-      const bool c_lane = gather && attached && 4 * lane < C_ROWS;
-      int tok[4] = {0, 0, 0, 0}, tokc[4] = {0, 0, 0, 0};
-      if (g_lane) {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) tok[u] = g.gather_rows[min(g_first + 4 * lane + u, last)];
-      }
-      if (c_lane) {
-#pragma unroll
-        for (int u = 0; u < 4; ++u) tokc[u] = g.gather_rows[min(c_row + 4 * lane + u, last)];
-      }
-      const uint32_t tx_bytes = attached ? 2u * STAGE_BYTES
-                                : (!gather || !swapped)
-                                    ? 2u * AB_BYTES
-                                    : 2u * (uint32_t)(A_BYTES + g_rows * BK * 2);
+      const uint32_t tx_bytes = 2u * (attached ? STAGE_BYTES : AB_BYTES);
       for (int kb = 0; kb < nk; ++kb) {
-        lok = 1;
-        if (lane == 0)
-          lok = mbar_wait_cluster(empty_bar(stage), phase ^ 1u, wc, SITE_TC_PRODUCER) ? 1 : 0;
-        if (!__shfl_sync(0xffffffffu, lok, 0)) {
+        if (!mbar_wait_cluster(empty_bar(stage), phase ^ 1u, wc, SITE_TC_PRODUCER)) {
           ok = false;
           break;
         }
         const uint32_t sa = base + stage * STAGE_BYTES, sb = sa + A_BYTES, sc = sb + B_BYTES;
         const uint32_t fb = map_to_rank(full_bar(stage), 0);
         const int ka = g.a_kwrap ? (kb * BK) % g.a_kwrap : kb * BK;
-        if (lane == 0 && leader) mbar_arrive_expect_tx(full_bar(stage), tx_bytes);
-        if (attached) {
-          if (gather) {
-            if (c_lane)
-              tma_gather4_pair(sc + (uint32_t)(4 * lane * BK * 2), &map_act, fb, ka, tokc[0],
-                               tokc[1], tokc[2], tokc[3]);
-          } else if (lane == 0) {
-            tma_load_2d_pair(sc, &map_rem, fb, ka, c_row);
-          }
-        }
+        if (leader) mbar_arrive_expect_tx(full_bar(stage), tx_bytes);
         if (!swapped) {
-          if (gather) {
-            if (g_lane)
-              tma_gather4_pair(sa + (uint32_t)(4 * lane * BK * 2), &map_act, fb, ka, tok[0],
-                               tok[1], tok[2], tok[3]);
-          } else if (lane == 0) {
-            tma_load_2d_pair(sa, &map_act, fb, ka, a_row);
-          }
-          if (lane == 0) tma_load_3d_pair(sb, &map_w, fb, kb * BK, b_row, ent.x);
+          tma_load_2d_pair(sa, &map_act, fb, ka, a_row);
+          tma_load_3d_pair(sb, &map_w, fb, kb * BK, b_row, ent.x);
+          if (attached) tma_load_2d_pair(sc, &map_rem, fb, ka, c_row);
         } else {
-          if (lane == 0) tma_load_3d_pair(sa, &map_w, fb, kb * BK, a_row, ent.x);
-          if (gather) {
-            if (g_lane)
-              tma_gather4_pair(sb + (uint32_t)(4 * lane * BK * 2), &map_act, fb, ka, tok[0],
-                               tok[1], tok[2], tok[3]);
-          } else if (lane == 0) {
-            tma_load_2d_pair(sb, &map_act, fb, ka, b_row);
-          }
+          tma_load_3d_pair(sa, &map_w, fb, kb * BK, a_row, ent.x);
+          tma_load_2d_pair(sb, &map_act, fb, ka, b_row);
         }
         ++issued;
         if (++stage == STAGES) {
@@ -258,7 +202,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       }
     }
-    if (!ok && leader && lane == 0) {
+    if (!ok && leader) {
       // the leader's stage barriers count both CTAs' copies: wait for those in flight
       const long first = issued > STAGES ? issued - STAGES : 0;
       for (long i = first; i < issued; ++i)
@@ -297,28 +241,53 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t idesc2 = make_idesc_bf16(MP, attached ? swap_n(ent.z - MP) : 16);
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * NT);
       const uint32_t d2_tmem = tmem_base + (uint32_t)(acc2 * NT);
-      for (int kb = 0; kb < nk; ++kb) {
-        if (!mbar_wait_cluster(full_bar(stage), phase, wc, SITE_TC_MMA)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t sa = base + stage * STAGE_BYTES, sb = sa + A_BYTES, sc = sb + B_BYTES;
+      // Two copies of the K loop: the MMA stream of an ordinary tile keeps no
+      // branch between its MMAs (a conditional second MMA in the same loop cost
+      // about 15 % of throughput on every tile, measured)
+      if (!attached) {
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait_cluster(full_bar(stage), phase, wc, SITE_TC_MMA)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = base + stage * STAGE_BYTES, sb = sa + A_BYTES;
 #pragma unroll
-        for (int kk = 0; kk < BK / UMMA_K; ++kk) {
-          umma_bf16_pair(d_tmem, make_sdesc_sw128(sa + kk * UMMA_K * 2),
-                         make_sdesc_sw128(sb + kk * UMMA_K * 2), idesc, (kb | kk) != 0);
-          // attached remainder: the staged weight rows on M, the remainder rows on N
-          if (attached)
+          for (int kk = 0; kk < BK / UMMA_K; ++kk)
+            umma_bf16_pair(d_tmem, make_sdesc_sw128(sa + kk * UMMA_K * 2),
+                           make_sdesc_sw128(sb + kk * UMMA_K * 2), idesc, (kb | kk) != 0);
+          any = true;
+          umma_commit_pair(empty_bar(stage));
+          umma_commit_pair(map_to_rank(empty_bar(stage), 1));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      } else {
+        for (int kb = 0; kb < nk; ++kb) {
+          if (!mbar_wait_cluster(full_bar(stage), phase, wc, SITE_TC_MMA)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = base + stage * STAGE_BYTES, sb = sa + A_BYTES, sc = sb + B_BYTES;
+#pragma unroll
+          for (int kk = 0; kk < BK / UMMA_K; ++kk)
+            umma_bf16_pair(d_tmem, make_sdesc_sw128(sa + kk * UMMA_K * 2),
+                           make_sdesc_sw128(sb + kk * UMMA_K * 2), idesc, (kb | kk) != 0);
+          // attached partial tile: the staged weight rows on M, its rows on N
+#pragma unroll
+          for (int kk = 0; kk < BK / UMMA_K; ++kk)
             umma_bf16_pair(d2_tmem, make_sdesc_sw128(sb + kk * UMMA_K * 2),
                            make_sdesc_sw128(sc + kk * UMMA_K * 2), idesc2, (kb | kk) != 0);
-        }
-        any = true;
-        umma_commit_pair(empty_bar(stage));
-        umma_commit_pair(map_to_rank(empty_bar(stage), 1));
-        if (++stage == STAGES) {
-          stage = 0;
-          phase ^= 1u;
+          any = true;
+          umma_commit_pair(empty_bar(stage));
+          umma_commit_pair(map_to_rank(empty_bar(stage), 1));
+          if (++stage == STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
         }
       }
       if (!ok) break;
@@ -395,35 +364,39 @@ __global__ void __launch_bounds__(THREADS, 1)
             if (valid && c + j < rows) tc::epi_elem(g, r0 + c + j, f, v[j]);
         }
       };
-      if (!acquire(it)) break;
-      const uint32_t tq = tmem_base + ((uint32_t)(qw * 32) << 16) + (uint32_t)((it & 1) * NT);
-      if (ent.w != 1) {
-        // accumulator lane = token row, column = output feature
-        const int row = (int)rank * HALF + qw * 32 + lane;
-        const bool valid = row < min(ent.z, MP);
-        for (int c = 0; c < n_eff; c += 32) {
-          float v[32];
-          tmem_ld_x32(tq + (uint32_t)c, v);
-          if (valid) tc::epi_row32(g, ent.y + row, n0 + c, v);
+      // a kind-2 tile holds two accumulator uses: the full tile, then the
+      // attached partial tile; one loop keeps a single copy of each path
+      const int parts = ent.w == 2 ? 2 : 1;
+      bool live = true;
+      for (int part = 0; part < parts; ++part) {
+        const int u = it + part;
+        if (!acquire(u)) {
+          live = false;
+          break;
         }
-      } else {
-        // weights on M: this CTA's 128 weight rows start at n0 + rank * 128
-        swapped_rows(tq, ent.y, ent.z, n0 + (int)rank * HALF, g.N);
+        const uint32_t tq = tmem_base + ((uint32_t)(qw * 32) << 16) + (uint32_t)((u & 1) * NT);
+        if (part == 0 && ent.w != 1) {
+          // accumulator lane = token row, column = output feature
+          const int row = (int)rank * HALF + qw * 32 + lane;
+          const bool valid = row < min(ent.z, MP);
+          for (int c = 0; c < n_eff; c += 32) {
+            float v[32];
+            tmem_ld_x32(tq + (uint32_t)c, v);
+            if (valid) tc::epi_row32(g, ent.y + row, n0 + c, v);
+          }
+        } else {
+          // kind 1: weights on M, this CTA's 128 weight rows start at
+          // n0 + rank * 128.  Attached partial tile: the weight rows of the B
+          // slot on M (this CTA's n_eff / 2 rows start at n0 + rank * n_eff / 2)
+          const int f0 = n0 + (int)rank * (part == 0 ? HALF : n_eff / 2);
+          const int f_end = part == 0 ? g.N : min(g.N, f0 + n_eff / 2);
+          swapped_rows(tq, part == 0 ? ent.y : ent.y + MP, part == 0 ? ent.z : ent.z - MP, f0,
+                       f_end);
+        }
+        release(u);
       }
-      release(it);
-      if (ent.w == 2) {
-        // attached remainder: the weight rows of the B slot on M (this CTA's
-        // n_eff / 2 rows start at n0 + rank * n_eff / 2), remainder rows on N
-        if (!acquire(it + 1)) break;
-        const uint32_t tq2 =
-            tmem_base + ((uint32_t)(qw * 32) << 16) + (uint32_t)(((it + 1) & 1) * NT);
-        const int f0 = n0 + (int)rank * (n_eff / 2);
-        swapped_rows(tq2, ent.y + MP, ent.z - MP, f0, min(g.N, f0 + n_eff / 2));
-        release(it + 1);
-        it += 2;
-      } else {
-        ++it;
-      }
+      if (!live) break;
+      it += parts;
     }
   }
   tc_fence_before();

@@ -183,9 +183,6 @@ static nh_status make_plan(const nh_moe_config* c, int64_t T, Plan* p) {
   L.tile_rows = tr;
   L.swap_ab = sw;
   L.x_direct = (sw && T <= 64) ? 1 : 0;   // every token fits one activation tile
-  // CTA-pair tiles (bf16, native weights, T > 64): the up projection gathers
-  // its activation rows from x by TMA, so no permuted copy of x is made
-  L.x_gather = (p->bf16 && !sw && c->weight_format == NH_WEIGHTS_NATIVE) ? 1 : 0;
   L.max_tiles = (int)((rows + tr - 1) / tr + p->E);
   L.n_chunks = (int)((T + PERM_CHUNK - 1) / PERM_CHUNK);
   L.rows_alloc = rows;
@@ -206,7 +203,7 @@ static nh_status make_plan(const nh_moe_config* c, int64_t T, Plan* p) {
   L.inv_row = take((size_t)rows * 4);
   L.tiles = take((size_t)L.max_tiles * 16);
   L.num_tiles = take(4);
-  L.x_perm = take((L.x_direct || L.x_gather) ? 0 : (size_t)rows * p->H * p->elem);
+  L.x_perm = take(L.x_direct ? 0 : (size_t)rows * p->H * p->elem);
   L.h = take((size_t)rows * p->I * p->elem);
   L.total_bytes = o;
   return NH_OK;
@@ -256,7 +253,7 @@ static PermuteOut permute_out(void* ws, const nh_moe_ws_layout& L, int* status) 
   o.x_perm = at<void>(ws, L.x_perm);
   o.status = status;
   o.sched_zero = reinterpret_cast<unsigned int*>(status + SCHED_UP);
-  o.gather = (L.x_direct || L.x_gather) ? 0 : 1;
+  o.gather = L.x_direct ? 0 : 1;
   return o;
 }
 
@@ -441,7 +438,6 @@ struct GemmCall {
   const float* perm_w;
   const int32_t* dst_row;    // routed down projection: token of each permuted row
   const int32_t* row_token;  // decode up projection reads x directly
-  const int32_t* gather_rows;  // prefill up projection gathers x rows by TMA (pair kernel)
   int* status;
   unsigned int* sched;  // tile scheduler counters (tensor-core path)
 };
@@ -452,7 +448,7 @@ static nh_status launch_tc(const GemmCall& c, int dev, cudaStream_t st) {
   CUtensorMap ma, mw;
   NH_TRY(map_2d(&ma, c.A, c.a_kwrap ? c.a_kwrap : c.K, c.rows, SWAP ? NT : tc::M));
   NH_TRY(map_3d(&mw, c.W, c.K, c.N, c.n_exp, SWAP ? tc::M : NT));
-  tc::TcArgs g;
+  tc::TcArgs g{};
   g.tiles = c.tiles;
   g.num_tiles = c.num_tiles;
   g.dense_rows = (int)c.rows;
@@ -466,7 +462,6 @@ static nh_status launch_tc(const GemmCall& c, int dev, cudaStream_t st) {
   g.perm_w = c.perm_w;
   g.dst_row = c.dst_row;
   g.row_token = c.row_token;
-  g.gather_rows = nullptr;
   g.status = c.status;
   g.timeout_ns = timeout_ns();
   g.sched = c.sched;
@@ -484,15 +479,11 @@ static nh_status launch_tc(const GemmCall& c, int dev, cudaStream_t st) {
 // the activations and half of the weight rows
 static nh_status launch_tc2(const GemmCall& c, int dev, cudaStream_t st) {
   CUtensorMap ma, mw, mr;
-  // gathered activations: a box one row high, four rows per TMA gather
-  NH_TRY(map_2d(&ma, c.A, c.a_kwrap ? c.a_kwrap : c.K, c.rows, c.gather_rows ? 1 : tc2::HALF));
+  NH_TRY(map_2d(&ma, c.A, c.a_kwrap ? c.a_kwrap : c.K, c.rows, tc2::HALF));
   NH_TRY(map_3d(&mw, c.W, c.K, c.N, c.n_exp, tc2::HALF));
-  // attached remainder rows (kind-2 tiles) when they are not gathered
-  if (c.gather_rows)
-    mr = ma;
-  else
-    NH_TRY(map_2d(&mr, c.A, c.a_kwrap ? c.a_kwrap : c.K, c.rows, tc2::C_ROWS));
-  tc::TcArgs g;
+  // rows of a partial tile attached to a full one (kind-2 tiles)
+  NH_TRY(map_2d(&mr, c.A, c.a_kwrap ? c.a_kwrap : c.K, c.rows, tc2::C_ROWS));
+  tc::TcArgs g{};
   g.tiles = c.tiles;
   g.num_tiles = c.num_tiles;
   g.dense_rows = (int)c.rows;
@@ -506,13 +497,11 @@ static nh_status launch_tc2(const GemmCall& c, int dev, cudaStream_t st) {
   g.perm_w = c.perm_w;
   g.dst_row = c.dst_row;
   g.row_token = nullptr;
-  g.gather_rows = c.gather_rows;
   g.status = c.status;
   g.timeout_ns = timeout_ns();
   g.sched = c.sched;
   if (!g.sched) return fail(NH_ERR_INVALID_ARG, "internal: no tile scheduler counters");
   if (c.tile_rows != tc2::MP) return fail(NH_ERR_INVALID_ARG, "internal: pair tiles are 256 rows");
-  if (c.gather_rows && c.a_kwrap) return fail(NH_ERR_INVALID_ARG, "internal: gather with K wrap");
   const int n_blocks = (c.N + tc2::NT - 1) / tc2::NT;
   const int64_t m_max = c.tiles ? c.max_tiles : (c.rows + c.tile_rows - 1) / c.tile_rows;
   const int64_t pairs = std::min<int64_t>(m_max * n_blocks, g_pair_clusters[dev]);
@@ -564,7 +553,7 @@ static nh_status launch_q4(const GemmCall& c, const nh_nvfp4_weight& w, int dev,
   NH_TRY(map_2d(&ma, c.A, c.K, c.rows, NT));
   NH_TRY(map_u8_3d(&mc, w.codes, c.K / 2, c.N, c.n_exp, q4::CODE_ROW, true));
   NH_TRY(map_u8_3d(&ms, w.scales, nvfp4_pitch(c.K), c.N, c.n_exp, q4::SCALE_BOX, false));
-  q4::Q4Args qa;
+  q4::Q4Args qa{};
   tc::TcArgs& g = qa.g;
   g.tiles = c.tiles;
   g.num_tiles = c.num_tiles;
@@ -579,7 +568,6 @@ static nh_status launch_q4(const GemmCall& c, const nh_nvfp4_weight& w, int dev,
   g.perm_w = c.perm_w;
   g.dst_row = c.dst_row;
   g.row_token = c.row_token;
-  g.gather_rows = nullptr;
   g.status = c.status;
   g.timeout_ns = timeout_ns();
   g.sched = c.sched;
@@ -596,7 +584,7 @@ static nh_status launch_q4(const GemmCall& c, const nh_nvfp4_weight& w, int dev,
 template <int NT>
 static nh_status launch_q4v(const GemmCall& c, const nh_nvfp4_weight& w, int dev,
                             cudaStream_t st) {
-  q4v::Args a;
+  q4v::Args a{};
   tc::TcArgs& g = a.g;
   g.tiles = c.tiles;
   g.num_tiles = c.num_tiles;
@@ -611,7 +599,6 @@ static nh_status launch_q4v(const GemmCall& c, const nh_nvfp4_weight& w, int dev
   g.perm_w = c.perm_w;
   g.dst_row = c.dst_row;
   g.row_token = c.row_token;
-  g.gather_rows = nullptr;
   g.status = c.status;
   g.timeout_ns = timeout_ns();
   g.sched = c.sched;
@@ -657,7 +644,7 @@ static nh_status run_gemm_q4(const GemmCall& c, const nh_nvfp4_weight* w, int de
 // 16 weight rows with K split over the warps (gemv_bf16.cuh)
 template <int NT>
 static nh_status launch_dgv(const GemmCall& c, int dev, cudaStream_t st) {
-  dgv::Args a;
+  dgv::Args a{};
   tc::TcArgs& g = a.g;
   g.tiles = nullptr;
   g.num_tiles = nullptr;
@@ -672,7 +659,6 @@ static nh_status launch_dgv(const GemmCall& c, int dev, cudaStream_t st) {
   g.perm_w = c.perm_w;
   g.dst_row = c.dst_row;
   g.row_token = nullptr;
-  g.gather_rows = nullptr;
   g.status = c.status;
   g.timeout_ns = timeout_ns();
   g.sched = c.sched;
@@ -1043,7 +1029,6 @@ nh_status nh_moe_permute(const nh_moe_config* cfg, int64_t T, const void* x,
         at<int32_t>(ws, L.perm_token), at<float>(ws, L.perm_w), at<int32_t>(ws, L.inv_row),
         at<__nv_bfloat16>(ws, L.x_perm), status, 0)));
     NH_TRY(launch_check("permute_scatter"));
-    if (L.x_gather) return NH_OK;   // the up projection gathers x rows itself
     NH_TRY((launch_k("permute_gather", permute_gather<__nv_bfloat16>, dim3(gather_blocks), dim3(256), 0, st, 
         static_cast<const __nv_bfloat16*>(x), at<int32_t>(ws, L.perm_token),
         at<int32_t>(ws, L.offsets), p.E, p.H, at<__nv_bfloat16>(ws, L.x_perm))));
@@ -1144,11 +1129,6 @@ static nh_status experts_phase(const nh_moe_config* cfg, int64_t T, const void* 
       c.A = x;
       c.rows = T;
       c.row_token = at<int32_t>(ws, L.perm_token);
-    } else if (L.x_gather && !nvfp4) {
-      // prefill: permuted row r is x[perm_token[r]], gathered by the GEMM's TMA
-      c.A = x;
-      c.rows = T;
-      c.gather_rows = at<int32_t>(ws, L.perm_token);
     } else {
       c.A = at<void>(ws, L.x_perm);
     }

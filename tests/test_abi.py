@@ -83,7 +83,7 @@ def test_workspace_layout(name):
                ("counts", cfg.E * 4),
                ("offsets", (cfg.E + 1) * 4), ("chunk_counts", L.n_chunks * cfg.E * 4),
                ("perm_token", rows * 4), ("perm_w", rows * 4), ("inv_row", rows * 4),
-               ("tiles", L.max_tiles * 16), ("num_tiles", 4), ("x_perm", 0 if (L.x_direct or L.x_gather) else rows * cfg.H * elem),
+               ("tiles", L.max_tiles * 16), ("num_tiles", 4), ("x_perm", 0 if L.x_direct else rows * cfg.H * elem),
                ("h", rows * cfg.I * elem)]
     spans = sorted((getattr(L, n), getattr(L, n) + sz, n) for n, sz in regions)
     for (a0, a1, an), (b0, b1, bn) in zip(spans, spans[1:]):
@@ -99,7 +99,6 @@ def test_workspace_layout(name):
         assert L.swap_ab == 1 and L.tile_rows >= T and L.tile_rows % 16 == 0
     else:
         assert L.swap_ab == 0 and L.tile_rows == 256     # CTA-pair tiles
-        assert L.x_gather == 1 and L.x_direct == 0       # rows gathered from x by TMA
     assert L.max_tiles >= -(-rows // L.tile_rows) + cfg.E - 1
 
 

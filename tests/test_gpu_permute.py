@@ -2,8 +2,7 @@
 
 Checks, for the single-block path (T <= 256), the multi-kernel path and the
 fused decode router+permute: counts, offsets, perm_token, perm_w, inv_row
-equal oracle.permute of the GPU's own routing; x_perm rows (where the plan
-makes them) equal x rows; the
+equal oracle.permute of the GPU's own routing; x_perm rows equal x rows; the
 tile table covers every expert's rows exactly once in order, with tiles no
 taller than the plan's tile height and the partial-tile kind flag set as
 documented (kind 1: an expert's partial last tile; kind 2: a full tile with
@@ -39,7 +38,7 @@ def check_permute(cfg, x_np, idx, w, ws, lay, x_dev):
     np.testing.assert_array_equal(region(ws, lay.inv_row, rows, np.int32).reshape(T, k),
                                   ref["inv_row"])
     elem = np.uint16 if cfg.dtype == "bf16" else np.float32
-    if not (lay.x_direct or lay.x_gather):   # else the up projection reads x itself
+    if not lay.x_direct:   # the decode orientation reads x directly (no x_perm)
         xp = region(ws, lay.x_perm, rows * cfg.H, elem).reshape(rows, cfg.H)
         np.testing.assert_array_equal(xp, x_np[ref["perm_token"]])
     nt = int(region(ws, lay.num_tiles, 1, np.int32)[0])
