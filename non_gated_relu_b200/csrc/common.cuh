@@ -314,6 +314,39 @@ __device__ __forceinline__ bool mbar_try_wait_cluster(uint32_t bar, uint32_t par
   return ok != 0;
 }
 
+// Test of a stage barrier without the sleep hint: the TMA -> MMA -> TMA hand-offs of
+// a pipeline stage complete through the barrier's transaction count and tcgen05
+// commits, so a CTA-scope test is enough, and the roles poll it without sleeping.
+__device__ __forceinline__ bool mbar_try_wait_spin(uint32_t bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// bounded wait on a stage barrier (mbar_try_wait_spin)
+__device__ __forceinline__ bool mbar_wait_spin(uint32_t bar, uint32_t parity, const WaitCtl& w,
+                                               int site) {
+  if (mbar_try_wait_spin(bar, parity)) return true;
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (mbar_try_wait_spin(bar, parity)) return true;
+    if ((i & 63u) == 0) {
+      if (*w.abort_flag) return false;
+      if (globaltimer_ns() - t0 > w.timeout_ns) {
+        *w.abort_flag = 1;
+        record_status(w.status, NH_ERR_TIMEOUT, site, (int)i);
+        return false;
+      }
+    }
+  }
+}
+
 // bounded wait with cluster-scope acquire (barriers that peers arrive on)
 __device__ __forceinline__ bool mbar_wait_cluster(uint32_t bar, uint32_t parity, const WaitCtl& w,
                                                   int site) {

@@ -57,6 +57,8 @@ struct TcArgs {
   int* status;
   uint64_t timeout_ns;
   unsigned int* sched;        // [2]: next tile, CTAs finished; zero on entry, reset on exit
+  int k_split;                // >1: each output tile is computed as k_split K slices by
+                              // separate tiles (additive epilogues only); 0 or 1: whole K
 };
 
 constexpr int TQ = 4;         // depth of the tile-id ring between the roles
@@ -211,8 +213,17 @@ __global__ void __launch_bounds__(THREADS, 1)
 
   const int num_m = g.tiles ? *g.num_tiles : (g.dense_rows + g.tile_rows - 1) / g.tile_rows;
   const int n_blocks = SWAP ? (g.N + M - 1) / M : (g.N + NT - 1) / NT;
-  const int total = num_m * n_blocks;
+  const int ks_n = g.k_split > 1 ? g.k_split : 1;
+  const int total = num_m * n_blocks * ks_n;
   const int nk = g.K / BK;
+  // tile id -> (tile entry m, feature block nb, K slice [kb_lo, kb_hi))
+  auto decode_tile = [&](int tile, int& m, int& nb, int& kb_lo, int& kb_hi) {
+    const int ks = tile % ks_n, rest = tile / ks_n;
+    m = rest / n_blocks;
+    nb = rest - m * n_blocks;
+    kb_lo = ks * nk / ks_n;
+    kb_hi = (ks + 1) * nk / ks_n;
+  };
 
   if (warp == 0 && lane == 0) {
     // ---------------- TMA producer + tile scheduler ----------------
@@ -231,9 +242,10 @@ __global__ void __launch_bounds__(THREADS, 1)
       tile_q[q] = tile;
       mbar_arrive(tq_full_bar(q));
       if (tile < 0) break;
-      const int m = tile / n_blocks, nb = tile - m * n_blocks;
+      int m, nb, kb_lo, kb_hi;
+      decode_tile(tile, m, nb, kb_lo, kb_hi);
       const int4 ent = tile_entry_of(g, m);
-      for (int kb = 0; kb < nk; ++kb) {
+      for (int kb = kb_lo; kb < kb_hi; ++kb) {
         if (!mbar_wait(empty_bar(stage), phase ^ 1u, wc, SITE_TC_PRODUCER)) {
           ok = false;
           break;
@@ -277,7 +289,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int tile = tile_q[q];
       mbar_arrive(tq_empty_bar(q));
       if (tile < 0) break;
-      const int m = tile / n_blocks, nb = tile - m * n_blocks;
+      int m, nb, kb_lo, kb_hi;
+      decode_tile(tile, m, nb, kb_lo, kb_hi);
       const int acc = it & 1;
       const uint32_t aph = (uint32_t)((it >> 1) & 1);
       if (!mbar_wait(tempty_bar(acc), aph ^ 1u, wc, SITE_TC_MMA)) {
@@ -289,7 +302,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const uint32_t idesc = make_idesc_bf16(M, n_mma);
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * S::ACC_COLS);
       (void)m;
-      for (int kb = 0; kb < nk; ++kb) {
+      for (int kb = kb_lo; kb < kb_hi; ++kb) {
         if (!mbar_wait(full_bar(stage), phase, wc, SITE_TC_MMA)) {
           ok = false;
           break;
@@ -299,7 +312,7 @@ __global__ void __launch_bounds__(THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < BK / UMMA_K; ++kk) {
           umma_bf16(d_tmem, make_sdesc_sw128(sa + kk * UMMA_K * 2),
-                    make_sdesc_sw128(sb + kk * UMMA_K * 2), idesc, (kb | kk) != 0);
+                    make_sdesc_sw128(sb + kk * UMMA_K * 2), idesc, (kb != kb_lo) | kk);
         }
         any = true;
         umma_commit(empty_bar(stage));
@@ -335,7 +348,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       ok = __shfl_sync(0xffffffffu, ok, 0);
       tile = __shfl_sync(0xffffffffu, tile, 0);
       if (!ok || tile < 0) break;
-      const int m = tile / n_blocks, nb = tile - m * n_blocks;
+      int m, nb, kb_lo, kb_hi;
+      decode_tile(tile, m, nb, kb_lo, kb_hi);
       const int acc = it & 1;
       const uint32_t aph = (uint32_t)((it >> 1) & 1);
       if (lane == 0) ok = mbar_wait(tfull_bar(acc), aph, wc, SITE_TC_EPILOGUE) ? 1 : 0;

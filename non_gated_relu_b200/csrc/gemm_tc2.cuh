@@ -30,7 +30,9 @@
 // MMA completion is committed to the stage / accumulator barriers of both
 // CTAs (two plain commits, no multicast); the peer's epilogue and scheduler
 // hand-backs arrive on the leader's barriers through shared::cluster
-// addresses.  All waits are bounded like the one-CTA kernel's.
+// addresses.  The per-stage waits (producer on empty, MMA on full) are
+// CTA-scope polls; the tile-id and accumulator hand-offs between the CTAs use
+// cluster-scope acquire.  All waits are bounded like the one-CTA kernel's.
 #pragma once
 
 #include "gemm_tc.cuh"
@@ -179,7 +181,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int c_row = ent.y + MP + (int)rank * (attached ? swap_n(ent.z - MP) / 2 : 0);
       const uint32_t tx_bytes = 2u * (attached ? STAGE_BYTES : AB_BYTES);
       for (int kb = 0; kb < nk; ++kb) {
-        if (!mbar_wait_cluster(empty_bar(stage), phase ^ 1u, wc, SITE_TC_PRODUCER)) {
+        if (!mbar_wait_spin(empty_bar(stage), phase ^ 1u, wc, SITE_TC_PRODUCER)) {
           ok = false;
           break;
         }
@@ -246,7 +248,7 @@ __global__ void __launch_bounds__(THREADS, 1)
       // about 15 % of throughput on every tile, measured)
       if (!attached) {
         for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait_cluster(full_bar(stage), phase, wc, SITE_TC_MMA)) {
+          if (!mbar_wait_spin(full_bar(stage), phase, wc, SITE_TC_MMA)) {
             ok = false;
             break;
           }
@@ -266,7 +268,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         }
       } else {
         for (int kb = 0; kb < nk; ++kb) {
-          if (!mbar_wait_cluster(full_bar(stage), phase, wc, SITE_TC_MMA)) {
+          if (!mbar_wait_spin(full_bar(stage), phase, wc, SITE_TC_MMA)) {
             ok = false;
             break;
           }

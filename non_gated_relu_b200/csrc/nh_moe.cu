@@ -440,6 +440,7 @@ struct GemmCall {
   const int32_t* row_token;  // decode up projection reads x directly
   int* status;
   unsigned int* sched;  // tile scheduler counters (tensor-core path)
+  int k_split;          // K slices per output tile (additive epilogues; 0/1 = none)
 };
 
 template <bool SWAP, int NT, int STAGES>
@@ -465,10 +466,13 @@ static nh_status launch_tc(const GemmCall& c, int dev, cudaStream_t st) {
   g.status = c.status;
   g.timeout_ns = timeout_ns();
   g.sched = c.sched;
+  g.k_split = c.k_split;
   if (!g.sched) return fail(NH_ERR_INVALID_ARG, "internal: no tile scheduler counters");
+  if (c.k_split > 1 && c.epi != EPI_DOWN_COMBINE && c.epi != EPI_ACC_F32)
+    return fail(NH_ERR_INVALID_ARG, "internal: K slices need an additive epilogue");
   const int n_blocks = SWAP ? (c.N + tc::M - 1) / tc::M : (c.N + NT - 1) / NT;
   const int64_t m_max = c.tiles ? c.max_tiles : (c.rows + c.tile_rows - 1) / c.tile_rows;
-  const int64_t work = m_max * n_blocks;
+  const int64_t work = m_max * n_blocks * (c.k_split > 1 ? c.k_split : 1);
   const int grid = (int)std::min<int64_t>(work, g_sm_count[dev]);
   if (grid <= 0) return NH_OK;
   NH_TRY((launch_k("tc_grouped_gemm", tc::tc_grouped_gemm<SWAP, NT, STAGES>, dim3(grid), dim3(tc::THREADS), S::SMEM, st, ma, mw, g)));
@@ -1147,6 +1151,10 @@ static nh_status experts_phase(const nh_moe_config* cfg, int64_t T, const void* 
     c.ldo = p.H;
     c.perm_w = at<float>(ws, L.perm_w);
     c.dst_row = at<int32_t>(ws, L.perm_token);
+    // decode tiles stream an expert's weights for a few tokens: two K slices
+    // per output block halve a tile's length (finer load balance at the end);
+    // the combine adds both slices into y_acc
+    if (L.swap_ab && !nvfp4 && p.I >= 2 * tc::BK) c.k_split = 2;
   }
   if (nvfp4) return run_gemm_q4(c, wq, dev, st);
   return run_gemm(p, c, dev, st);
