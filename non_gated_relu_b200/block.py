@@ -14,8 +14,9 @@ than 256 rows (one CTA-pair tile) per expert on average: the shared expert
 then fills what the routed path leaves idle.  With more rows per expert every
 GEMM is bound by the tensor cores, and running the shared expert's GEMMs beside
 the routed ones only makes them contend (their float32 adds into the same y_acc
-included); there every step runs on the caller's stream in turn: y_acc = 0,
-shared expert, route + permute, forward, finalize.
+included); there the zeroing of y_acc still runs on the side stream, beside
+route + permute, and the rest runs in turn on one stream: shared expert,
+forward, finalize.
 
 With latent projections (config ``latent_size`` L > 0; the modules
 fc1_latent_proj / fc2_latent_proj of the ModelOpt descriptor
@@ -192,45 +193,62 @@ class NemotronHMoE:
         fork = torch.cuda.Event()
         fork.record(caller)
         main.wait_event(fork)
-        # weight-streaming calls run the shared expert beside the routed path
-        E = self.c.n_routed_experts
-        side = self.side if T * self.k < self.concurrent_rows_per_expert * E else main
-        if side is not main:
-            side.wait_event(fork)
-        # the accumulators start at zero, then the shared expert adds into y_acc
+        self.side.wait_event(fork)
+        # the accumulators start at zero on the side stream (beside the router)
         push("zero_acc")
-        zero_acc(self.c, T, b.y_acc, stream=side)
+        zero_acc(self.c, T, b.y_acc, stream=self.side)
         if self.latent:
-            zero_acc(self.c_exp, T, b.y_lat_acc, stream=side)
+            zero_acc(self.c_exp, T, b.y_lat_acc, stream=self.side)
         pop()
         zero = torch.cuda.Event()
-        zero.record(side)
-        if self.has_shared:
+        zero.record(self.side)
+
+        def run_shared(stream):
+            if not self.has_shared:
+                return
             push("shared")
             if self.nvfp4:
                 shared_nvfp4(self.c, x, self.q4["shared_up"], self.q4["shared_down"], b.y_acc,
-                             b.ws_shared, stream=side)
+                             b.ws_shared, stream=stream)
             else:
                 shared(self.c, x, self.w_shared_up, self.w_shared_down, b.y_acc, b.ws_shared,
-                       stream=side)
+                       stream=stream)
             pop()
-        join = torch.cuda.Event()
-        join.record(side)
+
+        # weight-streaming calls run the shared expert beside the routed path;
+        # otherwise it runs on the main stream once y_acc is zero
+        E = self.c.n_routed_experts
+        concurrent = T * self.k < self.concurrent_rows_per_expert * E
+        join = None
+        if concurrent:
+            run_shared(self.side)
+            join = torch.cuda.Event()
+            join.record(self.side)
+
+        def shared_done():
+            if concurrent:
+                main.wait_event(join)
+            else:
+                run_shared(main)
+
         if self.latent:
-            out = self._forward_latent(x, b, main, zero, join, partial, push, pop)
+            out = self._forward_latent(x, b, main, zero, shared_done, partial, push, pop)
             self._join(caller, main)
             return out
         push("route_permute")
         route_permute(self.c, x, self.w_router, self.bias, b.topk_idx, b.topk_w, b.ws, stream=main)
         pop()
         main.wait_event(zero)
+        if not concurrent:
+            shared_done()
         push("forward")
         if self.nvfp4:
             forward_nvfp4(self.c, x, self.q4["up"], self.q4["down"], b.ws, b.y_acc, stream=main)
         else:
             forward(self.c, x, self.w_up, self.w_down, b.ws, b.y_acc, stream=main)
         pop()
-        main.wait_event(join)
+        if concurrent:
+            shared_done()
         if not partial:
             push("finalize")
             finalize(self.c, T, b.y_acc, b.y, stream=main)
@@ -244,7 +262,7 @@ class NemotronHMoE:
         done.record(main)
         caller.wait_event(done)
 
-    def _forward_latent(self, x, b, main, zero, join, partial, push, pop):
+    def _forward_latent(self, x, b, main, zero, shared_done, partial, push, pop):
         T = x.shape[0]
         push("route")
         route(self.c, x, self.w_router, self.bias, b.topk_idx, b.topk_w, b.ws_route, stream=main)
@@ -264,7 +282,7 @@ class NemotronHMoE:
             forward(ce, b.x_lat, self.w_up, self.w_down, b.ws, b.y_lat_acc, stream=main)
         finalize(ce, T, b.y_lat_acc, b.y_lat, stream=main)
         pop()
-        main.wait_event(join)
+        shared_done()     # y_acc holds the shared expert before fc2 adds into it
         push("latent_out")
         latent_out(self.c, T, b.y_lat, self.w_latent_fc2, b.y_acc, b.ws_lat, stream=main)
         pop()
