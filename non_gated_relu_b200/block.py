@@ -152,8 +152,10 @@ class NemotronHMoE:
         self._host: Dict[int, tuple] = {}
 
     # ------------------------------------------------------------------ buffers
-    def buffers(self, T: int) -> Buffers:
-        b = self._bufs.get(T)
+    def buffers(self, T: int, slot: int = 0) -> Buffers:
+        """Device buffers of a call with T tokens (``slot`` > 0: a further set, for
+        calls in flight together, see ``pipeline``)."""
+        b = self._bufs.get((T, slot))
         if b is None:
             dev = self.device
             ws = torch.empty(workspace_size(self.c_exp, T), dtype=torch.uint8, device=dev)
@@ -173,7 +175,7 @@ class NemotronHMoE:
                 b.x_lat = torch.empty((T, self.L), dtype=self.dtype, device=dev)
                 b.y_lat = torch.empty((T, self.L), dtype=self.dtype, device=dev)
                 b.y_lat_acc = torch.empty((T, self.L), dtype=torch.float32, device=dev)
-            self._bufs[T] = b
+            self._bufs[(T, slot)] = b
         return b
 
     # ------------------------------------------------------------------ compute
@@ -293,15 +295,16 @@ class NemotronHMoE:
         pop()
         return b.y
 
-    def capture(self, T: int):
-        """Capture the call sequence for T tokens in a CUDA graph.
+    def capture(self, T: int, slot: int = 0):
+        """Capture the call sequence for T tokens in a CUDA graph (on the buffer set
+        ``slot``).
 
         Returns (graph, x_static, y): write the input into ``x_static`` and
         ``graph.replay()`` writes ``y``."""
-        g = self._graphs.get(T)
+        g = self._graphs.get((T, slot))
         if g is None:
             x_static = torch.zeros((T, self.H), dtype=self.dtype, device=self.device)
-            b = self.buffers(T)
+            b = self.buffers(T, slot)
             s = torch.cuda.Stream(self.device)
             s.wait_stream(torch.cuda.current_stream(self.device))
             with torch.cuda.stream(s):           # warm up outside the graph
@@ -312,8 +315,72 @@ class NemotronHMoE:
             with torch.cuda.graph(graph):
                 y = self.forward(x_static, b)
             g = (graph, x_static, y)
-            self._graphs[T] = g
+            self._graphs[(T, slot)] = g
         return g
+
+    def pipeline(self, xs):
+        """y for a sequence of host batches (pinned tensors [T, H], one T), with the
+        host copies of one batch overlapping the block of another: the block runs
+        as a CUDA graph on the current stream, host-to-device copies on one stream
+        and device-to-host copies on another, over two buffer sets.  Every batch
+        still has its own copy in and copy out.
+
+        A generator: yields (index, y) in order, y a pinned host tensor [T, H] that
+        stays valid until the generator is resumed twice more (it is reused for the
+        batch after next); clone it to keep it."""
+        xs = list(xs)
+        if not xs:
+            return
+        T = xs[0].shape[0]
+        dev = self.device
+        comp = torch.cuda.current_stream(dev)
+        if not hasattr(self, "_h2d"):
+            with torch.cuda.device(dev):
+                self._h2d = torch.cuda.Stream()
+                self._d2h = torch.cuda.Stream()
+        slots = []
+        for s in (0, 1):
+            graph, x_static, y = self.capture(T, s)
+            key = ("pinned_out", T, s)
+            yh = self._host.get(key)
+            if yh is None:
+                yh = torch.empty((T, self.H), dtype=self.dtype).pin_memory()
+                self._host[key] = yh
+            slots.append((graph, x_static, y, yh))
+        in_free = [None, None]    # the slot's x_static was read by its last block call
+        out_free = [None, None]   # the slot's y was copied out
+        prev = None
+        for i, xh in enumerate(xs):
+            if xh.shape[0] != T:
+                raise ValueError("pipeline: every batch needs the same token count")
+            if not xh.is_pinned():
+                raise ValueError("pipeline: host batches must be in pinned memory")
+            graph, x_static, y, yh = slots[i % 2]
+            if in_free[i % 2] is not None:
+                self._h2d.wait_event(in_free[i % 2])
+            with torch.cuda.stream(self._h2d):
+                x_static.copy_(xh, non_blocking=True)
+            copied = torch.cuda.Event()
+            copied.record(self._h2d)
+            comp.wait_event(copied)
+            if out_free[i % 2] is not None:
+                comp.wait_event(out_free[i % 2])
+            graph.replay()
+            done = torch.cuda.Event()
+            done.record(comp)
+            in_free[i % 2] = done
+            self._d2h.wait_event(done)
+            with torch.cuda.stream(self._d2h):
+                yh.copy_(y, non_blocking=True)
+            out = torch.cuda.Event()
+            out.record(self._d2h)
+            out_free[i % 2] = out
+            if prev is not None:
+                prev[1].synchronize()
+                yield prev[0], prev[2]
+            prev = (i, out, yh)
+        prev[1].synchronize()
+        yield prev[0], prev[2]
 
     def check(self, T: int) -> int:
         """Status word of the last call for T tokens (synchronises)."""

@@ -140,6 +140,24 @@ def test_host_api_graph_matches_eager():
     assert_same_up_to_sum_order(y3, blk.forward(to_dev(x2)).float().cpu().numpy(), "bf16")
 
 
+@pytest.mark.parametrize("name", ["small_swap16", "small_prefill"])
+def test_host_pipeline_matches_eager(name):
+    """The pipelined host call (two buffer sets, copies on their own streams)
+    gives every batch the result of the eager call, in order."""
+    inp = synth.make_inputs(SMALL[name])
+    blk = make_block(inp)
+    rng = np.random.default_rng(3)
+    batches = [inp.x] + [np.ascontiguousarray(inp.x[rng.permutation(inp.x.shape[0])])
+                         for _ in range(4)]
+    ref = [blk.forward(to_dev(b)).float().cpu().numpy() for b in batches]
+    host = [torch.from_numpy(b).view(torch.bfloat16).pin_memory() for b in batches]
+    seen = []
+    for i, y in blk.pipeline(host):
+        seen.append(i)
+        assert_same_up_to_sum_order(y.float().numpy(), ref[i], "bf16")
+    assert seen == list(range(len(batches)))
+
+
 # ----------------------------------------------------------------------------- full size
 FULL = synth.CONFIG_ORDER
 
