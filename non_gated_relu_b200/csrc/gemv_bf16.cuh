@@ -4,12 +4,10 @@
 // These layers have one "tile entry" (all tokens) and N / 128 weight tiles,
 // so the tcgen05 kernel runs on N / 128 CTAs (29 for the shared up
 // projection) and cannot draw full HBM bandwidth.  Here a CTA task is 16
-// weight rows; its 8 warps split K in 128-feature blocks, load the weights
-// with 16-byte global loads straight into the A fragments of mma.sync
-// m16n8k16 (bf16 in, f32 accumulate; tokens on N = 8) and add their partial
-// tiles through shared memory in warp order (deterministic).  The feature
-// permutation inside a block is the one of gemv_q4.cuh: thread tq's 32
-// features are one contiguous run of 64 bytes per row.
+// weight rows, which reach shared memory by untiled bulk copies; the warps
+// feed them to mma.sync m16n8k16 (bf16 in, f32 accumulate; tokens on N = 8)
+// and add their partial tiles through shared memory in warp order
+// (deterministic).
 #pragma once
 
 #include "gemv_q4.cuh"
@@ -26,84 +24,141 @@ struct Args {
   const void* W;           // weights [N, K] bf16
 };
 
-// One block of BK features for one n-tile: the weight runs of rows gq (wa)
-// and gq + 8 (wb), BK/32 uint4 each (one uint4 = 8 features = two k-tiles),
-// and the activation run of token gq.
-template <int BK>
-__device__ __forceinline__ void block_mma(const uint4* wa, const uint4* wb,
-                                          const __nv_bfloat16* act, float* c0, float* c1) {
-  constexpr int KT = BK / 16;
-  uint2 bv[KT];
-#pragma unroll
-  for (int kt = 0; kt < KT; ++kt) bv[kt] = __ldg(reinterpret_cast<const uint2*>(act + 4 * kt));
-#pragma unroll
-  for (int u = 0; u < KT / 2; ++u) {
-    // k-tile 2u: run features 8u + {0,1} (.x) and {2,3} (.y); k-tile 2u + 1: .z, .w
-    q4v::mma_bf16_16816(c0, wa[u].x, wb[u].x, wa[u].y, wb[u].y, bv[2 * u].x, bv[2 * u].y);
-    q4v::mma_bf16_16816(c1, wa[u].z, wb[u].z, wa[u].w, wb[u].w, bv[2 * u + 1].x,
-                        bv[2 * u + 1].y);
-  }
-}
+// A CTA task is 16 weight rows over the whole K, split over the 8 warps in
+// units of 32 features (4 lanes x 8 bf16): warp w owns units
+// [w U / 8, (w + 1) U / 8) of the U = K / 32.  Each warp streams its share in
+// chunks of up to CH units through NBUF private buffers: one bulk copy per row
+// and chunk (row r's units are contiguous in W), completing on the buffer's
+// mbarrier.  One chunk of 11 units holds a warp's whole share for K up to
+// 2816, so for the shared expert's up projection (K = 2688) one round trip to
+// memory brings all of it; its down projection (K = 3712) takes a chunk of 11
+// and one of up to 4.  The first chunks of the CTA's first task are issued
+// before the grid waits on its predecessor (weights are inputs, never produced
+// by an earlier kernel), so a dependent launch streams its weights while the
+// kernel before it finishes.  Inside a unit, lane (gq, tq) reads the 16 bytes
+// at 16 tq of rows gq and gq + 8 -- features 8 tq .. 8 tq + 7 of the unit --
+// and the same features of its token's activations: k-tile 2u takes features
+// 8 tq + {0,1} / {2,3}, k-tile 2u + 1 takes 8 tq + {4,5} / {6,7}, a bijection
+// of the unit's 32 features onto the two k-tiles' slots.  Rows are PITCH bytes
+// apart in a buffer, 64 modulo 128, so the eight lanes of one shared-memory
+// wavefront (rows gq, gq + 1) hit disjoint banks.  K must be a multiple of 32
+// and W 16-byte aligned (both hold for every weight this library takes).
+constexpr int UNIT = 32;
+constexpr int CH = 11;
+constexpr int NBUF = 1;
+constexpr int PITCH = CH * UNIT * 2;
+constexpr int BUF_BYTES = MT * PITCH;
+constexpr int STAGED_SMEM = WARPS * NBUF * BUF_BYTES;
+static_assert(PITCH % 128 == 64, "rows gq and gq + 1 must use disjoint banks");
+static_assert(BUF_BYTES % 16 == 0, "bulk copy destinations are 16-byte aligned");
 
 template <int NT>
-__global__ void __launch_bounds__(WARPS * 32, 2) bf16_gemv_splitk(const Args a) {
+__global__ void __launch_bounds__(WARPS * 32, 2) bf16_gemv_staged(const Args a) {
+  extern __shared__ __align__(128) uint8_t stage_smem[];
   __shared__ float red[WARPS][32][4];
+  __shared__ __align__(8) uint64_t bars[WARPS][NBUF];
+  __shared__ int abort_flag;
   const tc::TcArgs& g = a.g;
-  pdl_wait();
-  pdl_trigger();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int gq = lane >> 2, tq = lane & 3;
   const int num_m = (g.dense_rows + g.tile_rows - 1) / g.tile_rows;
   const int n_rb = g.N / MT;
   const int total = num_m * n_rb;
   const int K = g.K;
-  const int nkb = K / 128, tail = K % 128;
+  const int U = K / UNIT;
+  const int u_lo = warp * U / WARPS, u_hi = (warp + 1) * U / WARPS;
+  const int nch = (u_hi - u_lo + CH - 1) / CH;
+  const uint8_t* const bufp = stage_smem + warp * NBUF * BUF_BYTES;
+  const uint32_t buf = smem_u32(bufp);
+  const uint32_t bar = smem_u32(&bars[warp][0]);
   const __nv_bfloat16* A = static_cast<const __nv_bfloat16*>(a.A);
   const __nv_bfloat16* W = static_cast<const __nv_bfloat16*>(a.W);
+  if (threadIdx.x == 0) abort_flag = 0;
+  if (lane == 0)
+    for (int b = 0; b < NBUF; ++b) mbar_init(bar + 8u * b, 1);
+  fence_barrier_init();
+  __syncthreads();
+  const WaitCtl wc{&abort_flag, g.status, g.timeout_ns};
+  uint32_t phase = 0u, pending = 0u;  // bit b: buffer b's next parity / a copy in flight
+  // chunk c of the task at weight row r0 into buffer c % NBUF
+  auto issue = [&](int r0, int c) {
+    const int b = c % NBUF;
+    const int ua = u_lo + c * CH, ub = min(ua + CH, u_hi);
+    const uint32_t bytes = (uint32_t)(ub - ua) * UNIT * 2;
+    if (lane == 0) mbar_arrive_expect_tx(bar + 8u * b, bytes * MT);
+    __syncwarp();
+    if (lane < MT)
+      bulk_load(buf + (uint32_t)(b * BUF_BYTES + lane * PITCH),
+                W + (size_t)(r0 + lane) * K + (size_t)ua * UNIT, bytes, bar + 8u * b);
+    pending |= 1u << b;
+  };
+  if ((int)blockIdx.x < total)
+    for (int c = 0; c < min(NBUF, nch); ++c) issue(((int)blockIdx.x % n_rb) * MT, c);
+  pdl_wait();
+  pdl_trigger();
+  bool ok = true;
   for (int task = blockIdx.x; task < total; task += gridDim.x) {
     const int m = task / n_rb, rb = task - m * n_rb;
     const int r0 = rb * MT;
     const int4 ent = tc::tile_entry_of(g, m);
     const int count = ent.z;
-    const __nv_bfloat16* wa_p = W + (size_t)(r0 + gq) * K;
-    const __nv_bfloat16* wb_p = wa_p + 8 * (size_t)K;
-    for (int n0 = 0; n0 < count; n0 += 8) {
-      const int j = min(n0 + gq, count - 1);
-      const __nv_bfloat16* act = A + (size_t)(ent.y + j) * K;
-      float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
-      for (int kb = warp; kb < nkb; kb += WARPS) {
-        uint4 wa[4], wb[4];
-        const uint4* pa = reinterpret_cast<const uint4*>(wa_p + kb * 128 + 32 * tq);
-        const uint4* pb = reinterpret_cast<const uint4*>(wb_p + kb * 128 + 32 * tq);
+    if (task != (int)blockIdx.x && ok)
+      for (int c = 0; c < min(NBUF, nch); ++c) issue(r0, c);
+    float c0[NT / 8][4], c1[NT / 8][4];
 #pragma unroll
-        for (int u = 0; u < 4; ++u) {
-          wa[u] = __ldg(pa + u);
-          wb[u] = __ldg(pb + u);
+    for (int p = 0; p < NT / 8; ++p)
+#pragma unroll
+      for (int i = 0; i < 4; ++i) c0[p][i] = c1[p][i] = 0.f;
+    for (int c = 0; c < nch; ++c) {
+      const int b = c % NBUF;
+      if (ok) ok = mbar_wait(bar + 8u * b, (phase >> b) & 1u, wc, SITE_GEMV_STAGE);
+      if (ok) {
+        phase ^= 1u << b;
+        pending &= ~(1u << b);
+        const int ua = u_lo + c * CH, nu = min(CH, u_hi - ua);
+        const uint8_t* bp = bufp + b * BUF_BYTES + tq * 16;
+#pragma unroll
+        for (int p = 0; p < NT / 8; ++p) {
+          if (p * 8 >= count) break;
+          // token p * 8 + gq (lanes past count re-read the last token; their
+          // columns are never stored)
+          const int j = min(p * 8 + gq, count - 1);
+          const __nv_bfloat16* act = A + (size_t)(ent.y + j) * K + (size_t)ua * UNIT + tq * 8;
+          uint4 xv[CH];
+#pragma unroll
+          for (int uu = 0; uu < CH; ++uu)
+            if (uu < nu) xv[uu] = __ldg(reinterpret_cast<const uint4*>(act + uu * UNIT));
+#pragma unroll
+          for (int uu = 0; uu < CH; ++uu) {
+            if (uu < nu) {
+              const uint4 wa = *reinterpret_cast<const uint4*>(bp + gq * PITCH + uu * 64);
+              const uint4 wb = *reinterpret_cast<const uint4*>(bp + (gq + 8) * PITCH + uu * 64);
+              q4v::mma_bf16_16816(c0[p], wa.x, wb.x, wa.y, wb.y, xv[uu].x, xv[uu].y);
+              q4v::mma_bf16_16816(c1[p], wa.z, wb.z, wa.w, wb.w, xv[uu].z, xv[uu].w);
+            }
+          }
         }
-        block_mma<128>(wa, wb, act + kb * 128 + 32 * tq, c0, c1);
       }
-      if (tail && warp == nkb % WARPS) {
-        // 64-feature tail: thread tq's run is features [16 tq, 16 tq + 16)
-        uint4 wa[2], wb[2];
-        const uint4* pa = reinterpret_cast<const uint4*>(wa_p + nkb * 128 + 16 * tq);
-        const uint4* pb = reinterpret_cast<const uint4*>(wb_p + nkb * 128 + 16 * tq);
-#pragma unroll
-        for (int u = 0; u < 2; ++u) {
-          wa[u] = __ldg(pa + u);
-          wb[u] = __ldg(pb + u);
-        }
-        block_mma<64>(wa, wb, act + nkb * 128 + 16 * tq, c0, c1);
+      // every lane is done with the buffer before it is refilled
+      __syncwarp();
+      if (ok && c + NBUF < nch) {
+        fence_proxy_async_smem();
+        issue(r0, c + NBUF);
       }
+    }
 #pragma unroll
-      for (int i = 0; i < 4; ++i) red[warp][lane][i] = c0[i] + c1[i];
+    for (int p = 0; p < NT / 8; ++p) {
+      if (p * 8 >= count) break;
+#pragma unroll
+      for (int i = 0; i < 4; ++i) red[warp][lane][i] = c0[p][i] + c1[p][i];
       __syncthreads();
-      if (warp == 0) {
+      if (warp == 0 && !abort_flag) {
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           float v = 0.f;
 #pragma unroll
           for (int w = 0; w < WARPS; ++w) v += red[w][lane][i];
-          const int jj = n0 + 2 * tq + (i & 1);
+          const int jj = p * 8 + 2 * tq + (i & 1);
           const int f = r0 + gq + (i >> 1) * 8;
           if (jj < count) tc::epi_elem(g, ent.y + jj, f, v);
         }
@@ -111,6 +166,9 @@ __global__ void __launch_bounds__(WARPS * 32, 2) bf16_gemv_splitk(const Args a) 
       __syncthreads();
     }
   }
+  // copies still in flight after a wait ran out land before the CTA exits
+  for (int b = 0; b < NBUF; ++b)
+    if (pending & (1u << b)) tc::mbar_drain(bar + 8u * b, (phase >> b) & 1u, g.timeout_ns, g.status);
 }
 
 }  // namespace dgv

@@ -290,6 +290,10 @@ static nh_status set_attrs(int dev) {
                                tc2::SMEM));
   NH_CUDA(cudaFuncSetAttribute(q4::tc_q4_gemm<64, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                q4::Shape<64, 4>::SMEM));
+  NH_CUDA(cudaFuncSetAttribute(dgv::bf16_gemv_staged<16>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, dgv::STAGED_SMEM));
+  NH_CUDA(cudaFuncSetAttribute(dgv::bf16_gemv_staged<32>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, dgv::STAGED_SMEM));
   NH_CUDA(cudaFuncSetAttribute(route_permute_small<__nv_bfloat16>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, ROUTE_PERMUTE_SMEM_MAX));
   NH_CUDA(cudaFuncSetAttribute(route_permute_small<float>,
@@ -671,8 +675,8 @@ static nh_status launch_dgv(const GemmCall& c, int dev, cudaStream_t st) {
   const int64_t tasks = (c.rows + c.tile_rows - 1) / c.tile_rows * (c.N / dgv::MT);
   const int64_t grid = std::min<int64_t>(tasks, (int64_t)g_sm_count[dev] * 2);
   if (grid <= 0) return NH_OK;
-  return launch_k("bf16_gemv_splitk", dgv::bf16_gemv_splitk<NT>, dim3((unsigned)grid),
-                  dim3(dgv::WARPS * 32), 0, st, a);
+  return launch_k("bf16_gemv_staged", dgv::bf16_gemv_staged<NT>, dim3((unsigned)grid),
+                  dim3(dgv::WARPS * 32), dgv::STAGED_SMEM, st, a);
 }
 
 static nh_status run_gemm(const Plan& p, const GemmCall& c, int dev, cudaStream_t st) {
