@@ -89,10 +89,6 @@ class NemotronHMoE:
     context), as one process per GPU does.
     """
 
-    #: the shared expert runs on a side stream, beside the routed path, while
-    #: T * k < concurrent_rows_per_expert * E (mean rows per routed expert)
-    concurrent_rows_per_expert = 256
-
     def __init__(self, cfg, w_router, w_up=None, w_down=None, w_shared_up=None,
                  w_shared_down=None, bias=None, device=None, nvfp4=None, w_latent_fc1=None,
                  w_latent_fc2=None):
@@ -205,33 +201,23 @@ class NemotronHMoE:
         zero = torch.cuda.Event()
         zero.record(self.side)
 
-        def run_shared(stream):
-            if not self.has_shared:
-                return
+        # the shared expert runs on the side stream beside the routed path (at
+        # decode it streams its weights while the router runs; at prefill its
+        # GEMMs take the SMs the routing and permute kernels leave idle)
+        if self.has_shared:
             push("shared")
             if self.nvfp4:
                 shared_nvfp4(self.c, x, self.q4["shared_up"], self.q4["shared_down"], b.y_acc,
-                             b.ws_shared, stream=stream)
+                             b.ws_shared, stream=self.side)
             else:
                 shared(self.c, x, self.w_shared_up, self.w_shared_down, b.y_acc, b.ws_shared,
-                       stream=stream)
+                       stream=self.side)
             pop()
-
-        # weight-streaming calls run the shared expert beside the routed path;
-        # otherwise it runs on the main stream once y_acc is zero
-        E = self.c.n_routed_experts
-        concurrent = T * self.k < self.concurrent_rows_per_expert * E
-        join = None
-        if concurrent:
-            run_shared(self.side)
-            join = torch.cuda.Event()
-            join.record(self.side)
+        join = torch.cuda.Event()
+        join.record(self.side)
 
         def shared_done():
-            if concurrent:
-                main.wait_event(join)
-            else:
-                run_shared(main)
+            main.wait_event(join)
 
         if self.latent:
             out = self._forward_latent(x, b, main, zero, shared_done, partial, push, pop)
@@ -241,16 +227,13 @@ class NemotronHMoE:
         route_permute(self.c, x, self.w_router, self.bias, b.topk_idx, b.topk_w, b.ws, stream=main)
         pop()
         main.wait_event(zero)
-        if not concurrent:
-            shared_done()
         push("forward")
         if self.nvfp4:
             forward_nvfp4(self.c, x, self.q4["up"], self.q4["down"], b.ws, b.y_acc, stream=main)
         else:
             forward(self.c, x, self.w_up, self.w_down, b.ws, b.y_acc, stream=main)
         pop()
-        if concurrent:
-            shared_done()
+        shared_done()
         if not partial:
             push("finalize")
             finalize(self.c, T, b.y_acc, b.y, stream=main)
