@@ -374,6 +374,9 @@ def kernel_times(blk, xs, b, nb, steps):
     main = torch.cuda.current_stream(blk.device)
     T = xs[0].shape[0]
     names = ["zero_acc", "route", "permute", "experts_up", "experts_down", "shared", "finalize"]
+    # bf16 decode batches (T <= 32): nh_moe_forward runs the up and down
+    # projections as one persistent launch
+    fused = (not blk.nvfp4) and T <= 32 and blk.cfg.dtype == "bf16"
     acc = {n: 0.0 for n in names}
     ev = {n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for n in names}
@@ -416,6 +419,10 @@ def kernel_times(blk, xs, b, nb, steps):
             # up and down run back to back in one call; each is timed as half
             timed("experts_up", lambda: nh.forward_nvfp4(blk.c, x, blk.q4["up"], blk.q4["down"],
                                                           b.ws, yacc, stream=main))
+        elif fused:
+            # decode: nh_moe_forward runs both projections as one launch
+            timed("experts_up", lambda: nh.forward(ce, xe, blk.w_up, blk.w_down, b.ws, yacc,
+                                                    stream=main))
         else:
             timed("experts_up", lambda: nh.experts_up(ce, xe, blk.w_up, b.ws, stream=main))
             timed("experts_down", lambda: nh.experts_down(ce, T, blk.w_down, b.ws, yacc,
@@ -430,12 +437,15 @@ def kernel_times(blk, xs, b, nb, steps):
             timed("finalize", lambda: nh.finalize(blk.c, T, b.y_acc, b.y, stream=main))
         torch.cuda.synchronize(blk.device)
         for n in names:
-            if (n == "shared" and not blk.has_shared) or (n == "experts_down" and blk.nvfp4):
+            if (n == "shared" and not blk.has_shared) or (n == "experts_down" and
+                                                            (blk.nvfp4 or fused)):
                 continue
             acc[n] += ev[n][0].elapsed_time(ev[n][1])
     out = {n: acc[n] / steps for n in names}
-    if blk.nvfp4:
+    if blk.nvfp4 or fused:
         out["experts_up"] = out["experts_down"] = acc["experts_up"] / steps / 2
+    if fused:
+        out["experts_fused"] = acc["experts_up"] / steps
     return out
 
 
@@ -496,9 +506,13 @@ def report(args, cfg, inp, world, steps, elapsed_ms, clk, kern, e2e_ms, blk, ds,
     # (eager), against the burst peaks
     decode = T <= 64
     dom = "experts_up" if kern["experts_up"] >= kern["experts_down"] else "experts_down"
+    if "experts_fused" in kern:
+        dom = "experts_fused"
     if decode:
         d_kern = cycled_mean(ds, ksteps)
         kb = d_kern * expert_bytes + rows * (cfg.HE + cfg.I) * elem
+        if dom == "experts_fused":
+            kb *= 2          # both projections in the launch
         ach = kb / (kern[dom] / 1e3) / 1e9
         peak = pk["hbm_gbs"]
         roof = {"bound": "hbm", "kernel": dom, "achieved": round(ach, 1), "peak": peak,

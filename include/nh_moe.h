@@ -137,6 +137,11 @@ typedef struct {
     size_t x_perm;        /* dtype [rows_alloc, H] x gathered in permuted order
                              (empty when x_direct: the GEMM reads x itself)   */
     size_t h;             /* dtype [rows_alloc, I] relu^2(up) in permuted order */
+    size_t ready;         /* int32 [max_tiles] per tile entry: up-projection tiles
+                             finished, when nh_moe_forward runs both projections
+                             of a decode batch as one launch; zero between
+                             launches (the permute zeroes it, and each such
+                             launch leaves it zero)                            */
     int64_t rows_alloc;   /* T * k rounded up to the tile height                */
     int32_t tile_rows;    /* rows per tile entry of this (cfg, T)               */
     int32_t max_tiles;

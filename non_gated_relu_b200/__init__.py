@@ -63,7 +63,7 @@ class Layout(ctypes.Structure):
     """nh_moe_ws_layout: byte offsets of the routed-path workspace regions."""
     _fields_ = [(n, ctypes.c_size_t) for n in (
         "total_bytes", "status", "logits", "router_w", "counts", "offsets", "chunk_counts", "perm_token",
-        "perm_w", "inv_row", "tiles", "num_tiles", "x_perm", "h")] + [
+        "perm_w", "inv_row", "tiles", "num_tiles", "x_perm", "h", "ready")] + [
         ("rows_alloc", ctypes.c_int64), ("tile_rows", ctypes.c_int32),
         ("max_tiles", ctypes.c_int32), ("n_chunks", ctypes.c_int32), ("swap_ab", ctypes.c_int32),
         ("x_direct", ctypes.c_int32)]

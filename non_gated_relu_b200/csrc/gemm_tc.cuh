@@ -59,6 +59,9 @@ struct TcArgs {
   unsigned int* sched;        // [2]: next tile, CTAs finished; zero on entry, reset on exit
   int k_split;                // >1: each output tile is computed as k_split K slices by
                               // separate tiles (additive epilogues only); 0 or 1: whole K
+  int* ready;                 // fused launch: per tile entry, epilogue warps done with its
+                              // first-GEMM tiles (zeroed by the permute); null otherwise
+  int ready_need;             // second GEMM: count that makes a tile entry's rows ready
 };
 
 constexpr int TQ = 4;         // depth of the tile-id ring between the roles
@@ -156,10 +159,42 @@ __device__ __forceinline__ void epi_elem(const TcArgs& g, int r, int f, float v)
   }
 }
 
+// Wait until a fused launch's first GEMM has finished every tile of tile entry
+// m (its epilogue warps have stored those rows and counted them), then order
+// those generic-proxy stores before this thread's tensor-memory-access loads.
+__device__ __forceinline__ bool wait_ready(const int* ready, int m, int need, const WaitCtl& w) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 0;; ++i) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(ready + m) : "memory");
+    if (v >= need) break;
+    if ((i & 63u) == 63u) {
+      if (*w.abort_flag) return false;
+      if (globaltimer_ns() - t0 > w.timeout_ns) {
+        *w.abort_flag = 1;
+        record_status(w.status, NH_ERR_TIMEOUT, SITE_TC_PRODUCER, m);
+        return false;
+      }
+    }
+  }
+  asm volatile("fence.proxy.async.global;" ::: "memory");
+  return true;
+}
+
+// map_act2 / map_w2 / g2: a second GEMM in the same launch (g2.N > 0), over the
+// same tile entries, whose activations are the first GEMM's output: the decode
+// up projection and down projection as one persistent grid.  Its tiles come
+// after all of the first GEMM's in the scheduler's order, and its producer
+// waits per tile entry until the first GEMM's epilogues have written those
+// rows (g.ready); since every CTA is resident and tiles are handed out in
+// order, the tiles waited on are already running.  The SMs that finish the
+// first GEMM's last tiles early go on to the second GEMM's instead of idling.
 template <bool SWAP, int NT, int STAGES>
 __global__ void __launch_bounds__(THREADS, 1)
     tc_grouped_gemm(const __grid_constant__ CUtensorMap map_act,
-                    const __grid_constant__ CUtensorMap map_w, const TcArgs g) {
+                    const __grid_constant__ CUtensorMap map_w, const TcArgs g,
+                    const __grid_constant__ CUtensorMap map_act2,
+                    const __grid_constant__ CUtensorMap map_w2, const TcArgs g2) {
   using S = Shape<SWAP, NT, STAGES>;
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
@@ -197,6 +232,10 @@ __global__ void __launch_bounds__(THREADS, 1)
     fence_barrier_init();
     tma_prefetch_map(&map_act);
     tma_prefetch_map(&map_w);
+    if (g2.N > 0) {
+      tma_prefetch_map(&map_act2);
+      tma_prefetch_map(&map_w2);
+    }
   }
   if (warp == 1) {
     tmem_alloc(smem_u32(tmem_slot), S::TMEM_COLS);
@@ -212,12 +251,17 @@ __global__ void __launch_bounds__(THREADS, 1)
   const WaitCtl wc{abort_flag, g.status, g.timeout_ns};
 
   const int num_m = g.tiles ? *g.num_tiles : (g.dense_rows + g.tile_rows - 1) / g.tile_rows;
-  const int n_blocks = SWAP ? (g.N + M - 1) / M : (g.N + NT - 1) / NT;
-  const int ks_n = g.k_split > 1 ? g.k_split : 1;
-  const int total = num_m * n_blocks * ks_n;
-  const int nk = g.K / BK;
-  // tile id -> (tile entry m, feature block nb, K slice [kb_lo, kb_hi))
-  auto decode_tile = [&](int tile, int& m, int& nb, int& kb_lo, int& kb_hi) {
+  const bool fused = g2.N > 0;
+  auto n_blocks_of = [&](const TcArgs& a) { return SWAP ? (a.N + M - 1) / M : (a.N + NT - 1) / NT; };
+  auto ks_of = [&](const TcArgs& a) { return a.k_split > 1 ? a.k_split : 1; };
+  const int total1 = num_m * n_blocks_of(g) * ks_of(g);
+  const int total = total1 + (fused ? num_m * n_blocks_of(g2) * ks_of(g2) : 0);
+  // tile id -> (GEMM ph, tile entry m, feature block nb, K slice [kb_lo, kb_hi))
+  auto decode_tile = [&](int tile, int& ph, int& m, int& nb, int& kb_lo, int& kb_hi) {
+    ph = tile >= total1 ? 1 : 0;
+    const TcArgs& a = ph ? g2 : g;
+    if (ph) tile -= total1;
+    const int ks_n = ks_of(a), n_blocks = n_blocks_of(a), nk = a.K / BK;
     const int ks = tile % ks_n, rest = tile / ks_n;
     m = rest / n_blocks;
     nb = rest - m * n_blocks;
@@ -242,23 +286,30 @@ __global__ void __launch_bounds__(THREADS, 1)
       tile_q[q] = tile;
       mbar_arrive(tq_full_bar(q));
       if (tile < 0) break;
-      int m, nb, kb_lo, kb_hi;
-      decode_tile(tile, m, nb, kb_lo, kb_hi);
-      const int4 ent = tile_entry_of(g, m);
+      int ph, m, nb, kb_lo, kb_hi;
+      decode_tile(tile, ph, m, nb, kb_lo, kb_hi);
+      const TcArgs& a = ph ? g2 : g;
+      const CUtensorMap* mact = ph ? &map_act2 : &map_act;
+      const CUtensorMap* mw = ph ? &map_w2 : &map_w;
+      const int4 ent = tile_entry_of(a, m);
+      if (ph && !wait_ready(g.ready, m, g2.ready_need, wc)) {
+        ok = false;
+        break;
+      }
       for (int kb = kb_lo; kb < kb_hi; ++kb) {
         if (!mbar_wait(empty_bar(stage), phase ^ 1u, wc, SITE_TC_PRODUCER)) {
           ok = false;
           break;
         }
         const uint32_t sa = base + stage * S::STAGE_BYTES, sb = sa + S::A_BYTES;
-        const int ka = g.a_kwrap ? (kb * BK) % g.a_kwrap : kb * BK;
+        const int ka = a.a_kwrap ? (kb * BK) % a.a_kwrap : kb * BK;
         mbar_arrive_expect_tx(full_bar(stage), S::STAGE_BYTES);
         if (!SWAP) {
-          tma_load_2d(sa, &map_act, full_bar(stage), ka, ent.y);
-          tma_load_3d(sb, &map_w, full_bar(stage), kb * BK, nb * NT, ent.x);
+          tma_load_2d(sa, mact, full_bar(stage), ka, ent.y);
+          tma_load_3d(sb, mw, full_bar(stage), kb * BK, nb * NT, ent.x);
         } else {
-          tma_load_3d(sa, &map_w, full_bar(stage), kb * BK, nb * M, ent.x);
-          tma_load_2d(sb, &map_act, full_bar(stage), ka, g.row_token ? 0 : ent.y);
+          tma_load_3d(sa, mw, full_bar(stage), kb * BK, nb * M, ent.x);
+          tma_load_2d(sb, mact, full_bar(stage), ka, a.row_token ? 0 : ent.y);
         }
         ++issued;
         if (++stage == STAGES) {
@@ -289,8 +340,8 @@ __global__ void __launch_bounds__(THREADS, 1)
       const int tile = tile_q[q];
       mbar_arrive(tq_empty_bar(q));
       if (tile < 0) break;
-      int m, nb, kb_lo, kb_hi;
-      decode_tile(tile, m, nb, kb_lo, kb_hi);
+      int ph, m, nb, kb_lo, kb_hi;
+      decode_tile(tile, ph, m, nb, kb_lo, kb_hi);
       const int acc = it & 1;
       const uint32_t aph = (uint32_t)((it >> 1) & 1);
       if (!mbar_wait(tempty_bar(acc), aph ^ 1u, wc, SITE_TC_MMA)) {
@@ -298,7 +349,7 @@ __global__ void __launch_bounds__(THREADS, 1)
         break;
       }
       tc_fence_after();
-      const int n_mma = SWAP ? NT : min(NT, g.N - nb * NT);
+      const int n_mma = SWAP ? NT : min(NT, (ph ? g2 : g).N - nb * NT);
       const uint32_t idesc = make_idesc_bf16(M, n_mma);
       const uint32_t d_tmem = tmem_base + (uint32_t)(acc * S::ACC_COLS);
       (void)m;
@@ -348,49 +399,56 @@ __global__ void __launch_bounds__(THREADS, 1)
       ok = __shfl_sync(0xffffffffu, ok, 0);
       tile = __shfl_sync(0xffffffffu, tile, 0);
       if (!ok || tile < 0) break;
-      int m, nb, kb_lo, kb_hi;
-      decode_tile(tile, m, nb, kb_lo, kb_hi);
+      int ph, m, nb, kb_lo, kb_hi;
+      decode_tile(tile, ph, m, nb, kb_lo, kb_hi);
+      const TcArgs& a = ph ? g2 : g;
       const int acc = it & 1;
       const uint32_t aph = (uint32_t)((it >> 1) & 1);
       if (lane == 0) ok = mbar_wait(tfull_bar(acc), aph, wc, SITE_TC_EPILOGUE) ? 1 : 0;
       ok = __shfl_sync(0xffffffffu, ok, 0);
       if (!ok) break;
       tc_fence_after();
-      const int4 ent = tile_entry_of(g, m);
+      const int4 ent = tile_entry_of(a, m);
       const uint32_t tq = tmem_base + ((uint32_t)(q * 32) << 16) + (uint32_t)(acc * S::ACC_COLS);
       if (!SWAP) {
         const int row = q * 32 + lane;
         const bool valid = row < ent.z;
         const int n0 = nb * NT;
-        const int n_eff = min(NT, g.N - n0);
+        const int n_eff = min(NT, a.N - n0);
         for (int c = 0; c < n_eff; c += 32) {
           float v[32];
           tmem_ld_x32(tq + (uint32_t)c, v);
-          if (valid) epi_row32(g, ent.y + row, n0 + c, v);
+          if (valid) epi_row32(a, ent.y + row, n0 + c, v);
         }
       } else {
         const int f = nb * M + q * 32 + lane;
-        const bool valid = f < g.N;
+        const bool valid = f < a.N;
 #pragma unroll
         for (int c = 0; c < NT; c += 16) {
           float v[16];
           tmem_ld_x16(tq + (uint32_t)c, v);
-          if (g.row_token) {
+          if (a.row_token) {
             // accumulator columns are tokens: row r of the expert takes column row_token[r]
             for (int j = 0; j < ent.z; ++j) {
-              const int t = g.row_token[ent.y + j] - c;
+              const int t = a.row_token[ent.y + j] - c;
               if (t < 0 || t >= 16) continue;
               float val = 0.f;
 #pragma unroll
               for (int u = 0; u < 16; ++u) val = (u == t) ? v[u] : val;
-              if (valid) epi_elem(g, ent.y + j, f, val);
+              if (valid) epi_elem(a, ent.y + j, f, val);
             }
           } else {
 #pragma unroll
             for (int j = 0; j < 16; ++j)
-              if (valid && c + j < ent.z) epi_elem(g, ent.y + c + j, f, v[j]);
+              if (valid && c + j < ent.z) epi_elem(a, ent.y + c + j, f, v[j]);
           }
         }
+      }
+      if (fused && ph == 0) {
+        // this warp's rows of the tile are stored: count them for the second GEMM
+        __threadfence();
+        __syncwarp();
+        if (lane == 0) atomicAdd(g.ready + m, 1);
       }
       tc_fence_before();
       mbar_arrive(tempty_bar(acc));
@@ -404,11 +462,14 @@ __global__ void __launch_bounds__(THREADS, 1)
     tmem_dealloc(tmem_base, S::TMEM_COLS);
   }
   if (threadIdx.x == 0) {
-    // the last CTA to finish resets the scheduler for the next launch
+    // the last CTA to finish resets the scheduler (and a fused launch's ready
+    // counters) for the next launch
     __threadfence();
     if (atomicAdd(g.sched + 1, 1u) == gridDim.x - 1) {
       atomicExch(g.sched, 0u);
       atomicExch(g.sched + 1, 0u);
+      if (fused)
+        for (int i = 0; i < num_m; ++i) g.ready[i] = 0;
     }
   }
 }

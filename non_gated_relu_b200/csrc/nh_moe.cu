@@ -205,6 +205,7 @@ static nh_status make_plan(const nh_moe_config* c, int64_t T, Plan* p) {
   L.num_tiles = take(4);
   L.x_perm = take(L.x_direct ? 0 : (size_t)rows * p->H * p->elem);
   L.h = take((size_t)rows * p->I * p->elem);
+  L.ready = take((size_t)L.max_tiles * 4);
   L.total_bytes = o;
   return NH_OK;
 }
@@ -254,6 +255,8 @@ static PermuteOut permute_out(void* ws, const nh_moe_ws_layout& L, int* status) 
   o.status = status;
   o.sched_zero = reinterpret_cast<unsigned int*>(status + SCHED_UP);
   o.gather = L.x_direct ? 0 : 1;
+  o.ready = at<int>(ws, L.ready);
+  o.n_ready = L.max_tiles;
   return o;
 }
 
@@ -447,12 +450,7 @@ struct GemmCall {
   int k_split;          // K slices per output tile (additive epilogues; 0/1 = none)
 };
 
-template <bool SWAP, int NT, int STAGES>
-static nh_status launch_tc(const GemmCall& c, int dev, cudaStream_t st) {
-  using S = tc::Shape<SWAP, NT, STAGES>;
-  CUtensorMap ma, mw;
-  NH_TRY(map_2d(&ma, c.A, c.a_kwrap ? c.a_kwrap : c.K, c.rows, SWAP ? NT : tc::M));
-  NH_TRY(map_3d(&mw, c.W, c.K, c.N, c.n_exp, SWAP ? tc::M : NT));
+static tc::TcArgs tc_args(const GemmCall& c) {
   tc::TcArgs g{};
   g.tiles = c.tiles;
   g.num_tiles = c.num_tiles;
@@ -471,15 +469,65 @@ static nh_status launch_tc(const GemmCall& c, int dev, cudaStream_t st) {
   g.timeout_ns = timeout_ns();
   g.sched = c.sched;
   g.k_split = c.k_split;
-  if (!g.sched) return fail(NH_ERR_INVALID_ARG, "internal: no tile scheduler counters");
+  return g;
+}
+
+static nh_status check_tc_call(const GemmCall& c) {
+  if (!c.sched) return fail(NH_ERR_INVALID_ARG, "internal: no tile scheduler counters");
   if (c.k_split > 1 && c.epi != EPI_DOWN_COMBINE && c.epi != EPI_ACC_F32)
     return fail(NH_ERR_INVALID_ARG, "internal: K slices need an additive epilogue");
+  return NH_OK;
+}
+
+// output tiles of one call: tile entries x feature blocks x K slices
+template <bool SWAP, int NT>
+static int64_t tc_work(const GemmCall& c) {
   const int n_blocks = SWAP ? (c.N + tc::M - 1) / tc::M : (c.N + NT - 1) / NT;
   const int64_t m_max = c.tiles ? c.max_tiles : (c.rows + c.tile_rows - 1) / c.tile_rows;
-  const int64_t work = m_max * n_blocks * (c.k_split > 1 ? c.k_split : 1);
+  return m_max * n_blocks * (c.k_split > 1 ? c.k_split : 1);
+}
+
+template <bool SWAP, int NT, int STAGES>
+static nh_status launch_tc(const GemmCall& c, int dev, cudaStream_t st) {
+  using S = tc::Shape<SWAP, NT, STAGES>;
+  CUtensorMap ma, mw;
+  NH_TRY(map_2d(&ma, c.A, c.a_kwrap ? c.a_kwrap : c.K, c.rows, SWAP ? NT : tc::M));
+  NH_TRY(map_3d(&mw, c.W, c.K, c.N, c.n_exp, SWAP ? tc::M : NT));
+  NH_TRY(check_tc_call(c));
+  const tc::TcArgs g = tc_args(c);
+  const int grid = (int)std::min<int64_t>(tc_work<SWAP, NT>(c), g_sm_count[dev]);
+  if (grid <= 0) return NH_OK;
+  const tc::TcArgs none{};
+  NH_TRY((launch_k("tc_grouped_gemm", tc::tc_grouped_gemm<SWAP, NT, STAGES>, dim3(grid), dim3(tc::THREADS), S::SMEM, st, ma, mw, g, ma, mw, none)));
+  return launch_check("tc_grouped_gemm");
+}
+
+// Decode up and down projections as one persistent launch (weights on the MMA
+// M side): c1 writes h, c2 reads it; c2's tiles of a tile entry start once
+// the 4 epilogue warps of each of c1's feature blocks of that entry have
+// counted their rows into `ready` (zeroed by the permute).
+template <int NT, int STAGES>
+static nh_status launch_tc_fused(const GemmCall& c1, const GemmCall& c2, int* ready, int dev,
+                                 cudaStream_t st) {
+  using S = tc::Shape<true, NT, STAGES>;
+  CUtensorMap ma1, mw1, ma2, mw2;
+  NH_TRY(map_2d(&ma1, c1.A, c1.a_kwrap ? c1.a_kwrap : c1.K, c1.rows, NT));
+  NH_TRY(map_3d(&mw1, c1.W, c1.K, c1.N, c1.n_exp, tc::M));
+  NH_TRY(map_2d(&ma2, c2.A, c2.a_kwrap ? c2.a_kwrap : c2.K, c2.rows, NT));
+  NH_TRY(map_3d(&mw2, c2.W, c2.K, c2.N, c2.n_exp, tc::M));
+  NH_TRY(check_tc_call(c1));
+  NH_TRY(check_tc_call(c2));
+  if (c1.k_split > 1 || c1.tiles != c2.tiles)
+    return fail(NH_ERR_INVALID_ARG, "internal: fused GEMMs share the tile table, whole-K first");
+  tc::TcArgs g1 = tc_args(c1), g2 = tc_args(c2);
+  g1.ready = ready;
+  g2.ready = ready;
+  g2.ready_need = 4 * ((c1.N + tc::M - 1) / tc::M);
+  const int64_t work = tc_work<true, NT>(c1) + tc_work<true, NT>(c2);
   const int grid = (int)std::min<int64_t>(work, g_sm_count[dev]);
   if (grid <= 0) return NH_OK;
-  NH_TRY((launch_k("tc_grouped_gemm", tc::tc_grouped_gemm<SWAP, NT, STAGES>, dim3(grid), dim3(tc::THREADS), S::SMEM, st, ma, mw, g)));
+  NH_TRY((launch_k("tc_grouped_gemm", tc::tc_grouped_gemm<true, NT, STAGES>, dim3(grid),
+                   dim3(tc::THREADS), S::SMEM, st, ma1, mw1, g1, ma2, mw2, g2)));
   return launch_check("tc_grouped_gemm");
 }
 
@@ -1101,24 +1149,10 @@ nh_status nh_moe_route_permute(const nh_moe_config* cfg, int64_t T, const void* 
                   static_cast<const float*>(x), w_router, a, p.H, done, o);
 }
 
-static nh_status experts_phase(const nh_moe_config* cfg, int64_t T, const void* x, const void* w,
-                               void* ws, size_t ws_bytes, float* y_acc, void* stream,
-                               bool up_phase, const nh_nvfp4_weight* wq = nullptr) {
-  NH_TRY(no_latent(cfg, "routed experts"));
-  Plan p;
-  NH_TRY(make_plan(cfg, T, &p));
-  NH_TRY(check_ws(p, ws, ws_bytes));
-  const bool nvfp4 = cfg->weight_format == NH_WEIGHTS_NVFP4;
-  if (nvfp4 != (wq != nullptr))
-    return fail(NH_ERR_INVALID_ARG, nvfp4 ? "config has NVFP4 weights: use the _nvfp4 entry points"
-                                          : "config has native weights: use nh_moe_forward");
-  if (T == 0) return NH_OK;
-  if (!nvfp4) NH_TRY(check_ptr(w, up_phase ? "w_up" : "w_down"));
-  if (up_phase) NH_TRY(check_ptr(x, "x"));
-  else NH_TRY(check_ptr(y_acc, "y_acc"));
-  int dev;
-  NH_TRY(device_setup(&dev));
-  cudaStream_t st = static_cast<cudaStream_t>(stream);
+// GemmCall of one routed projection on the workspace: up (x -> h, relu^2) or
+// down (h -> y_acc, the weighted combine)
+static GemmCall routed_call(const Plan& p, void* ws, int64_t T, const void* x, const void* w,
+                            float* y_acc, bool up_phase, bool nvfp4) {
   const nh_moe_ws_layout& L = p.lay;
   GemmCall c{};
   c.rows = p.rows;
@@ -1160,6 +1194,28 @@ static nh_status experts_phase(const nh_moe_config* cfg, int64_t T, const void* 
     // the combine adds both slices into y_acc
     if (L.swap_ab && !nvfp4 && p.I >= 2 * tc::BK) c.k_split = 2;
   }
+  return c;
+}
+
+static nh_status experts_phase(const nh_moe_config* cfg, int64_t T, const void* x, const void* w,
+                               void* ws, size_t ws_bytes, float* y_acc, void* stream,
+                               bool up_phase, const nh_nvfp4_weight* wq = nullptr) {
+  NH_TRY(no_latent(cfg, "routed experts"));
+  Plan p;
+  NH_TRY(make_plan(cfg, T, &p));
+  NH_TRY(check_ws(p, ws, ws_bytes));
+  const bool nvfp4 = cfg->weight_format == NH_WEIGHTS_NVFP4;
+  if (nvfp4 != (wq != nullptr))
+    return fail(NH_ERR_INVALID_ARG, nvfp4 ? "config has NVFP4 weights: use the _nvfp4 entry points"
+                                          : "config has native weights: use nh_moe_forward");
+  if (T == 0) return NH_OK;
+  if (!nvfp4) NH_TRY(check_ptr(w, up_phase ? "w_up" : "w_down"));
+  if (up_phase) NH_TRY(check_ptr(x, "x"));
+  else NH_TRY(check_ptr(y_acc, "y_acc"));
+  int dev;
+  NH_TRY(device_setup(&dev));
+  cudaStream_t st = static_cast<cudaStream_t>(stream);
+  const GemmCall c = routed_call(p, ws, T, x, w, y_acc, up_phase, nvfp4);
   if (nvfp4) return run_gemm_q4(c, wq, dev, st);
   return run_gemm(p, c, dev, st);
 }
@@ -1185,6 +1241,19 @@ nh_status nh_moe_forward(const nh_moe_config* cfg, int64_t T, const void* x, con
   NH_TRY(check_ptr(w_up, "w_up"));
   NH_TRY(check_ptr(w_down, "w_down"));
   NH_TRY(check_ptr(y_acc, "y_acc"));
+  const nh_moe_ws_layout& L = p.lay;
+  if (p.bf16 && L.x_direct && cfg->weight_format == NH_WEIGHTS_NATIVE && !cfg->latent_size &&
+      (L.tile_rows == 16 || L.tile_rows == 32)) {
+    // decode: both projections in one persistent launch
+    int dev;
+    NH_TRY(device_setup(&dev));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const GemmCall up = routed_call(p, ws, T, x, w_up, y_acc, true, false);
+    const GemmCall down = routed_call(p, ws, T, x, w_down, y_acc, false, false);
+    int* ready = at<int>(ws, L.ready);
+    if (L.tile_rows == 16) return launch_tc_fused<16, 8>(up, down, ready, dev, st);
+    return launch_tc_fused<32, 8>(up, down, ready, dev, st);
+  }
   NH_TRY(nh_moe_experts_up(cfg, T, x, w_up, ws, ws_bytes, stream));
   return nh_moe_experts_down(cfg, T, w_down, ws, ws_bytes, y_acc, stream);
 }

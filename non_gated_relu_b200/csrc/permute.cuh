@@ -264,10 +264,13 @@ __device__ __forceinline__ void permute_block(
     int tile_rows, int max_tiles, int32_t* __restrict__ counts, int32_t* __restrict__ offsets,
     int4* __restrict__ tiles, int32_t* __restrict__ num_tiles, int32_t* __restrict__ perm_token,
     float* __restrict__ perm_w, int32_t* __restrict__ inv_row, Tin* __restrict__ x_perm,
-    int* status, unsigned int* sched_zero, int* cnt, int* pos, int* warp_sums, bool gather) {
+    int* status, unsigned int* sched_zero, int* cnt, int* pos, int* warp_sums, bool gather,
+    int* ready_zero, int n_ready) {
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int n = T * k;
   if (threadIdx.x < 4) sched_zero[threadIdx.x] = 0u;  // up/down GEMM tile schedulers
+  // per-tile-entry counters of a fused up + down launch
+  for (int i = threadIdx.x; i < n_ready; i += blockDim.x) ready_zero[i] = 0;
   for (int e = threadIdx.x; e < E; e += blockDim.x) cnt[e] = 0;
   __syncthreads();
   for (int a = threadIdx.x; a < n; a += blockDim.x) {
@@ -339,6 +342,8 @@ struct PermuteOut {
   int* status;
   unsigned int* sched_zero;
   int gather;   // 0: no x_perm (decode orientation reads x directly)
+  int* ready;   // [n_ready] zeroed: the fused decode GEMM's per-entry counters
+  int n_ready;
 };
 
 // Whole permute in one block for T <= PERM_CHUNK tokens (decode).
@@ -354,7 +359,7 @@ __global__ void __launch_bounds__(512) permute_small(const int32_t* __restrict__
   pdl_trigger();
   permute_block(idx, w, x, T, k, E, H, o.tile_rows, o.max_tiles, o.counts, o.offsets, o.tiles,
                 o.num_tiles, o.perm_token, o.perm_w, o.inv_row, static_cast<Tin*>(o.x_perm),
-                o.status, o.sched_zero, sm, sm + E, warp_sums, o.gather != 0);
+                o.status, o.sched_zero, sm, sm + E, warp_sums, o.gather != 0, o.ready, o.n_ready);
 }
 
 }  // namespace nh

@@ -44,7 +44,7 @@ __global__ void __launch_bounds__(256) route_permute_small(const Tin* __restrict
   __syncthreads();
   permute_block(s_idx, s_w, x, T, k, E, H, o.tile_rows, o.max_tiles, o.counts, o.offsets, o.tiles,
                 o.num_tiles, o.perm_token, o.perm_w, o.inv_row, static_cast<Tin*>(o.x_perm),
-                o.status, o.sched_zero, cnt, pos, warp_sums, o.gather != 0);
+                o.status, o.sched_zero, cnt, pos, warp_sums, o.gather != 0, o.ready, o.n_ready);
   if (threadIdx.x == 0) *done = 0u;
 }
 

@@ -158,6 +158,36 @@ def test_host_pipeline_matches_eager(name):
     assert seen == list(range(len(batches)))
 
 
+@pytest.mark.parametrize("name", ["small_swap16", "small_swap32"])
+def test_fused_decode_forward_matches_two_launches(name):
+    """For decode batches nh_moe_forward runs the up and down projections as one
+    persistent launch (the down tiles of a tile entry wait for its up tiles).
+    Called twice after one permute, it gives the y_acc of the separate
+    experts_up + experts_down launches, up to float32 summation order."""
+    import non_gated_relu_b200 as nh
+    inp = synth.make_inputs(SMALL[name])
+    blk = make_block(inp)
+    x = to_dev(inp.x)
+    T = x.shape[0]
+    b = blk.buffers(T)
+    blk.forward(x, b)
+    fused = [torch.zeros_like(b.y_acc) for _ in range(2)]
+    for acc in fused:
+        nh.forward(blk.c, x, blk.w_up, blk.w_down, b.ws, acc)
+    two = torch.zeros_like(b.y_acc)
+    nh.experts_up(blk.c, x, blk.w_up, b.ws)
+    nh.experts_down(blk.c, T, blk.w_down, b.ws, two)
+    torch.cuda.synchronize()
+    assert blk.check(T) == 0
+    ref = two.cpu().numpy()
+    assert np.abs(ref).max() > 0
+    for acc in fused:
+        assert_same_up_to_sum_order(acc.cpu().numpy(), ref, "f32")
+    L = nh.workspace_layout(blk.c, T)
+    ready = b.ws.view(torch.uint8)[L.ready:L.ready + 4 * L.max_tiles]
+    assert (ready == 0).all(), "a fused launch leaves its ready counters zero"
+
+
 # ----------------------------------------------------------------------------- full size
 FULL = synth.CONFIG_ORDER
 
