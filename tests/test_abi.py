@@ -84,7 +84,7 @@ def test_workspace_layout(name):
                ("offsets", (cfg.E + 1) * 4), ("chunk_counts", L.n_chunks * cfg.E * 4),
                ("perm_token", rows * 4), ("perm_w", rows * 4), ("inv_row", rows * 4),
                ("tiles", L.max_tiles * 16), ("num_tiles", 4), ("x_perm", 0 if L.x_direct else rows * cfg.H * elem),
-               ("h", rows * cfg.I * elem)]
+               ("h", rows * cfg.I * elem), ("ready", L.max_tiles * 4)]
     spans = sorted((getattr(L, n), getattr(L, n) + sz, n) for n, sz in regions)
     for (a0, a1, an), (b0, b1, bn) in zip(spans, spans[1:]):
         assert a1 <= b0, (an, bn)
