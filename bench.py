@@ -374,9 +374,9 @@ def kernel_times(blk, xs, b, nb, steps):
     main = torch.cuda.current_stream(blk.device)
     T = xs[0].shape[0]
     names = ["zero_acc", "route", "permute", "experts_up", "experts_down", "shared", "finalize"]
-    # bf16 decode batches (T <= 32): nh_moe_forward runs the up and down
-    # projections as one persistent launch
-    fused = (not blk.nvfp4) and T <= 32 and blk.cfg.dtype == "bf16"
+    # decode batches (T <= 32, bf16 or NVFP4 experts): nh_moe_forward[_nvfp4]
+    # runs the up and down projections as one launch
+    fused = T <= 32 and (blk.nvfp4 or blk.cfg.dtype == "bf16")
     acc = {n: 0.0 for n in names}
     ev = {n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for n in names}
@@ -419,7 +419,7 @@ def kernel_times(blk, xs, b, nb, steps):
             # up and down run back to back in one call; each is timed as half
             timed("experts_up", lambda: nh.forward_nvfp4(blk.c, x, blk.q4["up"], blk.q4["down"],
                                                           b.ws, yacc, stream=main))
-        elif fused:
+        elif fused and not blk.nvfp4:
             # decode: nh_moe_forward runs both projections as one launch
             timed("experts_up", lambda: nh.forward(ce, xe, blk.w_up, blk.w_down, b.ws, yacc,
                                                     stream=main))
@@ -452,22 +452,23 @@ def kernel_times(blk, xs, b, nb, steps):
 def launches_per_step(cfg):
     """Kernels of one block call (memsets excluded), as nh_moe.cu launches them."""
     T = cfg.T
+    # routed up and down: one launch for decode batches (bf16 or NVFP4 experts)
+    experts = 1 if T <= 32 and (cfg.dtype == "bf16" or cfg.weight_format == "nvfp4") else 2
+    shared = 2 if cfg.n_shared_experts else 0
     if getattr(cfg, "latent_size", 0):
-        # route (no fused permute), fc1, permute, up, down, finalize, fc2, cast, shared
+        # route, fc1, permute, experts, finalize of the latent sum, fc2, cast, shared
         n = 1 if T <= 32 else (3 if cfg.dtype == "bf16" and cfg.E % 32 == 0 else 2)
-        n += 1 + (1 if T <= 256 else 4) + 2 + 1 + 1 + 1
-        return n + (2 if cfg.n_shared_experts else 0)
+        n += 1 + (1 if T <= 256 else 4) + experts + 1 + 1 + 1
+        return n + shared
     if T <= 32:
-        n = 1                                   # fused router
-    elif cfg.dtype == "bf16" and cfg.E % 32 == 0:
-        n = 3                                   # weight split, tensor-core logits, select
+        n = 1                                   # router and permute in one launch
     else:
-        n = 2                                   # logits, select
-    n += 1 if T <= 256 else 4                   # permute (fused, or hist/scan/scatter/gather)
-    n += 2                                      # routed up, routed down
-    n += 2 if cfg.n_shared_experts else 0       # shared up, shared down
-    n += 1                                      # finalize
-    return n
+        if cfg.dtype == "bf16" and cfg.E % 32 == 0:
+            n = 3                               # weight split, tensor-core logits, select
+        else:
+            n = 2                               # logits, select
+        n += 1 if T <= 256 else 4               # permute (one block, or hist/scan/scatter/gather)
+    return n + experts + shared + 1             # + finalize
 
 
 def distinct_experts(cfg, idx):

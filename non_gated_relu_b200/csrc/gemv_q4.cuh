@@ -53,14 +53,32 @@ __device__ __forceinline__ void mma_bf16_16816(float* c, uint32_t a0, uint32_t a
 // scale multipliers of the run's groups, and the activation row of token gq.
 // Word w of the run holds k-tiles 2w and 2w + 1; even and odd k-tiles go to
 // two accumulators (c0, c1) so consecutive MMAs do not wait on each other.
+// Activation loads: through the read-only path, or (`coherent`) from L2 for
+// activations that an earlier part of the same launch wrote.
+__device__ __forceinline__ uint2 ld_act2(const __nv_bfloat16* p, bool coherent) {
+  if (!coherent) return __ldg(reinterpret_cast<const uint2*>(p));
+  uint2 v;
+  asm volatile("ld.global.cg.v2.u32 {%0, %1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
+  return v;
+}
+__device__ __forceinline__ uint4 ld_act4(const __nv_bfloat16* p, bool coherent) {
+  if (!coherent) return __ldg(reinterpret_cast<const uint4*>(p));
+  uint4 v;
+  asm volatile("ld.global.cg.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(v.x), "=r"(v.y), "=r"(v.z), "=r"(v.w)
+               : "l"(p));
+  return v;
+}
+
 template <int BK>
 __device__ __forceinline__ void block_mma(const uint32_t* ca, const uint32_t* cb,
                                           const uint32_t* ma, const uint32_t* mb,
-                                          const __nv_bfloat16* act, float* c0, float* c1) {
+                                          const __nv_bfloat16* act, float* c0, float* c1,
+                                          bool coherent = false) {
   constexpr int KT = BK / 16;
   uint2 bv[KT];
 #pragma unroll
-  for (int kt = 0; kt < KT; ++kt) bv[kt] = __ldg(reinterpret_cast<const uint2*>(act + 4 * kt));
+  for (int kt = 0; kt < KT; ++kt) bv[kt] = ld_act2(act + 4 * kt, coherent);
 #pragma unroll
   for (int w = 0; w < KT / 2; ++w) {
     uint32_t pa[4], pb[4];
@@ -182,27 +200,74 @@ __global__ void __launch_bounds__(WARPS * 32, 3) q4_gemv_splitk(const Args a) {
   }
 }
 
+// Wait until every up-projection warp task of tile entry m has counted itself
+// (a fused launch); false if the launch's status word already holds an error
+// or the wait runs out (then it records NH_ERR_TIMEOUT).
+__device__ __forceinline__ bool wait_entry_ready(const int* ready, int m, int need, int* status,
+                                                 uint64_t timeout_ns) {
+  const uint64_t t0 = globaltimer_ns();
+  for (uint32_t i = 0;; ++i) {
+    int v;
+    asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(ready + m) : "memory");
+    if (v >= need) return true;
+    if ((i & 63u) == 63u) {
+      if (status && *reinterpret_cast<volatile int*>(status) != 0) return false;
+      if (globaltimer_ns() - t0 > timeout_ns) {
+        record_status(status, NH_ERR_TIMEOUT, SITE_GEMV_STAGE, m);
+        return false;
+      }
+    }
+  }
+}
+
 // Many tasks (the routed experts).  Warp tasks (tile entry, 16 weight rows)
 // are dealt round-robin over all warps of the grid; each warp runs the whole
 // K with the next block's codes, scale bytes and activation run in flight.  An entry with more than 8 tokens
 // takes one pass per 8 tokens (the codes are re-read from L1/L2).
+//
+// With a2.g.N > 0 the launch also runs a second GEMM over the same tile
+// entries whose activations are the first one's output (the decode up and
+// down projections): warps then fetch tasks from a counter (a.g.sched), all
+// of the first GEMM's before any of the second's; a warp that finishes an up
+// task counts it into a.g.ready[m], and a down task of entry m first waits
+// for a2.g.ready_need counts (the up tasks it waits on were handed out
+// earlier, to running warps, and wait on nothing) and reads h from L2.
 template <int NT>
-__global__ void __launch_bounds__(WARPS * 32, 2) q4_gemv_rows(const Args a) {
-  const tc::TcArgs& g = a.g;
+__global__ void __launch_bounds__(WARPS * 32, 2) q4_gemv_rows(const Args a1, const Args a2) {
   pdl_wait();
   pdl_trigger();
   const int lane = threadIdx.x & 31;
   const int gq = lane >> 2, tq = lane & 3;
-  const int num_m = g.tiles ? *g.num_tiles : (g.dense_rows + g.tile_rows - 1) / g.tile_rows;
-  const int n_rb = g.N / MT;
-  const int total = num_m * n_rb;
-  const int K = g.K;
-  const int nkb = K / 128, tail = K % 128;
-  const size_t row_bytes = (size_t)K / 2;
-  const __nv_bfloat16* A = static_cast<const __nv_bfloat16*>(a.A);
+  const bool fused = a2.g.N > 0;
+  const int num_m =
+      a1.g.tiles ? *a1.g.num_tiles : (a1.g.dense_rows + a1.g.tile_rows - 1) / a1.g.tile_rows;
+  const int total1 = num_m * (a1.g.N / MT);
+  const int total = total1 + (fused ? num_m * (a2.g.N / MT) : 0);
   const int nwarps = gridDim.x * WARPS;
-  for (int task = blockIdx.x * WARPS + (threadIdx.x >> 5); task < total; task += nwarps) {
-    const int m = task / n_rb, rb = task - m * n_rb;
+  int task = fused ? 0 : blockIdx.x * WARPS + (threadIdx.x >> 5);
+  for (;; task += nwarps) {
+    if (fused) {
+      int t = 0;
+      if (lane == 0) t = (int)atomicAdd(a1.g.sched, 1u);
+      task = __shfl_sync(0xffffffffu, t, 0);
+    }
+    if (task >= total) break;
+    const bool second = task >= total1;
+    const Args& a = second ? a2 : a1;
+    const tc::TcArgs& g = a.g;
+    const int t = second ? task - total1 : task;
+    const int n_rb = g.N / MT;
+    const int m = t / n_rb, rb = t - m * n_rb;
+    if (second) {
+      int ok = 1;
+      if (lane == 0)
+        ok = wait_entry_ready(a1.g.ready, m, a2.g.ready_need, g.status, g.timeout_ns) ? 1 : 0;
+      if (!__shfl_sync(0xffffffffu, ok, 0)) break;
+    }
+    const int K = g.K;
+    const int nkb = K / 128, tail = K % 128;
+    const size_t row_bytes = (size_t)K / 2;
+    const __nv_bfloat16* A = static_cast<const __nv_bfloat16*>(a.A);
     const int r0 = rb * MT;
     const int4 ent = tc::tile_entry_of(g, m);
     const int count = ent.z;
@@ -223,9 +288,9 @@ __global__ void __launch_bounds__(WARPS * 32, 2) q4_gemv_rows(const Args a) {
       auto fetch = [&](int kb, uint4& fa, uint4& fb, uint4* fx, uint32_t& fsa, uint32_t& fsb) {
         fa = __ldg(reinterpret_cast<const uint4*>(ca_p + (size_t)kb * 64 + 16 * tq));
         fb = __ldg(reinterpret_cast<const uint4*>(cb_p + (size_t)kb * 64 + 16 * tq));
-        const uint4* xr = reinterpret_cast<const uint4*>(act + kb * 128 + 32 * tq);
+        const __nv_bfloat16* xr = act + kb * 128 + 32 * tq;
 #pragma unroll
-        for (int u = 0; u < 4; ++u) fx[u] = __ldg(xr + u);
+        for (int u = 0; u < 4; ++u) fx[u] = ld_act4(xr + 8 * u, second);
         // thread tq's 32 features are scale groups 8 kb + 2 tq and + 1
         fsa = *reinterpret_cast<const uint16_t*>(sa_p + kb * 8 + 2 * tq);
         fsb = *reinterpret_cast<const uint16_t*>(sb_p + kb * 8 + 2 * tq);
@@ -253,13 +318,31 @@ __global__ void __launch_bounds__(WARPS * 32, 2) q4_gemv_rows(const Args a) {
         const uint32_t ma[1] = {q4::scale_mult(sa_p[nkb * 8 + tq])};
         const uint32_t mb[1] = {q4::scale_mult(sb_p[nkb * 8 + tq])};
         const uint32_t cwa[2] = {ta.x, ta.y}, cwb[2] = {tb.x, tb.y};
-        block_mma<64>(cwa, cwb, ma, mb, act + nkb * 128 + 16 * tq, c0, c1);
+        block_mma<64>(cwa, cwb, ma, mb, act + nkb * 128 + 16 * tq, c0, c1, second);
       }
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const int jj = n0 + 2 * tq + (i & 1);
         const int f = r0 + gq + (i >> 1) * 8;
         if (jj < count) tc::epi_elem(g, ent.y + jj, f, (c0[i] + c1[i]) * gs);
+      }
+    }
+    if (fused && !second) {
+      // this warp's rows of h are stored: count the task for the down projection
+      __threadfence();
+      __syncwarp();
+      if (lane == 0) atomicAdd(a1.g.ready + m, 1);
+    }
+  }
+  if (fused) {
+    // the last CTA to finish resets the task counter and the ready counters
+    __syncthreads();
+    if (threadIdx.x == 0) {
+      __threadfence();
+      if (atomicAdd(a1.g.sched + 1, 1u) == gridDim.x - 1) {
+        atomicExch(a1.g.sched, 0u);
+        atomicExch(a1.g.sched + 1, 0u);
+        for (int i = 0; i < num_m; ++i) a1.g.ready[i] = 0;
       }
     }
   }

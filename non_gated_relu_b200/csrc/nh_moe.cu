@@ -636,10 +636,7 @@ static nh_status launch_q4(const GemmCall& c, const nh_nvfp4_weight& w, int dev,
                   st, ma, mc, ms, qa);
 }
 
-// decode-sized tiles: warp-level MMAs from registers (gemv_q4.cuh)
-template <int NT>
-static nh_status launch_q4v(const GemmCall& c, const nh_nvfp4_weight& w, int dev,
-                            cudaStream_t st) {
+static q4v::Args q4v_args(const GemmCall& c, const nh_nvfp4_weight& w) {
   q4v::Args a{};
   tc::TcArgs& g = a.g;
   g.tiles = c.tiles;
@@ -663,6 +660,22 @@ static nh_status launch_q4v(const GemmCall& c, const nh_nvfp4_weight& w, int dev
   a.scales = w.scales;
   a.gscale = w.global_scale;
   a.pitch = (int)nvfp4_pitch(c.K);
+  return a;
+}
+
+static nh_status check_q4(const nh_nvfp4_weight* w) {
+  if (!w || !w->codes || !w->scales || !w->global_scale)
+    return fail(NH_ERR_INVALID_ARG, "NVFP4 weight with a NULL pointer");
+  if (reinterpret_cast<uintptr_t>(w->codes) % 16 || reinterpret_cast<uintptr_t>(w->scales) % 16)
+    return fail(NH_ERR_INVALID_ARG, "NVFP4 codes / scales must be 16-byte aligned");
+  return NH_OK;
+}
+
+// decode-sized tiles: warp-level MMAs from registers (gemv_q4.cuh)
+template <int NT>
+static nh_status launch_q4v(const GemmCall& c, const nh_nvfp4_weight& w, int dev,
+                            cudaStream_t st) {
+  const q4v::Args a = q4v_args(c, w);
   // tasks: (tile entry, 16 weight rows).  Few tasks (dense rows: shared
   // expert, latent projections): one per CTA with K split over its warps;
   // many (routed experts): one per warp.
@@ -678,16 +691,33 @@ static nh_status launch_q4v(const GemmCall& c, const nh_nvfp4_weight& w, int dev
   const int64_t grid = std::min<int64_t>((tasks + q4v::WARPS - 1) / q4v::WARPS,
                                          (int64_t)g_sm_count[dev] * 2);
   return launch_k("q4_gemv_rows", q4v::q4_gemv_rows<NT>, dim3((unsigned)grid),
-                  dim3(q4v::WARPS * 32), 0, st, a);
+                  dim3(q4v::WARPS * 32), 0, st, a, q4v::Args{});
+}
+
+// NVFP4 decode: the routed up and down projections as one launch of the rows
+// GEMV, warps fetching tasks from a counter (up tasks first); a down task of a
+// tile entry waits until the entry's up tasks have counted themselves into
+// `ready` (zeroed by the permute and by each such launch).
+template <int NT>
+static nh_status launch_q4v_fused(const GemmCall& c1, const nh_nvfp4_weight& w1,
+                                  const GemmCall& c2, const nh_nvfp4_weight& w2, int* ready,
+                                  int dev, cudaStream_t st) {
+  q4v::Args a1 = q4v_args(c1, w1), a2 = q4v_args(c2, w2);
+  a1.g.ready = ready;
+  a2.g.ready = ready;
+  a2.g.ready_need = c1.N / q4v::MT;
+  const int64_t tasks = (int64_t)c1.max_tiles * (c1.N / q4v::MT + c2.N / q4v::MT);
+  if (tasks <= 0) return NH_OK;
+  const int64_t grid = std::min<int64_t>((tasks + q4v::WARPS - 1) / q4v::WARPS,
+                                         (int64_t)g_sm_count[dev] * 2);
+  return launch_k("q4_gemv_rows", q4v::q4_gemv_rows<NT>, dim3((unsigned)grid),
+                  dim3(q4v::WARPS * 32), 0, st, a1, a2);
 }
 
 static nh_status run_gemm_q4(const GemmCall& c, const nh_nvfp4_weight* w, int dev,
                              cudaStream_t st) {
   if (c.rows == 0) return NH_OK;
-  if (!w || !w->codes || !w->scales || !w->global_scale)
-    return fail(NH_ERR_INVALID_ARG, "NVFP4 weight with a NULL pointer");
-  if (reinterpret_cast<uintptr_t>(w->codes) % 16 || reinterpret_cast<uintptr_t>(w->scales) % 16)
-    return fail(NH_ERR_INVALID_ARG, "NVFP4 codes / scales must be 16-byte aligned");
+  NH_TRY(check_q4(w));
   switch (c.tile_rows) {
     case 16: return launch_q4v<16>(c, *w, dev, st);
     case 32: return launch_q4v<32>(c, *w, dev, st);
@@ -1263,6 +1293,25 @@ nh_status nh_moe_forward_nvfp4(const nh_moe_config* cfg, int64_t T, const void* 
                                void* ws, size_t ws_bytes, float* y_acc, void* stream) {
   if (!w_up || !w_down) return fail(NH_ERR_INVALID_ARG, "w_up / w_down is NULL");
   if (T > 0) NH_TRY(check_ptr(y_acc, "y_acc"));
+  Plan p;
+  NH_TRY(make_plan(cfg, T, &p));
+  const nh_moe_ws_layout& L = p.lay;
+  if (T > 0 && cfg->weight_format == NH_WEIGHTS_NVFP4 && !cfg->latent_size && L.x_direct &&
+      (L.tile_rows == 16 || L.tile_rows == 32)) {
+    // decode: both projections in one launch of the rows GEMV
+    NH_TRY(check_ws(p, ws, ws_bytes));
+    NH_TRY(check_ptr(x, "x"));
+    NH_TRY(check_q4(w_up));
+    NH_TRY(check_q4(w_down));
+    int dev;
+    NH_TRY(device_setup(&dev));
+    cudaStream_t st = static_cast<cudaStream_t>(stream);
+    const GemmCall up = routed_call(p, ws, T, x, nullptr, y_acc, true, true);
+    const GemmCall down = routed_call(p, ws, T, x, nullptr, y_acc, false, true);
+    int* ready = at<int>(ws, L.ready);
+    if (L.tile_rows == 16) return launch_q4v_fused<16>(up, *w_up, down, *w_down, ready, dev, st);
+    return launch_q4v_fused<32>(up, *w_up, down, *w_down, ready, dev, st);
+  }
   NH_TRY(experts_phase(cfg, T, x, nullptr, ws, ws_bytes, nullptr, stream, true, w_up));
   return experts_phase(cfg, T, x, nullptr, ws, ws_bytes, y_acc, stream, false, w_down);
 }

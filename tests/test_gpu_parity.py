@@ -188,6 +188,38 @@ def test_fused_decode_forward_matches_two_launches(name):
     assert (ready == 0).all(), "a fused launch leaves its ready counters zero"
 
 
+@pytest.mark.parametrize("name", ["small_nvfp4_t5", "small_nvfp4_t29"])
+def test_fused_nvfp4_decode_forward_repeats(name):
+    """For NVFP4 decode batches nh_moe_forward_nvfp4 runs both projections as one
+    launch of the rows GEMV (down tasks wait for their entry's up tasks).  Called
+    twice after one permute it gives the same y_acc up to float32 summation
+    order, matches the block (whose output the oracle checks), and leaves its
+    ready counters zero."""
+    import non_gated_relu_b200 as nh
+    inp = synth.make_inputs(SMALL[name])
+    blk = make_block(inp)
+    x = to_dev(inp.x)
+    T = x.shape[0]
+    b = blk.buffers(T)
+    blk.forward(x, b)
+    torch.cuda.synchronize()
+    ref = b.y_acc.cpu().numpy().copy()
+    outs = []
+    for _ in range(2):
+        acc = torch.zeros_like(b.y_acc)
+        if blk.has_shared:
+            nh.shared_nvfp4(blk.c, x, blk.q4["shared_up"], blk.q4["shared_down"], acc, b.ws_shared)
+        nh.forward_nvfp4(blk.c, x, blk.q4["up"], blk.q4["down"], b.ws, acc)
+        outs.append(acc)
+    torch.cuda.synchronize()
+    assert blk.check(T) == 0
+    for acc in outs:
+        assert_same_up_to_sum_order(acc.cpu().numpy(), ref, "f32")
+    L = nh.workspace_layout(blk.c, T)
+    ready = b.ws.view(torch.uint8)[L.ready:L.ready + 4 * L.max_tiles]
+    assert (ready == 0).all(), "a fused launch leaves its ready counters zero"
+
+
 # ----------------------------------------------------------------------------- full size
 FULL = synth.CONFIG_ORDER
 
