@@ -169,7 +169,11 @@ __device__ __forceinline__ bool wait_ready(const int* ready, int m, int need, co
     asm volatile("ld.acquire.gpu.global.s32 %0, [%1];" : "=r"(v) : "l"(ready + m) : "memory");
     if (v >= need) break;
     if ((i & 63u) == 63u) {
-      if (*w.abort_flag) return false;
+      // another CTA's wait already ran out (the status word holds an error): stop
+      if (*w.abort_flag || (w.status && *reinterpret_cast<volatile int*>(w.status) != 0)) {
+        *w.abort_flag = 1;
+        return false;
+      }
       if (globaltimer_ns() - t0 > w.timeout_ns) {
         *w.abort_flag = 1;
         record_status(w.status, NH_ERR_TIMEOUT, SITE_TC_PRODUCER, m);

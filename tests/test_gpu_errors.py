@@ -4,6 +4,9 @@
   NH_ERR_TIMEOUT in the status word and returns; the context stays usable;
 * an expert id out of range reaching the permute is caught by the kernel's
   own bounds check (NH_ERR_DEVICE_CHECK) and skipped;
+* a fused decode launch whose down tiles wait on up tiles that can never
+  complete them (the ready counters set out of reach) runs out of its bounded
+  wait, records NH_ERR_TIMEOUT and returns;
 * argument errors are reported before anything is enqueued.
 """
 import numpy as np
@@ -47,6 +50,39 @@ def test_out_of_range_expert_id_is_caught_on_device():
     nh.permute(blk.c, x, b.topk_idx, b.topk_w, b.ws)
     assert nh.check_device(b.ws) == nh.NH_ERR_DEVICE_CHECK
     # the next block call starts clean (route clears the status word)
+    y, _, _, _ = run_block(inp, blk)
+    assert np.isfinite(y).all()
+
+
+@pytest.mark.parametrize("fmt", ["bf16", "nvfp4"])
+def test_fused_decode_wait_times_out(fmt):
+    """A decode batch runs the up and down projections as one launch whose down
+    tasks wait (bounded) for their tile entry's up tasks.  With the entry
+    counters set far below zero after the permute, the waits can never end:
+    the launch must record NH_ERR_TIMEOUT and return, and the next block call
+    must run clean (the launch leaves its counters zero)."""
+    cfg = small_cfg(T=8)
+    if fmt == "nvfp4":
+        import dataclasses
+        cfg = dataclasses.replace(cfg, weight_format="nvfp4")
+    inp = synth.make_inputs(cfg)
+    blk = make_block(inp)
+    T = cfg.T
+    b = blk.buffers(T)
+    x = to_dev(inp.x)
+    nh.route_permute(blk.c, x, blk.w_router, None, b.topk_idx, b.topk_w, b.ws)
+    L = nh.workspace_layout(blk.c, T)
+    num = int(b.ws[L.num_tiles:L.num_tiles + 4].view(torch.int32).item())
+    assert num > 0
+    ready = b.ws[L.ready:L.ready + 4 * L.max_tiles].view(torch.int32)
+    ready[:num].fill_(-(1 << 24))
+    if fmt == "nvfp4":
+        nh.forward_nvfp4(blk.c, x, blk.q4["up"], blk.q4["down"], b.ws, b.y_acc)
+    else:
+        nh.forward(blk.c, x, blk.w_up, blk.w_down, b.ws, b.y_acc)
+    torch.cuda.synchronize()
+    assert nh.check_device(b.ws) == nh.NH_ERR_TIMEOUT
+    assert (ready == 0).all(), "the launch leaves the counters of its tile entries zero"
     y, _, _, _ = run_block(inp, blk)
     assert np.isfinite(y).all()
 
