@@ -224,7 +224,8 @@ nh_status nh_moe_route_noalloc(const nh_moe_config *cfg, int64_t T, const void *
  * Token permute: per-expert histogram, exclusive scan, stable scatter of the
  * (t, j) assignments in (t, j) order, the tile table of the expert GEMMs and
  * (unless the layout's x_direct is set) the gather
- * x_perm[row] = x[perm_token[row]].  The routed experts are
+ * x_perm[row] = x[perm_token[row]].  It also zeroes the layout's `ready`
+ * counters and the expert GEMMs' tile schedulers.  The routed experts are
  * applied per expert id (MLX SwitchMLP fc1/fc2 indexed by the router's
  * expert ids, exo commit "Add support for Nemotron sharding").
  *   topk_idx / topk_w as produced by nh_moe_route (any valid ids in [0, E)
@@ -251,7 +252,10 @@ nh_status nh_moe_permute(const nh_moe_config *cfg, int64_t T, const void *x,
  *   hold its starting value (zeros from nh_moe_zero_acc, optionally plus the
  *   shared expert) before the down projection runs, and no other stream may
  *   write it meanwhile except nh_moe_shared's adds.
- * Needs nh_moe_permute's workspace contents.
+ * Needs nh_moe_permute's workspace contents.  For bf16 batches of at most 32
+ * tokens both projections run as one launch (down tiles of a tile entry start
+ * once its up tiles have stored h); larger batches take one launch each.  The
+ * call may be repeated after one permute.
  */
 nh_status nh_moe_forward(const nh_moe_config *cfg, int64_t T, const void *x, const void *w_up,
                          const void *w_down, void *ws, size_t ws_bytes, float *y_acc,
@@ -264,7 +268,8 @@ nh_status nh_moe_forward(const nh_moe_config *cfg, int64_t T, const void *x, con
  * bf16): for tiles of up to 32 tokens per expert straight into warp-level MMA
  * fragments, for 64-token tiles into tensor memory as the A operand of
  * tcgen05.mma.  The float32 matrix scale is applied in the epilogue.  Adds
- * into y_acc exactly like nh_moe_forward.
+ * into y_acc exactly like nh_moe_forward; batches of at most 32 tokens run
+ * both projections as one launch, as there.
  */
 nh_status nh_moe_forward_nvfp4(const nh_moe_config *cfg, int64_t T, const void *x,
                                const nh_nvfp4_weight *w_up, const nh_nvfp4_weight *w_down,
