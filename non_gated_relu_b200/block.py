@@ -9,14 +9,10 @@ call runs, on the caller's stream and a side stream:
     main: route + permute -> forward: y_acc += routed experts (x) ---+-> finalize: y = dtype(y_acc)
                       (forward's down projection waits for y_acc = 0)
 
-That is the schedule while the routed experts stream their weights, with fewer
-than 256 rows (one CTA-pair tile) per expert on average: the shared expert
-then fills what the routed path leaves idle.  With more rows per expert every
-GEMM is bound by the tensor cores, and running the shared expert's GEMMs beside
-the routed ones only makes them contend (their float32 adds into the same y_acc
-included); there the zeroing of y_acc still runs on the side stream, beside
-route + permute, and the rest runs in turn on one stream: shared expert,
-forward, finalize.
+The shared expert runs beside the routed path at every size: at decode its
+GEMVs stream their weights while the router runs, and at prefill its GEMMs take
+the SMs that the routing and permute kernels leave idle (measured faster than
+running it in turn on one stream, from 6144 to 16384 tokens).
 
 With latent projections (config ``latent_size`` L > 0; the modules
 fc1_latent_proj / fc2_latent_proj of the ModelOpt descriptor
