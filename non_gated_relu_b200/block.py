@@ -7,7 +7,7 @@ call runs, on the caller's stream and a side stream:
 
     side: y_acc = 0 --+-> shared expert: y_acc += shared(x) ----------+
     main: route + permute -> forward: y_acc += routed experts (x) ---+-> finalize: y = dtype(y_acc)
-                      (forward's down projection waits for y_acc = 0)
+                      (forward waits for y_acc = 0)
 
 The shared expert runs beside the routed path at every size: at decode its
 GEMVs stream their weights while the router runs, and at prefill its GEMMs take
