@@ -300,6 +300,18 @@ nh_status nh_moe_shared(const nh_moe_config *cfg, int64_t T, const void *x, cons
                         const void *w_shared_down, float *y_acc, void *ws_shared,
                         size_t ws_shared_bytes, void *stream);
 
+/*
+ * The shared expert as the accumulator's starting value instead of an add:
+ *   y_acc = relu(x W_su^T)^2 W_sd^T      (float32 stores, each element once)
+ * Same arguments as nh_moe_shared.  It replaces nh_moe_zero_acc plus
+ * nh_moe_shared when it completes before any routed add into y_acc (the
+ * caller orders them, e.g. nh_moe_experts_down after an event of this call's
+ * stream), saving the zero fill and the read half of the shared adds.
+ */
+nh_status nh_moe_shared_store(const nh_moe_config *cfg, int64_t T, const void *x,
+                              const void *w_shared_up, const void *w_shared_down, float *y_acc,
+                              void *ws_shared, size_t ws_shared_bytes, void *stream);
+
 /* nh_moe_shared with NVFP4 shared-expert weights: w_shared_up [1][S][H],
  * w_shared_down [1][H][S]. */
 nh_status nh_moe_shared_nvfp4(const nh_moe_config *cfg, int64_t T, const void *x,

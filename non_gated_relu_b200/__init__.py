@@ -91,7 +91,8 @@ _lib = None
 _EXPORTS = ["nh_moe_validate", "nh_moe_workspace_size", "nh_moe_workspace_layout",
             "nh_moe_shared_workspace_size", "nh_moe_route", "nh_moe_route_noalloc", "nh_moe_route_permute",
             "nh_moe_permute", "nh_moe_forward", "nh_moe_experts_up", "nh_moe_experts_down",
-            "nh_moe_forward_nvfp4", "nh_moe_shared", "nh_moe_shared_nvfp4", "nh_moe_zero_acc",
+            "nh_moe_forward_nvfp4", "nh_moe_shared", "nh_moe_shared_store", "nh_moe_shared_nvfp4",
+            "nh_moe_zero_acc",
             "nh_moe_finalize",
             "nh_moe_latent_config", "nh_moe_latent_workspace_size", "nh_moe_latent_in",
             "nh_moe_latent_out", "nh_moe_reset_status", "nh_moe_check_device",
@@ -255,6 +256,14 @@ def shared(cfg, x, w_shared_up, w_shared_down, y_acc, ws_shared, stream=None):
     _check(load().nh_moe_shared(ctypes.byref(c), x.shape[0], _p(x), _p(w_shared_up),
                                 _p(w_shared_down), _p(y_acc), _p(ws_shared),
                                 _nbytes(ws_shared), _stream(stream)))
+
+
+def shared_store(cfg, x, w_shared_up, w_shared_down, y_acc, ws_shared, stream=None):
+    """Shared expert as y_acc's starting value: y_acc = relu(x W_su^T)^2 W_sd^T."""
+    c = config_from(cfg)
+    _check(load().nh_moe_shared_store(ctypes.byref(c), x.shape[0], _p(x), _p(w_shared_up),
+                                      _p(w_shared_down), _p(y_acc), _p(ws_shared),
+                                      _nbytes(ws_shared), _stream(stream)))
 
 
 def nvfp4_weight(codes, scales, global_scale) -> NvFp4Weight:

@@ -12,7 +12,13 @@ call runs, on the caller's stream and a side stream:
 The shared expert runs beside the routed path at every size: at decode its
 GEMVs stream their weights while the router runs, and at prefill its GEMMs take
 the SMs that the routing and permute kernels leave idle (measured faster than
-running it in turn on one stream, from 6144 to 16384 tokens).
+running it in turn on one stream, from 6144 to 16384 tokens).  For more than
+32 tokens with native weights its down projection writes y_acc's starting
+value instead of adding into zeros (no fill, no read of the zeros), and the
+routed down projection waits for it:
+
+    side: shared expert: y_acc = shared(x) ----------------------------+
+    main: route + permute -> experts_up -> (wait) experts_down: y_acc += routed -> finalize
 
 With latent projections (config ``latent_size`` L > 0; the modules
 fc1_latent_proj / fc2_latent_proj of the ModelOpt descriptor
@@ -33,9 +39,11 @@ from typing import Dict, Optional
 import numpy as np
 import torch
 
-from . import (check_device, config_from, finalize, forward, forward_nvfp4, latent_config,
+from . import (check_device, config_from, experts_down, experts_up, finalize, forward,
+               forward_nvfp4, latent_config,
                latent_in, latent_out, latent_workspace_size, nvfp4_weight, permute, reset_status,
-               route, route_permute, shared, shared_nvfp4, shared_workspace_size, validate,
+               route, route_permute, shared, shared_nvfp4, shared_store, shared_workspace_size,
+               validate,
                workspace_layout, workspace_size, zero_acc, NH_BF16, NH_WEIGHTS_NVFP4)
 
 
@@ -188,12 +196,17 @@ class NemotronHMoE:
         fork.record(caller)
         main.wait_event(fork)
         self.side.wait_event(fork)
-        # the accumulators start at zero on the side stream (beside the router)
-        push("zero_acc")
-        zero_acc(self.c, T, b.y_acc, stream=self.side)
-        if self.latent:
-            zero_acc(self.c_exp, T, b.y_lat_acc, stream=self.side)
-        pop()
+        # batches of more than 32 tokens with native weights: the shared expert's
+        # down projection writes y_acc's starting value (no zero fill, no read
+        # of the zeros), and the routed down projection waits for it
+        store = (self.has_shared and not self.nvfp4 and not self.latent and T > 32)
+        if not store:
+            # the accumulators start at zero on the side stream (beside the router)
+            push("zero_acc")
+            zero_acc(self.c, T, b.y_acc, stream=self.side)
+            if self.latent:
+                zero_acc(self.c_exp, T, b.y_lat_acc, stream=self.side)
+            pop()
         zero = torch.cuda.Event()
         zero.record(self.side)
 
@@ -204,6 +217,9 @@ class NemotronHMoE:
             push("shared")
             if self.nvfp4:
                 shared_nvfp4(self.c, x, self.q4["shared_up"], self.q4["shared_down"], b.y_acc,
+                             b.ws_shared, stream=self.side)
+            elif store:
+                shared_store(self.c, x, self.w_shared_up, self.w_shared_down, b.y_acc,
                              b.ws_shared, stream=self.side)
             else:
                 shared(self.c, x, self.w_shared_up, self.w_shared_down, b.y_acc, b.ws_shared,
@@ -222,11 +238,17 @@ class NemotronHMoE:
         push("route_permute")
         route_permute(self.c, x, self.w_router, self.bias, b.topk_idx, b.topk_w, b.ws, stream=main)
         pop()
-        main.wait_event(zero)
         push("forward")
-        if self.nvfp4:
+        if store:
+            # y_acc holds the shared expert before the routed adds begin
+            experts_up(self.c, x, self.w_up, b.ws, stream=main)
+            shared_done()
+            experts_down(self.c, T, self.w_down, b.ws, b.y_acc, stream=main)
+        elif self.nvfp4:
+            main.wait_event(zero)
             forward_nvfp4(self.c, x, self.q4["up"], self.q4["down"], b.ws, b.y_acc, stream=main)
         else:
+            main.wait_event(zero)
             forward(self.c, x, self.w_up, self.w_down, b.ws, b.y_acc, stream=main)
         pop()
         shared_done()

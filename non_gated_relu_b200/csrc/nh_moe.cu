@@ -1319,7 +1319,7 @@ nh_status nh_moe_forward_nvfp4(const nh_moe_config* cfg, int64_t T, const void* 
 static nh_status shared_impl(const nh_moe_config* cfg, int64_t T, const void* x, const void* w_su,
                              const void* w_sd, const nh_nvfp4_weight* q_su,
                              const nh_nvfp4_weight* q_sd, float* y_acc, void* ws_shared,
-                             size_t ws_shared_bytes, void* stream);
+                             size_t ws_shared_bytes, void* stream, bool store = false);
 
 nh_status nh_moe_shared_nvfp4(const nh_moe_config* cfg, int64_t T, const void* x,
                               const nh_nvfp4_weight* w_su, const nh_nvfp4_weight* w_sd,
@@ -1337,10 +1337,17 @@ nh_status nh_moe_shared(const nh_moe_config* cfg, int64_t T, const void* x, cons
                      ws_shared_bytes, stream);
 }
 
+nh_status nh_moe_shared_store(const nh_moe_config* cfg, int64_t T, const void* x,
+                              const void* w_su, const void* w_sd, float* y_acc, void* ws_shared,
+                              size_t ws_shared_bytes, void* stream) {
+  return shared_impl(cfg, T, x, w_su, w_sd, nullptr, nullptr, y_acc, ws_shared,
+                     ws_shared_bytes, stream, true);
+}
+
 static nh_status shared_impl(const nh_moe_config* cfg, int64_t T, const void* x, const void* w_su,
                              const void* w_sd, const nh_nvfp4_weight* q_su,
                              const nh_nvfp4_weight* q_sd, float* y_acc, void* ws_shared,
-                             size_t ws_shared_bytes, void* stream) {
+                             size_t ws_shared_bytes, void* stream, bool store) {
   Plan p;
   NH_TRY(make_plan(cfg, T, &p));
   const bool nvfp4 = cfg->weight_format == NH_WEIGHTS_NVFP4;
@@ -1387,7 +1394,9 @@ static nh_status shared_impl(const nh_moe_config* cfg, int64_t T, const void* x,
   dn.W = w_sd;
   dn.N = p.H;
   dn.K = p.S;
-  dn.epi = EPI_ACC_F32;   // y_acc += shared expert, beside the routed combine
+  // y_acc += shared expert, beside the routed combine; or y_acc = shared
+  // expert, the accumulator's starting value (each element is written once)
+  dn.epi = store ? EPI_STORE_F32 : EPI_ACC_F32;
   dn.out = y_acc;
   dn.ldo = p.H;
   dn.sched = reinterpret_cast<unsigned int*>(status + 6);

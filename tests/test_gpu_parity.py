@@ -220,6 +220,26 @@ def test_fused_nvfp4_decode_forward_repeats(name):
     assert (ready == 0).all(), "a fused launch leaves its ready counters zero"
 
 
+@pytest.mark.parametrize("name", ["small_prefill", "small_swap16", "small_f32_odd"])
+def test_shared_store_equals_add_into_zeros(name):
+    """nh_moe_shared_store writes the shared expert as y_acc's starting value:
+    bit-equal to nh_moe_shared adding into zeros (each element is computed once,
+    and 0 + v == v), whatever y_acc held before."""
+    import non_gated_relu_b200 as nh
+    inp = synth.make_inputs(SMALL[name])
+    blk = make_block(inp)
+    x = to_dev(inp.x)
+    T = x.shape[0]
+    b = blk.buffers(T)
+    added = torch.zeros_like(b.y_acc)
+    nh.shared(blk.c, x, blk.w_shared_up, blk.w_shared_down, added, b.ws_shared)
+    stored = torch.full_like(b.y_acc, float("nan"))
+    nh.shared_store(blk.c, x, blk.w_shared_up, blk.w_shared_down, stored, b.ws_shared)
+    torch.cuda.synchronize()
+    assert torch.equal(stored, added)
+    assert added.abs().max().item() > 0
+
+
 # ----------------------------------------------------------------------------- full size
 FULL = synth.CONFIG_ORDER
 
