@@ -377,6 +377,7 @@ def kernel_times(blk, xs, b, nb, steps):
     # decode batches (T <= 32, bf16 or NVFP4 experts): nh_moe_forward[_nvfp4]
     # runs the up and down projections as one launch
     fused = T <= 32 and (blk.nvfp4 or blk.cfg.dtype == "bf16")
+    store = blk.has_shared and not blk.nvfp4 and not blk.latent and T > 32
     acc = {n: 0.0 for n in names}
     ev = {n: (torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
           for n in names}
@@ -389,9 +390,14 @@ def kernel_times(blk, xs, b, nb, steps):
         if blk.latent:
             timed("zero_acc", lambda: (nh.zero_acc(blk.c, T, b.y_acc, stream=main),
                                        nh.zero_acc(blk.c_exp, T, b.y_lat_acc, stream=main)))
-        else:
+        elif not store:
             timed("zero_acc", lambda: nh.zero_acc(blk.c, T, b.y_acc, stream=main))
-        if blk.has_shared and blk.nvfp4:
+        if store:
+            # the block's schedule for these batches: the shared expert writes
+            # y_acc's starting value, no zero fill
+            timed("shared", lambda: nh.shared_store(blk.c, x, blk.w_shared_up, blk.w_shared_down,
+                                                     b.y_acc, b.ws_shared, stream=main))
+        elif blk.has_shared and blk.nvfp4:
             timed("shared", lambda: nh.shared_nvfp4(blk.c, x, blk.q4["shared_up"],
                                                      blk.q4["shared_down"], b.y_acc,
                                                      b.ws_shared, stream=main))
@@ -437,8 +443,8 @@ def kernel_times(blk, xs, b, nb, steps):
             timed("finalize", lambda: nh.finalize(blk.c, T, b.y_acc, b.y, stream=main))
         torch.cuda.synchronize(blk.device)
         for n in names:
-            if (n == "shared" and not blk.has_shared) or (n == "experts_down" and
-                                                            (blk.nvfp4 or fused)):
+            if ((n == "shared" and not blk.has_shared) or (n == "zero_acc" and store) or
+                    (n == "experts_down" and (blk.nvfp4 or fused))):
                 continue
             acc[n] += ev[n][0].elapsed_time(ev[n][1])
     out = {n: acc[n] / steps for n in names}
