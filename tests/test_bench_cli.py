@@ -58,3 +58,15 @@ def test_product_arm_has_no_cpu_path():
     out = run_bench("--steps", "1", "--warmup", "3")
     assert out.returncode != 0
     assert not any(ln.lstrip().startswith("{") for ln in out.stdout.splitlines())
+
+
+def test_launches_per_step_match_the_profiled_launch_lists():
+    """The kernel count per step that bench.py reports as gpu_launches, against the
+    ncu launch lists in profiles/ (kernels per graph replay: 36 in 3 prefill steps,
+    100 in 20 decode steps, 100 in 20 NVFP4 decode steps, 180 in 20 latent steps)."""
+    import bench
+    import synth
+    want = {"prefill_bf16_t16384": 12, "decode_bf16_t8": 5, "decode_nvfp4_t8": 5,
+            "decode_latent_bf16_t8": 9}
+    for name, n in want.items():
+        assert bench.launches_per_step(synth.CONFIGS[name]) == n, name
