@@ -146,28 +146,31 @@ __global__ void __launch_bounds__(WARPS * 32, 3) q4_gemv_splitk(const Args a) {
       const int arow = g.row_token ? g.row_token[ent.y + j] : ent.y + j;
       const __nv_bfloat16* act = A + (size_t)arow * K;
       float c0[4] = {0.f, 0.f, 0.f, 0.f}, c1[4] = {0.f, 0.f, 0.f, 0.f};
+      // the warp's blocks kb, kb + WARPS, ...: the next one's codes are in flight
+      // while one is used, in two register sets taken in turn (no copies)
       int kb = warp;
-      uint4 qa = make_uint4(0, 0, 0, 0), qb = qa;
-      if (kb < nkb) {
-        qa = __ldg(reinterpret_cast<const uint4*>(ca_p + (size_t)kb * 64 + 16 * tq));
-        qb = __ldg(reinterpret_cast<const uint4*>(cb_p + (size_t)kb * 64 + 16 * tq));
-      }
-      for (; kb < nkb; kb += WARPS) {
-        // the warp's next block is in flight while this one is used
-        uint4 na = qa, nbq = qb;
-        if (kb + WARPS < nkb) {
-          na = __ldg(reinterpret_cast<const uint4*>(ca_p + (size_t)(kb + WARPS) * 64 + 16 * tq));
-          nbq = __ldg(reinterpret_cast<const uint4*>(cb_p + (size_t)(kb + WARPS) * 64 + 16 * tq));
-        }
-        // thread tq's 32 features are scale groups 8 kb + 2 tq and + 1
-        const uint32_t sa2 = *reinterpret_cast<const uint16_t*>(sa_p + kb * 8 + 2 * tq);
-        const uint32_t sb2 = *reinterpret_cast<const uint16_t*>(sb_p + kb * 8 + 2 * tq);
+      uint4 qa = make_uint4(0, 0, 0, 0), qb = qa, qa2 = qa, qb2 = qa;
+      auto load = [&](int k, uint4& fa, uint4& fb) {
+        fa = __ldg(reinterpret_cast<const uint4*>(ca_p + (size_t)k * 64 + 16 * tq));
+        fb = __ldg(reinterpret_cast<const uint4*>(cb_p + (size_t)k * 64 + 16 * tq));
+      };
+      auto use = [&](int k, const uint4& fa, const uint4& fb) {
+        // thread tq's 32 features are scale groups 8 k + 2 tq and + 1
+        const uint32_t sa2 = *reinterpret_cast<const uint16_t*>(sa_p + k * 8 + 2 * tq);
+        const uint32_t sb2 = *reinterpret_cast<const uint16_t*>(sb_p + k * 8 + 2 * tq);
         const uint32_t ma[2] = {q4::scale_mult(sa2 & 0xffu), q4::scale_mult(sa2 >> 8)};
         const uint32_t mb[2] = {q4::scale_mult(sb2 & 0xffu), q4::scale_mult(sb2 >> 8)};
-        const uint32_t cwa[4] = {qa.x, qa.y, qa.z, qa.w}, cwb[4] = {qb.x, qb.y, qb.z, qb.w};
-        block_mma<128>(cwa, cwb, ma, mb, act + kb * 128 + 32 * tq, c0, c1);
-        qa = na;
-        qb = nbq;
+        const uint32_t cwa[4] = {fa.x, fa.y, fa.z, fa.w}, cwb[4] = {fb.x, fb.y, fb.z, fb.w};
+        block_mma<128>(cwa, cwb, ma, mb, act + k * 128 + 32 * tq, c0, c1);
+      };
+      if (kb < nkb) load(kb, qa, qb);
+      for (; kb < nkb; kb += 2 * WARPS) {
+        if (kb + WARPS < nkb) load(kb + WARPS, qa2, qb2);
+        use(kb, qa, qb);
+        if (kb + WARPS < nkb) {
+          if (kb + 2 * WARPS < nkb) load(kb + 2 * WARPS, qa, qb);
+          use(kb + WARPS, qa2, qb2);
+        }
       }
       if (tail && warp == nkb % WARPS) {
         // 64-feature tail: thread tq's run is features [16 tq, 16 tq + 16), one group
@@ -295,21 +298,23 @@ __global__ void __launch_bounds__(WARPS * 32, 2) q4_gemv_rows(const Args a1, con
         fsa = *reinterpret_cast<const uint16_t*>(sa_p + kb * 8 + 2 * tq);
         fsb = *reinterpret_cast<const uint16_t*>(sb_p + kb * 8 + 2 * tq);
       };
+      // two register sets used in turn (blocks kb and kb + 1): no copies between them
+      uint4 qa2 = qa, qb2 = qb, xb2[4] = {qa, qa, qa, qa};
+      uint32_t sa2b = 0, sb2b = 0;
+      auto use = [&](const uint4& fa, const uint4& fb, const uint4* fx, uint32_t fsa, uint32_t fsb) {
+        const uint32_t ma[2] = {q4::scale_mult(fsa & 0xffu), q4::scale_mult(fsa >> 8)};
+        const uint32_t mb[2] = {q4::scale_mult(fsb & 0xffu), q4::scale_mult(fsb >> 8)};
+        const uint32_t cwa[4] = {fa.x, fa.y, fa.z, fa.w}, cwb[4] = {fb.x, fb.y, fb.z, fb.w};
+        block_mma_b(cwa, cwb, ma, mb, fx, c0, c1);
+      };
       if (nkb > 0) fetch(0, qa, qb, xb, sa2, sb2);
-      for (int kb = 0; kb < nkb; ++kb) {
-        uint4 na = qa, nbq = qb, nx[4] = {xb[0], xb[1], xb[2], xb[3]};
-        uint32_t nsa = sa2, nsb = sb2;
-        if (kb + 1 < nkb) fetch(kb + 1, na, nbq, nx, nsa, nsb);
-        const uint32_t ma[2] = {q4::scale_mult(sa2 & 0xffu), q4::scale_mult(sa2 >> 8)};
-        const uint32_t mb[2] = {q4::scale_mult(sb2 & 0xffu), q4::scale_mult(sb2 >> 8)};
-        const uint32_t cwa[4] = {qa.x, qa.y, qa.z, qa.w}, cwb[4] = {qb.x, qb.y, qb.z, qb.w};
-        block_mma_b(cwa, cwb, ma, mb, xb, c0, c1);
-        qa = na;
-        qb = nbq;
-#pragma unroll
-        for (int u = 0; u < 4; ++u) xb[u] = nx[u];
-        sa2 = nsa;
-        sb2 = nsb;
+      for (int kb = 0; kb < nkb; kb += 2) {
+        if (kb + 1 < nkb) fetch(kb + 1, qa2, qb2, xb2, sa2b, sb2b);
+        use(qa, qb, xb, sa2, sb2);
+        if (kb + 1 < nkb) {
+          if (kb + 2 < nkb) fetch(kb + 2, qa, qb, xb, sa2, sb2);
+          use(qa2, qb2, xb2, sa2b, sb2b);
+        }
       }
       if (tail) {
         const size_t off = (size_t)nkb * 64 + 8 * tq;
