@@ -99,6 +99,18 @@ __device__ __forceinline__ void tmem_st_x32_wait(uint32_t taddr, const uint32_t*
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// Two E4M3 scale bytes (low byte first) -> two bf16x2 multipliers, each holding
+// its scale * 2^118 in both halves (exact): one conversion for both bytes, the
+// same arithmetic as scale_mult byte by byte.
+__device__ __forceinline__ void scale_mult2(uint32_t two, uint32_t* m) {
+  uint32_t h;
+  asm("cvt.rn.f16x2.e4m3x2 %0, %1;" : "=r"(h) : "h"((uint16_t)two));
+  const float s0 = __half2float(__ushort_as_half((uint16_t)(h & 0xffffu))) * 0x1p118f;
+  const float s1 = __half2float(__ushort_as_half((uint16_t)(h >> 16))) * 0x1p118f;
+  m[0] = pack_bf16x2(s0, s0);
+  m[1] = pack_bf16x2(s1, s1);
+}
+
 // E4M3 scale byte -> bf16x2 holding scale * 2^118 in both halves (exact)
 __device__ __forceinline__ uint32_t scale_mult(uint32_t byte) {
   uint32_t h;

@@ -158,8 +158,9 @@ __global__ void __launch_bounds__(WARPS * 32, 3) q4_gemv_splitk(const Args a) {
         // thread tq's 32 features are scale groups 8 k + 2 tq and + 1
         const uint32_t sa2 = *reinterpret_cast<const uint16_t*>(sa_p + k * 8 + 2 * tq);
         const uint32_t sb2 = *reinterpret_cast<const uint16_t*>(sb_p + k * 8 + 2 * tq);
-        const uint32_t ma[2] = {q4::scale_mult(sa2 & 0xffu), q4::scale_mult(sa2 >> 8)};
-        const uint32_t mb[2] = {q4::scale_mult(sb2 & 0xffu), q4::scale_mult(sb2 >> 8)};
+        uint32_t ma[2], mb[2];
+        q4::scale_mult2(sa2, ma);
+        q4::scale_mult2(sb2, mb);
         const uint32_t cwa[4] = {fa.x, fa.y, fa.z, fa.w}, cwb[4] = {fb.x, fb.y, fb.z, fb.w};
         block_mma<128>(cwa, cwb, ma, mb, act + k * 128 + 32 * tq, c0, c1);
       };
@@ -302,8 +303,9 @@ __global__ void __launch_bounds__(WARPS * 32, 2) q4_gemv_rows(const Args a1, con
       uint4 qa2 = qa, qb2 = qb, xb2[4] = {qa, qa, qa, qa};
       uint32_t sa2b = 0, sb2b = 0;
       auto use = [&](const uint4& fa, const uint4& fb, const uint4* fx, uint32_t fsa, uint32_t fsb) {
-        const uint32_t ma[2] = {q4::scale_mult(fsa & 0xffu), q4::scale_mult(fsa >> 8)};
-        const uint32_t mb[2] = {q4::scale_mult(fsb & 0xffu), q4::scale_mult(fsb >> 8)};
+        uint32_t ma[2], mb[2];
+        q4::scale_mult2(fsa, ma);
+        q4::scale_mult2(fsb, mb);
         const uint32_t cwa[4] = {fa.x, fa.y, fa.z, fa.w}, cwb[4] = {fb.x, fb.y, fb.z, fb.w};
         block_mma_b(cwa, cwb, ma, mb, fx, c0, c1);
       };
