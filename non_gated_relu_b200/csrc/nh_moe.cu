@@ -1116,8 +1116,8 @@ nh_status nh_moe_permute(const nh_moe_config* cfg, int64_t T, const void* x,
         at<__nv_bfloat16>(ws, L.x_perm), status, 0)));
     NH_TRY(launch_check("permute_scatter"));
     NH_TRY((launch_k("permute_gather", permute_gather<__nv_bfloat16>, dim3(gather_blocks), dim3(256), 0, st, 
-        static_cast<const __nv_bfloat16*>(x), at<int32_t>(ws, L.perm_token),
-        at<int32_t>(ws, L.offsets), p.E, p.H, at<__nv_bfloat16>(ws, L.x_perm))));
+        static_cast<const __nv_bfloat16*>(x), at<int32_t>(ws, L.inv_row), (int)T, p.k, p.H,
+        at<__nv_bfloat16>(ws, L.x_perm))));
   } else {
     NH_TRY((launch_k("permute_scatter", permute_scatter<float>, dim3(L.n_chunks), dim3(32), smem, st, 
         topk_idx, topk_w, static_cast<const float*>(x), (int)T, p.k, p.E, p.H, chunk,
@@ -1125,8 +1125,8 @@ nh_status nh_moe_permute(const nh_moe_config* cfg, int64_t T, const void* x,
         at<float>(ws, L.x_perm), status, 0)));
     NH_TRY(launch_check("permute_scatter"));
     NH_TRY((launch_k("permute_gather", permute_gather<float>, dim3(gather_blocks), dim3(256), 0, st, 
-        static_cast<const float*>(x), at<int32_t>(ws, L.perm_token), at<int32_t>(ws, L.offsets),
-        p.E, p.H, at<float>(ws, L.x_perm))));
+        static_cast<const float*>(x), at<int32_t>(ws, L.inv_row), (int)T, p.k, p.H,
+        at<float>(ws, L.x_perm))));
   }
   return launch_check("permute_gather");
 }

@@ -239,19 +239,56 @@ __device__ __forceinline__ void copy_row(const Tin* __restrict__ src, Tin* __res
   }
 }
 
-// x_perm[p] = x[perm_token[p]] for every permuted row (one warp per row)
+// x_perm[inv_row[t k + j]] = x[t] for every token t and choice j: one warp per
+// token reads the row once, GATHER_CH 16-byte words per lane at a time, and
+// stores it to each of the token's permuted rows (rows of dropped choices,
+// inv_row < 0, do not exist).  Every permuted row is written exactly once.
+constexpr int GATHER_CH = 8;
+
 template <typename Tin>
 __global__ void __launch_bounds__(256) permute_gather(const Tin* __restrict__ x,
-                                                      const int32_t* __restrict__ perm_token,
-                                                      const int32_t* __restrict__ offsets, int E,
-                                                      int H, Tin* __restrict__ x_perm) {
+                                                      const int32_t* __restrict__ inv_row, int T,
+                                                      int k, int H, Tin* __restrict__ x_perm) {
   pdl_wait();
   pdl_trigger();
   const int lane = threadIdx.x & 31;
-  const int rows = offsets[E];
   const int nw = (gridDim.x * blockDim.x) >> 5;
-  for (int p = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; p < rows; p += nw)
-    copy_row(x + (size_t)perm_token[p] * H, x_perm + (size_t)p * H, H, lane);
+  const size_t row_bytes = (size_t)H * sizeof(Tin);
+  for (int t = (blockIdx.x * blockDim.x + threadIdx.x) >> 5; t < T; t += nw) {
+    const Tin* src = x + (size_t)t * H;
+    for (int j0 = 0; j0 < k; j0 += 32) {
+      const int nj = min(32, k - j0);
+      const int dst = lane < nj ? inv_row[(size_t)t * k + j0 + lane] : -1;
+      if (row_bytes % 16 == 0) {
+        const int nv = (int)(row_bytes / 16);
+        const uint4* s4 = reinterpret_cast<const uint4*>(src);
+        for (int v0 = 0; v0 < nv; v0 += 32 * GATHER_CH) {
+          uint4 r[GATHER_CH];
+#pragma unroll
+          for (int u = 0; u < GATHER_CH; ++u) {
+            const int i = v0 + 32 * u + lane;
+            if (i < nv) r[u] = s4[i];
+          }
+          for (int j = 0; j < nj; ++j) {
+            const int p = __shfl_sync(0xffffffffu, dst, j);
+            if (p < 0) continue;
+            uint4* d4 = reinterpret_cast<uint4*>(x_perm + (size_t)p * H);
+#pragma unroll
+            for (int u = 0; u < GATHER_CH; ++u) {
+              const int i = v0 + 32 * u + lane;
+              if (i < nv) d4[i] = r[u];
+            }
+          }
+        }
+      } else {
+        for (int j = 0; j < nj; ++j) {
+          const int p = __shfl_sync(0xffffffffu, dst, j);
+          if (p >= 0)
+            for (int i = lane; i < H; i += 32) x_perm[(size_t)p * H + i] = src[i];
+        }
+      }
+    }
+  }
 }
 
 // Whole permute of T <= PERM_CHUNK tokens by one block of blockDim.x >= E
