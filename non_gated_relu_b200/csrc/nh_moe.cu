@@ -270,6 +270,7 @@ static int g_pair_clusters[MAX_DEVICES];  // co-resident 2-CTA clusters of tc2_g
 static nh_status g_attr_status[MAX_DEVICES];
 
 using TcPrefill = tc::Shape<false, 256, 4>;
+using TcPrefill128 = tc::Shape<false, 128, 6>;
 using TcSwap16 = tc::Shape<true, 16, 8>;
 using TcSwap32 = tc::Shape<true, 32, 8>;
 using TcSwap64 = tc::Shape<true, 64, 6>;
@@ -283,6 +284,8 @@ static nh_status set_attrs(int dev) {
                 prop.major, prop.minor);
   NH_CUDA(cudaFuncSetAttribute(tc::tc_grouped_gemm<false, 256, 4>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, TcPrefill::SMEM));
+  NH_CUDA(cudaFuncSetAttribute(tc::tc_grouped_gemm<false, 128, 6>,
+                               cudaFuncAttributeMaxDynamicSharedMemorySize, TcPrefill128::SMEM));
   NH_CUDA(cudaFuncSetAttribute(tc::tc_grouped_gemm<true, 16, 8>,
                                cudaFuncAttributeMaxDynamicSharedMemorySize, TcSwap16::SMEM));
   NH_CUDA(cudaFuncSetAttribute(tc::tc_grouped_gemm<true, 32, 8>,
@@ -992,7 +995,12 @@ nh_status nh_moe_route(const nh_moe_config* cfg, int64_t T, const void* x, const
     c.ldo = p.E;
     c.status = status;
     c.sched = reinterpret_cast<unsigned int*>(status + SCHED_ROUTER);
-    NH_TRY((launch_tc<false, 256, 4>(c, dev, st)));
+    // up to 128 experts fit one 128-wide N tile (a 256-wide tile would spend
+    // half of its MMA work on zero-filled weight rows)
+    if (p.E <= 128)
+      NH_TRY((launch_tc<false, 128, 6>(c, dev, st)));
+    else
+      NH_TRY((launch_tc<false, 256, 4>(c, dev, st)));
   } else {
     dim3 grid((unsigned)((T + RT_BT - 1) / RT_BT), (unsigned)((p.E + RT_BE - 1) / RT_BE));
     if (p.bf16)
