@@ -12,7 +12,10 @@ call runs, on the caller's stream and a side stream:
 The shared expert runs beside the routed path at every size: at decode its
 GEMVs stream their weights while the router runs, and at prefill its GEMMs take
 the SMs that the routing and permute kernels leave idle (measured faster than
-running it in turn on one stream, from 6144 to 16384 tokens).  For more than
+running it in turn on one stream, from 6144 to 16384 tokens).  For bf16 decode
+batches (at most 32 tokens) the router is launched before the shared expert, so
+that its blocks reach the SMs first; the streams and their joins are the same.
+For more than
 32 tokens with native weights its down projection writes y_acc's starting
 value instead of adding into zeros (no fill, no read of the zeros), and the
 routed down projection waits for it:
@@ -200,6 +203,16 @@ class NemotronHMoE:
         # down projection writes y_acc's starting value (no zero fill, no read
         # of the zeros), and the routed down projection waits for it
         store = (self.has_shared and not self.nvfp4 and not self.latent and T > 32)
+        # bf16 decode batches: the router goes to the GPU ahead of the shared
+        # expert's GEMV, whose CTAs would otherwise hold the registers that the
+        # router's blocks wait for (1 % of the step, measured; with NVFP4
+        # weights and at prefill the shared expert first is as fast or faster)
+        route_first = not self.latent and not self.nvfp4 and T <= 32
+        if route_first:
+            push("route_permute")
+            route_permute(self.c, x, self.w_router, self.bias, b.topk_idx, b.topk_w, b.ws,
+                          stream=main)
+            pop()
         if not store:
             # the accumulators start at zero on the side stream (beside the router)
             push("zero_acc")
@@ -235,9 +248,11 @@ class NemotronHMoE:
             out = self._forward_latent(x, b, main, zero, shared_done, partial, push, pop)
             self._join(caller, main)
             return out
-        push("route_permute")
-        route_permute(self.c, x, self.w_router, self.bias, b.topk_idx, b.topk_w, b.ws, stream=main)
-        pop()
+        if not route_first:
+            push("route_permute")
+            route_permute(self.c, x, self.w_router, self.bias, b.topk_idx, b.topk_w, b.ws,
+                          stream=main)
+            pop()
         push("forward")
         if store:
             # y_acc holds the shared expert before the routed adds begin
